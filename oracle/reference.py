@@ -1,0 +1,288 @@
+"""Plain float64 CPU oracle for content-routed block-sparse attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+benchmark's CPU-baseline leg may import this module.  It shares no code with
+the CUDA path (no kernels, headers, helpers, tables or pre-/post-processing);
+the two meet only in the seeded input generator, which holds none of the
+method's arithmetic.
+
+What it computes, step by step, in the order the method states it
+(jonsmirl/ssa README: the introduction, "Algorithm and complexity" and
+"Mathematical status"; SingleZombie/LLSA README, "Minimum Usage" for the
+non-causal variant):
+
+1. Upcast bf16 Q, K, V to float64 (exact).
+2. Query head h reads KV head h // (Hq / Hkv) (consecutive grouped-query
+   attention, the "native grouped-query attention" of the SSA 10M run).
+3. Block summaries: mu_c = mean of the Bk keys of key block c; the query
+   block qb is summarised by qbar = mean of its Bq queries.  (SSA's routing
+   score r_c(q) = <q, mu_c> + (beta/2) q^T Sigma_c q is taken with beta = 0:
+   mean pooling only.  Because the score is linear in q, scoring the mean
+   query equals averaging the per-query scores over the block.)
+4. Admissible key blocks of query block qb: causal -- the completed blocks
+   that end at or before the block's first query, (c+1)*Bk <= qb*Bq, so no
+   summary averages a future key; non-causal -- every key block.
+5. Score s_c = <qbar, mu_c> (unscaled: a positive scale does not change the
+   ranking).
+6. Selection: the first min(top_k, |A|) admissible blocks in the order
+   (score descending, block index ascending) -- ties go to the lower index --
+   stored ascending by block index, padded with -1, with their count.
+7. Key set of query i as a SET: the keys of its query block's selected blocks
+   united with the local causal window {j : i - W < j <= i} and cut at i
+   (causal); only the selected blocks' keys (non-causal).  A key that is both
+   routed and in the window counts once.
+8. Exact softmax over that set: l_j = scale * <q_i, k_j>, scale = 1/sqrt(D)
+   by default; o_i = sum_j softmax(l)_j v_j; lse_i = max l + log sum exp(l - max l)
+   (natural log).  The dense N x N matrix is never needed: the masked-dense
+   form builds one query block's rows at a time.
+
+Two attend forms are provided and must agree: ``attend_masked_dense`` (a
+[Bq, N] logit slab with -inf outside each row's set) and ``attend_gathered``
+(each query's explicit key-index set).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+import math
+
+import numpy as np
+
+__all__ = [
+    "Params", "upcast_bf16", "block_summary", "admissible_blocks", "route",
+    "RouteResult", "key_set", "attend_masked_dense", "attend_gathered", "forward",
+    "near_tie_rows",
+]
+
+NEAR_TIE_REL = 1e-4   # relative score gap under which two blocks count as tied
+
+
+@dataclass(frozen=True)
+class Params:
+    """Method parameters (names follow the pages' notation)."""
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    D: int
+    block_k: int
+    block_q: int
+    top_k: int
+    window: int
+    causal: bool
+    scale: float = 0.0          # 0 -> 1/sqrt(D)
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def n_kblocks(self) -> int:
+        return self.N // self.block_k
+
+    @property
+    def n_qblocks(self) -> int:
+        return self.N // self.block_q
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale > 0 else 1.0 / math.sqrt(self.D)
+
+    @staticmethod
+    def of(w) -> "Params":
+        """Build from any object with the same field names (e.g. a workload)."""
+        return Params(w.B, w.Hq, w.Hkv, w.N, w.D, w.block_k, w.block_q, w.top_k,
+                      w.window, bool(w.causal), getattr(w, "scale", 0.0))
+
+
+def upcast_bf16(u16: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float64.  A bf16 value is a float32 whose low 16
+    bits are zero, so the upcast is exact."""
+    u32 = np.asarray(u16, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u32.view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# step 3: block summaries
+# --------------------------------------------------------------------------
+def block_summary(x: np.ndarray, block: int) -> np.ndarray:
+    """Mean of every ``block`` consecutive rows of ``x[..., N, D]``.
+
+    jonsmirl/ssa README, "Algorithm and complexity": mu_c is block c's mean
+    key (the first cumulant of the second-cumulant routing score)."""
+    n, d = x.shape[-2], x.shape[-1]
+    if n % block:
+        raise ValueError("sequence length must be a multiple of the block size")
+    return x.reshape(*x.shape[:-2], n // block, block, d).mean(axis=-2)
+
+
+# --------------------------------------------------------------------------
+# step 4: admissible blocks
+# --------------------------------------------------------------------------
+def admissible_blocks(qb: int, p: Params) -> np.ndarray:
+    """Key blocks query block ``qb`` may route to.
+
+    Causal: only completed blocks that end at or before the query block's
+    first token, (c + 1) * Bk <= qb * Bq -- a routed set is causal only once
+    it is cut at each query's position (jonsmirl/ssa README, "Mathematical
+    status" and "Known limitations"); taking whole past blocks keeps every
+    summary free of future keys, and the current partial block is reached
+    through the local window.  Non-causal: all key blocks (LLSA)."""
+    if not p.causal:
+        return np.arange(p.n_kblocks)
+    last = (qb * p.block_q) // p.block_k          # blocks 0 .. last-1 are complete
+    return np.arange(min(last, p.n_kblocks))
+
+
+# --------------------------------------------------------------------------
+# steps 5-6: scores and top-k
+# --------------------------------------------------------------------------
+@dataclass
+class RouteResult:
+    idx: np.ndarray        # int32 [B, Hq, NQB, top_k], ascending, -1 padded
+    cnt: np.ndarray        # int32 [B, Hq, NQB]
+    kth: np.ndarray        # float64 [B, Hq, NQB]: k-th best score (nan if none)
+    next: np.ndarray       # float64 [B, Hq, NQB]: (k+1)-th best score (nan if none)
+
+
+def route_row(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, top_k: int):
+    """Select from candidate blocks ``cand`` for one query-block summary.
+
+    Returns (selected ascending, k-th score, (k+1)-th score)."""
+    if len(cand) == 0 or top_k == 0:
+        return np.zeros(0, dtype=np.int64), math.nan, math.nan
+    s = mu[cand] @ qbar
+    # order: score descending, then block index ascending (lower index wins a tie)
+    order = np.lexsort((cand, -s))
+    take = min(top_k, len(cand))
+    chosen = np.sort(cand[order[:take]])
+    kth = s[order[take - 1]]
+    nxt = s[order[take]] if take < len(cand) else math.nan
+    return chosen, kth, nxt
+
+
+def route(qsum: np.ndarray, ksum: np.ndarray, p: Params, rows=None) -> RouteResult:
+    """Top-k routing for every (b, query head, query block).
+
+    ``qsum`` [B, Hq, NQB, D] and ``ksum`` [B, Hkv, NB, D] are block summaries
+    (float64).  ``rows`` optionally restricts the work to a list of
+    (b, h, qb) triples; the arrays keep their full shape and rows not listed
+    stay at idx = -1, cnt = 0, scores nan."""
+    nqb = p.n_qblocks
+    idx = np.full((p.B, p.Hq, nqb, p.top_k), -1, dtype=np.int32)
+    cnt = np.zeros((p.B, p.Hq, nqb), dtype=np.int32)
+    kth = np.full((p.B, p.Hq, nqb), math.nan)
+    nxt = np.full((p.B, p.Hq, nqb), math.nan)
+    todo = rows if rows is not None else [
+        (b, h, qb) for b in range(p.B) for h in range(p.Hq) for qb in range(nqb)]
+    for b, h, qb in todo:
+        mu = ksum[b, h // p.group]
+        sel, a, c = route_row(qsum[b, h, qb], mu, admissible_blocks(qb, p), p.top_k)
+        idx[b, h, qb, :len(sel)] = sel
+        cnt[b, h, qb] = len(sel)
+        kth[b, h, qb], nxt[b, h, qb] = a, c
+    return RouteResult(idx, cnt, kth, nxt)
+
+
+def near_tie_rows(r: RouteResult, rel: float = NEAR_TIE_REL) -> np.ndarray:
+    """Rows whose k-th and (k+1)-th scores differ by less than ``rel`` of the
+    larger magnitude: at such a row either choice is an acceptable top-k."""
+    a, c = r.kth, r.next
+    with np.errstate(invalid="ignore"):
+        gap = np.abs(a - c)
+        tol = rel * np.maximum(np.abs(a), np.abs(c))
+        return np.isfinite(gap) & (gap <= tol)
+
+
+# --------------------------------------------------------------------------
+# step 7: key sets
+# --------------------------------------------------------------------------
+def key_set(i: int, sel_blocks: np.ndarray, p: Params) -> np.ndarray:
+    """Sorted key positions query ``i`` attends to (a set: no duplicates)."""
+    routed = (np.asarray(sel_blocks, dtype=np.int64)[:, None] * p.block_k
+              + np.arange(p.block_k)[None, :]).ravel()
+    if not p.causal:
+        return np.unique(routed)
+    window = np.arange(max(0, i - p.window + 1), i + 1)
+    s = np.union1d(routed, window)
+    return s[s <= i]
+
+
+# --------------------------------------------------------------------------
+# step 8: exact softmax over each query's set
+# --------------------------------------------------------------------------
+def _softmax_read(logits: np.ndarray, vals: np.ndarray):
+    m = logits.max(axis=-1, keepdims=True)
+    w = np.exp(logits - m)
+    z = w.sum(axis=-1, keepdims=True)
+    return (w @ vals) / z, (m + np.log(z))[..., 0]
+
+
+def attend_masked_dense(q, k, v, idx, cnt, p: Params, blocks=None):
+    """Masked-dense form: for each query block, a [Bq, N] logit slab with -inf
+    outside each row's key set.
+
+    ``q`` [B, Hq, N, D], ``k``/``v`` [B, Hkv, N, *] float64.  ``blocks``
+    optionally restricts the work to a list of (b, h, qb) triples; the
+    returned arrays are then [len(blocks), Bq, Dv] and [len(blocks), Bq].
+    Otherwise returns O [B, Hq, N, Dv] and LSE [B, Hq, N]."""
+    scale = p.softmax_scale
+    dv = v.shape[-1]
+    todo = blocks if blocks is not None else [
+        (b, h, qb) for b in range(p.B) for h in range(p.Hq) for qb in range(p.n_qblocks)]
+    o_out = np.zeros((len(todo), p.block_q, dv))
+    l_out = np.zeros((len(todo), p.block_q))
+    jpos = np.arange(p.N)
+    jblk = jpos // p.block_k
+    for t, (b, h, qb) in enumerate(todo):
+        g = h // p.group
+        rows = np.arange(qb * p.block_q, (qb + 1) * p.block_q)
+        routed = np.zeros(p.n_kblocks, dtype=bool)
+        routed[idx[b, h, qb, :cnt[b, h, qb]]] = True
+        allow = np.broadcast_to(routed[jblk][None, :], (len(rows), p.N)).copy()
+        if p.causal:
+            allow |= jpos[None, :] > rows[:, None] - p.window
+            allow &= jpos[None, :] <= rows[:, None]
+        logits = (q[b, h, rows] @ k[b, g].T) * scale
+        logits = np.where(allow, logits, -np.inf)
+        o_out[t], l_out[t] = _softmax_read(logits, v[b, g])
+    if blocks is not None:
+        return o_out, l_out
+    o = o_out.reshape(p.B, p.Hq, p.N, dv)
+    lse = l_out.reshape(p.B, p.Hq, p.N)
+    return o, lse
+
+
+def attend_gathered(q, k, v, idx, cnt, p: Params, queries=None):
+    """Gathered form: each query's explicit key set, then softmax over it.
+
+    ``queries`` optionally lists (b, h, i) triples; the result is then
+    ([len, Dv], [len]).  Otherwise returns O [B, Hq, N, Dv], LSE [B, Hq, N]."""
+    scale = p.softmax_scale
+    dv = v.shape[-1]
+    todo = queries if queries is not None else [
+        (b, h, i) for b in range(p.B) for h in range(p.Hq) for i in range(p.N)]
+    o_out = np.zeros((len(todo), dv))
+    l_out = np.zeros(len(todo))
+    for t, (b, h, i) in enumerate(todo):
+        g = h // p.group
+        qb = i // p.block_q
+        s = key_set(i, idx[b, h, qb, :cnt[b, h, qb]], p)
+        logits = (k[b, g, s] @ q[b, h, i]) * scale
+        o1, l1 = _softmax_read(logits[None, :], v[b, g, s])
+        o_out[t], l_out[t] = o1[0], l1[0]
+    if queries is not None:
+        return o_out, l_out
+    return o_out.reshape(p.B, p.Hq, p.N, dv), l_out.reshape(p.B, p.Hq, p.N)
+
+
+def forward(q, k, v, p: Params, form: str = "dense"):
+    """Whole path: summaries -> routing -> attend.  Inputs float64 arrays
+    (use ``upcast_bf16`` on bf16 bit patterns).  Returns a dict with
+    ``o``, ``lse``, ``idx``, ``cnt``, ``route`` (RouteResult), ``qsum``, ``ksum``."""
+    ksum = block_summary(k, p.block_k)
+    qsum = block_summary(q, p.block_q)
+    r = route(qsum, ksum, p)
+    attend = attend_masked_dense if form == "dense" else attend_gathered
+    o, lse = attend(q, k, v, r.idx, r.cnt, p)
+    return {"o": o, "lse": lse, "idx": r.idx, "cnt": r.cnt, "route": r,
+            "qsum": qsum, "ksum": ksum}

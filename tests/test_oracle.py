@@ -1,0 +1,357 @@
+"""Pins for the float64 oracle against facts fixed outside it.
+
+Each test checks the oracle against something other than itself: a
+hand-derived worked example (tests/golden), a library routine in a special
+case the method reduces to (torch SDPA in float64 on the CPU), closed forms,
+or invariants (set semantics, the lower-index tie rule, weights summing to 1,
+the append law of the softmax read, causality).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _params(**kw):
+    base = dict(B=1, Hq=1, Hkv=1, N=8, D=2, block_k=2, block_q=2, top_k=1,
+                window=2, causal=True, scale=0.0)
+    base.update(kw)
+    return O.Params(**base)
+
+
+def _worked_inputs():
+    k = np.array([[1, 0], [1, 0], [0, 1], [0, 1], [-1, 0], [-1, 0], [0, -1], [0, -1]],
+                 dtype=np.float64)
+    q = np.tile(np.array([[0.0, 2.0]]), (8, 1))
+    v = np.stack([np.arange(8.0), np.ones(8)], axis=1)
+    return q[None, None], k[None, None], v[None, None]
+
+
+def _read_worked_golden():
+    rows = []
+    with open(os.path.join(GOLDEN, "worked_example_4block.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            kk, i, expr = line.split(maxsplit=2)
+            rows.append((int(kk), int(i), expr))
+    return rows
+
+
+# ---------------------------------------------------------------- worked example
+@pytest.mark.parametrize("form", ["dense", "gathered"])
+def test_worked_example_matches_hand_derivation(form):
+    q, k, v = _worked_inputs()
+    E = math.exp(math.sqrt(2.0))
+    rows = _read_worked_golden()
+    assert len(rows) == 26
+    by_k = {}
+    for kk, i, expr in rows:
+        by_k.setdefault(kk, []).append((i, eval(expr, {"E": E})))
+    for kk, items in by_k.items():
+        p = _params(top_k=kk)
+        out = O.forward(q, k, v, p, form=form)
+        for i, want in items:
+            assert out["o"][0, 0, i, 0] == pytest.approx(want, abs=1e-12), (kk, i)
+        np.testing.assert_allclose(out["o"][0, 0, :, 1], 1.0, atol=1e-14)
+
+
+def test_worked_example_routing_and_tie_rule():
+    q, k, v = _worked_inputs()
+    p1 = O.forward(q, k, v, _params(top_k=1))
+    assert p1["idx"][0, 0, :, 0].tolist() == [-1, 0, 1, 1]
+    assert p1["cnt"][0, 0].tolist() == [0, 1, 1, 1]
+    p2 = O.forward(q, k, v, _params(top_k=2))
+    # qb3 scores (0, 2, 0): block 1, then the tie between blocks 0 and 2 goes to 0
+    assert p2["idx"][0, 0, 3].tolist() == [0, 1]
+    assert p2["idx"][0, 0, 2].tolist() == [0, 1]
+    assert p2["idx"][0, 0, 1].tolist() == [0, -1]
+    assert p2["cnt"][0, 0].tolist() == [0, 1, 2, 2]
+    # block means are the hand values
+    np.testing.assert_array_equal(p2["ksum"][0, 0], [[1, 0], [0, 1], [-1, 0], [0, -1]])
+
+
+# ---------------------------------------------------------------- summaries
+def test_block_summary_closed_form():
+    # rows K[t, :] = t (exact in binary): the mean of block c is c*Bk + (Bk-1)/2
+    for bk in (1, 2, 16, 64):
+        n = bk * 5
+        x = np.tile(np.arange(n, dtype=np.float64)[:, None], (1, 3))[None, None]
+        s = O.block_summary(x, bk)
+        want = np.arange(5) * bk + (bk - 1) / 2
+        np.testing.assert_array_equal(s[0, 0, :, 0], want)
+
+
+def test_block_summary_rejects_ragged():
+    with pytest.raises(ValueError):
+        O.block_summary(np.zeros((1, 1, 10, 2)), 4)
+
+
+# ---------------------------------------------------------------- routing
+def _route_property_check(qsum, ksum, r, p):
+    """Selection property written pairwise: every selected admissible block
+    beats every unselected one in (score desc, index asc)."""
+    for b in range(p.B):
+        for h in range(p.Hq):
+            mu = ksum[b, h // p.group]
+            for qb in range(p.n_qblocks):
+                if p.causal:
+                    adm = [c for c in range(p.n_kblocks) if (c + 1) * p.block_k <= qb * p.block_q]
+                else:
+                    adm = list(range(p.n_kblocks))
+                c_n = int(r.cnt[b, h, qb])
+                sel = r.idx[b, h, qb, :c_n].tolist()
+                assert c_n == min(p.top_k, len(adm))
+                assert (r.idx[b, h, qb, c_n:] == -1).all()
+                assert sel == sorted(sel) and len(set(sel)) == c_n
+                assert set(sel) <= set(adm)
+                s = {c: float(np.dot(qsum[b, h, qb], mu[c])) for c in adm}
+                for a in sel:
+                    for u in set(adm) - set(sel):
+                        assert (s[a] > s[u]) or (s[a] == s[u] and a < u), (qb, a, u)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_route_selection_property_with_planted_ties(causal):
+    # entries in {-1, 0, 1} with Bk = 2 make block means multiples of 1/2 and
+    # scores multiples of 1/4: exact ties are frequent, so the lower-index rule
+    # is exercised many times
+    rng = np.random.default_rng(7)
+    p = _params(B=2, Hq=4, Hkv=2, N=48, D=3, block_k=2, block_q=4, top_k=3,
+                window=3, causal=causal)
+    q = rng.integers(-1, 2, size=(2, 4, 48, 3)).astype(np.float64)
+    k = rng.integers(-1, 2, size=(2, 2, 48, 3)).astype(np.float64)
+    qs, ks = O.block_summary(q, 4), O.block_summary(k, 2)
+    r = O.route(qs, ks, p)
+    _route_property_check(qs, ks, r, p)
+    ties = 0
+    for b in range(2):
+        for h in range(4):
+            for qb in range(p.n_qblocks):
+                sc = ks[b, h // 2] @ qs[b, h, qb]
+                ties += len(sc) - len(np.unique(sc))
+    assert ties > 20
+
+
+def test_route_all_equal_keys_pick_lowest_indices():
+    p = _params(N=64, D=4, block_k=4, block_q=4, top_k=5, window=4)
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((1, 1, 64, 4))
+    k = np.ones((1, 1, 64, 4))
+    r = O.route(O.block_summary(q, 4), O.block_summary(k, 4), p)
+    for qb in range(16):
+        n = min(5, qb)
+        assert r.idx[0, 0, qb, :n].tolist() == list(range(n))
+        assert r.cnt[0, 0, qb] == n
+
+
+def test_route_brute_force_tiny():
+    # brute force: enumerate every subset of the admissible blocks of the right
+    # size; the chosen one is the unique subset that beats its complement
+    import itertools
+    rng = np.random.default_rng(3)
+    p = _params(N=24, D=2, block_k=3, block_q=3, top_k=3, window=1)
+    q = rng.standard_normal((1, 1, 24, 2))
+    k = rng.standard_normal((1, 1, 24, 2))
+    qs, ks = O.block_summary(q, 3), O.block_summary(k, 3)
+    r = O.route(qs, ks, p)
+    for qb in range(8):
+        adm = list(range(qb))
+        s = ks[0, 0, :qb] @ qs[0, 0, qb]
+        n = min(3, qb)
+        best = max(itertools.combinations(adm, n), key=lambda sub: sorted(s[list(sub)])[::-1])
+        assert sorted(best) == r.idx[0, 0, qb, :n].tolist()
+
+
+# ---------------------------------------------------------------- attend: special cases
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _sdpa(q, k, v, mask=None, causal=False, gqa=False):
+    t = [torch.from_numpy(np.ascontiguousarray(a)) for a in (q, k, v)]
+    m = None if mask is None else torch.from_numpy(mask)
+    return F.scaled_dot_product_attention(t[0], t[1], t[2], attn_mask=m, is_causal=causal,
+                                          enable_gqa=gqa).numpy()
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,bk", [(16, 2, 2, 8), (32, 4, 2, 16), (64, 6, 2, 32)])
+def test_dense_causal_when_topk_covers_every_block(D, Hq, Hkv, bk):
+    N = 8 * bk
+    p = _params(B=2, Hq=Hq, Hkv=Hkv, N=N, D=D, block_k=bk, block_q=bk, top_k=N // bk,
+                window=bk)
+    q, k, v = _rand((2, Hq, N, D), 1), _rand((2, Hkv, N, D), 2), _rand((2, Hkv, N, D), 3)
+    out = O.forward(q, k, v, p)
+    want = _sdpa(q, k, v, causal=True, gqa=Hq != Hkv)
+    np.testing.assert_allclose(out["o"], want, atol=1e-12, rtol=0)
+
+
+def test_dense_noncausal_when_topk_covers_every_block():
+    N, D, bk = 128, 16, 16
+    p = _params(B=1, Hq=2, Hkv=1, N=N, D=D, block_k=bk, block_q=bk, top_k=N // bk,
+                window=0, causal=False)
+    q, k, v = _rand((1, 2, N, D), 4), _rand((1, 1, N, D), 5), _rand((1, 1, N, D), 6)
+    out = O.forward(q, k, v, p)
+    want = _sdpa(q, k, v, gqa=True)
+    np.testing.assert_allclose(out["o"], want, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("W", [1, 5, 16, 40])
+def test_sliding_window_when_topk_is_zero(W):
+    N, D = 96, 8
+    p = _params(B=1, Hq=1, Hkv=1, N=N, D=D, block_k=16, block_q=16, top_k=0, window=W)
+    q, k, v = _rand((1, 1, N, D), 8), _rand((1, 1, N, D), 9), _rand((1, 1, N, D), 10)
+    out = O.forward(q, k, v, p)
+    # textbook sliding-window attention: query i sees the W most recent keys
+    band = np.zeros((N, N), dtype=bool)
+    for i in range(N):
+        band[i, max(0, i - W + 1):i + 1] = True
+    want = _sdpa(q, k, v, mask=band)
+    np.testing.assert_allclose(out["o"], want, atol=1e-12, rtol=0)
+
+
+def test_explicit_scale_is_used():
+    N, D = 64, 8
+    p = _params(B=1, Hq=1, Hkv=1, N=N, D=D, block_k=8, block_q=8, top_k=8, window=8,
+                scale=0.37)
+    q, k, v = _rand((1, 1, N, D), 11), _rand((1, 1, N, D), 12), _rand((1, 1, N, D), 13)
+    out = O.forward(q, k, v, p)
+    t = [torch.from_numpy(a) for a in (q, k, v)]
+    want = F.scaled_dot_product_attention(*t, is_causal=True, scale=0.37).numpy()
+    np.testing.assert_allclose(out["o"], want, atol=1e-12, rtol=0)
+
+
+# ---------------------------------------------------------------- attend: invariants
+@pytest.mark.parametrize("causal", [True, False])
+def test_weights_are_a_distribution_on_the_key_set(causal):
+    # V = identity makes O the attention-weight matrix itself
+    N, D = 48, 4
+    p = _params(B=1, Hq=1, Hkv=1, N=N, D=D, block_k=4, block_q=4, top_k=3,
+                window=5 if causal else 0, causal=causal)
+    q, k = _rand((1, 1, N, D), 14), _rand((1, 1, N, D), 15)
+    v = np.eye(N)[None, None]
+    out = O.forward(q, k, v, p)
+    wts = out["o"][0, 0]
+    np.testing.assert_allclose(wts.sum(axis=1), 1.0, atol=1e-14)
+    assert (wts >= 0).all()
+    scale = 1 / math.sqrt(D)
+    for i in range(N):
+        qb = i // 4
+        sel = out["idx"][0, 0, qb, :out["cnt"][0, 0, qb]]
+        # key set written from the definition: routed blocks' keys, plus the
+        # causal window, cut at i
+        member = np.zeros(N, dtype=bool)
+        for c in sel:
+            member[c * 4:(c + 1) * 4] = True
+        if causal:
+            member[max(0, i - 4):i + 1] = True
+            member[i + 1:] = False
+        assert (wts[i, ~member] == 0).all()
+        assert (wts[i, member] > 0).all()
+        logits = k[0, 0] @ q[0, 0, i] * scale
+        j0 = np.flatnonzero(member)[0]
+        np.testing.assert_allclose(wts[i, member] / wts[i, j0],
+                                   np.exp(logits[member] - logits[j0]), rtol=1e-12)
+
+
+def test_key_set_is_a_set_and_obeys_cardinality_bound():
+    # routed block overlapping the window must be counted once, and
+    # |S_i| <= W + k*Bk (jonsmirl/ssa README, "Mathematical status": union with
+    # a fixed carrier has a uniform W + C cardinality bound)
+    p = _params(N=256, D=4, block_k=16, block_q=16, top_k=4, window=40)
+    rng = np.random.default_rng(0)
+    for i in rng.integers(0, 256, size=60):
+        qb = i // 16
+        sel = rng.choice(max(qb, 1), size=min(4, qb), replace=False) if qb else np.zeros(0, int)
+        s = O.key_set(int(i), np.sort(sel), p)
+        assert len(s) == len(np.unique(s))
+        assert len(s) <= p.window + p.top_k * p.block_k
+        assert s.max() <= i and (s >= max(0, i - 39)).sum() >= min(40, i + 1)
+
+
+def test_append_law_of_the_read():
+    # jonsmirl/ssa README, "Mathematical status": appending a fresh item of mass
+    # a to an old mass Z moves the read by a/(Z+a) times the fresh value's
+    # displacement from the old read, and the potential by log(1 + a/Z).
+    # With Bk = 1, non-causal, every block is one key; selecting one more block
+    # appends exactly one item.
+    N, D = 32, 6
+    p2 = _params(N=N, D=D, block_k=1, block_q=1, top_k=2, window=0, causal=False)
+    p3 = _params(N=N, D=D, block_k=1, block_q=1, top_k=3, window=0, causal=False)
+    q, k, v = _rand((1, 1, N, D), 21), _rand((1, 1, N, D), 22), _rand((1, 1, N, 5), 23)
+    idx2 = np.full((1, 1, N, 2), -1, np.int32)
+    idx3 = np.full((1, 1, N, 3), -1, np.int32)
+    rng = np.random.default_rng(5)
+    extra = np.zeros(N, int)
+    for i in range(N):
+        trio = rng.choice(N, size=3, replace=False)
+        idx2[0, 0, i] = np.sort(trio[:2])
+        idx3[0, 0, i] = np.sort(trio)
+        extra[i] = trio[2]
+    cnt2 = np.full((1, 1, N), 2, np.int32)
+    cnt3 = np.full((1, 1, N), 3, np.int32)
+    o2, l2 = O.attend_gathered(q, k, v, idx2, cnt2, p2)
+    o3, l3 = O.attend_gathered(q, k, v, idx3, cnt3, p3)
+    scale = 1 / math.sqrt(D)
+    for i in range(N):
+        ell = float(k[0, 0, extra[i]] @ q[0, 0, i]) * scale
+        a_over_z = math.exp(ell - l2[0, 0, i])             # a / Z
+        assert l3[0, 0, i] == pytest.approx(l2[0, 0, i] + math.log1p(a_over_z), abs=1e-12)
+        frac = a_over_z / (1 + a_over_z)                   # a / (Z + a)
+        want = o2[0, 0, i] + frac * (v[0, 0, extra[i]] - o2[0, 0, i])
+        np.testing.assert_allclose(o3[0, 0, i], want, atol=1e-12)
+
+
+def test_future_keys_do_not_move_past_outputs():
+    N, D = 128, 8
+    p = _params(B=1, Hq=2, Hkv=1, N=N, D=D, block_k=8, block_q=16, top_k=3, window=10)
+    q, k, v = _rand((1, 2, N, D), 31), _rand((1, 1, N, D), 32), _rand((1, 1, N, D), 33)
+    base = O.forward(q, k, v, p)
+    for cut in (15, 47, 96):
+        k2, v2 = k.copy(), v.copy()
+        k2[:, :, cut + 1:] = _rand(k2[:, :, cut + 1:].shape, cut)
+        v2[:, :, cut + 1:] = _rand(v2[:, :, cut + 1:].shape, cut + 1)
+        out = O.forward(q, k2, v2, p)
+        # every query at or before the cut is unchanged, bit for bit
+        np.testing.assert_array_equal(out["o"][:, :, :cut + 1], base["o"][:, :, :cut + 1])
+
+
+def test_masked_dense_and_gathered_forms_agree():
+    N, D = 192, 16
+    p = _params(B=2, Hq=4, Hkv=2, N=N, D=D, block_k=16, block_q=32, top_k=3, window=23)
+    q, k, v = _rand((2, 4, N, D), 41), _rand((2, 2, N, D), 42), _rand((2, 2, N, D), 43)
+    a = O.forward(q, k, v, p, form="dense")
+    b = O.forward(q, k, v, p, form="gathered")
+    np.testing.assert_allclose(a["o"], b["o"], atol=1e-12, rtol=0)
+    np.testing.assert_allclose(a["lse"], b["lse"], atol=1e-12, rtol=0)
+
+
+def test_lse_against_dense_logsumexp():
+    N, D = 64, 8
+    p = _params(N=N, D=D, block_k=8, block_q=8, top_k=8, window=8)
+    q, k, v = _rand((1, 1, N, D), 51), _rand((1, 1, N, D), 52), _rand((1, 1, N, D), 53)
+    out = O.forward(q, k, v, p)
+    t = torch.from_numpy(q[0, 0]) @ torch.from_numpy(k[0, 0]).T / math.sqrt(D)
+    t = t.masked_fill(torch.triu(torch.ones(N, N, dtype=torch.bool), 1), float("-inf"))
+    np.testing.assert_allclose(out["lse"][0, 0], torch.logsumexp(t, dim=1).numpy(), atol=1e-12)
+
+
+def test_near_tie_rows_flags_only_close_scores():
+    r = O.RouteResult(idx=None, cnt=None,
+                      kth=np.array([1.0, 1.0, -2.0, 5.0, np.nan]),
+                      next=np.array([0.99995, 0.9, -2.0001, np.nan, np.nan]))
+    assert O.near_tie_rows(r).tolist() == [True, False, True, False, False]
+
+
+def test_bf16_upcast_is_exact():
+    u = np.array([0x3F80, 0xBF80, 0x0000, 0x7F7F, 0x0001, 0x4049], dtype=np.uint16)
+    want = torch.from_numpy(u.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.upcast_bf16(u), want)
