@@ -1,0 +1,513 @@
+#!/usr/bin/env python
+"""Benchmark of content-routed block-sparse attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ssa|reference]
+
+A step is one pass of the whole path (K/Q block summaries, routing, fused
+attend) over one batch of the synthetic workload, inputs resident in HBM.
+Default workload: the GQA clustered-key prefill (1 x 14/2 heads, N = 32768,
+D = 64, Bk = Bq = 64, top-k 16, W = 512).  Prints one JSON line on rank 0.
+
+* value     whole-job prefill tokens/s (device time, CUDA events per step,
+            L2 flushed between steps by a 256 MiB write outside the events)
+* e2e       the same metric through the public call from pinned host buffers
+            (H2D of Q, K, V and D2H of O inside the timed region)
+* roofline  the attend kernel: algorithmic gathered bytes (distinct routed +
+            window key blocks of every query block, K and V, plus the Q read
+            and O / LSE writes) per launch / its event-timed duration, against
+            the measured HBM copy bandwidth
+* cpu_baseline  the float64 oracle on the host cores over a bounded sample
+
+With --gpus N > 1 (torchrun) every rank runs an independent replica of the
+workload (the path shards into independent problems; there is no exchange
+step), the per-step time is the max over ranks, and value sums all ranks.
+--impl reference times the oracle instead (host cores, bounded samples).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn prefill tokens/s; selected-key TFLOP/s as % of B200 roofline"
+UNIT = "tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attend_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ssa", choices=["ssa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attend.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "content_routed_block_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.samples = []
+        self.proc = None
+        self.thread = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", self.gpu_id, "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        if which == "start":
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for t, line in self.samples:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != 7:
+                continue
+            rows.append((t, parts))
+        inside = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= (self.t1 or 1e30)]
+        use = inside if inside else rows
+        sm = [float(p[0]) for _, p in use if p[0].replace(".", "").isdigit()]
+        smax = [float(p[1]) for _, p in use if p[1].replace(".", "").isdigit()]
+        reasons = sorted({self.NAMES[i] for _, p in use for i in range(4) if p[3 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(use), "in_timed_region": bool(inside)}
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work of one forward (from the routed lists)
+# ----------------------------------------------------------------------------
+def algorithmic_work(w, idx, cnt):
+    """Mean distinct keys per query (|S_i|), selected-key flops, and the attend
+    kernel's algorithmic bytes: per query block, the distinct key blocks it
+    needs (routed U window) x Bk rows x K and V, plus Q read, O and LSE write."""
+    import numpy as np
+    B, Hq, N, D, Bk, Bq, W = w.B, w.Hq, w.N, w.D, w.block_k, w.block_q, w.window
+    nqb = N // Bq
+    qb = np.arange(nqb)
+    k = w.top_k
+    keys_total = 0.0
+    blocks_total = 0
+    for b in range(B):
+        for h in range(Hq):
+            sel = idx[b, h] if k > 0 else np.zeros((nqb, 0), np.int64)
+            valid = (np.arange(k)[None, :] < cnt[b, h][:, None]) if k > 0 else sel.astype(bool)
+            if not w.causal:
+                keys_total += float(cnt[b, h].sum()) * Bk * Bq
+                blocks_total += int(cnt[b, h].sum())
+                continue
+            # rows i of block qb: i = qb*Bq + r
+            r = np.arange(Bq)
+            i = qb[:, None] * Bq + r[None, :]                           # [nqb, Bq]
+            win = np.minimum(W, i + 1)                                 # window keys
+            lo = np.maximum(0, i - W + 1)                              # first window key
+            c0 = sel.astype(np.int64) * Bk                             # [nqb, k]
+            c1 = c0 + Bk - 1
+            # overlap of routed block [c0, c1] with window [lo, i] (routed blocks end before i)
+            ov = np.clip(c1[:, None, :] - np.maximum(c0[:, None, :], lo[:, :, None]) + 1, 0, Bk)
+            ov = np.where(valid[:, None, :], ov, 0)
+            routed = np.where(valid, Bk, 0).sum(axis=1)[:, None]        # [nqb, 1]
+            keys_total += float((win + routed - ov.sum(axis=2)).sum())
+            # distinct key blocks per query block: routed U window blocks
+            wlo = np.maximum(0, qb * Bq - W + 1) // Bk
+            whi = (qb * Bq + Bq - 1) // Bk
+            in_win = (sel >= wlo[:, None]) & (sel <= whi[:, None]) & valid
+            blocks_total += int(((whi - wlo + 1) + valid.sum(axis=1) - in_win.sum(axis=1)).sum())
+    kpq = keys_total / (B * Hq * N)
+    flops = 4.0 * B * Hq * N * kpq * D
+    gathered = blocks_total * Bk * 2 * D * 2
+    io = B * Hq * N * D * 2 * 2 + B * Hq * N * 4
+    return {"keys_per_query": kpq, "flops": flops, "gathered_bytes": gathered,
+            "attend_bytes": gathered + io, "nominal_keys_per_query": k * Bk + W}
+
+
+# ----------------------------------------------------------------------------
+# oracle on the host cores (cpu_baseline and the reference arm)
+# ----------------------------------------------------------------------------
+def _cpu_worker(args):
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle as O
+    from content_routed_block_b200.workloads import CONFIGS, make_inputs
+    cfg, b, h, blocks, seconds = args
+    w = CONFIGS[cfg]
+    g = w.Hq // w.Hkv
+    x = make_inputs(w, q_heads=[h], kv_heads=[h // g])
+    sub = w.with_(Hq=1, Hkv=1, B=1)
+    p = O.Params.of(sub)
+    q = O.upcast_bf16(x["q"][b:b + 1])
+    k = O.upcast_bf16(x["k"][b:b + 1])
+    v = O.upcast_bf16(x["v"][b:b + 1])
+    t0 = time.perf_counter()
+    ksum = O.block_summary(k, p.block_k)
+    done = 0
+    idx = np.full((1, 1, p.n_qblocks, p.top_k), -1, np.int32)
+    cnt = np.zeros((1, 1, p.n_qblocks), np.int32)
+    for qb in blocks:
+        qbar = O.block_summary(q[:, :, qb * p.block_q:(qb + 1) * p.block_q], p.block_q)[0, 0, 0]
+        sel, _, _ = O.route_row(qbar, ksum[0, 0], O.admissible_blocks(qb, p), p.top_k)
+        idx[0, 0, qb, :len(sel)] = sel
+        cnt[0, 0, qb] = len(sel)
+        O.attend_masked_dense(q, k, v, idx, cnt, p, blocks=[(0, 0, qb)])
+        done += 1
+        if time.perf_counter() - t0 > seconds:
+            break
+    return done, time.perf_counter() - t0
+
+
+class OraclePool:
+    def __init__(self, cfg: int):
+        import multiprocessing as mp
+        self.cfg = cfg
+        self.cores = max(1, min(len(os.sched_getaffinity(0)), 64))
+        old = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        for k in old:
+            os.environ[k] = "1"
+        self.pool = mp.get_context("spawn").Pool(self.cores)
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+        self.step = 0
+
+    def run(self, seconds: float):
+        """Each worker runs the oracle's whole path for seconds on its own
+        (b, head) and a spread of query blocks; returns (tokens/s, blocks)."""
+        import numpy as np
+        from content_routed_block_b200.workloads import CONFIGS
+        w = CONFIGS[self.cfg]
+        nqb = w.N // w.block_q
+        tasks = []
+        rng = np.random.default_rng(self.step)
+        self.step += 1
+        for c in range(self.cores):
+            b = c % w.B
+            h = (c // w.B) % w.Hq
+            blocks = rng.permutation(nqb).tolist()
+            tasks.append((self.cfg, b, h, blocks, seconds))
+        res = self.pool.map(_cpu_worker, tasks)
+        blocks = sum(r[0] for r in res)
+        wall = max(r[1] for r in res)
+        return blocks * w.block_q / wall, blocks, wall
+
+    def close(self):
+        self.pool.terminate()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from content_routed_block_b200.workloads import CONFIGS
+    w = CONFIGS[args.config]
+    per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
+    pool = OraclePool(args.config)
+    try:
+        for _ in range(args.warmup):
+            pool.run(per_step)
+        vals, blocks = [], 0
+        t0 = time.time()
+        for _ in range(args.steps):
+            v, nb, _ = pool.run(per_step)
+            vals.append(v)
+            blocks += nb
+        wall = time.time() - t0
+    finally:
+        pool.close()
+    value = statistics.mean(vals)
+    sample = (f"{blocks} query blocks of {w.block_q} tokens over {args.steps} steps, "
+              f"~{per_step:.1f} s of oracle work per core per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * wall / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, args):
+    return {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} D={w.D} "
+                        f"Bk={w.block_k} Bq={w.block_q} top_k={w.top_k} W={w.window} "
+                        f"{'causal' if w.causal else 'non-causal'} {w.kind}",
+            "global_batch": w.B * args.gpus, "seq_len": w.N, "parallelism": f"replicas{args.gpus}",
+            "l2": "flushed between timed steps (256 MiB write)"}
+
+
+# ----------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------
+def run_ssa(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from content_routed_block_b200 import build, ssa
+    from content_routed_block_b200.workloads import CONFIGS, make_inputs
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    ssa.lib()
+
+    w = CONFIGS[args.config]
+    p = ssa.params_of(w)
+    x = make_inputs(w)
+    host = {n: torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16) for n in "qkv"}
+    qd, kd, vd = (host[n].to(dev) for n in "qkv")
+    ws = torch.empty(ssa.workspace_size(p), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    idx = torch.empty((w.B, w.Hq, w.N // w.block_q, w.top_k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.Hq, w.N // w.block_q), dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        ssa.forward(qd, kd, vd, p, workspace=ws, out=o, lse_out=lse, idx_out=idx, cnt_out=cnt)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    ssa.check_error()
+
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = str(getattr(props, "uuid", "")) or str(local)
+    if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) > 8:
+        gpu_id = "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark("start")
+    for s in range(args.steps):
+        flush.zero_()
+        starts[s].record()
+        step()
+        ends[s].record()
+    torch.cuda.synchronize()
+    sampler.mark("end")
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    ssa.check_error()
+    times = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    ms = statistics.mean(times)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = w.B * w.N * world
+    value = tokens / (ms * 1e-3)
+
+    # per-kernel split: the same path as separate calls with events between them
+    n_split = min(args.steps, 200)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_split)]
+    ks = torch.empty((w.B, w.Hkv, w.N // w.block_k, w.D), dtype=torch.float32, device=dev)
+    qs = torch.empty((w.B, w.Hq, w.N // w.block_q, w.D), dtype=torch.float32, device=dev)
+    L = ssa.lib()
+    import ctypes
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    pp = ctypes.byref(p)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    for s in range(n_split):
+        flush.zero_()
+        e = ev[s]
+        e[0].record()
+        assert L.ssa_block_summary(pp, P(kd), w.Hkv, w.block_k, P(ks), st) == 0
+        e[1].record()
+        assert L.ssa_block_summary(pp, P(qd), w.Hq, w.block_q, P(qs), st) == 0
+        e[2].record()
+        assert L.ssa_route(pp, P(qs), P(ks), P(idx) if w.top_k else None, P(cnt), st) == 0
+        e[3].record()
+        assert L.ssa_attend(pp, P(qd), P(kd), P(vd), P(idx) if w.top_k else None, P(cnt),
+                            P(o), P(lse), st) == 0
+        e[4].record()
+    torch.cuda.synchronize()
+    ssa.check_error()
+    seg = lambda i: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(n_split))  # noqa: E731
+    pool_k_ms, pool_q_ms, route_ms, attend_ms = seg(0), seg(1), seg(2), seg(3)
+
+    work = algorithmic_work(w, idx.cpu().numpy(), cnt.cpu().numpy())
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    achieved = work["attend_bytes"] / (attend_ms * 1e-3) / 1e9
+    tflops = work["flops"] / (ms * 1e-3) / 1e12
+    attend_tflops = work["flops"] / (attend_ms * 1e-3) / 1e12
+    t_roof = max(work["flops"] / (float(peaks["bf16_tflops"]) * 1e12),
+                 work["attend_bytes"] / (hbm * 1e9))
+    traffic = None
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            tr = json.load(f)
+        if tr.get("kernel_hash") == kernel_source_hash():
+            traffic = tr.get("bytes_per_launch", {}).get(str(args.config))
+
+    # end to end through the public call, from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (host[n].pin_memory() for n in "qkv")
+        oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+        bufs = {"q": qd, "k": kd, "v": vd, "o": o}
+        n_e2e = min(args.steps, 100)
+        for _ in range(3):
+            ssa.forward_host(qh, kh, vh, p, oh, device=dev, workspace=ws, dev_bufs=bufs)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_e2e):
+            ssa.forward_host(qh, kh, vh, p, oh, device=dev, workspace=ws, dev_bufs=bufs)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+        e2e = {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": oh.numel() * oh.element_size(), "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        pool = OraclePool(args.config)
+        try:
+            v, nb, wall = pool.run(args.cpu_seconds)
+        finally:
+            pool.close()
+        cpu = {"value": v, "unit": UNIT, "cores": pool.cores, "kind": "oracle",
+               "sample": f"{nb} query blocks ({nb * w.block_q} tokens) of this workload, whole "
+                         f"path (summaries, routing, masked-dense attend) in float64, "
+                         f"{pool.cores} processes x ~{args.cpu_seconds:.0f} s"}
+
+    clocks = sampler.summary()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ssa",
+        "config": workload_config(w, args),
+        "selected_tflops": tflops,
+        "keys_per_query": work["keys_per_query"],
+        "nominal_keys_per_query": work["nominal_keys_per_query"],
+        "kernels_ms": {"pool_k": pool_k_ms, "pool_q": pool_q_ms, "route": route_ms,
+                       "attend": attend_ms},
+        "roofline": {"bound": "hbm", "kernel": "attend_kernel", "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
+                     "peak_source": f"{peak_kind} hbm_gbs",
+                     "bytes_per_launch": work["attend_bytes"],
+                     "attend_tflops": attend_tflops,
+                     "attend_tensor_frac": attend_tflops / float(peaks["bf16_tflops"]),
+                     "path_frac_of_roofline": t_roof / (ms * 1e-3)},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ssa(args)
+
+
+if __name__ == "__main__":
+    main()

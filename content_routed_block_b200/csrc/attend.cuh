@@ -1,0 +1,528 @@
+// K3: fused attend over the routed blocks and the local window.
+//
+// jonsmirl/ssa README, introduction: for each query, select a small set of
+// key blocks, add a local causal window, and compute ordinary softmax
+// attention over the selected keys without forming the dense n x n matrix;
+// "Mathematical status": the routed set is causal once it is masked at each
+// query's original position.  For query i in query block qb the key set is
+// (keys of the routed blocks of qb) U {i-W < j <= i}, cut at j <= i (causal)
+// or the routed blocks' keys alone (non-causal), each key counted once; the
+// read is exact softmax over that set.  The append law on the same page
+// (adding mass a to Z moves the read by a/(Z+a) of the displacement) is the
+// online-softmax merge this kernel performs chunk by chunk.
+//
+// B200 design (one CTA = 128 query rows of one (b, head), i.e. 128/Bq query
+// blocks; 192 threads):
+//  * The CTA first builds the sorted union of its query blocks' routed
+//    blocks and the window's blocks in shared memory, each entry carrying a
+//    bitmask of which query blocks routed it.  The union is walked in chunks
+//    of 64 keys (one or more whole blocks, or a 64-row slice of a larger
+//    block), so every key block is fetched once per CTA.
+//  * Warp 4 (one lane) gathers each chunk's K and V rows with tiled TMA loads
+//    (one box per block, no multicast) into a 128-byte-swizzled ring of
+//    STAGES stages; Q (128 x D) is loaded once.
+//  * Warp 5 (one lane) issues tcgen05.mma: S = Q K^T (M=128, N=64, fp32 in
+//    TMEM, two S buffers) and O += P V (A = P read from TMEM, B = V as an
+//    MN-major shared-memory operand, N = D, fp32 accumulator in TMEM).
+//  * Warps 0-3 own one query row each per thread (TMEM lane = row): they
+//    load S, apply the row's mask (routed bit of its query block, window,
+//    causal cut), keep the running max / sum in fp32, write P as bf16 back
+//    over S in TMEM, and rescale O in TMEM only when the max has grown by
+//    more than 2^8 (the result is exact either way; the lazy update only
+//    bounds the magnitudes).  The epilogue divides by the sum, rounds to
+//    bf16 and writes O and the natural-log LSE.
+//  * Every wait is bounded (mbar_wait): on a timeout the CTA raises a shared
+//    abort flag, each role leaves its loop, the producer and the MMA issuer
+//    wait for their copies / MMAs in flight, and TMEM is freed.
+#pragma once
+
+#include "common.cuh"
+
+namespace ssa {
+
+constexpr int kAtQT = 128;       // query rows per CTA (MMA M)
+constexpr int kAtKT = 64;        // keys per chunk (MMA N of S)
+constexpr int kAtLCap = 1024;    // window entries capacity
+constexpr int kAtFarCap = 512;   // routed entries outside the window (>= 8 * 64)
+constexpr int kAtThreads = 192;
+constexpr uint32_t kAtTmemCols = 256;
+constexpr float kAtTau = 8.0f;   // lazy-rescale threshold, log2 units
+
+template <int D>
+struct AtLayout {
+  static constexpr int STAGES = (D == 64) ? 3 : 2;
+  static constexpr uint32_t HALF_Q = kAtQT * 128;      // one 64-column half of Q
+  static constexpr uint32_t Q_BYTES = kAtQT * D * 2;
+  static constexpr uint32_t HALF_KV = kAtKT * 128;     // one 64-column half of a chunk
+  static constexpr uint32_t KV_BYTES = kAtKT * D * 2;  // one K (or V) chunk
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+  static constexpr uint32_t OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr uint32_t OFF_WIN = OFF_V + STAGES * KV_BYTES;   // uint32 [kAtLCap]
+  static constexpr uint32_t OFF_FAR = OFF_WIN + kAtLCap * 4;       // int32 [kAtFarCap]
+  static constexpr uint32_t OFF_FARU = OFF_FAR + kAtFarCap * 4;    // int32 [kAtFarCap]
+  static constexpr int NBAR = 1 + 2 * STAGES + 2 + 2 + 2 + 1;
+  static constexpr uint32_t OFF_BAR = OFF_FARU + kAtFarCap * 4;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr uint32_t USED = OFF_MISC + 64;
+  // request enough shared memory that at most two CTAs share an SM, so the
+  // two 256-column TMEM allocations always fit in the SM's 512 columns
+  static constexpr uint32_t MIN_REQ = 80 * 1024;
+  static constexpr uint32_t SMEM_BYTES = (USED + 1024 > MIN_REQ) ? USED + 1024 : MIN_REQ;
+  // TMEM columns: S buffers at 0 and 64 (P overwrites the first 32 columns of
+  // its S buffer as packed bf16 pairs); O at 128 .. 128 + D
+  static constexpr uint32_t TM_S0 = 0, TM_O = 128;
+};
+
+struct AttendArgs {
+  const int32_t* idx;    // [B*Hq, NQB, top_k]
+  const int32_t* cnt;    // [B*Hq, NQB]
+  __nv_bfloat16* o;      // [B*Hq, N, D]
+  float* lse;            // [B*Hq, N] or null
+  int32_t Hq, Hkv, N, NQB, NB, Bq, Bk, top_k, window, causal;
+  int32_t n_qtiles;
+  float scale_log2;      // softmax scale * log2(e)
+  uint64_t timeout_ns;
+};
+
+// union entry: (block << 8) | routed-bits (bit r: query block r of the tile
+// routed this block)
+__device__ __forceinline__ uint32_t at_entry(const int32_t* faru, const uint32_t* win, int nf,
+                                             int wlo, int e) {
+  if (e < nf) return static_cast<uint32_t>(faru[e]);
+  const int w = e - nf;
+  return (static_cast<uint32_t>(wlo + w) << 8) | (win[w] & 0xFFu);
+}
+
+// bits [lo, hi) of a 64-bit word
+__device__ __forceinline__ uint64_t bit_range(int lo, int hi) {
+  if (hi <= lo) return 0ull;
+  const int n = hi - lo;
+  const uint64_t m = (n >= 64) ? ~0ull : ((1ull << n) - 1ull);
+  return m << lo;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAtThreads, 2)
+    attend_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                  const __grid_constant__ CUtensorMap tv, const AttendArgs a) {
+  using L = AtLayout<D>;
+  constexpr int S = L::STAGES;
+  extern __shared__ uint8_t at_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(at_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint32_t* win = reinterpret_cast<uint32_t*>(smem + L::OFF_WIN);
+  int32_t* far = reinterpret_cast<int32_t*>(smem + L::OFF_FAR);
+  int32_t* faru = reinterpret_cast<int32_t*>(smem + L::OFF_FARU);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_kv_full = bars + 1;
+  uint64_t* bar_kv_empty = bars + 1 + S;
+  uint64_t* bar_s_full = bars + 1 + 2 * S;
+  uint64_t* bar_p_full = bar_s_full + 2;
+  uint64_t* bar_pv_done = bar_p_full + 2;
+  uint64_t* bar_drain = bar_pv_done + 2;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  // misc[0] TMEM base, misc[1] raw far count, misc[2] unique far count,
+  // misc[3] abort flag
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[3]);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x / a.n_qtiles;
+  const int qt = blockIdx.x % a.n_qtiles;
+  const int b = bh / a.Hq, h = bh % a.Hq;
+  const int bkv = b * a.Hkv + h / (a.Hq / a.Hkv);
+  const int q0 = qt * kAtQT;
+  const int qend = min(a.N, q0 + kAtQT);
+  const int qb0 = q0 / a.Bq;
+  const int R = min(kAtQT / a.Bq, a.NQB - qb0);
+  int wlo = 0, nwin = 0;
+  if (a.causal) {
+    wlo = max(0, q0 - a.window + 1) / a.Bk;
+    nwin = (qend - 1) / a.Bk - wlo + 1;
+  }
+
+  // ---------------------------------------------------------------- setup
+  if (tid == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&bar_kv_full[s], 1);
+      mbar_init(&bar_kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_s_full[s], 1);
+      mbar_init(&bar_p_full[s], 128);
+      mbar_init(&bar_pv_done[s], 1);
+    }
+    mbar_init(bar_drain, 1);
+    misc[1] = 0;
+    misc[2] = 0;
+    misc[3] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&misc[0], kAtTmemCols);
+    tmem_relinquish();
+  }
+  for (int w = tid; w < nwin; w += kAtThreads) win[w] = 0u;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  // Q does not depend on the routing: start its load now
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+    mbar_arrive_expect_tx(bar_q, L::Q_BYTES);
+#pragma unroll
+    for (int half = 0; half < D / 64; ++half)
+      tma_load_3d(smem + L::OFF_Q + half * L::HALF_Q, &tq, bar_q, half * 64, q0, bh);
+  }
+
+  // ------------------------------------------ union of routed and window blocks
+  {
+    const int total = R * a.top_k;
+    for (int t = tid; t < total; t += kAtThreads) {
+      const int r = t / a.top_k, e = t % a.top_k;
+      const int64_t row = static_cast<int64_t>(bh) * a.NQB + qb0 + r;
+      int n = a.cnt[row];
+      if (n > a.top_k || n < 0) {
+        record_error(kErrCheck, kSiteIdx);
+        n = min(max(n, 0), a.top_k);
+      }
+      if (e >= n) continue;
+      const int c = a.idx[row * a.top_k + e];
+      if (c < 0 || c >= a.NB) {
+        record_error(kErrCheck, kSiteIdx);
+        continue;
+      }
+      const uint32_t bit = 1u << r;
+      if (a.causal && c >= wlo) {
+        if (c - wlo < nwin) atomicOr(&win[c - wlo], bit);
+        // a block entirely after the tile's last query contributes nothing
+      } else {
+        const int pos = static_cast<int>(atomicAdd(&misc[1], 1u));
+        far[pos] = (c << 8) | static_cast<int>(bit);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int nfar = static_cast<int>(misc[1]);
+    int P = 1;
+    while (P < nfar) P <<= 1;
+    for (int i = nfar + lane; i < P; i += 32) far[i] = 0x7FFFFFFF;
+    __syncwarp();
+    for (int k = 2; k <= P; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = lane; i < P; i += 32) {
+          const int l = i ^ j;
+          if (l > i) {
+            const int x = far[i], y = far[l];
+            const bool asc = (i & k) == 0;
+            if ((x > y) == asc) {
+              far[i] = y;
+              far[l] = x;
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+    int base = 0;
+    for (int i0 = 0; i0 < nfar; i0 += 32) {
+      const int i = i0 + lane;
+      bool head = false;
+      int ent = 0;
+      if (i < nfar) {
+        const int c = far[i] >> 8;
+        head = (i == 0) || ((far[i - 1] >> 8) != c);
+        if (head) {
+          int bits = 0;
+          for (int k = i; k < nfar && (far[k] >> 8) == c; ++k) bits |= far[k] & 0xFF;
+          ent = (c << 8) | bits;
+        }
+      }
+      const uint32_t hm = __ballot_sync(0xffffffffu, head);
+      if (head) faru[base + __popc(hm & ((1u << lane) - 1u))] = ent;
+      base += __popc(hm);
+    }
+    if (lane == 0) misc[2] = static_cast<uint32_t>(base);
+  }
+  __syncthreads();
+
+  const int nf = static_cast<int>(misc[2]);
+  const int n_entries = nf + nwin;
+  const int G = (a.Bk < kAtKT) ? kAtKT / a.Bk : 1;           // blocks per chunk
+  const int SUBS = (a.Bk > kAtKT) ? a.Bk / kAtKT : 1;        // chunks per block
+  const int T = (a.Bk >= kAtKT) ? n_entries * SUBS : (n_entries + G - 1) / G;
+  int issued = 0;  // chunks the producer has put in flight
+
+  if (warp == 4) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      for (int t = 0; t < T; ++t) {
+        const int st = t % S;
+        if (t >= S && !mbar_wait(&bar_kv_empty[st], ((t / S) - 1) & 1, a.timeout_ns, abort_flag,
+                                 kSiteKvEmpty))
+          break;
+        mbar_arrive_expect_tx(&bar_kv_full[st], 2 * L::KV_BYTES);
+        uint8_t* kdst = smem + L::OFF_K + st * L::KV_BYTES;
+        uint8_t* vdst = smem + L::OFF_V + st * L::KV_BYTES;
+        if (a.Bk >= kAtKT) {
+          const int e = t / SUBS, sub = t % SUBS;
+          const int c = static_cast<int>(at_entry(faru, win, nf, wlo, e) >> 8);
+          const int row0 = c * a.Bk + sub * kAtKT;
+#pragma unroll
+          for (int half = 0; half < D / 64; ++half) {
+            tma_load_3d(kdst + half * L::HALF_KV, &tk, &bar_kv_full[st], half * 64, row0, bkv);
+            tma_load_3d(vdst + half * L::HALF_KV, &tv, &bar_kv_full[st], half * 64, row0, bkv);
+          }
+        } else {
+          for (int s = 0; s < G; ++s) {
+            int e = t * G + s;
+            if (e >= n_entries) e = t * G;  // pad a short last chunk with a real block (masked)
+            const int c = static_cast<int>(at_entry(faru, win, nf, wlo, e) >> 8);
+            const int row0 = c * a.Bk;
+#pragma unroll
+            for (int half = 0; half < D / 64; ++half) {
+              tma_load_3d(kdst + half * L::HALF_KV + s * a.Bk * 128, &tk, &bar_kv_full[st],
+                          half * 64, row0, bkv);
+              tma_load_3d(vdst + half * L::HALF_KV + s * a.Bk * 128, &tv, &bar_kv_full[st],
+                          half * 64, row0, bkv);
+            }
+          }
+        }
+        ++issued;
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(kAtQT, kAtKT, false, false);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(kAtQT, D, false, true);
+      bool ok = mbar_wait(bar_q, 0, a.timeout_ns, abort_flag, kSiteQFull);
+      auto issue_pv = [&](int u) -> bool {
+        if (!mbar_wait(&bar_p_full[u & 1], (u >> 1) & 1, a.timeout_ns, abort_flag, kSitePFull))
+          return false;
+        tc_fence_after();
+        const uint32_t vbase = sbase + L::OFF_V + (u % S) * L::KV_BYTES;
+        const uint32_t pcol = tmem + L::TM_S0 + (u & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < kAtKT / 16; ++kk) {
+          const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, L::HALF_KV, 1024);
+          mma_ts(tmem + L::TM_O, pcol + kk * 8, bdesc, IDESC_O, (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bar_pv_done[u & 1]);
+        mma_commit(&bar_kv_empty[u % S]);
+        return true;
+      };
+      for (int t = 0; ok && t < T; ++t) {
+        const int st = t % S;
+        if (!mbar_wait(&bar_kv_full[st], (t / S) & 1, a.timeout_ns, abort_flag, kSiteKvFull)) {
+          ok = false;
+          break;
+        }
+        // S buffer t&1 is free once PV(t-2), which read P(t-2) from it, is done
+        if (t >= 2 && !mbar_wait(&bar_pv_done[t & 1], ((t - 2) >> 1) & 1, a.timeout_ns,
+                                 abort_flag, kSitePvDone)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t kbase = sbase + L::OFF_K + st * L::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qa = sbase + L::OFF_Q + (kk / 4) * L::HALF_Q + (kk % 4) * 32;
+          const uint32_t kb = kbase + (kk / 4) * L::HALF_KV + (kk % 4) * 32;
+          mma_ss(tmem + L::TM_S0 + (t & 1) * 64, sdesc_sw128(qa, 16, 1024),
+                 sdesc_sw128(kb, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bar_s_full[t & 1]);
+        if (t >= 1 && !issue_pv(t - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok) issue_pv(T - 1);
+      // every MMA issued so far must finish before TMEM is released
+      mma_commit(bar_drain);
+      mbar_wait(bar_drain, 0, a.timeout_ns, nullptr, kSiteDrain);
+    }
+  } else {
+    // ------------------------------------------------------- softmax warps
+    const int r = tid;  // row in the tile == TMEM lane
+    const int i = q0 + r;
+    const bool row_ok = i < qend;
+    const int qbr = row_ok ? r / a.Bq : 0;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+
+    for (int t = 0; t < T; ++t) {
+      const bool got = mbar_wait(&bar_s_full[t & 1], (t >> 1) & 1, a.timeout_ns, abort_flag,
+                                 kSiteSFull);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t s0[32], s1[32];
+      tmem_ld32(trow + L::TM_S0 + (t & 1) * 64, s0);
+      tmem_ld32(trow + L::TM_S0 + (t & 1) * 64 + 32, s1);
+      tmem_ld_wait(s0);
+      tmem_ld_wait(s1);
+
+      // allowed keys of this row within the chunk
+      uint64_t mask = 0ull;
+      if (row_ok) {
+        if (a.Bk >= kAtKT) {
+          const int e = t / SUBS, sub = t % SUBS;
+          const uint32_t ent = at_entry(faru, win, nf, wlo, e);
+          const int j0 = static_cast<int>(ent >> 8) * a.Bk + sub * kAtKT;
+          const bool routed = (ent >> qbr) & 1u;
+          int lo = 0, hi = 0;
+          if (a.causal) {
+            hi = min(kAtKT, i - j0 + 1);
+            lo = routed ? 0 : max(0, i - a.window + 1 - j0);
+          } else {
+            hi = routed ? kAtKT : 0;
+          }
+          mask = bit_range(lo, hi);
+        } else {
+          for (int s = 0; s < G; ++s) {
+            const int e = t * G + s;
+            if (e >= n_entries) break;
+            const uint32_t ent = at_entry(faru, win, nf, wlo, e);
+            const int j0 = static_cast<int>(ent >> 8) * a.Bk;
+            const bool routed = (ent >> qbr) & 1u;
+            int lo = 0, hi = 0;
+            if (a.causal) {
+              hi = min(a.Bk, i - j0 + 1);
+              lo = routed ? 0 : max(0, i - a.window + 1 - j0);
+            } else {
+              hi = routed ? a.Bk : 0;
+            }
+            mask |= bit_range(lo, hi) << (s * a.Bk);
+          }
+        }
+      }
+
+      float x[64];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        x[c] = ((mask >> c) & 1ull) ? __uint_as_float(s0[c]) * a.scale_log2 : -INFINITY;
+        x[c + 32] =
+            ((mask >> (c + 32)) & 1ull) ? __uint_as_float(s1[c]) * a.scale_log2 : -INFINITY;
+      }
+#pragma unroll
+      for (int c = 0; c < 64; ++c) mx = fmaxf(mx, x[c]);
+      const float m_new = fmaxf(m_ref, mx);
+      const bool need = (m_ref != -INFINITY) && (m_new > m_ref + kAtTau);
+      if (__any_sync(0xffffffffu, need)) {
+        // rescale the O row in TMEM; PV(t-1) must have landed first
+        if (t >= 1) {
+          const bool g2 = mbar_wait(&bar_pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1, a.timeout_ns,
+                                    abort_flag, kSitePvDone);
+          if (!__all_sync(0xffffffffu, g2)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const float alpha = (m_ref == -INFINITY || m_new == m_ref) ? 1.f : ex2_approx(m_ref - m_new);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          tmem_ld32(trow + L::TM_O + cc * 32, ov);
+          tmem_ld_wait(ov);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+          tmem_st32(trow + L::TM_O + cc * 32, ov);
+        }
+        tmem_st_wait();
+        l_sum *= alpha;
+        m_ref = m_new;
+      } else if (m_ref == -INFINITY) {
+        m_ref = m_new;  // first keys of this row: O and the sum are still zero
+      }
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      uint32_t p[32];
+      float part = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = ex2_approx(x[2 * c] - m_use);
+        const float p1 = ex2_approx(x[2 * c + 1] - m_use);
+        part += p0 + p1;
+        p[c] = pack_bf16x2(p0, p1);
+      }
+      l_sum += part;
+      tmem_st32(trow + L::TM_S0 + (t & 1) * 64, p);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bar_p_full[t & 1]);
+    }
+
+    // ------------------------------------------------------- epilogue
+    if (ok && T > 0) {
+      const bool got = mbar_wait(&bar_pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, a.timeout_ns,
+                                 abort_flag, kSitePvDone);
+      ok = __all_sync(0xffffffffu, got);
+    }
+    if (ok && !*abort_flag) {
+      tc_fence_after();
+      const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
+      __nv_bfloat16* orow = a.o + (static_cast<int64_t>(bh) * a.N + i) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t ov[32];
+        if (T > 0) {
+          tmem_ld32(trow + L::TM_O + cc * 32, ov);
+          tmem_ld_wait(ov);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov[c] = 0u;
+        }
+        if (row_ok) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            pk[c] = pack_bf16x2(__uint_as_float(ov[2 * c]) * inv, __uint_as_float(ov[2 * c + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      if (row_ok && a.lse != nullptr) {
+        const float lse2 = (l_sum > 0.f) ? m_ref + __log2f(l_sum) : -INFINITY;
+        a.lse[static_cast<int64_t>(bh) * a.N + i] = lse2 * 0.69314718055994530942f;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  // After an abort some copies may still be in flight: they must land before
+  // the CTA exits.  On the normal path every chunk and Q were consumed, so
+  // these waits return at once; Q is unconsumed when there was no chunk.
+  if (warp == 4 && lane == 0) {
+    if (*abort_flag) {
+      for (int t = max(0, issued - S); t < issued; ++t)
+        mbar_wait(&bar_kv_full[t % S], (t / S) & 1, a.timeout_ns, nullptr, kSiteDrain);
+    }
+    if (T == 0 || *abort_flag) mbar_wait(bar_q, 0, a.timeout_ns, nullptr, kSiteDrain);
+  }
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kAtTmemCols);
+  }
+}
+
+}  // namespace ssa

@@ -1,0 +1,305 @@
+// K2: routing -- block scores and top-k per query block.
+//
+// jonsmirl/ssa README, "Algorithm and complexity": block c is scored by
+// r_c(q) = <q, mu_c> + (beta/2) q^T Sigma_c q; here beta = 0 (mean pooling
+// only) and q is the query block's mean.  Each query block keeps the top_k
+// admissible blocks; ties go to the lower block index (an explicit
+// deterministic order; the same page notes that without a margin a
+// deterministic index order is needed to name one top set).  The selected
+// blocks are written in ascending order, padded with -1, with their count.
+//
+// Design (sm_100a):
+//  * One CTA owns 64 consecutive query blocks of one (b, head) and streams
+//    the key summaries of its KV head in tiles of 64 blocks through shared
+//    memory, so each summary tile is read once per 64 query blocks.  Scores
+//    are fp32 FMA dot products (a 4x4 register tile per thread): fp32 keeps
+//    the ranking exact up to ~1e-6 relative, which tensor-core bf16/tf32
+//    products would not.
+//  * Causal row tiles have triangular work; the grid visits the heaviest
+//    (last) tiles first.
+//  * Each warp owns 8 query-block rows and keeps each row's running top list
+//    in registers as 64-bit keys (orderable score bits << 32 | ~block), so
+//    "score descending, index ascending" is one unsigned compare and every
+//    key is distinct.  A new batch of 32 candidates is filtered by a ballot
+//    against the current k-th key; a few survivors are inserted by a warp
+//    shift, many are sorted with a register bitonic network (shuffles) and
+//    merged into the list with a bitonic merge.
+#pragma once
+
+#include "common.cuh"
+
+namespace ssa {
+
+constexpr int kRouteRows = 64;     // query blocks per CTA
+constexpr int kRouteCands = 64;    // key blocks per summary tile
+constexpr int kRouteThreads = 256;
+
+struct RouteArgs {
+  const float* qsum;   // [B*Hq, NQB, D]
+  const float* ksum;   // [B*Hkv, NB, D]
+  int32_t* idx;        // [B*Hq, NQB, top_k]
+  int32_t* cnt;        // [B*Hq, NQB]
+  int32_t Hq, Hkv, NQB, NB, Bq, Bk, top_k, causal;
+  int32_t n_row_tiles;
+};
+
+// orderable 64-bit key: larger key <=> (higher score, then lower index)
+__device__ __forceinline__ uint64_t route_key(float s, int c) {
+  s = (s == 0.0f) ? 0.0f : s;  // -0 and +0 are the same score
+  const uint32_t u = __float_as_uint(s);
+  const uint32_t hi = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<uint64_t>(hi) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(c));
+}
+
+__device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
+__device__ __forceinline__ uint64_t umin64(uint64_t a, uint64_t b) { return a < b ? a : b; }
+
+// bitonic sort of one key per lane, descending over lanes
+__device__ __forceinline__ uint64_t warp_sort_desc(uint64_t x, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint64_t y = __shfl_xor_sync(0xffffffffu, x, j);
+      const bool desc_block = (lane & k) == 0;
+      const bool low = (lane & j) == 0;
+      x = (low == desc_block) ? umax64(x, y) : umin64(x, y);
+    }
+  }
+  return x;
+}
+
+// list element e = lane + 32*r, sorted descending over e
+template <int R>
+__device__ __forceinline__ uint64_t list_get(const uint64_t (&v)[R], int e) {
+  uint64_t src = v[0];
+#pragma unroll
+  for (int r = 1; r < R; ++r)
+    if ((e >> 5) == r) src = v[r];
+  return __shfl_sync(0xffffffffu, src, e & 31);
+}
+
+// insert one key (same value in every lane) that beats the current k-th key
+template <int R>
+__device__ __forceinline__ void list_insert(uint64_t (&v)[R], uint64_t y, int lane) {
+  int pos = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) pos += __popc(__ballot_sync(0xffffffffu, v[r] > y));
+  uint64_t carry = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    uint64_t up = __shfl_up_sync(0xffffffffu, v[r], 1);
+    const uint64_t last = __shfl_sync(0xffffffffu, v[r], 31);
+    if (lane == 0) up = carry;
+    const int e = lane + 32 * r;
+    v[r] = (e < pos) ? v[r] : (e == pos ? y : up);
+    carry = last;
+  }
+}
+
+// merge 32 keys sorted descending (one per lane) into the list, keeping the
+// top 32*R: max against the reversed batch makes a bitonic sequence, which a
+// bitonic merge sorts
+template <int R>
+__device__ __forceinline__ void list_merge(uint64_t (&v)[R], uint64_t sorted, int lane) {
+  const uint64_t rev = __shfl_sync(0xffffffffu, sorted, 31 - lane);
+  v[R - 1] = umax64(v[R - 1], rev);
+  if (R == 2) {
+    const uint64_t a = v[0], b = v[R - 1];
+    v[0] = umax64(a, b);
+    v[R - 1] = umin64(a, b);
+  }
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const bool low = (lane & j) == 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const uint64_t y = __shfl_xor_sync(0xffffffffu, v[r], j);
+      v[r] = low ? umax64(v[r], y) : umin64(v[r], y);
+    }
+  }
+}
+
+// offer one candidate key per lane (0 = no candidate)
+template <int R>
+__device__ __forceinline__ void list_offer(uint64_t (&v)[R], uint64_t& thr, uint64_t x, int k,
+                                           int lane) {
+  const bool pass = x > thr;
+  uint32_t m = __ballot_sync(0xffffffffu, pass);
+  if (m == 0) return;
+  if (__popc(m) <= 4) {
+    while (m) {
+      const int src = __ffs(m) - 1;
+      m &= m - 1;
+      const uint64_t y = __shfl_sync(0xffffffffu, x, src);
+      if (y > thr) {
+        list_insert<R>(v, y, lane);
+        thr = list_get<R>(v, k - 1);
+      }
+    }
+  } else {
+    const uint64_t s = warp_sort_desc(pass ? x : 0ull, lane);
+    list_merge<R>(v, s, lane);
+    thr = list_get<R>(v, k - 1);
+  }
+}
+
+// ascending bitonic sort of 32*R ints spread as e = lane + 32*r
+template <int R>
+__device__ __forceinline__ void warp_sort_asc_i32(int (&a)[R], int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32 * R; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {
+        // only when R == 2 and k == 64: the whole sequence is one ascending block
+        const int x0 = a[0], x1 = a[R - 1];
+        a[0] = min(x0, x1);
+        a[R - 1] = max(x0, x1);
+      } else {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int e = lane + 32 * r;
+          const int y = __shfl_xor_sync(0xffffffffu, a[r], j);
+          const bool asc = (e & k) == 0;
+          const bool low = (lane & j) == 0;
+          a[r] = (low == asc) ? min(a[r], y) : max(a[r], y);
+        }
+      }
+    }
+  }
+}
+
+template <int D, int R>
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a) {
+  extern __shared__ __align__(16) float rsm[];
+  float* qsT = rsm;                         // [D][64]   query summaries, transposed
+  float* ksT = qsT + D * kRouteRows;        // [D][64]   key summaries, transposed
+  float* sc = ksT + D * kRouteCands;        // [64][65]  score tile
+  constexpr int SC_LD = kRouteCands + 1;
+  constexpr int ROWS_PER_WARP = kRouteRows / (kRouteThreads / 32);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.y;
+  const int b = bh / a.Hq, h = bh % a.Hq;
+  const int bkv = b * a.Hkv + h / (a.Hq / a.Hkv);
+  const int rt = a.causal ? (a.n_row_tiles - 1 - static_cast<int>(blockIdx.x))
+                          : static_cast<int>(blockIdx.x);
+  const int qb0 = rt * kRouteRows;
+  const int qb_last = min(qb0 + kRouteRows - 1, a.NQB - 1);
+  const int lim_max =
+      a.top_k == 0 ? 0
+      : a.causal   ? min(a.NB, static_cast<int>((static_cast<int64_t>(qb_last) * a.Bq) / a.Bk))
+                   : a.NB;
+  const int n_tiles = (lim_max + kRouteCands - 1) / kRouteCands;
+
+  const float* qsrc = a.qsum + static_cast<int64_t>(bh) * a.NQB * D;
+  const float* ksrc = a.ksum + static_cast<int64_t>(bkv) * a.NB * D;
+
+  // query summaries of this row tile, transposed (consecutive threads take
+  // consecutive rows so the shared-memory stores do not conflict)
+  for (int i = tid; i < kRouteRows * (D / 4); i += kRouteThreads) {
+    const int r = i % kRouteRows, d4 = i / kRouteRows;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (qb0 + r < a.NQB)
+      v = *reinterpret_cast<const float4*>(qsrc + static_cast<int64_t>(qb0 + r) * D + d4 * 4);
+    qsT[(d4 * 4 + 0) * kRouteRows + r] = v.x;
+    qsT[(d4 * 4 + 1) * kRouteRows + r] = v.y;
+    qsT[(d4 * 4 + 2) * kRouteRows + r] = v.z;
+    qsT[(d4 * 4 + 3) * kRouteRows + r] = v.w;
+  }
+
+  uint64_t list[ROWS_PER_WARP][R];
+  uint64_t thr[ROWS_PER_WARP];
+  int lim[ROWS_PER_WARP];
+#pragma unroll
+  for (int rr = 0; rr < ROWS_PER_WARP; ++rr) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) list[rr][r] = 0ull;
+    thr[rr] = 0ull;
+    const int qb = qb0 + warp * ROWS_PER_WARP + rr;
+    lim[rr] = a.causal ? min(a.NB, static_cast<int>((static_cast<int64_t>(qb) * a.Bq) / a.Bk))
+                       : a.NB;
+    if (qb >= a.NQB) lim[rr] = 0;
+  }
+
+  const int ty = tid / 16, tx = tid % 16;
+  for (int tile = 0; tile < n_tiles; ++tile) {
+    const int c0 = tile * kRouteCands;
+    for (int i = tid; i < kRouteCands * (D / 4); i += kRouteThreads) {
+      const int c = i % kRouteCands, d4 = i / kRouteCands;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c0 + c < a.NB)
+        v = *reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(c0 + c) * D + d4 * 4);
+      ksT[(d4 * 4 + 0) * kRouteCands + c] = v.x;
+      ksT[(d4 * 4 + 1) * kRouteCands + c] = v.y;
+      ksT[(d4 * 4 + 2) * kRouteCands + c] = v.z;
+      ksT[(d4 * 4 + 3) * kRouteCands + c] = v.w;
+    }
+    __syncthreads();
+
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+    for (int d = 0; d < D; ++d) {
+      const float4 qa = *reinterpret_cast<const float4*>(qsT + d * kRouteRows + ty * 4);
+      const float4 kb = *reinterpret_cast<const float4*>(ksT + d * kRouteCands + tx * 4);
+      const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
+      const float kv[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qv[i], kv[j], acc[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sc[(ty * 4 + i) * SC_LD + tx * 4 + j] = acc[i][j];
+    __syncthreads();
+
+#pragma unroll
+    for (int rr = 0; rr < ROWS_PER_WARP; ++rr) {
+      const int row = warp * ROWS_PER_WARP + rr;
+      if (c0 < lim[rr]) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int cl = half * 32 + lane;
+          const int c = c0 + cl;
+          const uint64_t key = (c < lim[rr]) ? route_key(sc[row * SC_LD + cl], c) : 0ull;
+          list_offer<R>(list[rr], thr[rr], key, a.top_k, lane);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // epilogue: the first top_k keys, as block indices in ascending order
+#pragma unroll
+  for (int rr = 0; rr < ROWS_PER_WARP; ++rr) {
+    const int qb = qb0 + warp * ROWS_PER_WARP + rr;
+    if (qb >= a.NQB) continue;
+    int vals[R];
+    int n_valid = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int e = lane + 32 * r;
+      const bool ok = e < a.top_k && list[rr][r] != 0ull;
+      vals[r] = ok ? static_cast<int>(~static_cast<uint32_t>(list[rr][r] & 0xFFFFFFFFull))
+                   : 0x7FFFFFFF;
+      n_valid += __popc(__ballot_sync(0xffffffffu, ok));
+    }
+    warp_sort_asc_i32<R>(vals, lane);
+    int32_t* dst = a.idx + (static_cast<int64_t>(bh) * a.NQB + qb) * a.top_k;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int e = lane + 32 * r;
+      if (e < a.top_k) dst[e] = e < n_valid ? vals[r] : -1;
+    }
+    if (lane == 0) a.cnt[static_cast<int64_t>(bh) * a.NQB + qb] = n_valid;
+  }
+}
+
+}  // namespace ssa

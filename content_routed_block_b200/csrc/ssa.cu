@@ -1,0 +1,407 @@
+// libssa.so: C ABI of content-routed block-sparse attention on B200.
+//
+// Host side: argument validation (synchronous, before any launch), TMA
+// tensor-map encoding, and the launches of the three sm_100a kernels on the
+// caller's stream.  The library allocates no device memory; its device state
+// is the error word below.  The CUDA runtime is linked statically and the
+// driver's tensor-map encoder is looked up at first use, so the library loads
+// on a machine without a GPU (calls then fail with SSA_ERR_CUDA).
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "../../include/ssa.h"
+#include "attend.cuh"
+#include "common.cuh"
+#include "pool.cuh"
+#include "route.cuh"
+
+namespace ssa {
+__global__ void probe_wait_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // nothing ever arrives: the wait must give up on its own
+    mbar_wait(&bar, 0, timeout_ns, &abort_flag, kSiteProbe);
+  }
+  __syncthreads();
+}
+}  // namespace ssa
+
+namespace {
+
+constexpr int32_t kVersion = 1;
+thread_local std::string g_msg;
+
+ssa_status fail(ssa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+ssa_status fail(ssa_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_msg = buf;
+  return s;
+}
+
+ssa_status ok() {
+  g_msg.clear();
+  return SSA_OK;
+}
+
+ssa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool pow2_in(int32_t x, int32_t lo, int32_t hi) {
+  return x >= lo && x <= hi && (x & (x - 1)) == 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+ssa_status validate(const ssa_params* p) {
+  if (p == nullptr) return fail(SSA_ERR_INVALID_ARG, "params is NULL");
+  if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->N < 1 || p->D < 1)
+    return fail(SSA_ERR_INVALID_ARG, "B, Hq, Hkv, N, D must be positive");
+  if (p->Hq % p->Hkv != 0) return fail(SSA_ERR_INVALID_ARG, "Hq must be a multiple of Hkv");
+  if (p->D != 64 && p->D != 128) return fail(SSA_ERR_UNSUPPORTED, "D must be 64 or 128");
+  if (!pow2_in(p->block_k, 16, 128) || !pow2_in(p->block_q, 16, 128))
+    return fail(SSA_ERR_UNSUPPORTED, "block_k and block_q must be powers of two in [16, 128]");
+  if (p->N % p->block_k != 0 || p->N % p->block_q != 0)
+    return fail(SSA_ERR_UNSUPPORTED, "N must be a multiple of block_k and block_q");
+  if (p->top_k < 0 || p->top_k > 64) return fail(SSA_ERR_UNSUPPORTED, "top_k must be in 0..64");
+  if (p->window < 0) return fail(SSA_ERR_INVALID_ARG, "window must be >= 0");
+  if (p->causal != 0 && p->causal != 1) return fail(SSA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (p->causal && p->window < 1)
+    return fail(SSA_ERR_INVALID_ARG, "causal attention needs window >= 1 (every query sees itself)");
+  if (!p->causal && p->window != 0)
+    return fail(SSA_ERR_INVALID_ARG, "the non-causal variant has no window (window must be 0)");
+  if (!p->causal && p->top_k < 1)
+    return fail(SSA_ERR_INVALID_ARG, "the non-causal variant needs top_k >= 1");
+  if (!(p->scale >= 0.f) || !std::isfinite(p->scale))
+    return fail(SSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (p->wait_timeout_us < 0) return fail(SSA_ERR_INVALID_ARG, "wait_timeout_us must be >= 0");
+  const int64_t nb = p->N / p->block_k;
+  if (nb >= (1 << 23)) return fail(SSA_ERR_UNSUPPORTED, "N / block_k must be below 2^23");
+  const int64_t rows = static_cast<int64_t>(p->B) * p->Hq * p->N;
+  if (rows > (static_cast<int64_t>(1) << 31) - 1)
+    return fail(SSA_ERR_UNSUPPORTED, "B * Hq * N must fit in int32");
+  if (p->causal) {
+    const int64_t nwin = (static_cast<int64_t>(p->window) + ssa::kAtQT - 2) / p->block_k + 2;
+    if (nwin > ssa::kAtLCap)
+      return fail(SSA_ERR_UNSUPPORTED, "window spans more than %d key blocks per query tile",
+                  ssa::kAtLCap);
+  }
+  return SSA_OK;
+}
+
+uint64_t timeout_ns(const ssa_params* p) {
+  return p->wait_timeout_us > 0 ? static_cast<uint64_t>(p->wait_timeout_us) * 1000ull
+                                : 2000000000ull;
+}
+
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+ssa_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (g_encode == nullptr)
+    return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (no CUDA driver?)");
+  return SSA_OK;
+}
+
+// 3-D view [heads, N, D] of a bf16 tensor, box {64 columns, rows, 1}, 128B swizzle
+ssa_status make_map(CUtensorMap* m, const void* base, int64_t heads, int64_t n, int64_t d,
+                    uint32_t box_rows) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2),
+                                 static_cast<cuuint64_t>(n * d * 2)};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return SSA_OK;
+}
+
+// ---------------------------------------------------------------- launches
+ssa_status launch_pool(const ssa_params* p, const void* x0, int32_t H0, int32_t blk0, float* out0,
+                       const void* x1, int32_t H1, int32_t blk1, float* out1,
+                       cudaStream_t stream) {
+  const int G = p->D / 8;
+  ssa::PoolJob j0{static_cast<const uint4*>(x0), out0,
+                  static_cast<int64_t>(p->B) * H0 * (p->N / blk0), blk0, 1.0f / blk0};
+  ssa::PoolJob j1 = j0;
+  int64_t n1 = 0;
+  if (x1 != nullptr) {
+    j1 = ssa::PoolJob{static_cast<const uint4*>(x1), out1,
+                      static_cast<int64_t>(p->B) * H1 * (p->N / blk1), blk1, 1.0f / blk1};
+    n1 = j1.n_blocks * G;
+  }
+  const int64_t split = j0.n_blocks * G;
+  const int64_t total = split + n1;
+  const int64_t grid = (total + 255) / 256;
+  if (p->D == 64)
+    ssa::block_mean_kernel<64><<<static_cast<unsigned>(grid), 256, 0, stream>>>(j0, j1, split);
+  else
+    ssa::block_mean_kernel<128><<<static_cast<unsigned>(grid), 256, 0, stream>>>(j0, j1, split);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "block_mean_kernel launch");
+  return SSA_OK;
+}
+
+template <int D, int R>
+cudaError_t launch_route_t(const ssa::RouteArgs& a, int B, cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(2 * D * 64 + 64 * 65) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(ssa::route_kernel<D, R>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.n_row_tiles, B * a.Hq);
+  ssa::route_kernel<D, R><<<grid, ssa::kRouteThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksum, int32_t* idx,
+                        int32_t* cnt, cudaStream_t stream) {
+  ssa::RouteArgs a;
+  a.qsum = qsum;
+  a.ksum = ksum;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.NQB = p->N / p->block_q;
+  a.NB = p->N / p->block_k;
+  a.Bq = p->block_q;
+  a.Bk = p->block_k;
+  a.top_k = p->top_k;
+  a.causal = p->causal;
+  a.n_row_tiles = (a.NQB + ssa::kRouteRows - 1) / ssa::kRouteRows;
+  cudaError_t e;
+  if (p->D == 64)
+    e = p->top_k <= 32 ? launch_route_t<64, 1>(a, p->B, stream) : launch_route_t<64, 2>(a, p->B, stream);
+  else
+    e = p->top_k <= 32 ? launch_route_t<128, 1>(a, p->B, stream)
+                       : launch_route_t<128, 2>(a, p->B, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "route_kernel launch");
+  return SSA_OK;
+}
+
+template <int D>
+cudaError_t launch_attend_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const ssa::AttendArgs& a, int n_ctas, cudaStream_t stream) {
+  const uint32_t smem = ssa::AtLayout<D>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(ssa::attend_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  ssa::attend_kernel<D><<<n_ctas, ssa::kAtThreads, smem, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+ssa_status launch_attend(const ssa_params* p, const void* q, const void* k, const void* v,
+                         const int32_t* idx, const int32_t* cnt, void* o, float* lse,
+                         cudaStream_t stream) {
+  ssa_status s = get_encoder();
+  if (s != SSA_OK) return s;
+  CUtensorMap tq, tk, tv;
+  const uint32_t kv_rows = static_cast<uint32_t>(p->block_k < 64 ? p->block_k : 64);
+  if ((s = make_map(&tq, q, static_cast<int64_t>(p->B) * p->Hq, p->N, p->D, 128)) != SSA_OK) return s;
+  if ((s = make_map(&tk, k, static_cast<int64_t>(p->B) * p->Hkv, p->N, p->D, kv_rows)) != SSA_OK)
+    return s;
+  if ((s = make_map(&tv, v, static_cast<int64_t>(p->B) * p->Hkv, p->N, p->D, kv_rows)) != SSA_OK)
+    return s;
+  ssa::AttendArgs a;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.N = p->N;
+  a.NQB = p->N / p->block_q;
+  a.NB = p->N / p->block_k;
+  a.Bq = p->block_q;
+  a.Bk = p->block_k;
+  a.top_k = p->top_k;
+  a.window = p->window;
+  a.causal = p->causal;
+  a.n_qtiles = (p->N + ssa::kAtQT - 1) / ssa::kAtQT;
+  const float scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.timeout_ns = timeout_ns(p);
+  const int64_t n_ctas = static_cast<int64_t>(p->B) * p->Hq * a.n_qtiles;
+  if (n_ctas > 0x7FFFFFFF) return fail(SSA_ERR_UNSUPPORTED, "too many query tiles");
+  const cudaError_t e =
+      p->D == 64 ? launch_attend_t<64>(tq, tk, tv, a, static_cast<int>(n_ctas), stream)
+                 : launch_attend_t<128>(tq, tk, tv, a, static_cast<int>(n_ctas), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "attend_kernel launch");
+  return SSA_OK;
+}
+
+struct WsLayout {
+  size_t ksum, qsum, idx, cnt, total;
+};
+
+WsLayout ws_layout(const ssa_params* p) {
+  WsLayout w;
+  const size_t nb = p->N / p->block_k, nqb = p->N / p->block_q;
+  const size_t ks = static_cast<size_t>(p->B) * p->Hkv * nb * p->D * sizeof(float);
+  const size_t qs = static_cast<size_t>(p->B) * p->Hq * nqb * p->D * sizeof(float);
+  const size_t ix = static_cast<size_t>(p->B) * p->Hq * nqb * p->top_k * sizeof(int32_t);
+  const size_t cn = static_cast<size_t>(p->B) * p->Hq * nqb * sizeof(int32_t);
+  w.ksum = 0;
+  w.qsum = align256(ks);
+  w.idx = w.qsum + align256(qs);
+  w.cnt = w.idx + align256(ix);
+  w.total = w.cnt + align256(cn);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssa_workspace_size(const ssa_params* p) {
+  if (validate(p) != SSA_OK) return 0;
+  return ws_layout(p).total;
+}
+
+ssa_status ssa_block_summary(const ssa_params* p, const void* x, int32_t H, int32_t block,
+                             float* out, ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (x == nullptr || out == nullptr) return fail(SSA_ERR_INVALID_ARG, "x and out must be non-NULL");
+  if (!aligned16(x) || !aligned16(out))
+    return fail(SSA_ERR_INVALID_ARG, "x and out must be 16-byte aligned");
+  if (H < 1) return fail(SSA_ERR_INVALID_ARG, "H must be positive");
+  if (!pow2_in(block, 1, 1 << 20) || p->N % block != 0)
+    return fail(SSA_ERR_INVALID_ARG, "block must be a power of two dividing N");
+  s = launch_pool(p, x, H, block, out, nullptr, 0, 0, nullptr, static_cast<cudaStream_t>(stream));
+  return s == SSA_OK ? ok() : s;
+}
+
+ssa_status ssa_route(const ssa_params* p, const float* qsum, const float* ksum, int32_t* idx,
+                     int32_t* cnt, ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (qsum == nullptr || ksum == nullptr || cnt == nullptr || (p->top_k > 0 && idx == nullptr))
+    return fail(SSA_ERR_INVALID_ARG, "qsum, ksum, cnt (and idx when top_k > 0) must be non-NULL");
+  if (!aligned16(qsum) || !aligned16(ksum) || !aligned16(cnt) || (idx && !aligned16(idx)))
+    return fail(SSA_ERR_INVALID_ARG, "routing buffers must be 16-byte aligned");
+  s = launch_route(p, qsum, ksum, idx, cnt, static_cast<cudaStream_t>(stream));
+  return s == SSA_OK ? ok() : s;
+}
+
+ssa_status ssa_attend(const ssa_params* p, const void* q, const void* k, const void* v,
+                      const int32_t* idx, const int32_t* cnt, void* o, float* lse,
+                      ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (!q || !k || !v || !o || !cnt || (p->top_k > 0 && !idx))
+    return fail(SSA_ERR_INVALID_ARG, "q, k, v, o, cnt (and idx when top_k > 0) must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return fail(SSA_ERR_INVALID_ARG, "q, k, v, o and lse must be 16-byte aligned");
+  s = launch_attend(p, q, k, v, idx, cnt, o, lse, static_cast<cudaStream_t>(stream));
+  return s == SSA_OK ? ok() : s;
+}
+
+ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const void* v, void* o,
+                       float* lse, int32_t* idx_out, int32_t* cnt_out, void* workspace,
+                       size_t workspace_bytes, ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (!q || !k || !v || !o) return fail(SSA_ERR_INVALID_ARG, "q, k, v, o must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)) ||
+      (idx_out && !aligned16(idx_out)) || (cnt_out && !aligned16(cnt_out)))
+    return fail(SSA_ERR_INVALID_ARG, "all buffers must be 16-byte aligned");
+  const WsLayout w = ws_layout(p);
+  if (workspace == nullptr || workspace_bytes < w.total)
+    return fail(SSA_ERR_WORKSPACE, "workspace needs %zu bytes", w.total);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* ksum = reinterpret_cast<float*>(ws + w.ksum);
+  float* qsum = reinterpret_cast<float*>(ws + w.qsum);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + w.idx);
+  int32_t* cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(ws + w.cnt);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = launch_pool(p, k, p->Hkv, p->block_k, ksum, q, p->Hq, p->block_q, qsum, st)) != SSA_OK)
+    return s;
+  if ((s = launch_route(p, qsum, ksum, idx, cnt, st)) != SSA_OK) return s;
+  if ((s = launch_attend(p, q, k, v, idx, cnt, o, lse, st)) != SSA_OK) return s;
+  return ok();
+}
+
+ssa_status ssa_check_error(ssa_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  uint32_t flags = 0, site = 0;
+  if ((e = cudaMemcpyFromSymbol(&flags, ssa::g_err_flags, sizeof(flags))) != cudaSuccess)
+    return cuda_fail(e, "read error word");
+  if ((e = cudaMemcpyFromSymbol(&site, ssa::g_err_site, sizeof(site))) != cudaSuccess)
+    return cuda_fail(e, "read error site");
+  const uint32_t zero = 0;
+  if ((e = cudaMemcpyToSymbol(ssa::g_err_flags, &zero, sizeof(zero))) != cudaSuccess)
+    return cuda_fail(e, "clear error word");
+  if ((e = cudaMemcpyToSymbol(ssa::g_err_site, &zero, sizeof(zero))) != cudaSuccess)
+    return cuda_fail(e, "clear error site");
+  if (flags & ssa::kErrTimeout)
+    return fail(SSA_ERR_TIMEOUT, "a device-side wait ran out (site %u)", site);
+  if (flags & ssa::kErrCheck)
+    return fail(SSA_ERR_DEVICE_CHECK, "a device-side check failed (site %u)", site);
+  return ok();
+}
+
+ssa_status ssa_probe_wait_timeout(int32_t timeout_us, ssa_stream_t stream) {
+  if (timeout_us < 1 || timeout_us > 10000000)
+    return fail(SSA_ERR_INVALID_ARG, "timeout_us must be in 1..10^7");
+  ssa::probe_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_us) * 1000ull);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "probe_wait_kernel launch");
+  return ok();
+}
+
+const char* ssa_status_string(ssa_status s) {
+  switch (s) {
+    case SSA_OK: return "ok";
+    case SSA_ERR_INVALID_ARG: return "invalid argument";
+    case SSA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SSA_ERR_WORKSPACE: return "workspace too small";
+    case SSA_ERR_CUDA: return "CUDA error";
+    case SSA_ERR_TIMEOUT: return "device wait timed out";
+    case SSA_ERR_DEVICE_CHECK: return "device check failed";
+  }
+  return "unknown status";
+}
+
+const char* ssa_last_error_message(void) { return g_msg.c_str(); }
+
+int32_t ssa_version(void) { return kVersion; }
+
+}  // extern "C"

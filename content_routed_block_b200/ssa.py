@@ -1,0 +1,224 @@
+"""Thin Python binding of libssa.so (ctypes, argument marshalling only).
+
+Every step of the path runs in the library's CUDA kernels; this module only
+checks tensor shapes / dtypes / devices, allocates outputs with PyTorch and
+passes raw pointers plus the current CUDA stream.  There is no fallback: if
+libssa.so is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+__all__ = [
+    "Params", "SsaError", "lib", "make_params", "params_of", "workspace_size", "block_summary",
+    "route", "attend", "forward", "forward_host", "check_error", "probe_wait_timeout",
+    "declared_functions", "LIB_PATH", "HEADER_PATH",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "ssa.h")
+
+SSA_OK = 0
+
+
+class SsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"ssa status {status}: {message}")
+        self.status = status
+        self.message = message
+
+
+class Params(ctypes.Structure):
+    """Mirror of ``ssa_params`` in include/ssa.h."""
+    _fields_ = [
+        ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+        ("N", ctypes.c_int32), ("D", ctypes.c_int32), ("block_k", ctypes.c_int32),
+        ("block_q", ctypes.c_int32), ("top_k", ctypes.c_int32), ("window", ctypes.c_int32),
+        ("causal", ctypes.c_int32), ("scale", ctypes.c_float),
+        ("wait_timeout_us", ctypes.c_int32),
+    ]
+
+    @property
+    def n_kblocks(self) -> int:
+        return self.N // self.block_k
+
+    @property
+    def n_qblocks(self) -> int:
+        return self.N // self.block_q
+
+
+def make_params(B, Hq, Hkv, N, D, block_k, block_q, top_k, window, causal, scale=0.0,
+                wait_timeout_us=0) -> Params:
+    return Params(B, Hq, Hkv, N, D, block_k, block_q, top_k, window, int(bool(causal)),
+                  float(scale), wait_timeout_us)
+
+
+def params_of(w, **over) -> Params:
+    """Params from any object with the workload field names."""
+    f = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=w.N, D=w.D, block_k=w.block_k, block_q=w.block_q,
+             top_k=w.top_k, window=w.window, causal=w.causal, scale=getattr(w, "scale", 0.0))
+    f.update(over)
+    return make_params(**f)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libssa.so once.  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m content_routed_block_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(Params)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    sig = {
+        "ssa_workspace_size": (sz, [P]),
+        "ssa_block_summary": (i32, [P, vp, i32, i32, vp, vp]),
+        "ssa_route": (i32, [P, vp, vp, vp, vp, vp]),
+        "ssa_attend": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "ssa_forward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ssa_check_error": (i32, [vp]),
+        "ssa_probe_wait_timeout": (i32, [i32, vp]),
+        "ssa_status_string": (ctypes.c_char_p, [i32]),
+        "ssa_last_error_message": (ctypes.c_char_p, []),
+        "ssa_version": (i32, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def declared_functions() -> list[str]:
+    """Entry points declared in include/ssa.h."""
+    src = open(HEADER_PATH).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssa_[a-z_]+)\s*\(", src)))
+
+
+def _check(status: int):
+    if status != SSA_OK:
+        L = lib()
+        raise SsaError(status, f"{L.ssa_status_string(status).decode()}: "
+                               f"{L.ssa_last_error_message().decode()}")
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, shape, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def workspace_size(p: Params) -> int:
+    return int(lib().ssa_workspace_size(ctypes.byref(p)))
+
+
+def block_summary(x: torch.Tensor, block: int, p: Params) -> torch.Tensor:
+    """fp32 [B, H, N/block, D] means of every ``block`` rows of bf16 x [B, H, N, D]."""
+    H = x.shape[1]
+    _need(x, torch.bfloat16, (p.B, H, p.N, p.D), "x")
+    out = torch.empty((p.B, H, p.N // block, p.D), dtype=torch.float32, device=x.device)
+    _check(lib().ssa_block_summary(ctypes.byref(p), _ptr(x), H, block, _ptr(out), _stream()))
+    return out
+
+
+def route(qsum: torch.Tensor, ksum: torch.Tensor, p: Params):
+    """(idx int32 [B, Hq, NQB, top_k], cnt int32 [B, Hq, NQB])."""
+    _need(qsum, torch.float32, (p.B, p.Hq, p.n_qblocks, p.D), "qsum")
+    _need(ksum, torch.float32, (p.B, p.Hkv, p.n_kblocks, p.D), "ksum")
+    dev = qsum.device
+    idx = torch.empty((p.B, p.Hq, p.n_qblocks, p.top_k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((p.B, p.Hq, p.n_qblocks), dtype=torch.int32, device=dev)
+    _check(lib().ssa_route(ctypes.byref(p), _ptr(qsum), _ptr(ksum),
+                           _ptr(idx) if p.top_k else None, _ptr(cnt), _stream()))
+    return idx, cnt
+
+
+def attend(q, k, v, idx, cnt, p: Params, with_lse: bool = True):
+    """(o bf16 [B, Hq, N, D], lse fp32 [B, Hq, N] or None)."""
+    _need(q, torch.bfloat16, (p.B, p.Hq, p.N, p.D), "q")
+    _need(k, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "k")
+    _need(v, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "v")
+    _need(idx, torch.int32, (p.B, p.Hq, p.n_qblocks, p.top_k), "idx")
+    _need(cnt, torch.int32, (p.B, p.Hq, p.n_qblocks), "cnt")
+    o = torch.empty_like(q)
+    lse = torch.empty((p.B, p.Hq, p.N), dtype=torch.float32, device=q.device) if with_lse else None
+    _check(lib().ssa_attend(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                            _ptr(idx) if p.top_k else None, _ptr(cnt), _ptr(o), _ptr(lse),
+                            _stream()))
+    return o, lse
+
+
+def forward(q, k, v, p: Params, workspace: torch.Tensor | None = None, with_lse: bool = True,
+            out: torch.Tensor | None = None, lse_out: torch.Tensor | None = None,
+            idx_out: torch.Tensor | None = None, cnt_out: torch.Tensor | None = None):
+    """Whole path in one library call.  Returns (o, lse, idx, cnt); idx/cnt are
+    the caller's ``idx_out``/``cnt_out`` if given, else fresh tensors."""
+    _need(q, torch.bfloat16, (p.B, p.Hq, p.N, p.D), "q")
+    _need(k, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "k")
+    _need(v, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "v")
+    dev = q.device
+    ws = workspace_size(p)
+    if workspace is None or workspace.numel() < ws:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+    o = out if out is not None else torch.empty_like(q)
+    lse = lse_out if lse_out is not None else (
+        torch.empty((p.B, p.Hq, p.N), dtype=torch.float32, device=dev) if with_lse else None)
+    idx = idx_out if idx_out is not None else torch.empty(
+        (p.B, p.Hq, p.n_qblocks, max(p.top_k, 0)), dtype=torch.int32, device=dev)
+    cnt = cnt_out if cnt_out is not None else torch.empty(
+        (p.B, p.Hq, p.n_qblocks), dtype=torch.int32, device=dev)
+    _check(lib().ssa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                             _ptr(idx) if p.top_k else None, _ptr(cnt), _ptr(workspace),
+                             workspace.numel(), _stream()))
+    return o, lse, idx, cnt
+
+
+def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
+                 device: torch.device | str = "cuda", workspace: torch.Tensor | None = None,
+                 dev_bufs: dict | None = None):
+    """End-to-end call from host memory: copy pinned bf16 Q, K, V to the
+    device, run the path, copy O back into ``o_host`` (pinned).  ``dev_bufs``
+    may hold preallocated device tensors (keys q, k, v, o) to reuse."""
+    d = dev_bufs if dev_bufs is not None else {}
+    for name, src in (("q", q_host), ("k", k_host), ("v", v_host)):
+        if name not in d:
+            d[name] = torch.empty(src.shape, dtype=src.dtype, device=device)
+        d[name].copy_(src, non_blocking=True)
+    if "o" not in d:
+        d["o"] = torch.empty(q_host.shape, dtype=torch.bfloat16, device=device)
+    forward(d["q"], d["k"], d["v"], p, workspace=workspace, with_lse=False, out=d["o"])
+    o_host.copy_(d["o"], non_blocking=True)
+    return o_host
+
+
+def check_error(stream=None):
+    """Synchronise the stream and raise if a kernel recorded a device error."""
+    s = _stream() if stream is None else stream
+    _check(lib().ssa_check_error(s))
+
+
+def probe_wait_timeout(timeout_us: int):
+    _check(lib().ssa_probe_wait_timeout(int(timeout_us), _stream()))

@@ -1,0 +1,143 @@
+/*
+ * ssa.h -- C ABI of libssa.so: content-routed block-sparse exact attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operation (jonsmirl/ssa README, introduction and "Algorithm and
+ * complexity"; SingleZombie/LLSA README, "Minimum Usage" for the non-causal
+ * variant): keys are mean-pooled into blocks of Bk rows; every query block of
+ * Bq rows scores the summaries of its admissible key blocks, keeps the top-k
+ * (ties go to the lower block index), adds the local causal window of W
+ * tokens, and runs ordinary exact softmax attention over that union only.
+ * The dense N x N score matrix is never formed.
+ *
+ * Conventions for every entry point
+ *   Layout     Q: bf16 [B, Hq, N, D]; K, V: bf16 [B, Hkv, N, D]; O like Q.
+ *              Contiguous, row-major, D innermost.  Query head h reads KV
+ *              head h / (Hq / Hkv).
+ *   Pointers   Device pointers unless stated otherwise.  Q, K, V, O must be
+ *              16-byte aligned (the kernels move them with TMA / 16-byte
+ *              vectors); float and int32 buffers 16-byte aligned.
+ *   Ownership  The caller owns every buffer.  The library allocates no device
+ *              memory: its only device state is a file-scope error word per
+ *              device that ssa_check_error reads and clears.
+ *   Streams    Every call is asynchronous on the caller's stream (a
+ *              cudaStream_t passed as ssa_stream_t; NULL = legacy default
+ *              stream).  Calls on one stream run in order.
+ *   Errors     Argument errors are returned synchronously before any launch,
+ *              with a message in ssa_last_error_message().  Launch failures
+ *              return SSA_ERR_CUDA.  Device-side failures (a bounded wait
+ *              that ran out, a failed bounds check) set the device error
+ *              word; ssa_check_error() reports them.  Kernels never trap.
+ *   Threading  Thread-safe; the last-error message is per host thread.
+ */
+#ifndef SSA_H_
+#define SSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* ssa_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  SSA_OK = 0,
+  SSA_ERR_INVALID_ARG = 1,  /* a size, pointer or alignment is invalid       */
+  SSA_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels implement  */
+  SSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required    */
+  SSA_ERR_CUDA = 4,         /* a CUDA runtime call or a launch failed        */
+  SSA_ERR_TIMEOUT = 5,      /* a device-side bounded wait ran out            */
+  SSA_ERR_DEVICE_CHECK = 6  /* a device-side bounds/consistency check failed */
+} ssa_status;
+
+/* Method parameters.  Names follow the pages' notation. */
+typedef struct {
+  int32_t B;               /* batch                                            */
+  int32_t Hq;              /* query heads                                      */
+  int32_t Hkv;             /* key/value heads; Hq % Hkv == 0                   */
+  int32_t N;               /* tokens; multiple of block_k and of block_q       */
+  int32_t D;               /* head dim: 64 or 128                              */
+  int32_t block_k;         /* Bk: key block, power of two in [16, 128]         */
+  int32_t block_q;         /* Bq: query block, power of two in [16, 128]       */
+  int32_t top_k;           /* k: routed blocks per query block, 0..64          */
+  int32_t window;          /* W: local causal window in tokens (i-W < j <= i)  */
+  int32_t causal;          /* 1 causal (requires W >= 1); 0 non-causal (W = 0, k >= 1) */
+  float scale;             /* softmax scale; 0 -> 1/sqrt(D)                    */
+  int32_t wait_timeout_us; /* bound on every device-side wait; 0 -> 2 s        */
+} ssa_params;
+
+/* Bytes of device workspace ssa_forward needs for these parameters:
+ * K summaries, Q summaries, the routed index list and counts, each 256-byte
+ * aligned.  Returns 0 if the parameters are invalid. */
+size_t ssa_workspace_size(const ssa_params* p);
+
+/* Block summary (step 1 of the path; jonsmirl/ssa README, "Algorithm and
+ * complexity": mu_c, block c's mean key).
+ *   x    bf16 [B, H, N, D] (device)
+ *   out  fp32 [B, H, N / block, D] (device): out[..., c, :] = mean of rows
+ *        c*block .. c*block + block - 1, summed in fp32 then scaled by
+ *        1/block (exact: block is a power of two).
+ * H is the head count of x (Hq for queries, Hkv for keys); block is Bk or Bq.
+ * B, N and D are taken from p.  One kernel launch. */
+ssa_status ssa_block_summary(const ssa_params* p, const void* x, int32_t H,
+                             int32_t block, float* out, ssa_stream_t stream);
+
+/* Routing (steps 2-3; jonsmirl/ssa README, "Algorithm and complexity": the
+ * block score <q, mu_c>, here with the second-cumulant weight beta = 0).
+ *   qsum fp32 [B, Hq, N/Bq, D], ksum fp32 [B, Hkv, N/Bk, D] (device)
+ *   idx  int32 [B, Hq, N/Bq, top_k] (device, out): for each query block the
+ *        selected key blocks in ascending order, padded with -1
+ *   cnt  int32 [B, Hq, N/Bq] (device, out): number of selected blocks,
+ *        min(top_k, |admissible|)
+ * Admissible blocks: causal -- completed blocks ending at or before the
+ * query block's first token, (c+1)*Bk <= qb*Bq; non-causal -- all blocks.
+ * Scores are fp32 dot products of the summaries; the top_k largest win, ties
+ * to the lower block index.  top_k == 0 writes cnt = 0 only.  One launch. */
+ssa_status ssa_route(const ssa_params* p, const float* qsum, const float* ksum,
+                     int32_t* idx, int32_t* cnt, ssa_stream_t stream);
+
+/* Attend (step 4; jonsmirl/ssa README, introduction: ordinary softmax over
+ * the selected keys; "Mathematical status": the routed set is cut at each
+ * query's position).  For query i in query block qb the key set is
+ *   causal:     {keys of idx[qb]} U {i-W < j <= i}, cut at j <= i
+ *   non-causal: {keys of idx[qb]}
+ * counted once each; o_i = softmax(scale * q_i . k_j) . v_j over the set.
+ *   q, k, v  bf16 (device), layouts above
+ *   idx/cnt  as written by ssa_route (any valid lists: ascending, distinct,
+ *            admissible, cnt <= top_k)
+ *   o        bf16 [B, Hq, N, D] (device, out), round-to-nearest-even
+ *   lse      fp32 [B, Hq, N] (device, out, may be NULL): natural-log
+ *            log-sum-exp of the scaled logits over the key set
+ * One launch of the fused TMA + tcgen05 kernel. */
+ssa_status ssa_attend(const ssa_params* p, const void* q, const void* k, const void* v,
+                      const int32_t* idx, const int32_t* cnt, void* o, float* lse,
+                      ssa_stream_t stream);
+
+/* The whole path in one call: summaries of K and Q (one launch), routing,
+ * attend.  workspace must hold ssa_workspace_size(p) bytes (device, 256-byte
+ * aligned).  idx_out / cnt_out (device, may be NULL) receive the routed lists
+ * when given; otherwise they live in the workspace.  lse may be NULL. */
+ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const void* v,
+                       void* o, float* lse, int32_t* idx_out, int32_t* cnt_out,
+                       void* workspace, size_t workspace_bytes, ssa_stream_t stream);
+
+/* Synchronise the stream, then read and clear this device's error word.
+ * Returns SSA_OK, SSA_ERR_TIMEOUT, SSA_ERR_DEVICE_CHECK or SSA_ERR_CUDA. */
+ssa_status ssa_check_error(ssa_stream_t stream);
+
+/* Diagnostic: launch one block that waits, with the same bounded wait the
+ * kernels use, on a barrier nothing ever arrives on; the wait gives up after
+ * timeout_us microseconds and records SSA_ERR_TIMEOUT in the error word.
+ * Lets a caller check the timeout path without a hang. */
+ssa_status ssa_probe_wait_timeout(int32_t timeout_us, ssa_stream_t stream);
+
+const char* ssa_status_string(ssa_status s);
+const char* ssa_last_error_message(void);
+int32_t ssa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSA_H_ */

@@ -50,7 +50,7 @@ import numpy as np
 __all__ = [
     "Params", "upcast_bf16", "block_summary", "admissible_blocks", "route",
     "RouteResult", "key_set", "attend_masked_dense", "attend_gathered", "forward",
-    "near_tie_rows",
+    "near_tie_rows", "acceptable_selections", "route_row",
 ]
 
 NEAR_TIE_REL = 1e-4   # relative score gap under which two blocks count as tied
@@ -191,6 +191,34 @@ def near_tie_rows(r: RouteResult, rel: float = NEAR_TIE_REL) -> np.ndarray:
         gap = np.abs(a - c)
         tol = rel * np.maximum(np.abs(a), np.abs(c))
         return np.isfinite(gap) & (gap <= tol)
+
+
+def acceptable_selections(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, top_k: int,
+                          rel: float = NEAR_TIE_REL, limit: int = 256) -> list:
+    """Every selection that the near-tie rule accepts, ascending.
+
+    Scores are fp64.  Let s_k be the k-th best score.  Blocks whose score is
+    within ``rel`` (relative) of s_k form the tie band; blocks above the band
+    are always selected and the remaining slots may be filled by any blocks of
+    the band.  With no near-tie the list holds exactly the ``route_row``
+    selection.  At most ``limit`` selections are listed."""
+    import itertools
+    if len(cand) == 0 or top_k == 0:
+        return [np.zeros(0, dtype=np.int64)]
+    s = mu[cand] @ qbar
+    order = np.lexsort((cand, -s))
+    take = min(top_k, len(cand))
+    sk = s[order[take - 1]]
+    band = np.abs(s - sk) <= rel * np.maximum(np.abs(s), abs(sk))
+    sure = cand[(s > sk) & ~band]
+    pool = cand[band]
+    need = take - len(sure)
+    out = []
+    for combo in itertools.combinations(pool.tolist(), need):
+        out.append(np.sort(np.concatenate([sure, np.array(combo, dtype=sure.dtype)])))
+        if len(out) >= limit:
+            break
+    return out
 
 
 # --------------------------------------------------------------------------

@@ -1,0 +1,92 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, and rejects invalid arguments synchronously, before any launch."""
+import ctypes
+
+import pytest
+
+from content_routed_block_b200 import build, ssa
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ssa.lib()
+
+
+def test_every_declared_function_is_exported(L):
+    names = ssa.declared_functions()
+    assert {"ssa_block_summary", "ssa_route", "ssa_attend", "ssa_forward",
+            "ssa_workspace_size", "ssa_check_error"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_status_strings(L):
+    assert L.ssa_version() == 1
+    for s in range(7):
+        assert L.ssa_status_string(s).decode() not in ("", "unknown status")
+    assert L.ssa_status_string(99).decode() == "unknown status"
+
+
+def _p(**kw):
+    base = dict(B=1, Hq=14, Hkv=2, N=32768, D=64, block_k=64, block_q=64, top_k=16,
+                window=512, causal=True)
+    base.update(kw)
+    return ssa.make_params(**base)
+
+
+def test_workspace_layout(L):
+    p = _p()
+    ks = 1 * 2 * 512 * 64 * 4
+    qs = 1 * 14 * 512 * 64 * 4
+    ix = 1 * 14 * 512 * 16 * 4
+    cn = 1 * 14 * 512 * 4
+    a = lambda x: (x + 255) // 256 * 256
+    assert ssa.workspace_size(p) == a(ks) + a(qs) + a(ix) + a(cn)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=96), 2), (dict(D=32), 2), (dict(Hq=3, Hkv=2), 1), (dict(N=1000), 2),
+    (dict(top_k=65), 2), (dict(top_k=-1), 2), (dict(block_k=48), 2), (dict(block_k=256), 2),
+    (dict(block_q=8), 2), (dict(window=0), 1), (dict(causal=False), 1),
+    (dict(causal=False, window=0, top_k=0), 1), (dict(window=-3), 1), (dict(B=0), 1),
+    (dict(scale=float("nan")), 1), (dict(scale=-1.0), 1), (dict(wait_timeout_us=-5), 1),
+    (dict(N=16 * 2 ** 23, block_k=16, block_q=16, B=1, Hq=1, Hkv=1), 2),
+    (dict(window=200000, block_k=16, block_q=16), 2),
+])
+def test_invalid_params_are_rejected_before_launch(L, kw, status):
+    p = _p(**kw)
+    assert L.ssa_workspace_size(ctypes.byref(p)) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    st = L.ssa_forward(ctypes.byref(p), fake, fake, fake, fake, None, None, None, fake,
+                       1 << 40, None)
+    assert st == status, L.ssa_last_error_message()
+    assert L.ssa_last_error_message().decode()
+
+
+def test_bad_pointers_and_workspace_are_rejected_before_launch(L):
+    p = _p()
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    ws = ssa.workspace_size(p)
+    f = L.ssa_forward
+    assert f(ctypes.byref(p), None, good, good, good, None, None, None, good, ws, None) == 1
+    assert f(ctypes.byref(p), odd, good, good, good, None, None, None, good, ws, None) == 1
+    assert f(ctypes.byref(p), good, good, good, good, None, None, None, good, ws - 1, None) == 3
+    assert f(ctypes.byref(p), good, good, good, good, None, None, None, None, ws, None) == 3
+    assert f(ctypes.byref(p), good, good, good, good, None, None, None,
+             ctypes.c_void_p((1 << 20) + 16), ws, None) == 1
+    assert L.ssa_attend(ctypes.byref(p), good, good, good, None, good, good, None, None) == 1
+    assert L.ssa_route(ctypes.byref(p), good, good, good, None, None) == 1
+    assert L.ssa_block_summary(ctypes.byref(p), good, 14, 48, good, None) == 1
+    assert L.ssa_block_summary(ctypes.byref(p), odd, 14, 64, good, None) == 1
+    assert L.ssa_probe_wait_timeout(0, None) == 1
+    assert L.ssa_forward(None, good, good, good, good, None, None, None, good, ws, None) == 1
+
+
+def test_binding_rejects_wrong_tensors():
+    import torch
+    p = _p(N=1024, Hq=2, Hkv=2, top_k=4, window=128)
+    q = torch.zeros(1, 2, 1024, 64, dtype=torch.bfloat16)   # CPU tensor: refused by the binding
+    with pytest.raises(ValueError):
+        ssa.forward(q, q, q, p)

@@ -1,0 +1,221 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Per-kernel checks isolate each step: K1 summaries against fp64 means, K2
+selections against the oracle's top-k (bit-exact except at counted near-ties,
+where the GPU's choice must be one the oracle itself enumerates as
+acceptable), K3 fed the oracle's own selections against the oracle's attend.
+Then the whole forward on small shapes (every row) and on the five workloads
+at full size (sampled query blocks, plus properties that hold for every row).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from content_routed_block_b200 import build, ssa
+from content_routed_block_b200.workloads import CONFIGS, Workload, make_inputs
+from parity_utils import (Case, assert_close, check_forward, check_route_rows, gpu_rows,
+                          oracle_attend_rows, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    ssa.lib()
+    torch.cuda.init()
+    ssa.check_error()
+
+
+def W(name, **kw):
+    base = dict(B=1, Hq=2, Hkv=2, N=1024, D=64, block_k=64, block_q=64, top_k=4, window=128,
+                causal=True, kind="iid", seed=11)
+    base.update(kw)
+    return Workload(name, **base)
+
+
+SMALL = [
+    CONFIGS[1],
+    W("ragged-gqa2", B=2, Hq=4, Hkv=2, N=1216, top_k=4, window=200),
+    W("d128-gqa8", Hq=8, Hkv=1, D=128, top_k=3, window=96),
+    W("window1", N=640, top_k=2, window=1),
+    W("sliding-k0", N=640, top_k=0, window=100),
+    W("dense-causal", N=768, top_k=12, window=64),
+    W("bk16", N=512, block_k=16, block_q=16, top_k=5, window=40),
+    W("bk32-bq64", N=768, block_k=32, block_q=64, top_k=6, window=70),
+    W("bq128-bk16", N=1024, block_k=16, block_q=128, top_k=8, window=130),
+    W("bk128", N=1024, block_k=128, block_q=128, top_k=2, window=128),
+    W("bk128-bq32", N=1024, block_k=128, block_q=32, top_k=2, window=50),
+    W("noncausal-bk16", B=1, Hq=2, Hkv=2, N=1024, block_k=16, block_q=16, top_k=8, window=0,
+      causal=False, kind="image"),
+    W("noncausal-k64", N=4096, top_k=64, window=0, causal=False),
+    W("k40", N=4096, top_k=40, window=64, Hq=2, Hkv=1),
+    W("tiny", N=64, Hq=1, Hkv=1, block_k=16, block_q=16, top_k=2, window=20),
+    W("gqa7-clustered", Hq=14, Hkv=2, N=2048, top_k=8, window=256, kind="clustered", centres=16),
+    W("needles-d128", Hq=2, Hkv=2, N=5120, D=128, top_k=4, window=256, kind="needles",
+      needles=4),
+]
+
+
+# ------------------------------------------------------------------ error path
+def test_bounded_wait_reports_timeout_and_context_survives():
+    ssa.probe_wait_timeout(2000)
+    with pytest.raises(ssa.SsaError) as e:
+        ssa.check_error()
+    assert e.value.status == 5
+    ssa.check_error()                       # the word was cleared
+    check_forward(Case(CONFIGS[1]))         # and the context still works
+
+
+# ------------------------------------------------------------------ K1
+@pytest.mark.parametrize("D,block", [(64, 16), (64, 32), (64, 64), (128, 64), (128, 128)])
+def test_block_summary_matches_fp64_means(D, block):
+    w = W("pool", B=2, Hq=3, Hkv=3, N=1024, D=D)
+    x = make_inputs(w)["q"]
+    p = ssa.params_of(w)
+    g = ssa.block_summary(to_dev(x), block, p).cpu().numpy().astype(np.float64)
+    ref = O.block_summary(O.upcast_bf16(x), block)
+    np.testing.assert_allclose(g, ref, rtol=0, atol=1e-5)
+
+
+def test_block_summary_exact_on_integer_inputs():
+    rng = np.random.default_rng(5)
+    vals = rng.integers(-64, 65, size=(1, 2, 2048, 64)).astype(np.float32)
+    from content_routed_block_b200.workloads import to_bf16_bits
+    x = to_bf16_bits(vals)
+    p = ssa.make_params(1, 2, 2, 2048, 64, 64, 64, 4, 64, True)
+    g = ssa.block_summary(to_dev(x), 64, p).cpu().numpy().astype(np.float64)
+    np.testing.assert_array_equal(g, O.block_summary(vals.astype(np.float64), 64))
+
+
+# ------------------------------------------------------------------ K2
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_route_matches_oracle(w):
+    case = Case(w)
+    p = case.p
+    ks = ssa.block_summary(case.kd, w.block_k, p)
+    qs = ssa.block_summary(case.qd, w.block_q, p)
+    idx, cnt = ssa.route(qs, ks, p)
+    ssa.check_error()
+    check_route_rows(case, idx.cpu().numpy(), cnt.cpu().numpy(), case.all_rows())
+
+
+def test_route_equal_scores_take_lowest_indices():
+    w = W("flat", N=2048, Hq=2, Hkv=1, top_k=7, window=64)
+    x = make_inputs(w)
+    x["k"][:] = x["k"][:, :, :1, :]            # every key row equal -> every score equal
+    case = Case(w, x)
+    p = case.p
+    ks = ssa.block_summary(case.kd, 64, p)
+    qs = ssa.block_summary(case.qd, 64, p)
+    idx, cnt = ssa.route(qs, ks, p)
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    for qb in range(32):
+        n = min(7, qb)
+        assert cnt[0, 0, qb] == n and cnt[0, 1, qb] == n
+        assert idx[0, 0, qb, :n].tolist() == list(range(n))
+        assert idx[0, 1, qb, :n].tolist() == list(range(n))
+
+
+# ------------------------------------------------------------------ K3
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_attend_with_oracle_selection(w):
+    case = Case(w)
+    op = case.op
+    r = O.route(case.qsum64, case.ksum64, op)
+    idx = torch.from_numpy(r.idx).cuda()
+    cnt = torch.from_numpy(r.cnt).cuda()
+    o, lse = ssa.attend(case.qd, case.kd, case.vd, idx, cnt, case.p)
+    ssa.check_error()
+    rows = case.all_rows()
+    o_ref, l_ref = oracle_attend_rows(case, r.idx, r.cnt, rows)
+    assert_close(gpu_rows(o, rows, op.block_q), o_ref, gpu_rows(lse, rows, op.block_q), l_ref,
+                 what=w.name)
+
+
+# ------------------------------------------------------------------ whole path
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_forward_small_every_row(w):
+    check_forward(Case(w))
+
+
+def _route_properties_all_rows(case, idx, cnt):
+    op = case.op
+    qb = np.arange(op.n_qblocks)
+    if op.causal:
+        n_adm = np.minimum((qb * op.block_q) // op.block_k, op.n_kblocks)
+    else:
+        n_adm = np.full(op.n_qblocks, op.n_kblocks)
+    want = np.minimum(op.top_k, n_adm)
+    assert (cnt == want[None, None, :]).all()
+    if op.top_k == 0:
+        return
+    e = np.arange(op.top_k)
+    valid = e[None, None, None, :] < cnt[..., None]
+    assert (idx[~valid] == -1).all()
+    sel = np.where(valid, idx, -1)
+    assert (sel[valid] >= 0).all()
+    lim = n_adm[None, None, :, None]
+    assert (np.where(valid, sel < lim, True)).all()
+    d = np.diff(sel, axis=-1)
+    vpair = valid[..., 1:]
+    assert (np.where(vpair, d > 0, True)).all()
+
+
+@pytest.mark.parametrize("cfg,rows", [(2, 48), (3, 48), (4, 48)])
+def test_forward_full_size_sampled(cfg, rows):
+    case = Case(CONFIGS[cfg])
+    rep = check_forward(case, rows=case.sample_rows(rows, seed=cfg))
+    _route_properties_all_rows(case, rep["idx"], rep["cnt"])
+    assert torch.isfinite(rep["o"]).all()
+
+
+def test_forward_million_tokens_sampled():
+    case = Case(CONFIGS[5])
+    rep = check_forward(case, rows=case.sample_rows(16, seed=5))
+    _route_properties_all_rows(case, rep["idx"], rep["cnt"])
+    assert torch.isfinite(rep["o"]).all()
+
+
+def test_forward_is_deterministic():
+    case = Case(CONFIGS[1].with_(N=2048, Hq=4, Hkv=2, top_k=6))
+    a = ssa.forward(case.qd, case.kd, case.vd, case.p)
+    b = ssa.forward(case.qd, case.kd, case.vd, case.p)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_attend_without_lse_matches_with_lse():
+    case = Case(CONFIGS[1])
+    r = O.route(case.qsum64, case.ksum64, case.op)
+    idx, cnt = torch.from_numpy(r.idx).cuda(), torch.from_numpy(r.cnt).cuda()
+    o1, _ = ssa.attend(case.qd, case.kd, case.vd, idx, cnt, case.p, with_lse=True)
+    o2, l2 = ssa.attend(case.qd, case.kd, case.vd, idx, cnt, case.p, with_lse=False)
+    assert l2 is None and torch.equal(o1, o2)
+
+
+def test_out_of_range_block_is_reported_not_read():
+    case = Case(CONFIGS[1])
+    r = O.route(case.qsum64, case.ksum64, case.op)
+    bad = r.idx.copy()
+    bad[0, 1, 9, 0] = case.op.n_kblocks + 5
+    o, _ = ssa.attend(case.qd, case.kd, case.vd, torch.from_numpy(bad).cuda(),
+                      torch.from_numpy(r.cnt).cuda(), case.p)
+    with pytest.raises(ssa.SsaError) as e:
+        ssa.check_error()
+    assert e.value.status == 6
+    # rows of other query tiles are untouched by the bad entry
+    rows = [(0, 0, qb) for qb in range(16)]
+    o_ref, _ = oracle_attend_rows(case, r.idx, r.cnt, rows)
+    assert_close(gpu_rows(o, rows, 64), o_ref, what="other rows")
+
+
+def test_forward_host_roundtrip():
+    case = Case(CONFIGS[1])
+    qh, kh, vh = (t.cpu().pin_memory() for t in (case.qd, case.kd, case.vd))
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    ssa.forward_host(qh, kh, vh, case.p, oh)
+    torch.cuda.synchronize()
+    o, _, _, _ = ssa.forward(case.qd, case.kd, case.vd, case.p)
+    assert torch.equal(oh, o.cpu())

@@ -355,3 +355,18 @@ def test_bf16_upcast_is_exact():
     u = np.array([0x3F80, 0xBF80, 0x0000, 0x7F7F, 0x0001, 0x4049], dtype=np.uint16)
     want = torch.from_numpy(u.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
     np.testing.assert_array_equal(O.upcast_bf16(u), want)
+
+
+def test_acceptable_selections_cover_near_ties():
+    # scores 3, 2, 1.99999, 1.99998, 0 with k = 2: block 0 is sure, then any
+    # one of the three band blocks 1, 2, 3
+    mu = np.array([[3.0], [2.0], [1.99999], [1.99998], [0.0]])
+    q = np.array([1.0])
+    cand = np.arange(5)
+    acc = O.acceptable_selections(q, mu, cand, 2)
+    assert [a.tolist() for a in acc] == [[0, 1], [0, 2], [0, 3]]
+    sel, kth, nxt = O.route_row(q, mu, cand, 2)
+    assert sel.tolist() == [0, 1]
+    # no near tie: exactly the lexicographic selection
+    acc = O.acceptable_selections(q, mu[[0, 1, 4]], np.arange(3), 2)
+    assert [a.tolist() for a in acc] == [[0, 1]]
