@@ -36,6 +36,13 @@ __global__ void probe_wait_kernel(uint64_t timeout_ns) {
   }
   __syncthreads();
 }
+// Scratch of ssa_forward_static: summaries, routed lists and counts live
+// here instead of in a caller-provided workspace.  It is part of the loaded
+// module, so every device that loads this library holds these bytes until the
+// process exits.  Host code must not use the name as a pointer: on the host it
+// is only a stand-in; the device address comes from cudaGetSymbolAddress.
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(32) << 20;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 }  // namespace ssa
 
 namespace {
@@ -355,6 +362,48 @@ ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const 
   if ((s = launch_route(p, qsum, ksum, idx, cnt, st)) != SSA_OK) return s;
   if ((s = launch_attend(p, q, k, v, idx, cnt, o, lse, st)) != SSA_OK) return s;
   return ok();
+}
+
+// Device address of the static scratch on the current device, looked up
+// once per device (the first call on a device does the lookup).
+std::mutex g_static_mu;
+constexpr int kMaxDevices = 256;
+void* g_static_ptr[kMaxDevices] = {};
+
+ssa_status static_scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, ssa::g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_static_ptr[dev] = ptr;
+  }
+  *out = g_static_ptr[dev];
+  return SSA_OK;
+}
+
+ssa_status ssa_forward_static(const ssa_params* p, const void* q, const void* k, const void* v,
+                              void* o, float* lse, int32_t* idx_out, int32_t* cnt_out,
+                              ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  const size_t need = ws_layout(p).total;
+  if (need > ssa::kStaticScratchBytes)
+    return fail(SSA_ERR_WORKSPACE,
+                "this shape needs %zu bytes of scratch; the built-in scratch holds %zu bytes "
+                "(use ssa_forward with a caller workspace)",
+                need, ssa::kStaticScratchBytes);
+  void* scratch = nullptr;
+  if ((s = static_scratch_address(&scratch)) != SSA_OK) return s;
+  // Every buffer in the scratch is fully written by the kernels before it is
+  // read (summaries by the pool kernel, lists and counts by the router), so
+  // nothing has to be cleared between calls.
+  return ssa_forward(p, q, k, v, o, lse, idx_out, cnt_out, scratch, ssa::kStaticScratchBytes,
+                     stream);
 }
 
 ssa_status ssa_check_error(ssa_stream_t stream) {

@@ -18,8 +18,9 @@
  *              16-byte aligned (the kernels move them with TMA / 16-byte
  *              vectors); float and int32 buffers 16-byte aligned.
  *   Ownership  The caller owns every buffer.  The library allocates no device
- *              memory: its only device state is a file-scope error word per
- *              device that ssa_check_error reads and clears.
+ *              memory: its device state is a file-scope error word per device
+ *              that ssa_check_error reads and clears, and the fixed scratch
+ *              of ssa_forward_static.
  *   Streams    Every call is asynchronous on the caller's stream (a
  *              cudaStream_t passed as ssa_stream_t; NULL = legacy default
  *              stream).  Calls on one stream run in order.
@@ -122,6 +123,31 @@ ssa_status ssa_attend(const ssa_params* p, const void* q, const void* k, const v
 ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const void* v,
                        void* o, float* lse, int32_t* idx_out, int32_t* cnt_out,
                        void* workspace, size_t workspace_bytes, ssa_stream_t stream);
+
+/* ssa_forward without a workspace argument, for callers that cannot allocate
+ * device memory at call time -- for example code running inside a host
+ * framework's launch callback or plugin, where cudaMalloc is forbidden (it can
+ * synchronise the device, is not allowed while a stream is being captured, and
+ * bypasses the framework's own memory pool), or code with no allocator at all.
+ * No counterpart on the pages: this is an interface convenience, not part of
+ * the method.
+ *
+ * The scratch (K and Q summaries, routed lists, counts) is a fixed 32 MiB
+ * array inside the library's device module; every device that loads the
+ * library keeps it until the process exits.  Shapes whose ssa_workspace_size
+ * exceeds 32 MiB (33554432 bytes) are rejected with SSA_ERR_WORKSPACE and
+ * nothing is launched.  The call allocates nothing: no cudaMalloc, cudaFree or
+ * allocating library routine.  The first call on each device looks up the
+ * scratch's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  All calls share the one
+ * scratch, which keeps the previous call's contents (every byte the path reads
+ * is rewritten first, so nothing needs clearing); calls that can overlap on the
+ * GPU -- on different streams, or from different host threads -- race on it
+ * and must be serialised by the caller.  Arguments and results are as for
+ * ssa_forward. */
+ssa_status ssa_forward_static(const ssa_params* p, const void* q, const void* k, const void* v,
+                              void* o, float* lse, int32_t* idx_out, int32_t* cnt_out,
+                              ssa_stream_t stream);
 
 /* Synchronise the stream, then read and clear this device's error word.
  * Returns SSA_OK, SSA_ERR_TIMEOUT, SSA_ERR_DEVICE_CHECK or SSA_ERR_CUDA. */
