@@ -359,7 +359,10 @@ __global__ void __launch_bounds__(kAtThreads, 2)
     const bool row_ok = i < qend;
     const int qbr = row_ok ? r / a.Bq : 0;
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float m_ref = -INFINITY, l_sum = 0.f;
+    const float sl2 = a.scale_log2;
+    // running max of the raw scores (the scale is positive, so the max of the
+    // scaled logits is sl2 times it) and running sum of 2^(x - max)
+    float m_raw = -INFINITY, l_sum = 0.f;
     bool ok = true;
 
     for (int t = 0; t < T; ++t) {
@@ -370,15 +373,12 @@ __global__ void __launch_bounds__(kAtThreads, 2)
         break;
       }
       tc_fence_after();
-      uint32_t s0[32], s1[32];
-      tmem_ld32(trow + L::TM_S0 + (t & 1) * 64, s0);
-      tmem_ld32(trow + L::TM_S0 + (t & 1) * 64 + 32, s1);
-      tmem_ld_wait(s0);
-      tmem_ld_wait(s1);
+      const uint32_t pcol = trow + L::TM_S0 + (t & 1) * 64;
 
-      // allowed keys of this row within the chunk
-      uint64_t mask = 0ull;
+      // allowed keys of this row within the chunk, as two 32-bit words
+      uint32_t mlo = 0u, mhi = 0u;
       if (row_ok) {
+        uint64_t mask = 0ull;
         if (a.Bk >= kAtKT) {
           const int e = t / SUBS, sub = t % SUBS;
           const uint32_t ent = at_entry(faru, win, nf, wlo, e);
@@ -409,20 +409,56 @@ __global__ void __launch_bounds__(kAtThreads, 2)
             mask |= bit_range(lo, hi) << (s * a.Bk);
           }
         }
+        mlo = static_cast<uint32_t>(mask);
+        mhi = static_cast<uint32_t>(mask >> 32);
       }
 
+      // no row of this warp sees any key of the chunk (it was routed by the
+      // tile's other query blocks only): P = 0 for these rows, nothing else
+      if (__all_sync(0xffffffffu, (mlo | mhi) == 0u)) {
+        uint32_t z[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) z[c] = 0u;
+        tmem_st32(pcol, z);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_p_full[t & 1]);
+        continue;
+      }
+
+      uint32_t s0[32], s1[32];
+      tmem_ld32(pcol, s0);
+      tmem_ld32(pcol + 32, s1);
+      tmem_ld_wait(s0);
+      tmem_ld_wait(s1);
       float x[64];
-      float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        x[c] = ((mask >> c) & 1ull) ? __uint_as_float(s0[c]) * a.scale_log2 : -INFINITY;
-        x[c + 32] =
-            ((mask >> (c + 32)) & 1ull) ? __uint_as_float(s1[c]) * a.scale_log2 : -INFINITY;
+        x[c] = __uint_as_float(s0[c]);
+        x[c + 32] = __uint_as_float(s1[c]);
       }
+      if (!__all_sync(0xffffffffu, (mlo & mhi) == 0xFFFFFFFFu)) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) mx = fmaxf(mx, x[c]);
-      const float m_new = fmaxf(m_ref, mx);
-      const bool need = (m_ref != -INFINITY) && (m_new > m_ref + kAtTau);
+        for (int c = 0; c < 32; ++c) {
+          x[c] = (mlo & (1u << c)) ? x[c] : -INFINITY;
+          x[c + 32] = (mhi & (1u << c)) ? x[c + 32] : -INFINITY;
+        }
+      }
+      // row max: three-input max tree
+      float mx;
+      {
+        float t1[22];
+#pragma unroll
+        for (int c = 0; c < 21; ++c) t1[c] = fmax3(x[3 * c], x[3 * c + 1], x[3 * c + 2]);
+        t1[21] = x[63];
+        float t2[8];
+#pragma unroll
+        for (int c = 0; c < 7; ++c) t2[c] = fmax3(t1[3 * c], t1[3 * c + 1], t1[3 * c + 2]);
+        t2[7] = t1[21];
+        mx = fmax3(fmax3(t2[0], t2[1], t2[2]), fmax3(t2[3], t2[4], t2[5]), fmaxf(t2[6], t2[7]));
+      }
+      const float m_new = fmaxf(m_raw, mx);
+      const bool need = (m_raw != -INFINITY) && ((m_new - m_raw) * sl2 > kAtTau);
       if (__any_sync(0xffffffffu, need)) {
         // rescale the O row in TMEM; PV(t-1) must have landed first
         if (t >= 1) {
@@ -434,7 +470,8 @@ __global__ void __launch_bounds__(kAtThreads, 2)
           }
           tc_fence_after();
         }
-        const float alpha = (m_ref == -INFINITY || m_new == m_ref) ? 1.f : ex2_approx(m_ref - m_new);
+        const float alpha =
+            (m_raw == -INFINITY || m_new == m_raw) ? 1.f : ex2_approx((m_raw - m_new) * sl2);
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t ov[32];
@@ -446,22 +483,28 @@ __global__ void __launch_bounds__(kAtThreads, 2)
         }
         tmem_st_wait();
         l_sum *= alpha;
-        m_ref = m_new;
-      } else if (m_ref == -INFINITY) {
-        m_ref = m_new;  // first keys of this row: O and the sum are still zero
+        m_raw = m_new;
+      } else if (m_raw == -INFINITY) {
+        m_raw = m_new;  // first keys of this row: O and the sum are still zero
       }
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // p = 2^(x*sl2 - m*sl2): one packed FMA per pair, one ex2 per score
+      const float moff = (m_raw == -INFINITY) ? 0.f : -m_raw * sl2;
       uint32_t p[32];
-      float part = 0.f;
+      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2_approx(x[2 * c] - m_use);
-        const float p1 = ex2_approx(x[2 * c + 1] - m_use);
-        part += p0 + p1;
+      for (int c = 0; c < 32; c += 2) {
+        float y0, y1, y2, y3;
+        ffma2_bc(y0, y1, x[2 * c], x[2 * c + 1], sl2, moff);
+        ffma2_bc(y2, y3, x[2 * c + 2], x[2 * c + 3], sl2, moff);
+        const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+        const float p2 = ex2_approx(y2), p3 = ex2_approx(y3);
+        fadd2(acc0, acc1, acc0, acc1, p0, p1);
+        fadd2(acc2, acc3, acc2, acc3, p2, p3);
         p[c] = pack_bf16x2(p0, p1);
+        p[c + 1] = pack_bf16x2(p2, p3);
       }
-      l_sum += part;
-      tmem_st32(trow + L::TM_S0 + (t & 1) * 64, p);
+      l_sum += (acc0 + acc1) + (acc2 + acc3);
+      tmem_st32(pcol, p);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bar_p_full[t & 1]);
@@ -499,7 +542,7 @@ __global__ void __launch_bounds__(kAtThreads, 2)
         }
       }
       if (row_ok && a.lse != nullptr) {
-        const float lse2 = (l_sum > 0.f) ? m_ref + __log2f(l_sum) : -INFINITY;
+        const float lse2 = (l_sum > 0.f) ? m_raw * sl2 + __log2f(l_sum) : -INFINITY;
         a.lse[static_cast<int64_t>(bh) * a.N + i] = lse2 * 0.69314718055994530942f;
       }
     }

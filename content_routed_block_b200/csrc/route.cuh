@@ -30,7 +30,6 @@
 
 namespace ssa {
 
-constexpr int kRouteRows = 64;     // query blocks per CTA
 constexpr int kRouteCands = 64;    // key blocks per summary tile
 constexpr int kRouteThreads = 256;
 
@@ -170,14 +169,17 @@ __device__ __forceinline__ void warp_sort_asc_i32(int (&a)[R], int lane) {
   }
 }
 
-template <int D, int R>
+// RT query blocks per CTA (64, or 16 when 64 would leave SMs idle)
+template <int D, int R, int RT>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a) {
+  constexpr int kRouteRows = RT;
   extern __shared__ __align__(16) float rsm[];
-  float* qsT = rsm;                         // [D][64]   query summaries, transposed
+  float* qsT = rsm;                         // [D][RT]   query summaries, transposed
   float* ksT = qsT + D * kRouteRows;        // [D][64]   key summaries, transposed
-  float* sc = ksT + D * kRouteCands;        // [64][65]  score tile
+  float* sc = ksT + D * kRouteCands;        // [RT][65]  score tile
   constexpr int SC_LD = kRouteCands + 1;
   constexpr int ROWS_PER_WARP = kRouteRows / (kRouteThreads / 32);
+  constexpr int RPT = kRouteRows / 16;      // score rows per thread
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.y;
@@ -238,26 +240,32 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     }
     __syncthreads();
 
-    float acc[4][4];
+    float acc[RPT][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < RPT; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 #pragma unroll 8
     for (int d = 0; d < D; ++d) {
-      const float4 qa = *reinterpret_cast<const float4*>(qsT + d * kRouteRows + ty * 4);
       const float4 kb = *reinterpret_cast<const float4*>(ksT + d * kRouteCands + tx * 4);
-      const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
       const float kv[4] = {kb.x, kb.y, kb.z, kb.w};
+      float qv[RPT];
+      if constexpr (RPT == 4) {
+        const float4 qa = *reinterpret_cast<const float4*>(qsT + d * kRouteRows + ty * 4);
+        qv[0] = qa.x; qv[1] = qa.y; qv[2] = qa.z; qv[3] = qa.w;
+      } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < RPT; ++i) qv[i] = qsT[d * kRouteRows + ty * RPT + i];
+      }
+#pragma unroll
+      for (int i = 0; i < RPT; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qv[i], kv[j], acc[i][j]);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < RPT; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) sc[(ty * 4 + i) * SC_LD + tx * 4 + j] = acc[i][j];
+      for (int j = 0; j < 4; ++j) sc[(ty * RPT + i) * SC_LD + tx * 4 + j] = acc[i][j];
     __syncthreads();
 
 #pragma unroll

@@ -158,19 +158,20 @@ ssa_status make_map(CUtensorMap* m, const void* base, int64_t heads, int64_t n, 
 ssa_status launch_pool(const ssa_params* p, const void* x0, int32_t H0, int32_t blk0, float* out0,
                        const void* x1, int32_t H1, int32_t blk1, float* out1,
                        cudaStream_t stream) {
-  const int G = p->D / 8;
+  // one warp per block; the kernel's split point is counted in warps
   ssa::PoolJob j0{static_cast<const uint4*>(x0), out0,
                   static_cast<int64_t>(p->B) * H0 * (p->N / blk0), blk0, 1.0f / blk0};
   ssa::PoolJob j1 = j0;
+  j1.n_blocks = 0;  // single job: the tail warps of the grid do nothing
   int64_t n1 = 0;
   if (x1 != nullptr) {
     j1 = ssa::PoolJob{static_cast<const uint4*>(x1), out1,
                       static_cast<int64_t>(p->B) * H1 * (p->N / blk1), blk1, 1.0f / blk1};
-    n1 = j1.n_blocks * G;
+    n1 = j1.n_blocks;
   }
-  const int64_t split = j0.n_blocks * G;
-  const int64_t total = split + n1;
-  const int64_t grid = (total + 255) / 256;
+  const int64_t split = j0.n_blocks;
+  const int64_t total_threads = (split + n1) * 32;
+  const int64_t grid = (total_threads + 255) / 256;
   if (p->D == 64)
     ssa::block_mean_kernel<64><<<static_cast<unsigned>(grid), 256, 0, stream>>>(j0, j1, split);
   else
@@ -180,16 +181,26 @@ ssa_status launch_pool(const ssa_params* p, const void* x0, int32_t H0, int32_t 
   return SSA_OK;
 }
 
-template <int D, int R>
-cudaError_t launch_route_t(const ssa::RouteArgs& a, int B, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(2 * D * 64 + 64 * 65) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(ssa::route_kernel<D, R>,
+template <int D, int R, int RT>
+cudaError_t launch_route_t(ssa::RouteArgs a, int B, cudaStream_t stream) {
+  a.n_row_tiles = (a.NQB + RT - 1) / RT;
+  const size_t smem = static_cast<size_t>(D * RT + D * 64 + RT * 65) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(ssa::route_kernel<D, R, RT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_row_tiles, B * a.Hq);
-  ssa::route_kernel<D, R><<<grid, ssa::kRouteThreads, smem, stream>>>(a);
+  ssa::route_kernel<D, R, RT><<<grid, ssa::kRouteThreads, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+template <int D, int R>
+cudaError_t launch_route_rt(const ssa::RouteArgs& a, int B, cudaStream_t stream) {
+  // 64 query blocks per CTA reuse each summary tile the most; use 16 when 64
+  // would give fewer than two CTAs per SM
+  const int64_t ctas64 = static_cast<int64_t>(B) * a.Hq * ((a.NQB + 63) / 64);
+  if (ctas64 < 2 * 148) return launch_route_t<D, R, 16>(a, B, stream);
+  return launch_route_t<D, R, 64>(a, B, stream);
 }
 
 ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksum, int32_t* idx,
@@ -207,13 +218,13 @@ ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksu
   a.Bk = p->block_k;
   a.top_k = p->top_k;
   a.causal = p->causal;
-  a.n_row_tiles = (a.NQB + ssa::kRouteRows - 1) / ssa::kRouteRows;
+  a.n_row_tiles = 0;
   cudaError_t e;
   if (p->D == 64)
-    e = p->top_k <= 32 ? launch_route_t<64, 1>(a, p->B, stream) : launch_route_t<64, 2>(a, p->B, stream);
+    e = p->top_k <= 32 ? launch_route_rt<64, 1>(a, p->B, stream) : launch_route_rt<64, 2>(a, p->B, stream);
   else
-    e = p->top_k <= 32 ? launch_route_t<128, 1>(a, p->B, stream)
-                       : launch_route_t<128, 2>(a, p->B, stream);
+    e = p->top_k <= 32 ? launch_route_rt<128, 1>(a, p->B, stream)
+                       : launch_route_rt<128, 2>(a, p->B, stream);
   if (e != cudaSuccess) return cuda_fail(e, "route_kernel launch");
   return SSA_OK;
 }
