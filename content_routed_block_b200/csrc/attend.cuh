@@ -50,7 +50,8 @@ constexpr float kAtTau = 8.0f;   // lazy-rescale threshold, log2 units
 
 template <int D>
 struct AtLayout {
-  static constexpr int STAGES = (D == 64) ? 3 : 2;
+  static constexpr int STAGES = (D == 64) ? 5 : 2;   // K/V ring depth
+  static constexpr int NS = (D == 64) ? 3 : 2;       // S/P buffers in TMEM
   static constexpr uint32_t HALF_Q = kAtQT * 128;      // one 64-column half of Q
   static constexpr uint32_t Q_BYTES = kAtQT * D * 2;
   static constexpr uint32_t HALF_KV = kAtKT * 128;     // one 64-column half of a chunk
@@ -61,7 +62,7 @@ struct AtLayout {
   static constexpr uint32_t OFF_WIN = OFF_V + STAGES * KV_BYTES;   // uint32 [kAtLCap]
   static constexpr uint32_t OFF_FAR = OFF_WIN + kAtLCap * 4;       // int32 [kAtFarCap]
   static constexpr uint32_t OFF_FARU = OFF_FAR + kAtFarCap * 4;    // int32 [kAtFarCap]
-  static constexpr int NBAR = 1 + 2 * STAGES + 2 + 2 + 2 + 1;
+  static constexpr int NBAR = 1 + 2 * STAGES + 3 * NS + 1;
   static constexpr uint32_t OFF_BAR = OFF_FARU + kAtFarCap * 4;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t USED = OFF_MISC + 64;
@@ -69,9 +70,10 @@ struct AtLayout {
   // two 256-column TMEM allocations always fit in the SM's 512 columns
   static constexpr uint32_t MIN_REQ = 80 * 1024;
   static constexpr uint32_t SMEM_BYTES = (USED + 1024 > MIN_REQ) ? USED + 1024 : MIN_REQ;
-  // TMEM columns: S buffers at 0 and 64 (P overwrites the first 32 columns of
-  // its S buffer as packed bf16 pairs); O at 128 .. 128 + D
-  static constexpr uint32_t TM_S0 = 0, TM_O = 128;
+  // TMEM columns: NS S buffers of 64 columns at 0, 64, ... (P overwrites the
+  // first 32 columns of its S buffer as packed bf16 pairs); O after them
+  static constexpr uint32_t TM_S0 = 0, TM_O = NS * 64;
+  static_assert(TM_O + D <= kAtTmemCols, "TMEM budget");
 };
 
 struct AttendArgs {
@@ -119,10 +121,11 @@ __global__ void __launch_bounds__(kAtThreads, 2)
   uint64_t* bar_q = bars;
   uint64_t* bar_kv_full = bars + 1;
   uint64_t* bar_kv_empty = bars + 1 + S;
+  constexpr int NS = L::NS;
   uint64_t* bar_s_full = bars + 1 + 2 * S;
-  uint64_t* bar_p_full = bar_s_full + 2;
-  uint64_t* bar_pv_done = bar_p_full + 2;
-  uint64_t* bar_drain = bar_pv_done + 2;
+  uint64_t* bar_p_full = bar_s_full + NS;
+  uint64_t* bar_pv_done = bar_p_full + NS;
+  uint64_t* bar_drain = bar_pv_done + NS;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   // misc[0] TMEM base, misc[1] raw far count, misc[2] unique far count,
   // misc[3] abort flag
@@ -150,9 +153,9 @@ __global__ void __launch_bounds__(kAtThreads, 2)
       mbar_init(&bar_kv_full[s], 1);
       mbar_init(&bar_kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&bar_s_full[s], 1);
-      mbar_init(&bar_p_full[s], 128);
+      mbar_init(&bar_p_full[s], 4);  // one arrival per softmax warp
       mbar_init(&bar_pv_done[s], 1);
     }
     mbar_init(bar_drain, 1);
@@ -301,53 +304,62 @@ __global__ void __launch_bounds__(kAtThreads, 2)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------- MMA issuer
+    // Event-driven: S(t) is issued as soon as chunk t has landed and its S
+    // buffer is free (PV(t-NS), which read P(t-NS) from that buffer, is done),
+    // up to NS chunks ahead of the PVs; PV(u) as soon as P(u) is written.
+    // Probes are non-blocking; the whole loop gives up after timeout_ns
+    // without progress.
     if (lane == 0 && T > 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(kAtQT, kAtKT, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(kAtQT, D, false, true);
       bool ok = mbar_wait(bar_q, 0, a.timeout_ns, abort_flag, kSiteQFull);
-      auto issue_pv = [&](int u) -> bool {
-        if (!mbar_wait(&bar_p_full[u & 1], (u >> 1) & 1, a.timeout_ns, abort_flag, kSitePFull))
-          return false;
-        tc_fence_after();
-        const uint32_t vbase = sbase + L::OFF_V + (u % S) * L::KV_BYTES;
-        const uint32_t pcol = tmem + L::TM_S0 + (u & 1) * 64;
+      int ns = 0, np = 0;
+      uint64_t t_last = globaltimer_ns();
+      while (ok && np < T) {
+        bool progress = false;
+        if (ns < T && ns < np + NS) {
+          bool ready = mbar_test(&bar_kv_full[ns % S], (ns / S) & 1);
+          if (ready && ns >= NS) ready = mbar_test(&bar_pv_done[ns % NS], ((ns - NS) / NS) & 1);
+          if (ready) {
+            tc_fence_after();
+            const uint32_t kbase = sbase + L::OFF_K + (ns % S) * L::KV_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < kAtKT / 16; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, L::HALF_KV, 1024);
-          mma_ts(tmem + L::TM_O, pcol + kk * 8, bdesc, IDESC_O, (u > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t qa = sbase + L::OFF_Q + (kk / 4) * L::HALF_Q + (kk % 4) * 32;
+              const uint32_t kb = kbase + (kk / 4) * L::HALF_KV + (kk % 4) * 32;
+              mma_ss(tmem + L::TM_S0 + (ns % NS) * 64, sdesc_sw128(qa, 16, 1024),
+                     sdesc_sw128(kb, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&bar_s_full[ns % NS]);
+            ++ns;
+            progress = true;
+          }
         }
-        mma_commit(&bar_pv_done[u & 1]);
-        mma_commit(&bar_kv_empty[u % S]);
-        return true;
-      };
-      for (int t = 0; ok && t < T; ++t) {
-        const int st = t % S;
-        if (!mbar_wait(&bar_kv_full[st], (t / S) & 1, a.timeout_ns, abort_flag, kSiteKvFull)) {
-          ok = false;
-          break;
-        }
-        // S buffer t&1 is free once PV(t-2), which read P(t-2) from it, is done
-        if (t >= 2 && !mbar_wait(&bar_pv_done[t & 1], ((t - 2) >> 1) & 1, a.timeout_ns,
-                                 abort_flag, kSitePvDone)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t kbase = sbase + L::OFF_K + st * L::KV_BYTES;
+        if (np < ns && mbar_test(&bar_p_full[np % NS], (np / NS) & 1)) {
+          tc_fence_after();
+          const uint32_t vbase = sbase + L::OFF_V + (np % S) * L::KV_BYTES;
+          const uint32_t pcol = tmem + L::TM_S0 + (np % NS) * 64;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qa = sbase + L::OFF_Q + (kk / 4) * L::HALF_Q + (kk % 4) * 32;
-          const uint32_t kb = kbase + (kk / 4) * L::HALF_KV + (kk % 4) * 32;
-          mma_ss(tmem + L::TM_S0 + (t & 1) * 64, sdesc_sw128(qa, 16, 1024),
-                 sdesc_sw128(kb, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kAtKT / 16; ++kk) {
+            const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, L::HALF_KV, 1024);
+            mma_ts(tmem + L::TM_O, pcol + kk * 8, bdesc, IDESC_O, (np > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar_pv_done[np % NS]);
+          mma_commit(&bar_kv_empty[np % S]);
+          ++np;
+          progress = true;
         }
-        mma_commit(&bar_s_full[t & 1]);
-        if (t >= 1 && !issue_pv(t - 1)) {
-          ok = false;
-          break;
+        if (progress) {
+          t_last = globaltimer_ns();
+        } else {
+          if (*abort_flag) break;
+          if (globaltimer_ns() - t_last > a.timeout_ns) {
+            *abort_flag = 1;
+            record_error(kErrTimeout, kSiteMma);
+            break;
+          }
         }
       }
-      if (ok) issue_pv(T - 1);
       // every MMA issued so far must finish before TMEM is released
       mma_commit(bar_drain);
       mbar_wait(bar_drain, 0, a.timeout_ns, nullptr, kSiteDrain);
@@ -366,14 +378,14 @@ __global__ void __launch_bounds__(kAtThreads, 2)
     bool ok = true;
 
     for (int t = 0; t < T; ++t) {
-      const bool got = mbar_wait(&bar_s_full[t & 1], (t >> 1) & 1, a.timeout_ns, abort_flag,
+      const bool got = mbar_wait(&bar_s_full[t % NS], (t / NS) & 1, a.timeout_ns, abort_flag,
                                  kSiteSFull);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t pcol = trow + L::TM_S0 + (t & 1) * 64;
+      const uint32_t pcol = trow + L::TM_S0 + (t % NS) * 64;
 
       // allowed keys of this row within the chunk, as two 32-bit words
       uint32_t mlo = 0u, mhi = 0u;
@@ -422,7 +434,8 @@ __global__ void __launch_bounds__(kAtThreads, 2)
         tmem_st32(pcol, z);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bar_p_full[t & 1]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_p_full[t % NS]);
         continue;
       }
 
@@ -462,8 +475,8 @@ __global__ void __launch_bounds__(kAtThreads, 2)
       if (__any_sync(0xffffffffu, need)) {
         // rescale the O row in TMEM; PV(t-1) must have landed first
         if (t >= 1) {
-          const bool g2 = mbar_wait(&bar_pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1, a.timeout_ns,
-                                    abort_flag, kSitePvDone);
+          const bool g2 = mbar_wait(&bar_pv_done[(t - 1) % NS], ((t - 1) / NS) & 1,
+                                    a.timeout_ns, abort_flag, kSitePvDone);
           if (!__all_sync(0xffffffffu, g2)) {
             ok = false;
             break;
@@ -507,12 +520,13 @@ __global__ void __launch_bounds__(kAtThreads, 2)
       tmem_st32(pcol, p);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bar_p_full[t & 1]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_p_full[t % NS]);
     }
 
     // ------------------------------------------------------- epilogue
     if (ok && T > 0) {
-      const bool got = mbar_wait(&bar_pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, a.timeout_ns,
+      const bool got = mbar_wait(&bar_pv_done[(T - 1) % NS], ((T - 1) / NS) & 1, a.timeout_ns,
                                  abort_flag, kSitePvDone);
       ok = __all_sync(0xffffffffu, got);
     }

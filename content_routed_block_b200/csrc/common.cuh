@@ -22,7 +22,7 @@ enum : uint32_t {
 enum : uint32_t {
   kSiteProbe = 1,
   kSiteQFull = 10, kSiteKvEmpty, kSiteKvFull, kSiteSFull, kSitePFull, kSitePvDone,
-  kSiteDrain, kSiteListCap = 30, kSiteIdx,
+  kSiteDrain, kSiteMma, kSiteListCap = 30, kSiteIdx,
 };
 
 // the library is a single translation unit, so the word is defined here
@@ -73,6 +73,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// non-blocking probe: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
