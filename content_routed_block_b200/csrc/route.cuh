@@ -40,6 +40,7 @@ struct RouteArgs {
   int32_t* cnt;        // [B*Hq, NQB]
   int32_t Hq, Hkv, NQB, NB, Bq, Bk, top_k, causal;
   int32_t n_row_tiles;
+  uint64_t timeout_ns;
 };
 
 // orderable 64-bit key: larger key <=> (higher score, then lower index)

@@ -11,6 +11,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 #include <string>
 
@@ -19,6 +20,7 @@
 #include "common.cuh"
 #include "pool.cuh"
 #include "route.cuh"
+#include "route_tc.cuh"
 
 namespace ssa {
 __global__ void probe_wait_kernel(uint64_t timeout_ns) {
@@ -194,6 +196,26 @@ cudaError_t launch_route_t(ssa::RouteArgs a, int B, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <int D, int KM>
+cudaError_t launch_route_tc_t(ssa::RouteArgs a, int B, cudaStream_t stream) {
+  a.n_row_tiles = (a.NQB + ssa::kRtcRows - 1) / ssa::kRtcRows;
+  const uint32_t smem = ssa::RtcLayout<D>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(ssa::route_tc_kernel<D, KM>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.n_row_tiles, B * a.Hq);
+  ssa::route_tc_kernel<D, KM><<<grid, ssa::kRtcThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_route_tc(const ssa::RouteArgs& a, int B, cudaStream_t stream) {
+  if (a.top_k <= 16) return launch_route_tc_t<D, 16>(a, B, stream);
+  if (a.top_k <= 32) return launch_route_tc_t<D, 32>(a, B, stream);
+  return launch_route_tc_t<D, 64>(a, B, stream);
+}
+
 template <int D, int R>
 cudaError_t launch_route_rt(const ssa::RouteArgs& a, int B, cudaStream_t stream) {
   // 64 query blocks per CTA reuse each summary tile the most; use 16 when 64
@@ -201,6 +223,16 @@ cudaError_t launch_route_rt(const ssa::RouteArgs& a, int B, cudaStream_t stream)
   const int64_t ctas64 = static_cast<int64_t>(B) * a.Hq * ((a.NQB + 63) / 64);
   if (ctas64 < 2 * 148) return launch_route_t<D, R, 16>(a, B, stream);
   return launch_route_t<D, R, 64>(a, B, stream);
+}
+
+// The tensor-core router ranks exactly like the fp32 one (see route_tc.cuh);
+// it is used whenever routing is non-trivial.  SSA_ROUTER=fp32 forces the
+// fp32 FMA kernel (both are exercised by the tests).
+bool use_tc_router(const ssa_params* p) {
+  const char* env = std::getenv("SSA_ROUTER");
+  if (env != nullptr && std::string(env) == "fp32") return false;
+  if (env != nullptr && std::string(env) == "tc") return p->top_k > 0;
+  return p->top_k > 0 && p->N / p->block_k > 64;
 }
 
 ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksum, int32_t* idx,
@@ -219,8 +251,11 @@ ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksu
   a.top_k = p->top_k;
   a.causal = p->causal;
   a.n_row_tiles = 0;
+  a.timeout_ns = timeout_ns(p);
   cudaError_t e;
-  if (p->D == 64)
+  if (use_tc_router(p)) {
+    e = p->D == 64 ? launch_route_tc<64>(a, p->B, stream) : launch_route_tc<128>(a, p->B, stream);
+  } else if (p->D == 64)
     e = p->top_k <= 32 ? launch_route_rt<64, 1>(a, p->B, stream) : launch_route_rt<64, 2>(a, p->B, stream);
   else
     e = p->top_k <= 32 ? launch_route_rt<128, 1>(a, p->B, stream)

@@ -219,3 +219,59 @@ def test_forward_host_roundtrip():
     torch.cuda.synchronize()
     o, _, _, _ = ssa.forward(case.qd, case.kd, case.vd, case.p)
     assert torch.equal(oh, o.cpu())
+
+
+# ------------------------------------------------------------------ router forms
+def _route_with(form, case):
+    import os
+    old = os.environ.get("SSA_ROUTER")
+    os.environ["SSA_ROUTER"] = form
+    try:
+        p = case.p
+        ks = ssa.block_summary(case.kd, case.w.block_k, p)
+        qs = ssa.block_summary(case.qd, case.w.block_q, p)
+        idx, cnt = ssa.route(qs, ks, p)
+        ssa.check_error()
+        return idx, cnt
+    finally:
+        if old is None:
+            os.environ.pop("SSA_ROUTER", None)
+        else:
+            os.environ["SSA_ROUTER"] = old
+
+
+@pytest.mark.parametrize("w", [w for w in SMALL if w.top_k > 0] + [CONFIGS[c] for c in (2, 3, 4, 5)],
+                         ids=lambda w: w.name)
+def test_tensor_core_router_equals_fp32_router(w):
+    # the tensor-core router ranks on the same fp32 scores as the FMA router
+    # (bf16 prefilter with a proven bound + exact rescoring): bit-identical lists
+    case = Case(w)
+    i1, c1 = _route_with("fp32", case)
+    i2, c2 = _route_with("tc", case)
+    assert torch.equal(c1, c2)
+    assert torch.equal(i1, i2)
+
+
+def test_tensor_core_router_on_flat_and_tied_scores():
+    # all-equal keys (every candidate inside the bound: all rescored) and
+    # integer-valued summaries with many exact ties
+    w = W("flat-tc", N=8192, Hq=2, Hkv=1, top_k=16, window=64)
+    x = make_inputs(w)
+    x["k"][:] = x["k"][:, :, :1, :]
+    case = Case(w, x)
+    i1, c1 = _route_with("fp32", case)
+    i2, c2 = _route_with("tc", case)
+    assert torch.equal(i1, i2) and torch.equal(c1, c2)
+    idx = i2.cpu().numpy()
+    for qb in (5, 40, 127):
+        n = min(16, qb)
+        assert idx[0, 0, qb, :n].tolist() == list(range(n))
+    from content_routed_block_b200.workloads import to_bf16_bits
+    rng = np.random.default_rng(9)
+    xi = {n: to_bf16_bits(rng.integers(-2, 3, size=s).astype(np.float32))
+          for n, s in (("q", (1, 2, 8192, 64)), ("k", (1, 1, 8192, 64)), ("v", (1, 1, 8192, 64)))}
+    case = Case(w, xi)
+    i1, c1 = _route_with("fp32", case)
+    i2, c2 = _route_with("tc", case)
+    assert torch.equal(i1, i2) and torch.equal(c1, c2)
+    check_route_rows(case, i2.cpu().numpy(), c2.cpu().numpy(), case.sample_rows(40, seed=1))
