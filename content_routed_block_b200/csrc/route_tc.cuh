@@ -4,31 +4,36 @@
 // jonsmirl/ssa README, "Algorithm and complexity": block c is scored by
 // <q, mu_c> (the second-cumulant weight beta is 0 here) and the top_k
 // admissible blocks of each query block are kept; ties go to the lower block
-// index.  The ranking must be decided on fp32 scores.  Scoring every
-// (query block, key block) pair in fp32 FMA costs NQB*NB*D*2 flops, which is
-// 240 GFLOP at a million tokens, so this kernel ranks in two passes:
+// index.  The ranking is decided on fp32 scores.  Scoring every (query block,
+// key block) pair with fp32 FMAs costs NQB*NB*D*2 flops (240 GFLOP at a
+// million tokens), so this kernel ranks in two passes over tensor-core scores:
 //
-//  pass 1  bf16 tensor-core scores sa_c (M = 128 query blocks, N = 256 or 128
-//          key blocks per MMA, fp32 accumulation in TMEM).  With bf16
-//          rounding of both operands (unit roundoff u = 2^-9) every score obeys
-//          |sa_c - s_c| <= (2u + u^2 + accumulation) ||qbar|| ||mu_c||
-//          < 2^-7 ||qbar|| ||mu_c|| =: E_c.  Each row keeps the k largest
-//          lower bounds sa_c - E_c; L is the k-th of them.
-//  pass 2  the same tensor-core scores again; every candidate whose upper
-//          bound sa_c + E_c reaches L is rescored exactly in fp32 (sequential
-//          FMA over d, the same arithmetic as the fp32 kernel) and offered to
-//          the row's exact top-k list (64-bit keys: orderable score bits << 32
-//          | ~block).  At least k candidates have s_c >= L, so every member of
-//          the true top-k has an upper bound >= L and is rescored: the result
-//          equals the fp32 top-k exactly.  (The filter is widened by
-//          2^-16 ||qbar|| max_c ||mu_c||, which covers the fp32 rounding of the
-//          rescored values themselves, at most ~2^-18 of the same product.)
+//  scores  each fp32 summary x is split into bf16 parts x = x_hi + x_lo + r
+//          (x_hi = bf16(x), x_lo = bf16(x - x_hi), |r| <= u^2 |x|, u = 2^-9)
+//          and sa_c = q_hi.mu_hi + q_hi.mu_lo + q_lo.mu_hi (three MMAs into
+//          one fp32 TMEM accumulator, M = 128 query blocks, N = 128 key
+//          blocks).  The dropped terms are below 3.1 u^2 sum_d |q_d mu_d| and
+//          the fp32 accumulation of 3*D products adds at most 3D 2^-23 of the
+//          same sum: 3.5e-5 (D = 64) or 5.8e-5 (D = 128) times ||qbar|| ||mu_c||.
+//          E_c = eps ||qbar|| ||mu_c|| with eps = 2^-13 (D = 64) or 2^-12
+//          (D = 128) bounds |sa_c - s_c| with a margin of 3.5x or more.
+//  pass 1  L = the k-th largest of the per-32-column maxima of the lower
+//          bounds sa_c - E_c.  Each maximum is the lower bound of a distinct
+//          candidate, so at least k candidates have s_c >= L.
+//  pass 2  every candidate whose upper bound sa_c + E_c reaches the filter is
+//          queued per row in shared memory; a warp's queues are rescored
+//          exactly in fp32 together (sequential FMA over d, the arithmetic of
+//          the fp32 kernel) and offered to the row's exact top-k list (64-bit
+//          keys: orderable score bits << 32 | ~block).  The filter starts at L
+//          and rises to the current exact k-th score once k are known.  Every
+//          member of the true top-k passes the filter, so the result equals
+//          the fp32 top-k exactly.  (The filter is widened by
+//          eps/2 ||qbar|| max_c ||mu_c||, covering the fp32 rounding of the
+//          rescored values themselves, ~2^-18 of the same product.)
 //
-// One CTA owns 128 query blocks of one (b, head) (thread r = row r = TMEM
-// lane r for the epilogue).  All 256 threads convert each fp32 key-summary
-// tile to bf16 in the 128-byte-swizzled K-major layout the MMA reads and
-// compute its row norms; one thread issues the MMAs; threads 0-127 run the
-// per-row bound test straight out of TMEM.
+// One CTA owns 128 query blocks of one (b, head): thread r = row r = TMEM
+// lane r runs the per-row tests straight out of TMEM; all 256 threads split
+// and stage each key-summary tile; one thread issues the MMAs.
 #pragma once
 
 #include "common.cuh"
@@ -38,20 +43,27 @@ namespace ssa {
 
 constexpr int kRtcRows = 128;
 constexpr int kRtcThreads = 256;
-constexpr float kRtcEps = 0.0078125f;  // 2^-7
+constexpr int kRtcNT = 128;               // key blocks per MMA (N)
+// error-bound factor of the split tensor-core scores (see above)
+template <int D>
+__host__ __device__ constexpr float rtc_eps() { return D == 64 ? 1.2207031e-4f : 2.4414062e-4f; }
+constexpr int kRtcCap = 32;               // queued candidates per row before a flush
 
 template <int D>
 struct RtcLayout {
-  static constexpr int NT = (D == 64) ? 256 : 128;    // key blocks per MMA (N)
-  static constexpr uint32_t HALF_Q = kRtcRows * 128;  // one 64-column bf16 half of the Q tile
+  static constexpr int NT = kRtcNT;
+  static constexpr uint32_t HALF_Q = kRtcRows * 128;  // one 64-column bf16 half of a Q tile
   static constexpr uint32_t Q_BYTES = kRtcRows * D * 2;
   static constexpr uint32_t HALF_K = NT * 128;
   static constexpr uint32_t K_BYTES = NT * D * 2;
-  static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
-  static constexpr uint32_t OFF_QF = OFF_K + K_BYTES;          // fp32 [D][128] query summaries
+  static constexpr uint32_t OFF_QH = 0;
+  static constexpr uint32_t OFF_QL = OFF_QH + Q_BYTES;
+  static constexpr uint32_t OFF_KH = OFF_QL + Q_BYTES;
+  static constexpr uint32_t OFF_KL = OFF_KH + K_BYTES;
+  static constexpr uint32_t OFF_QF = OFF_KL + K_BYTES;            // fp32 [D][128] query summaries
   static constexpr uint32_t OFF_NRM = OFF_QF + D * kRtcRows * 4;  // fp32 [NT] key-summary norms
-  static constexpr uint32_t OFF_BAR = OFF_NRM + NT * 4;
+  static constexpr uint32_t OFF_LIST = OFF_NRM + NT * 4;          // uint16 [kRtcCap][128]
+  static constexpr uint32_t OFF_BAR = OFF_LIST + kRtcCap * kRtcRows * 2;
   static constexpr uint32_t USED = OFF_BAR + 32;
   static constexpr uint32_t SMEM_BYTES = USED + 1024;
   static constexpr uint32_t TMEM_COLS = NT;
@@ -62,18 +74,31 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // byte offset of 16-byte chunk g (of D/8) of row r in a 128B-swizzled,
-// K-major bf16 tile of `rows` rows (64-column halves stacked)
+// K-major bf16 tile (64-column halves stacked)
 __device__ __forceinline__ uint32_t sw128_offset(int r, int g, uint32_t half_bytes) {
   return static_cast<uint32_t>(g >> 3) * half_bytes + static_cast<uint32_t>(r) * 128u +
          static_cast<uint32_t>(((g & 7) ^ (r & 7)) << 4);
 }
 
-// convert 8 fp32 to 8 bf16 (RNE) packed in a uint4; also accumulate squares
-__device__ __forceinline__ uint4 cvt8_bf16(const float4& a, const float4& b, float& sq) {
-  sq = fmaf(a.x, a.x, sq); sq = fmaf(a.y, a.y, sq); sq = fmaf(a.z, a.z, sq); sq = fmaf(a.w, a.w, sq);
-  sq = fmaf(b.x, b.x, sq); sq = fmaf(b.y, b.y, sq); sq = fmaf(b.z, b.z, sq); sq = fmaf(b.w, b.w, sq);
-  return make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                    pack_bf16x2(b.z, b.w));
+// split 8 fp32 into bf16 hi and lo parts (both round to nearest even);
+// accumulate the squares of the fp32 values
+__device__ __forceinline__ void split8_bf16(const float4& a, const float4& b, uint4& hi, uint4& lo,
+                                            float& sq) {
+  const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 hv = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    const float r0 = v[2 * i] - __bfloat162float(hv.x);
+    const float r1 = v[2 * i + 1] - __bfloat162float(hv.y);
+    const __nv_bfloat162 lv = __floats2bfloat162_rn(r0, r1);
+    h[i] = *reinterpret_cast<const uint32_t*>(&hv);
+    l[i] = *reinterpret_cast<const uint32_t*>(&lv);
+    sq = fmaf(v[2 * i], v[2 * i], sq);
+    sq = fmaf(v[2 * i + 1], v[2 * i + 1], sq);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 // insert v into a descending array (the smallest falls off the end)
@@ -84,8 +109,13 @@ __device__ __forceinline__ void sorted_insert(T (&arr)[KM], T v) {
   arr[0] = v > arr[0] ? v : arr[0];
 }
 
+__device__ __forceinline__ float key_score(uint64_t key) {
+  const uint32_t hi = static_cast<uint32_t>(key >> 32);
+  return __uint_as_float((hi & 0x80000000u) ? (hi & 0x7FFFFFFFu) : ~hi);
+}
+
 template <int D, int KM>
-__global__ void __launch_bounds__(kRtcThreads, (KM <= 16 && D == 64) ? 2 : 1)
+__global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     route_tc_kernel(const RouteArgs a) {
   using Lay = RtcLayout<D>;
   constexpr int NT = Lay::NT;
@@ -96,6 +126,7 @@ __global__ void __launch_bounds__(kRtcThreads, (KM <= 16 && D == 64) ? 2 : 1)
   const uint32_t sbase = smem_u32(smem);
   float* qf = reinterpret_cast<float*>(smem + Lay::OFF_QF);     // [D][128]
   float* nrm = reinterpret_cast<float*>(smem + Lay::OFF_NRM);   // [NT]
+  uint16_t* qlist = reinterpret_cast<uint16_t*>(smem + Lay::OFF_LIST);
   uint64_t* bar_mma = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_BAR + 8);
 
@@ -123,7 +154,7 @@ __global__ void __launch_bounds__(kRtcThreads, (KM <= 16 && D == 64) ? 2 : 1)
     tmem_alloc(tmem_slot, Lay::TMEM_COLS);
     tmem_relinquish();
   }
-  // query summaries: bf16 swizzled (MMA A operand) and fp32 transposed
+  // query summaries: bf16 hi / lo (MMA A operands) and fp32 transposed
   {
     constexpr int TPR = kRtcThreads / kRtcRows;   // 2 threads per row
     constexpr int CPT = (D / 8) / TPR;            // 16-byte chunks per thread
@@ -139,8 +170,10 @@ __global__ void __launch_bounds__(kRtcThreads, (KM <= 16 && D == 64) ? 2 : 1)
         v0 = *reinterpret_cast<const float4*>(src + g * 8);
         v1 = *reinterpret_cast<const float4*>(src + g * 8 + 4);
       }
-      *reinterpret_cast<uint4*>(smem + Lay::OFF_Q + sw128_offset(r, g, Lay::HALF_Q)) =
-          cvt8_bf16(v0, v1, sq);
+      uint4 hi, lo;
+      split8_bf16(v0, v1, hi, lo, sq);
+      *reinterpret_cast<uint4*>(smem + Lay::OFF_QH + sw128_offset(r, g, Lay::HALF_Q)) = hi;
+      *reinterpret_cast<uint4*>(smem + Lay::OFF_QL + sw128_offset(r, g, Lay::HALF_Q)) = lo;
       const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
       for (int e = 0; e < 8; ++e) qf[(g * 8 + e) * kRtcRows + r] = vv[e];
@@ -163,18 +196,19 @@ __global__ void __launch_bounds__(kRtcThreads, (KM <= 16 && D == 64) ? 2 : 1)
     float sq = 0.f;
 #pragma unroll 8
     for (int d = 0; d < D; ++d) sq = fmaf(qf[d * kRtcRows + r], qf[d * kRtcRows + r], sq);
-    // bound with a little slack for the fp32 norms themselves
-    e_row = kRtcEps * sqrtf(sq) * 1.001f;
+    e_row = rtc_eps<D>() * sqrtf(sq) * 1.001f;  // slack for the fp32 norms themselves
   }
   const int k = a.top_k;
   const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
   uint32_t phase = 0;
 
-  // one tile: convert key summaries, MMA, then `visit(col, score)` per column
-  auto run_tile = [&](int tile, auto&& visit) {
+  // one tile: split and stage key summaries, three MMAs, then for every
+  // 32-column group `group(cb, scores, nrm32, full)`: full means every column
+  // of the group is admissible for this row
+  auto run_tile = [&](int tile, auto&& group) {
     const int c0 = tile * NT;
     {
-      constexpr int TPR = kRtcThreads / NT;          // 1 (D=64) or 2 (D=128) threads per row
+      constexpr int TPR = kRtcThreads / NT;          // 2 threads per key row
       constexpr int CPT = (D / 8) / TPR;
       const int cr = tid / TPR, part = tid % TPR;
       const bool ok = c0 + cr < a.NB;
@@ -188,27 +222,34 @@ __global__ void __launch_bounds__(kRtcThreads, (KM <= 16 && D == 64) ? 2 : 1)
           v0 = *reinterpret_cast<const float4*>(src + g * 8);
           v1 = *reinterpret_cast<const float4*>(src + g * 8 + 4);
         }
-        *reinterpret_cast<uint4*>(smem + Lay::OFF_K + sw128_offset(cr, g, Lay::HALF_K)) =
-            cvt8_bf16(v0, v1, sq);
+        uint4 hi, lo;
+        split8_bf16(v0, v1, hi, lo, sq);
+        *reinterpret_cast<uint4*>(smem + Lay::OFF_KH + sw128_offset(cr, g, Lay::HALF_K)) = hi;
+        *reinterpret_cast<uint4*>(smem + Lay::OFF_KL + sw128_offset(cr, g, Lay::HALF_K)) = lo;
       }
-      if (TPR == 2) sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+      sq += __shfl_xor_sync(0xffffffffu, sq, 1);
       if (part == 0) nrm[cr] = sqrtf(sq) * 1.001f;
     }
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == kRtcRows) {  // warp 4, lane 0
       tc_fence_after();
+      const uint32_t oq[3] = {Lay::OFF_QH, Lay::OFF_QH, Lay::OFF_QL};
+      const uint32_t okk[3] = {Lay::OFF_KH, Lay::OFF_KL, Lay::OFF_KH};
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t qa = sbase + Lay::OFF_Q + (kk / 4) * Lay::HALF_Q + (kk % 4) * 32;
-        const uint32_t kb = sbase + Lay::OFF_K + (kk / 4) * Lay::HALF_K + (kk % 4) * 32;
-        mma_ss(tmem, sdesc_sw128(qa, 16, 1024), sdesc_sw128(kb, 16, 1024), IDESC,
-               kk > 0 ? 1u : 0u);
+      for (int term = 0; term < 3; ++term) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qa = sbase + oq[term] + (kk / 4) * Lay::HALF_Q + (kk % 4) * 32;
+          const uint32_t kb = sbase + okk[term] + (kk / 4) * Lay::HALF_K + (kk % 4) * 32;
+          mma_ss(tmem, sdesc_sw128(qa, 16, 1024), sdesc_sw128(kb, 16, 1024), IDESC,
+                 (term > 0 || kk > 0) ? 1u : 0u);
+        }
       }
       mma_commit(bar_mma);
     }
     if (is_row) {
-      // the MMA completes in bounded time; the wait is bounded anyway
+      // the MMAs complete in bounded time; the wait is bounded anyway
       mbar_wait(bar_mma, phase, a.timeout_ns, nullptr, kSiteMma);
       tc_fence_after();
 #pragma unroll 1
@@ -217,11 +258,7 @@ __global__ void __launch_bounds__(kRtcThreads, (KM <= 16 && D == 64) ? 2 : 1)
         tmem_ld32(trow + cc * 32, sv);
         tmem_ld_wait(sv);
         const int cb = c0 + cc * 32;
-        if (cb < lim) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (cb + j < lim) visit(cb + j, __uint_as_float(sv[j]), nrm[cc * 32 + j]);
-        }
+        group(cb, sv, nrm + cc * 32, cb + 32 <= lim);
       }
     }
     phase ^= 1u;
@@ -229,8 +266,8 @@ __global__ void __launch_bounds__(kRtcThreads, (KM <= 16 && D == 64) ? 2 : 1)
     __syncthreads();
   };
 
-  // pass 1: the k-th largest lower bound.  The array holds KM slots; the
-  // first KM - k are +inf sentinels, so slot KM-1 is the k-th real entry.
+  // pass 1: L = k-th largest per-group maximum of the lower bounds (the
+  // first KM - k slots of lb are +inf sentinels, so slot KM-1 is the k-th)
   float L = -INFINITY;
   float nmax = 0.f;
   {
@@ -238,38 +275,99 @@ __global__ void __launch_bounds__(kRtcThreads, (KM <= 16 && D == 64) ? 2 : 1)
 #pragma unroll
     for (int j = 0; j < KM; ++j) lb[j] = (j < KM - k) ? INFINITY : -INFINITY;
     for (int tile = 0; tile < n_tiles; ++tile) {
-      run_tile(tile, [&](int, float sa, float nc) {
-        nmax = fmaxf(nmax, nc);
-        const float v = fmaf(-e_row, nc, sa);
-        if (v > lb[KM - 1]) sorted_insert<KM>(lb, v);
+      run_tile(tile, [&](int cb, const uint32_t (&sv)[32], const float* nc, bool full) {
+        if (cb >= lim) return;
+        float gmax = -INFINITY, gn = 0.f;
+        if (full) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            gmax = fmaxf(gmax, fmaf(-e_row, nc[j], __uint_as_float(sv[j])));
+            gn = fmaxf(gn, nc[j]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (cb + j < lim) {
+              gmax = fmaxf(gmax, fmaf(-e_row, nc[j], __uint_as_float(sv[j])));
+              gn = fmaxf(gn, nc[j]);
+            }
+          }
+        }
+        nmax = fmaxf(nmax, gn);
+        if (gmax > lb[KM - 1]) sorted_insert<KM>(lb, gmax);
       });
     }
-    // widen by 2^-16 ||qbar|| max ||mu|| (e_row carries 2^-7 ||qbar||)
-    L = lb[KM - 1] - e_row * nmax * 0.0078125f;
+    L = lb[KM - 1];
   }
 
-  // pass 2: exact fp32 rescoring of every candidate whose upper bound reaches L
+  // pass 2: queue every candidate whose upper bound reaches the filter and
+  // rescore the queues exactly in fp32, a warp's rows together
   uint64_t keys[KM];
 #pragma unroll
   for (int j = 0; j < KM; ++j) keys[j] = (j < KM - k) ? ~0ull : 0ull;
-  for (int tile = 0; tile < n_tiles; ++tile) {
-    run_tile(tile, [&](int c, float sa, float nc) {
-      if (fmaf(e_row, nc, sa) >= L) {
-        const float4* mu = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(c) * D);
-        float acc = 0.f;
+  const float slack = e_row * nmax * 0.5f;  // >= 2^-14 ||qbar|| max ||mu||
+  float filt = L - slack;
+  int nq = 0;
+  auto rescore = [&](int c) -> float {
+    const float4* mu = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(c) * D);
+    float acc = 0.f;
 #pragma unroll 4
-        for (int d4 = 0; d4 < D / 4; ++d4) {
-          const float4 m = mu[d4];
-          acc = fmaf(qf[(d4 * 4 + 0) * kRtcRows + r], m.x, acc);
-          acc = fmaf(qf[(d4 * 4 + 1) * kRtcRows + r], m.y, acc);
-          acc = fmaf(qf[(d4 * 4 + 2) * kRtcRows + r], m.z, acc);
-          acc = fmaf(qf[(d4 * 4 + 3) * kRtcRows + r], m.w, acc);
-        }
-        const uint64_t key = route_key(acc, c);
+    for (int d4 = 0; d4 < D / 4; ++d4) {
+      const float4 m = mu[d4];
+      acc = fmaf(qf[(d4 * 4 + 0) * kRtcRows + r], m.x, acc);
+      acc = fmaf(qf[(d4 * 4 + 1) * kRtcRows + r], m.y, acc);
+      acc = fmaf(qf[(d4 * 4 + 2) * kRtcRows + r], m.z, acc);
+      acc = fmaf(qf[(d4 * 4 + 3) * kRtcRows + r], m.w, acc);
+    }
+    return acc;
+  };
+  auto flush = [&]() {
+    int rounds = nq;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+      rounds = max(rounds, __shfl_xor_sync(0xffffffffu, rounds, off));
+    for (int t = 0; t < rounds; t += 2) {
+      const bool h0 = t < nq, h1 = t + 1 < nq;
+      const int c0 = h0 ? qlist[t * kRtcRows + r] : 0;
+      const int c1 = h1 ? qlist[(t + 1) * kRtcRows + r] : c0;
+      float s0 = 0.f, s1 = 0.f;
+      if (h0) s0 = rescore(c0);
+      if (h1) s1 = rescore(c1);
+      if (h0) {
+        const uint64_t key = route_key(s0, c0);
         if (key > keys[KM - 1]) sorted_insert<KM>(keys, key);
+      }
+      if (h1) {
+        const uint64_t key = route_key(s1, c1);
+        if (key > keys[KM - 1]) sorted_insert<KM>(keys, key);
+      }
+    }
+    nq = 0;
+    // once k exact candidates are known, the k-th exact score bounds the rest
+    if (keys[KM - 1] != 0ull && keys[KM - 1] != ~0ull)
+      filt = fmaxf(filt, key_score(keys[KM - 1]) - slack);
+  };
+  for (int tile = 0; tile < n_tiles; ++tile) {
+    run_tile(tile, [&](int cb, const uint32_t (&sv)[32], const float* nc, bool full) {
+      uint32_t m = 0u;
+      if (cb < lim) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const bool adm = full || (cb + j < lim);
+          if (adm && fmaf(e_row, nc[j], __uint_as_float(sv[j])) >= filt) m |= 1u << j;
+        }
+      }
+      // flush (warp-uniform) only when a queue would overflow
+      if (__any_sync(0xffffffffu, nq + __popc(m) > kRtcCap)) flush();
+      while (m) {
+        const int j = __ffs(m) - 1;
+        m &= m - 1;
+        qlist[nq * kRtcRows + r] = static_cast<uint16_t>(cb + j);
+        ++nq;
       }
     });
   }
+  if (is_row) flush();
 
   // output: the real entries, ascending by block index
   if (is_row && qb < a.NQB) {
@@ -281,7 +379,6 @@ __global__ void __launch_bounds__(kRtcThreads, (KM <= 16 && D == 64) ? 2 : 1)
       sel[j] = real ? static_cast<int>(~static_cast<uint32_t>(keys[j] & 0xFFFFFFFFull)) : 0x7FFFFFFF;
       n += real ? 1 : 0;
     }
-    // insertion sort, ascending (KM <= 64, per thread)
 #pragma unroll
     for (int x = 1; x < KM; ++x) {
 #pragma unroll

@@ -225,14 +225,18 @@ cudaError_t launch_route_rt(const ssa::RouteArgs& a, int B, cudaStream_t stream)
   return launch_route_t<D, R, 64>(a, B, stream);
 }
 
-// The tensor-core router ranks exactly like the fp32 one (see route_tc.cuh);
-// it is used whenever routing is non-trivial.  SSA_ROUTER=fp32 forces the
-// fp32 FMA kernel (both are exercised by the tests).
+// The tensor-core router ranks exactly like the fp32 one (see route_tc.cuh).
+// Measured on B200 it wins once the score matrix is large (1M tokens: 6.6 vs
+// 10.6 ms) and loses on small ones (its per-tile steps are latency-bound), so
+// it takes problems with at least 2^26 (query block, key block) pairs.
+// SSA_ROUTER=fp32 / tc forces one form (the tests run both and compare).
 bool use_tc_router(const ssa_params* p) {
   const char* env = std::getenv("SSA_ROUTER");
+  const int64_t nb = p->N / p->block_k, nqb = p->N / p->block_q;
+  if (p->top_k == 0 || nb > 65535) return false;  // queued candidates are 16-bit offsets
   if (env != nullptr && std::string(env) == "fp32") return false;
-  if (env != nullptr && std::string(env) == "tc") return p->top_k > 0;
-  return p->top_k > 0 && p->N / p->block_k > 64;
+  if (env != nullptr && std::string(env) == "tc") return true;
+  return nb * nqb >= (static_cast<int64_t>(1) << 26);
 }
 
 ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksum, int32_t* idx,
