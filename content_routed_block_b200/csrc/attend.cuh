@@ -13,11 +13,12 @@
 //
 // B200 design (one CTA = 128 query rows of one (b, head), i.e. 128/Bq query
 // blocks; 192 threads):
-//  * The CTA first builds the sorted union of its query blocks' routed
-//    blocks and the window's blocks in shared memory, each entry carrying a
-//    bitmask of which query blocks routed it.  The union is walked in chunks
-//    of 64 keys (one or more whole blocks, or a 64-row slice of a larger
-//    block), so every key block is fetched once per CTA.
+//  * The CTA first builds the union of its query blocks' routed blocks and
+//    the window's blocks in shared memory (deduplicated), each entry carrying
+//    a bitmask of which query blocks routed it, with routed entries
+//    interleaved across the softmax warps that need them.  The union is
+//    walked in chunks of 64 keys (one or more whole blocks, or a 64-row slice
+//    of a larger block), so every key block is fetched once per CTA.
 //  * Warp 4 (one lane) gathers each chunk's K and V rows with tiled TMA loads
 //    (one box per block, no multicast) into a 128-byte-swizzled ring of
 //    STAGES stages; Q (128 x D) is loaded once.
@@ -252,6 +253,61 @@ __global__ void __launch_bounds__(kAtThreads, 2)
       const uint32_t hm = __ballot_sync(0xffffffffu, head);
       if (head) faru[base + __popc(hm & ((1u << lane) - 1u))] = ent;
       base += __popc(hm);
+    }
+    __syncwarp();
+    // Interleave: softmax warp w serves rows 32w..32w+31, and a chunk that
+    // none of its rows' query blocks routed costs it almost nothing, but the
+    // warps share the S/P buffers, so they can drift only a few chunks
+    // apart.  Order the routed entries round-robin over their "which warps
+    // need it" classes so that chunks exclusive to different warps alternate.
+    {
+      const int nf = base;
+      uint32_t qm[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int lo = (32 * w) / a.Bq, hi = min(R - 1, (32 * w + 31) / a.Bq);
+        qm[w] = (lo < R) ? ((2u << hi) - (1u << lo)) : 0u;
+      }
+      auto wmask = [&](int e) -> int {
+        const uint32_t bits = static_cast<uint32_t>(faru[e]) & 0xFFu;
+        int m = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) m |= ((bits & qm[w]) != 0u) << w;
+        return m;
+      };
+      int bc[16];
+#pragma unroll
+      for (int bkt = 0; bkt < 16; ++bkt) bc[bkt] = 0;
+      // class sizes
+      for (int i0 = 0; i0 < nf; i0 += 32) {
+        const int m = (i0 + lane < nf) ? wmask(i0 + lane) : -1;
+#pragma unroll
+        for (int bkt = 0; bkt < 16; ++bkt) bc[bkt] += __popc(__ballot_sync(0xffffffffu, m == bkt));
+      }
+      // round-robin position: entries of round r follow all entries of
+      // earlier rounds, and within a round go by class
+      int seen[16];
+#pragma unroll
+      for (int bkt = 0; bkt < 16; ++bkt) seen[bkt] = 0;
+      for (int i0 = 0; i0 < nf; i0 += 32) {
+        const int e = i0 + lane;
+        const int m = (e < nf) ? wmask(e) : -1;
+        int rank = 0;
+#pragma unroll
+        for (int bkt = 0; bkt < 16; ++bkt) {
+          const uint32_t bm = __ballot_sync(0xffffffffu, m == bkt);
+          if (m == bkt) rank = seen[bkt] + __popc(bm & ((1u << lane) - 1u));
+          seen[bkt] += __popc(bm);
+        }
+        if (e < nf) {
+          int pos = 0;
+#pragma unroll
+          for (int bkt = 0; bkt < 16; ++bkt) pos += min(bc[bkt], rank) + ((bkt < m && bc[bkt] > rank) ? 1 : 0);
+          far[pos] = faru[e];
+        }
+      }
+      __syncwarp();
+      for (int e = lane; e < nf; e += 32) faru[e] = far[e];
     }
     if (lane == 0) misc[2] = static_cast<uint32_t>(base);
   }
