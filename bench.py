@@ -57,6 +57,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="run the chosen workload's recipe at another sequence length "
+                         "(e.g. a smaller copy of the million-token workload for profiling)")
     return ap.parse_args(argv)
 
 
@@ -195,8 +198,10 @@ def _cpu_worker(args):
     sys.path.insert(0, ROOT)
     import oracle as O
     from content_routed_block_b200.workloads import CONFIGS, make_inputs
-    cfg, b, h, blocks, seconds = args
+    cfg, seq_len, b, h, blocks, seconds = args
     w = CONFIGS[cfg]
+    if seq_len:
+        w = w.with_(N=seq_len)
     g = w.Hq // w.Hkv
     x = make_inputs(w, q_heads=[h], kv_heads=[h // g])
     sub = w.with_(Hq=1, Hkv=1, B=1)
@@ -222,9 +227,10 @@ def _cpu_worker(args):
 
 
 class OraclePool:
-    def __init__(self, cfg: int):
+    def __init__(self, cfg: int, seq_len: int = 0):
         import multiprocessing as mp
         self.cfg = cfg
+        self.seq_len = seq_len
         self.cores = max(1, min(len(os.sched_getaffinity(0)), 64))
         old = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
         for k in old:
@@ -243,6 +249,8 @@ class OraclePool:
         import numpy as np
         from content_routed_block_b200.workloads import CONFIGS
         w = CONFIGS[self.cfg]
+        if self.seq_len:
+            w = w.with_(N=self.seq_len)
         nqb = w.N // w.block_q
         tasks = []
         rng = np.random.default_rng(self.step)
@@ -251,7 +259,7 @@ class OraclePool:
             b = c % w.B
             h = (c // w.B) % w.Hq
             blocks = rng.permutation(nqb).tolist()
-            tasks.append((self.cfg, b, h, blocks, seconds))
+            tasks.append((self.cfg, self.seq_len, b, h, blocks, seconds))
         res = self.pool.map(_cpu_worker, tasks)
         blocks = sum(r[0] for r in res)
         wall = max(r[1] for r in res)
@@ -265,10 +273,9 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from content_routed_block_b200.workloads import CONFIGS
-    w = CONFIGS[args.config]
+    w = workload_of(args)
     per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
-    pool = OraclePool(args.config)
+    pool = OraclePool(args.config, args.seq_len)
     try:
         for _ in range(args.warmup):
             pool.run(per_step)
@@ -295,6 +302,14 @@ def run_reference(args):
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def workload_of(args):
+    from content_routed_block_b200.workloads import CONFIGS
+    w = CONFIGS[args.config]
+    if args.seq_len:
+        w = w.with_(N=args.seq_len, name=f"{w.name}@{args.seq_len}")
+    return w
 
 
 def workload_config(w, args):
@@ -333,7 +348,7 @@ def run_ssa(args):
         dist.barrier()
     ssa.lib()
 
-    w = CONFIGS[args.config]
+    w = workload_of(args)
     p = ssa.params_of(w)
     x = make_inputs(w)
     host = {n: torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16) for n in "qkv"}
@@ -438,7 +453,7 @@ def run_ssa(args):
         bufs = {"q": qd, "k": kd, "v": vd, "o": o}
         n_e2e = min(args.steps, 100)
         for _ in range(3):
-            ssa.forward_host(qh, kh, vh, p, oh, device=dev, workspace=ws, dev_bufs=bufs)
+            ssa.forward_host(qh, kh, vh, p, oh, device=dev, dev_bufs=bufs)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -446,7 +461,7 @@ def run_ssa(args):
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(n_e2e):
-            ssa.forward_host(qh, kh, vh, p, oh, device=dev, workspace=ws, dev_bufs=bufs)
+            ssa.forward_host(qh, kh, vh, p, oh, device=dev, dev_bufs=bufs)
         e1.record()
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / n_e2e
@@ -460,7 +475,7 @@ def run_ssa(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        pool = OraclePool(args.config)
+        pool = OraclePool(args.config, args.seq_len)
         try:
             v, nb, wall = pool.run(args.cpu_seconds)
         finally:

@@ -196,21 +196,70 @@ def forward(q, k, v, p: Params, workspace: torch.Tensor | None = None, with_lse:
     return o, lse, idx, cnt
 
 
+def _forward_raw(p: Params, q: int, k: int, v: int, o: int, lse, idx, cnt, ws: torch.Tensor,
+                 stream) -> None:
+    """ssa_forward on raw device addresses (sub-problems of larger tensors)."""
+    vp = ctypes.c_void_p
+    _check(lib().ssa_forward(ctypes.byref(p), vp(q), vp(k), vp(v), vp(o), lse, idx, cnt,
+                             vp(ws.data_ptr()), ws.numel(), vp(stream.cuda_stream)))
+
+
 def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
-                 device: torch.device | str = "cuda", workspace: torch.Tensor | None = None,
-                 dev_bufs: dict | None = None):
-    """End-to-end call from host memory: copy pinned bf16 Q, K, V to the
-    device, run the path, copy O back into ``o_host`` (pinned).  ``dev_bufs``
-    may hold preallocated device tensors (keys q, k, v, o) to reuse."""
+                 device: torch.device | str = "cuda", dev_bufs: dict | None = None):
+    """End-to-end call from host memory: pinned bf16 Q, K, V in, O out.
+
+    Every (batch, query head) is an independent problem given its KV head, so
+    the call streams it: the K/V of a group and the Q of each head go to the
+    device on one copy stream, each head's forward (one ``ssa_forward`` on the
+    head's slice, B = Hq = Hkv = 1) runs on the compute stream as soon as its
+    inputs have landed, and its O returns on a second copy stream while later
+    heads are still arriving or computing.  ``dev_bufs`` may hold
+    preallocated device tensors and streams to reuse between calls.  The call
+    returns once all work is queued; the caller's current stream waits for it.
+    """
     d = dev_bufs if dev_bufs is not None else {}
+    dev = torch.device(device)
     for name, src in (("q", q_host), ("k", k_host), ("v", v_host)):
         if name not in d:
-            d[name] = torch.empty(src.shape, dtype=src.dtype, device=device)
-        d[name].copy_(src, non_blocking=True)
+            d[name] = torch.empty(src.shape, dtype=src.dtype, device=dev)
     if "o" not in d:
-        d["o"] = torch.empty(q_host.shape, dtype=torch.bfloat16, device=device)
-    forward(d["q"], d["k"], d["v"], p, workspace=workspace, with_lse=False, out=d["o"])
-    o_host.copy_(d["o"], non_blocking=True)
+        d["o"] = torch.empty(q_host.shape, dtype=torch.bfloat16, device=dev)
+    sub = make_params(1, 1, 1, p.N, p.D, p.block_k, p.block_q, p.top_k, p.window, p.causal,
+                      p.scale, p.wait_timeout_us)
+    if "ws" not in d:
+        d["ws"] = torch.empty(workspace_size(sub), dtype=torch.uint8, device=dev)
+    if "streams" not in d:
+        d["streams"] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    s_in, s_out = d["streams"]
+    compute = torch.cuda.current_stream(dev)
+    s_in.wait_stream(compute)       # buffers may still be read by earlier work
+    s_out.wait_stream(compute)
+    grp = p.Hq // p.Hkv
+    q, k, v, o = d["q"], d["k"], d["v"], d["o"]
+    row = p.N * p.D * 2             # bytes of one head
+    for b in range(p.B):
+        for g in range(p.Hkv):
+            with torch.cuda.stream(s_in):
+                k[b, g].copy_(k_host[b, g], non_blocking=True)
+                v[b, g].copy_(v_host[b, g], non_blocking=True)
+            for h in range(g * grp, (g + 1) * grp):
+                with torch.cuda.stream(s_in):
+                    q[b, h].copy_(q_host[b, h], non_blocking=True)
+                    ready = torch.cuda.Event()
+                    ready.record(s_in)
+                compute.wait_event(ready)
+                _forward_raw(sub, q.data_ptr() + (b * p.Hq + h) * row,
+                             k.data_ptr() + (b * p.Hkv + g) * row,
+                             v.data_ptr() + (b * p.Hkv + g) * row,
+                             o.data_ptr() + (b * p.Hq + h) * row, None, None, None, d["ws"],
+                             compute)
+                done = torch.cuda.Event()
+                done.record(compute)
+                s_out.wait_event(done)
+                with torch.cuda.stream(s_out):
+                    o_host[b, h].copy_(o[b, h], non_blocking=True)
+    compute.wait_stream(s_out)
+    compute.wait_stream(s_in)
     return o_host
 
 
