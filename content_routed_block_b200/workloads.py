@@ -65,6 +65,7 @@ class Workload:
     centres: int = 64          # clustered only
     needles: int = 64          # needles only
     needle_gap: int = 4096     # needles only: minimum query-after-key distance
+    consensus: bool = False    # one route per (batch, KV head, query block), voted by its heads
 
     @property
     def n_kblocks(self) -> int:

@@ -27,6 +27,12 @@ non-causal variant):
 6. Selection: the first min(top_k, |A|) admissible blocks in the order
    (score descending, block index ascending) -- ties go to the lower index --
    stored ascending by block index, padded with -1, with their count.
+6b. (Optional, ``Params.consensus``) GQA-shared consensus route: every query
+   head of a KV group votes for the blocks of its own selection, and the
+   group keeps the top_k blocks by (votes descending, block index ascending)
+   -- one list per (b, KV head, query block) that all of the group's heads
+   use ("Complete 10M transformer result": a cross-head consensus route
+   carrying the highest-vote blocks).
 7. Key set of query i as a SET: the keys of its query block's selected blocks
    united with the local causal window {j : i - W < j <= i} and cut at i
    (causal); only the selected blocks' keys (non-causal).  A key that is both
@@ -51,6 +57,7 @@ __all__ = [
     "Params", "upcast_bf16", "block_summary", "admissible_blocks", "route",
     "RouteResult", "key_set", "attend_masked_dense", "attend_gathered", "forward",
     "near_tie_rows", "acceptable_selections", "route_row",
+    "consensus_row", "route_consensus", "expand_consensus",
 ]
 
 NEAR_TIE_REL = 1e-4   # relative score gap under which two blocks count as tied
@@ -70,6 +77,7 @@ class Params:
     window: int
     causal: bool
     scale: float = 0.0          # 0 -> 1/sqrt(D)
+    consensus: bool = False     # GQA-shared (consensus) routing, see route_consensus
 
     @property
     def group(self) -> int:
@@ -91,7 +99,8 @@ class Params:
     def of(w) -> "Params":
         """Build from any object with the same field names (e.g. a workload)."""
         return Params(w.B, w.Hq, w.Hkv, w.N, w.D, w.block_k, w.block_q, w.top_k,
-                      w.window, bool(w.causal), getattr(w, "scale", 0.0))
+                      w.window, bool(w.causal), getattr(w, "scale", 0.0),
+                      bool(getattr(w, "consensus", False)))
 
 
 def upcast_bf16(u16: np.ndarray) -> np.ndarray:
@@ -222,6 +231,57 @@ def acceptable_selections(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, to
 
 
 # --------------------------------------------------------------------------
+# step 6b (optional): GQA-shared consensus route
+# --------------------------------------------------------------------------
+def consensus_row(head_selections, top_k: int) -> np.ndarray:
+    """One selection shared by the query heads of a KV group.
+
+    jonsmirl/ssa README, "Complete 10M transformer result": the first layer
+    forms one route across heads by consensus and carries the blocks with
+    the most votes forward; "Mathematical status": a highest-count reservoir
+    keeps the items that the per-head selectors voted for most often.  Here
+    every query head of the group votes once for each block of its own top-k
+    selection (step 6).  The shared selection is the first
+    min(top_k, #blocks with a vote) blocks in the order (votes descending,
+    block index ascending) -- the method's lower-index tie rule -- stored
+    ascending by block index."""
+    votes = {}
+    for sel in head_selections:
+        for c in np.asarray(sel, dtype=np.int64).tolist():
+            votes[c] = votes.get(c, 0) + 1
+    ranked = sorted(votes, key=lambda c: (-votes[c], c))
+    return np.array(sorted(ranked[:top_k]), dtype=np.int64)
+
+
+def route_consensus(idx: np.ndarray, cnt: np.ndarray, p: Params, rows=None):
+    """Consensus lists for every (b, KV head, query block) from the per-head
+    lists ``idx`` [B, Hq, NQB, top_k] / ``cnt`` [B, Hq, NQB] of step 6.
+
+    Returns (idx_kv int32 [B, Hkv, NQB, top_k] ascending and -1 padded,
+    cnt_kv int32 [B, Hkv, NQB]).  ``rows`` optionally lists (b, kv, qb)
+    triples; other rows stay empty.  The group of KV head kv is query heads
+    kv*g .. kv*g + g - 1 (step 2)."""
+    g = p.group
+    idx_kv = np.full((p.B, p.Hkv, p.n_qblocks, p.top_k), -1, dtype=np.int32)
+    cnt_kv = np.zeros((p.B, p.Hkv, p.n_qblocks), dtype=np.int32)
+    todo = rows if rows is not None else [
+        (b, kv, qb) for b in range(p.B) for kv in range(p.Hkv) for qb in range(p.n_qblocks)]
+    for b, kv, qb in todo:
+        heads = [idx[b, h, qb, :cnt[b, h, qb]] for h in range(kv * g, (kv + 1) * g)]
+        sel = consensus_row(heads, p.top_k)
+        idx_kv[b, kv, qb, :len(sel)] = sel
+        cnt_kv[b, kv, qb] = len(sel)
+    return idx_kv, cnt_kv
+
+
+def expand_consensus(idx_kv: np.ndarray, cnt_kv: np.ndarray, p: Params):
+    """Per-query-head view of consensus lists: query head h uses the list of
+    its KV head h // g.  The result feeds the attend forms unchanged."""
+    heads = np.arange(p.Hq) // p.group
+    return idx_kv[:, heads].copy(), cnt_kv[:, heads].copy()
+
+
+# --------------------------------------------------------------------------
 # step 7: key sets
 # --------------------------------------------------------------------------
 def key_set(i: int, sel_blocks: np.ndarray, p: Params) -> np.ndarray:
@@ -306,11 +366,20 @@ def attend_gathered(q, k, v, idx, cnt, p: Params, queries=None):
 def forward(q, k, v, p: Params, form: str = "dense"):
     """Whole path: summaries -> routing -> attend.  Inputs float64 arrays
     (use ``upcast_bf16`` on bf16 bit patterns).  Returns a dict with
-    ``o``, ``lse``, ``idx``, ``cnt``, ``route`` (RouteResult), ``qsum``, ``ksum``."""
+    ``o``, ``lse``, ``idx``, ``cnt``, ``route`` (RouteResult: the per-head
+    selections), ``qsum``, ``ksum``.  With ``p.consensus`` the per-head
+    selections are reduced to one list per (b, KV head, query block)
+    (``route_consensus``), which ``idx``/``cnt`` then hold, and every query
+    head of a group attends over its group's list."""
     ksum = block_summary(k, p.block_k)
     qsum = block_summary(q, p.block_q)
     r = route(qsum, ksum, p)
     attend = attend_masked_dense if form == "dense" else attend_gathered
-    o, lse = attend(q, k, v, r.idx, r.cnt, p)
-    return {"o": o, "lse": lse, "idx": r.idx, "cnt": r.cnt, "route": r,
+    if p.consensus:
+        idx, cnt = route_consensus(r.idx, r.cnt, p)
+        o, lse = attend(q, k, v, *expand_consensus(idx, cnt, p), p)
+    else:
+        idx, cnt = r.idx, r.cnt
+        o, lse = attend(q, k, v, idx, cnt, p)
+    return {"o": o, "lse": lse, "idx": idx, "cnt": cnt, "route": r,
             "qsum": qsum, "ksum": ksum}

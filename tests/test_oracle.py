@@ -370,3 +370,130 @@ def test_acceptable_selections_cover_near_ties():
     # no near tie: exactly the lexicographic selection
     acc = O.acceptable_selections(q, mu[[0, 1, 4]], np.arange(3), 2)
     assert [a.tolist() for a in acc] == [[0, 1]]
+
+
+# ---------------------------------------------------------------- consensus route
+def _read_consensus_votes():
+    cases = []
+    with open(os.path.join(GOLDEN, "consensus_votes.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, heads, want = (x.strip() for x in line.split("|"))
+            sels = [[int(c) for c in h.split()] for h in heads.split(";")]
+            cases.append((int(k), sels, [int(c) for c in want.split()]))
+    return cases
+
+
+def test_consensus_votes_match_hand_derivation():
+    cases = _read_consensus_votes()
+    assert len(cases) == 7
+    for k, sels, want in cases:
+        assert O.consensus_row(sels, k).tolist() == want, (k, sels)
+
+
+def test_consensus_brute_force_tiny():
+    # brute force: among all subsets of the voted blocks of the right size, the
+    # consensus is the unique one whose every member beats every non-member in
+    # (votes desc, index asc)
+    import itertools
+    rng = np.random.default_rng(5)
+    for trial in range(300):
+        g = int(rng.integers(1, 5))
+        k = int(rng.integers(1, 5))
+        sels = [sorted(rng.choice(9, size=int(rng.integers(0, k + 1)), replace=False).tolist())
+                for _ in range(g)]
+        votes = {}
+        for s in sels:
+            for c in s:
+                votes[c] = votes.get(c, 0) + 1
+        voted = sorted(votes)
+        m = min(k, len(voted))
+        ok = [sub for sub in itertools.combinations(voted, m)
+              if all((votes[a], -a) > (votes[u], -u) for a in sub for u in set(voted) - set(sub))]
+        assert len(ok) == 1
+        assert O.consensus_row(sels, k).tolist() == list(ok[0]), (sels, k)
+
+
+def _gqa_inputs(p, seed, same_heads=False):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((p.B, p.Hq, p.N, p.D))
+    if same_heads:
+        q = np.repeat(q[:, ::p.group], p.group, axis=1)
+    k = rng.standard_normal((p.B, p.Hkv, p.N, p.D))
+    v = rng.standard_normal((p.B, p.Hkv, p.N, p.D))
+    return q, k, v
+
+
+def test_consensus_with_groups_of_one_is_the_per_head_route():
+    p = _params(B=2, Hq=3, Hkv=3, N=96, D=4, block_k=8, block_q=8, top_k=3, window=8,
+                consensus=True)
+    q, k, v = _gqa_inputs(p, 21)
+    out = O.forward(q, k, v, p)
+    r = out["route"]
+    np.testing.assert_array_equal(out["idx"], r.idx)
+    np.testing.assert_array_equal(out["cnt"], r.cnt)
+    per_head = O.forward(q, k, v, O.Params(**{**p.__dict__, "consensus": False}))
+    np.testing.assert_array_equal(out["o"], per_head["o"])
+
+
+def test_consensus_of_identical_heads_is_their_own_route():
+    p = _params(B=1, Hq=6, Hkv=2, N=128, D=4, block_k=8, block_q=8, top_k=4, window=10,
+                consensus=True)
+    q, k, v = _gqa_inputs(p, 22, same_heads=True)
+    out = O.forward(q, k, v, p)
+    per_head = O.forward(q, k, v, O.Params(**{**p.__dict__, "consensus": False}))
+    for kv in range(2):
+        for h in range(kv * 3, kv * 3 + 3):
+            np.testing.assert_array_equal(out["idx"][:, kv], per_head["idx"][:, h])
+    np.testing.assert_allclose(out["o"], per_head["o"], atol=1e-13, rtol=0)
+
+
+def test_consensus_differs_from_per_head_routes_when_heads_disagree():
+    # not a tautology: with independent queries the shared list replaces many
+    # heads' own choices, and the outputs move
+    p = _params(B=1, Hq=4, Hkv=1, N=256, D=8, block_k=16, block_q=16, top_k=3, window=16,
+                consensus=True)
+    q, k, v = _gqa_inputs(p, 23)
+    out = O.forward(q, k, v, p)
+    own = out["route"].idx
+    shared = O.expand_consensus(out["idx"], out["cnt"], p)[0]
+    assert (own != shared).any(axis=-1).mean() > 0.3
+    per_head = O.forward(q, k, v, O.Params(**{**p.__dict__, "consensus": False}))
+    assert np.abs(out["o"] - per_head["o"]).max() > 1e-3
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,bk", [(16, 4, 2, 8), (32, 6, 2, 16)])
+def test_consensus_dense_causal_when_topk_covers_every_block(D, Hq, Hkv, bk):
+    N = 8 * bk
+    p = _params(B=2, Hq=Hq, Hkv=Hkv, N=N, D=D, block_k=bk, block_q=bk, top_k=N // bk,
+                window=bk, consensus=True)
+    q, k, v = _rand((2, Hq, N, D), 4), _rand((2, Hkv, N, D), 5), _rand((2, Hkv, N, D), 6)
+    out = O.forward(q, k, v, p)
+    want = _sdpa(q, k, v, causal=True, gqa=True)
+    np.testing.assert_allclose(out["o"], want, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("form", ["dense", "gathered"])
+def test_consensus_worked_example_matches_hand_derivation(form):
+    q0, k, v = _worked_inputs()
+    q1 = np.tile(np.array([[2.0, 0.0]]), (8, 1))[None, None]
+    q = np.concatenate([q0, q1], axis=1)
+    p = _params(Hq=2, Hkv=1, top_k=1, consensus=True)
+    out = O.forward(q, k, v, p, form=form)
+    assert out["route"].idx[0, :, :, 0].tolist() == [[-1, 0, 1, 1], [-1, 0, 0, 0]]
+    assert out["idx"][0, 0, :, 0].tolist() == [-1, 0, 0, 0]
+    E = math.exp(math.sqrt(2.0))
+    n = 0
+    with open(os.path.join(GOLDEN, "consensus_worked_example.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            h, i, expr = line.split(maxsplit=2)
+            assert out["o"][0, int(h), int(i), 0] == pytest.approx(eval(expr, {"E": E}),
+                                                                 abs=1e-12)
+            assert out["o"][0, int(h), int(i), 1] == pytest.approx(1.0, abs=1e-12)
+            n += 1
+    assert n == 16
