@@ -60,6 +60,9 @@ def parse_args(argv=None):
     ap.add_argument("--seq-len", type=int, default=0,
                     help="run the chosen workload's recipe at another sequence length "
                          "(e.g. a smaller copy of the million-token workload for profiling)")
+    ap.add_argument("--consensus", action="store_true",
+                    help="GQA-shared consensus routing: the query heads of a KV group vote "
+                         "and share one list per query block")
     return ap.parse_args(argv)
 
 
@@ -147,10 +150,14 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 def algorithmic_work(w, idx, cnt):
     """Mean distinct keys per query (|S_i|), selected-key flops, and the attend
-    kernel's algorithmic bytes: per query block, the distinct key blocks it
-    needs (routed U window) x Bk rows x K and V, plus Q read, O and LSE write."""
+    kernel's algorithmic bytes: per routed list (a query block of a query head;
+    of a KV group with consensus routing, where the group's heads share the
+    keys), the distinct key blocks it needs (routed U window) x Bk rows x K and
+    V, plus the Q read and the O and LSE writes."""
     import numpy as np
     B, Hq, N, D, Bk, Bq, W = w.B, w.Hq, w.N, w.D, w.block_k, w.block_q, w.window
+    g = w.Hq // w.Hkv
+    cons = bool(getattr(w, "consensus", False))
     nqb = N // Bq
     qb = np.arange(nqb)
     k = w.top_k
@@ -158,11 +165,13 @@ def algorithmic_work(w, idx, cnt):
     blocks_total = 0
     for b in range(B):
         for h in range(Hq):
-            sel = idx[b, h] if k > 0 else np.zeros((nqb, 0), np.int64)
-            valid = (np.arange(k)[None, :] < cnt[b, h][:, None]) if k > 0 else sel.astype(bool)
+            lh = h // g if cons else h             # the list this head reads
+            count_blocks = (not cons) or h % g == 0
+            sel = idx[b, lh] if k > 0 else np.zeros((nqb, 0), np.int64)
+            valid = (np.arange(k)[None, :] < cnt[b, lh][:, None]) if k > 0 else sel.astype(bool)
             if not w.causal:
-                keys_total += float(cnt[b, h].sum()) * Bk * Bq
-                blocks_total += int(cnt[b, h].sum())
+                keys_total += float(cnt[b, lh].sum()) * Bk * Bq
+                blocks_total += int(cnt[b, lh].sum()) if count_blocks else 0
                 continue
             # rows i of block qb: i = qb*Bq + r
             r = np.arange(Bq)
@@ -180,7 +189,8 @@ def algorithmic_work(w, idx, cnt):
             wlo = np.maximum(0, qb * Bq - W + 1) // Bk
             whi = (qb * Bq + Bq - 1) // Bk
             in_win = (sel >= wlo[:, None]) & (sel <= whi[:, None]) & valid
-            blocks_total += int(((whi - wlo + 1) + valid.sum(axis=1) - in_win.sum(axis=1)).sum())
+            if count_blocks:
+                blocks_total += int(((whi - wlo + 1) + valid.sum(axis=1) - in_win.sum(axis=1)).sum())
     kpq = keys_total / (B * Hq * N)
     flops = 4.0 * B * Hq * N * kpq * D
     gathered = blocks_total * Bk * 2 * D * 2
@@ -198,39 +208,51 @@ def _cpu_worker(args):
     sys.path.insert(0, ROOT)
     import oracle as O
     from content_routed_block_b200.workloads import CONFIGS, make_inputs
-    cfg, seq_len, b, h, blocks, seconds = args
+    cfg, seq_len, consensus, b, h, blocks, seconds = args
     w = CONFIGS[cfg]
     if seq_len:
         w = w.with_(N=seq_len)
     g = w.Hq // w.Hkv
-    x = make_inputs(w, q_heads=[h], kv_heads=[h // g])
-    sub = w.with_(Hq=1, Hkv=1, B=1)
+    # the unit of work: one query block of one query head, or (consensus) of
+    # every head of the KV group, which vote on one shared list
+    heads = list(range((h // g) * g, (h // g + 1) * g)) if consensus else [h]
+    x = make_inputs(w, q_heads=heads, kv_heads=[h // g])
+    sub = w.with_(Hq=len(heads), Hkv=1, B=1, consensus=consensus)
     p = O.Params.of(sub)
-    q = O.upcast_bf16(x["q"][b:b + 1])
+    q = O.upcast_bf16(x["q"][b:b + 1])           # the requested heads, in order
     k = O.upcast_bf16(x["k"][b:b + 1])
     v = O.upcast_bf16(x["v"][b:b + 1])
     t0 = time.perf_counter()
     ksum = O.block_summary(k, p.block_k)
     done = 0
-    idx = np.full((1, 1, p.n_qblocks, p.top_k), -1, np.int32)
-    cnt = np.zeros((1, 1, p.n_qblocks), np.int32)
+    nh = len(heads)
+    idx = np.full((1, nh, p.n_qblocks, p.top_k), -1, np.int32)
+    cnt = np.zeros((1, nh, p.n_qblocks), np.int32)
     for qb in blocks:
-        qbar = O.block_summary(q[:, :, qb * p.block_q:(qb + 1) * p.block_q], p.block_q)[0, 0, 0]
-        sel, _, _ = O.route_row(qbar, ksum[0, 0], O.admissible_blocks(qb, p), p.top_k)
-        idx[0, 0, qb, :len(sel)] = sel
-        cnt[0, 0, qb] = len(sel)
-        O.attend_masked_dense(q, k, v, idx, cnt, p, blocks=[(0, 0, qb)])
-        done += 1
+        for j in range(nh):
+            qbar = O.block_summary(q[:, j:j + 1, qb * p.block_q:(qb + 1) * p.block_q],
+                                   p.block_q)[0, 0, 0]
+            sel, _, _ = O.route_row(qbar, ksum[0, 0], O.admissible_blocks(qb, p), p.top_k)
+            idx[0, j, qb, :len(sel)] = sel
+            cnt[0, j, qb] = len(sel)
+        if consensus:
+            shared = O.consensus_row([idx[0, j, qb, :cnt[0, j, qb]] for j in range(nh)], p.top_k)
+            idx[0, :, qb] = -1
+            idx[0, :, qb, :len(shared)] = shared
+            cnt[0, :, qb] = len(shared)
+        O.attend_masked_dense(q, k, v, idx, cnt, p, blocks=[(0, j, qb) for j in range(nh)])
+        done += nh
         if time.perf_counter() - t0 > seconds:
             break
     return done, time.perf_counter() - t0
 
 
 class OraclePool:
-    def __init__(self, cfg: int, seq_len: int = 0):
+    def __init__(self, cfg: int, seq_len: int = 0, consensus: bool = False):
         import multiprocessing as mp
         self.cfg = cfg
         self.seq_len = seq_len
+        self.consensus = consensus
         self.cores = max(1, min(len(os.sched_getaffinity(0)), 64))
         old = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
         for k in old:
@@ -245,7 +267,10 @@ class OraclePool:
 
     def run(self, seconds: float):
         """Each worker runs the oracle's whole path for seconds on its own
-        (b, head) and a spread of query blocks; returns (tokens/s, blocks)."""
+        (b, head) and a spread of query blocks; returns (tokens/s, (head,
+        query block) units done, wall seconds).  One unit is 1/Hq of the work
+        of Bq tokens (tokens/s counts positions over all heads), so
+        tokens/s = units * Bq / Hq / wall."""
         import numpy as np
         from content_routed_block_b200.workloads import CONFIGS
         w = CONFIGS[self.cfg]
@@ -259,11 +284,11 @@ class OraclePool:
             b = c % w.B
             h = (c // w.B) % w.Hq
             blocks = rng.permutation(nqb).tolist()
-            tasks.append((self.cfg, self.seq_len, b, h, blocks, seconds))
+            tasks.append((self.cfg, self.seq_len, self.consensus, b, h, blocks, seconds))
         res = self.pool.map(_cpu_worker, tasks)
         blocks = sum(r[0] for r in res)
         wall = max(r[1] for r in res)
-        return blocks * w.block_q / wall, blocks, wall
+        return blocks * w.block_q / w.Hq / wall, blocks, wall
 
     def close(self):
         self.pool.terminate()
@@ -275,7 +300,7 @@ def run_reference(args):
         return
     w = workload_of(args)
     per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
-    pool = OraclePool(args.config, args.seq_len)
+    pool = OraclePool(args.config, args.seq_len, args.consensus)
     try:
         for _ in range(args.warmup):
             pool.run(per_step)
@@ -289,8 +314,9 @@ def run_reference(args):
     finally:
         pool.close()
     value = statistics.mean(vals)
-    sample = (f"{blocks} query blocks of {w.block_q} tokens over {args.steps} steps, "
-              f"~{per_step:.1f} s of oracle work per core per step")
+    sample = (f"{blocks} (query head, query block) units of this workload over {args.steps} "
+              f"steps, ~{per_step:.1f} s of oracle work per core per step; one unit is 1/Hq of "
+              f"the work of {w.block_q} tokens")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -309,13 +335,16 @@ def workload_of(args):
     w = CONFIGS[args.config]
     if args.seq_len:
         w = w.with_(N=args.seq_len, name=f"{w.name}@{args.seq_len}")
+    if getattr(args, "consensus", False):
+        w = w.with_(consensus=True, name=f"{w.name}+consensus")
     return w
 
 
 def workload_config(w, args):
     return {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} D={w.D} "
                         f"Bk={w.block_k} Bq={w.block_q} top_k={w.top_k} W={w.window} "
-                        f"{'causal' if w.causal else 'non-causal'} {w.kind}",
+                        f"{'causal' if w.causal else 'non-causal'} {w.kind}"
+                        f"{' consensus-routed' if w.consensus else ''}",
             "global_batch": w.B * args.gpus, "seq_len": w.N, "parallelism": f"replicas{args.gpus}",
             "l2": "flushed between timed steps (256 MiB write)"}
 
@@ -356,8 +385,11 @@ def run_ssa(args):
     ws = torch.empty(ssa.workspace_size(p), dtype=torch.uint8, device=dev)
     o = torch.empty_like(qd)
     lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
-    idx = torch.empty((w.B, w.Hq, w.N // w.block_q, w.top_k), dtype=torch.int32, device=dev)
-    cnt = torch.empty((w.B, w.Hq, w.N // w.block_q), dtype=torch.int32, device=dev)
+    LH = w.Hkv if w.consensus else w.Hq          # heads the attended lists span
+    idx = torch.empty((w.B, LH, w.N // w.block_q, w.top_k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, LH, w.N // w.block_q), dtype=torch.int32, device=dev)
+    idx_h = torch.empty((w.B, w.Hq, w.N // w.block_q, w.top_k), dtype=torch.int32, device=dev)
+    cnt_h = torch.empty((w.B, w.Hq, w.N // w.block_q), dtype=torch.int32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def step():
@@ -404,7 +436,7 @@ def run_ssa(args):
 
     # per-kernel split: the same path as separate calls with events between them
     n_split = min(args.steps, 200)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_split)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_split)]
     ks = torch.empty((w.B, w.Hkv, w.N // w.block_k, w.D), dtype=torch.float32, device=dev)
     qs = torch.empty((w.B, w.Hq, w.N // w.block_q, w.D), dtype=torch.float32, device=dev)
     L = ssa.lib()
@@ -420,30 +452,48 @@ def run_ssa(args):
         e[1].record()
         assert L.ssa_block_summary(pp, P(qd), w.Hq, w.block_q, P(qs), st) == 0
         e[2].record()
-        assert L.ssa_route(pp, P(qs), P(ks), P(idx) if w.top_k else None, P(cnt), st) == 0
-        e[3].record()
+        if w.consensus:
+            assert L.ssa_route(pp, P(qs), P(ks), P(idx_h) if w.top_k else None, P(cnt_h), st) == 0
+            e[3].record()
+            assert L.ssa_route_consensus(pp, P(idx_h) if w.top_k else None, P(cnt_h),
+                                         P(idx) if w.top_k else None, P(cnt), st) == 0
+        else:
+            assert L.ssa_route(pp, P(qs), P(ks), P(idx) if w.top_k else None, P(cnt), st) == 0
+            e[3].record()
+        e[4].record()
         assert L.ssa_attend(pp, P(qd), P(kd), P(vd), P(idx) if w.top_k else None, P(cnt),
                             P(o), P(lse), st) == 0
-        e[4].record()
+        e[5].record()
     torch.cuda.synchronize()
     ssa.check_error()
     seg = lambda i: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(n_split))  # noqa: E731
-    pool_k_ms, pool_q_ms, route_ms, attend_ms = seg(0), seg(1), seg(2), seg(3)
+    pool_k_ms, pool_q_ms, route_ms, cons_ms, attend_ms = seg(0), seg(1), seg(2), seg(3), seg(4)
 
     work = algorithmic_work(w, idx.cpu().numpy(), cnt.cpu().numpy())
     peaks, peak_kind = load_peaks()
     hbm = float(peaks["hbm_gbs"])
-    achieved = work["attend_bytes"] / (attend_ms * 1e-3) / 1e9
+    tensor = float(peaks["bf16_tflops"])
     tflops = work["flops"] / (ms * 1e-3) / 1e12
     attend_tflops = work["flops"] / (attend_ms * 1e-3) / 1e12
-    t_roof = max(work["flops"] / (float(peaks["bf16_tflops"]) * 1e12),
-                 work["attend_bytes"] / (hbm * 1e9))
+    t_hbm = work["attend_bytes"] / (hbm * 1e9)
+    t_tensor = work["flops"] / (tensor * 1e12)
+    t_roof = max(t_hbm, t_tensor)
+    # the attend kernel's binding roof: gathered bytes over HBM (per-head
+    # lists, ~64 flop/B), or bf16 flops over the tensor peak (consensus lists
+    # shared by g heads raise the intensity g-fold, past the B200 ridge)
+    if t_hbm >= t_tensor:
+        roof = {"bound": "hbm", "achieved": work["attend_bytes"] / (attend_ms * 1e-3) / 1e9,
+                "peak": hbm, "unit": "GB/s", "peak_source": f"{peak_kind} hbm_gbs"}
+    else:
+        roof = {"bound": "tensor", "achieved": attend_tflops, "peak": tensor, "unit": "TFLOP/s",
+                "peak_source": f"{peak_kind} bf16_tflops (burst)"}
     traffic = None
     if os.path.exists(TRAFFIC_FILE):
         with open(TRAFFIC_FILE) as f:
             tr = json.load(f)
         if tr.get("kernel_hash") == kernel_source_hash():
-            traffic = tr.get("bytes_per_launch", {}).get(str(args.config))
+            key = f"{args.config}{'c' if w.consensus else ''}" + (f"@{args.seq_len}" if args.seq_len else "")
+            traffic = tr.get("bytes_per_launch", {}).get(key)
 
     # end to end through the public call, from pinned host memory
     e2e = None
@@ -475,15 +525,16 @@ def run_ssa(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        pool = OraclePool(args.config, args.seq_len)
+        pool = OraclePool(args.config, args.seq_len, args.consensus)
         try:
             v, nb, wall = pool.run(args.cpu_seconds)
         finally:
             pool.close()
         cpu = {"value": v, "unit": UNIT, "cores": pool.cores, "kind": "oracle",
-               "sample": f"{nb} query blocks ({nb * w.block_q} tokens) of this workload, whole "
-                         f"path (summaries, routing, masked-dense attend) in float64, "
-                         f"{pool.cores} processes x ~{args.cpu_seconds:.0f} s"}
+               "sample": f"{nb} (query head, query block) units of this workload (each 1/Hq of "
+                         f"the work of {w.block_q} tokens), whole path (summaries, routing"
+                         f"{', consensus' if w.consensus else ''}, masked-dense attend) in "
+                         f"float64, {pool.cores} processes x ~{args.cpu_seconds:.0f} s"}
 
     clocks = sampler.summary()
     if world > 1:
@@ -500,17 +551,19 @@ def run_ssa(args):
         "keys_per_query": work["keys_per_query"],
         "nominal_keys_per_query": work["nominal_keys_per_query"],
         "kernels_ms": {"pool_k": pool_k_ms, "pool_q": pool_q_ms, "route": route_ms,
-                       "attend": attend_ms},
-        "roofline": {"bound": "hbm", "kernel": "attend_kernel", "achieved": achieved, "peak": hbm,
-                     "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
-                     "peak_source": f"{peak_kind} hbm_gbs",
+                       **({"consensus": cons_ms} if w.consensus else {}), "attend": attend_ms},
+        "roofline": {"bound": roof["bound"], "kernel": "attend_kernel",
+                     "achieved": roof["achieved"], "peak": roof["peak"], "unit": roof["unit"],
+                     "frac": roof["achieved"] / roof["peak"], "traffic": traffic,
+                     "peak_source": roof["peak_source"],
                      "bytes_per_launch": work["attend_bytes"],
+                     "hbm_frac": work["attend_bytes"] / (attend_ms * 1e-3) / 1e9 / hbm,
                      "attend_tflops": attend_tflops,
                      "attend_tensor_frac": attend_tflops / float(peaks["bf16_tflops"]),
                      "path_frac_of_roofline": t_roof / (ms * 1e-3)},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (4 if w.consensus else 3) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

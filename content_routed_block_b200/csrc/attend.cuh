@@ -12,7 +12,9 @@
 // online-softmax merge this kernel performs chunk by chunk.
 //
 // B200 design (one CTA = 128 query rows of one (b, head), i.e. 128/Bq query
-// blocks; 192 threads):
+// blocks; or, with GQA-shared consensus lists, 64 rows of each of two query
+// heads of one KV group, which read the same key set so that every chunk
+// serves all 128 rows; 192 threads):
 //  * The CTA first builds the union of its query blocks' routed blocks and
 //    the window's blocks in shared memory (deduplicated), each entry carrying
 //    a bitmask of which query blocks routed it, with routed entries
@@ -78,12 +80,15 @@ struct AtLayout {
 };
 
 struct AttendArgs {
-  const int32_t* idx;    // [B*Hq, NQB, top_k]
-  const int32_t* cnt;    // [B*Hq, NQB]
+  const int32_t* idx;    // [B*idx_heads, NQB, top_k]
+  const int32_t* cnt;    // [B*idx_heads, NQB]
   __nv_bfloat16* o;      // [B*Hq, N, D]
   float* lse;            // [B*Hq, N] or null
   int32_t Hq, Hkv, N, NQB, NB, Bq, Bk, top_k, window, causal;
-  int32_t n_qtiles;
+  int32_t idx_heads;     // Hq: a list per query head; Hkv: one list per KV group
+  int32_t pack;          // query heads per CTA: 1, or 2 (two heads of a group
+                         // sharing one list, 64 rows each)
+  int32_t n_qtiles;      // ceil(N / (kAtQT / pack))
   float scale_log2;      // softmax scale * log2(e)
   uint64_t timeout_ns;
 };
@@ -133,14 +138,35 @@ __global__ void __launch_bounds__(kAtThreads, 2)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[3]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x / a.n_qtiles;
+  // The tile is RH consecutive query positions of `pack` query heads: rows
+  // 0..RH-1 belong to head h0, rows RH..2RH-1 (pack == 2) to head h1 of the
+  // same KV group, which shares h0's routed lists.  With an odd group the
+  // last pair has no h1: its rows are loaded from h0 and never written.
+  const int RH = kAtQT / a.pack;
+  const int tile_bh = blockIdx.x / a.n_qtiles;
   const int qt = blockIdx.x % a.n_qtiles;
-  const int b = bh / a.Hq, h = bh % a.Hq;
-  const int bkv = b * a.Hkv + h / (a.Hq / a.Hkv);
-  const int q0 = qt * kAtQT;
-  const int qend = min(a.N, q0 + kAtQT);
+  const int grp = a.Hq / a.Hkv;
+  int b, h0, h1;
+  bool has_h1 = false;
+  if (a.pack == 1) {
+    b = tile_bh / a.Hq;
+    h0 = tile_bh % a.Hq;
+    h1 = h0;
+  } else {
+    const int npair = (grp + 1) / 2;
+    const int bk = tile_bh / npair, pr = tile_bh % npair;
+    b = bk / a.Hkv;
+    h0 = (bk % a.Hkv) * grp + 2 * pr;
+    has_h1 = 2 * pr + 1 < grp;
+    h1 = has_h1 ? h0 + 1 : h0;
+  }
+  const int bh = b * a.Hq + h0;
+  const int bkv = b * a.Hkv + h0 / grp;
+  const int ibh = (a.idx_heads == a.Hq) ? bh : bkv;  // row block of the routed lists
+  const int q0 = qt * RH;
+  const int qend = min(a.N, q0 + RH);
   const int qb0 = q0 / a.Bq;
-  const int R = min(kAtQT / a.Bq, a.NQB - qb0);
+  const int R = min(max(RH / a.Bq, 1), a.NQB - qb0);
   int wlo = 0, nwin = 0;
   if (a.causal) {
     wlo = max(0, q0 - a.window + 1) / a.Bk;
@@ -182,8 +208,13 @@ __global__ void __launch_bounds__(kAtThreads, 2)
     tma_prefetch_desc(&tv);
     mbar_arrive_expect_tx(bar_q, L::Q_BYTES);
 #pragma unroll
-    for (int half = 0; half < D / 64; ++half)
+    for (int half = 0; half < D / 64; ++half) {
+      // the tensor map's box is RH rows: one box per head
       tma_load_3d(smem + L::OFF_Q + half * L::HALF_Q, &tq, bar_q, half * 64, q0, bh);
+      if (a.pack == 2)
+        tma_load_3d(smem + L::OFF_Q + half * L::HALF_Q + 64 * 128, &tq, bar_q, half * 64, q0,
+                    b * a.Hq + h1);
+    }
   }
 
   // ------------------------------------------ union of routed and window blocks
@@ -191,7 +222,7 @@ __global__ void __launch_bounds__(kAtThreads, 2)
     const int total = R * a.top_k;
     for (int t = tid; t < total; t += kAtThreads) {
       const int r = t / a.top_k, e = t % a.top_k;
-      const int64_t row = static_cast<int64_t>(bh) * a.NQB + qb0 + r;
+      const int64_t row = static_cast<int64_t>(ibh) * a.NQB + qb0 + r;
       int n = a.cnt[row];
       if (n > a.top_k || n < 0) {
         record_error(kErrCheck, kSiteIdx);
@@ -265,7 +296,8 @@ __global__ void __launch_bounds__(kAtThreads, 2)
       uint32_t qm[4];
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        const int lo = (32 * w) / a.Bq, hi = min(R - 1, (32 * w + 31) / a.Bq);
+        const int i_lo = q0 + (32 * w) % RH;
+        const int lo = i_lo / a.Bq - qb0, hi = min(R - 1, (i_lo + 31) / a.Bq - qb0);
         qm[w] = (lo < R) ? ((2u << hi) - (1u << lo)) : 0u;
       }
       auto wmask = [&](int e) -> int {
@@ -423,9 +455,11 @@ __global__ void __launch_bounds__(kAtThreads, 2)
   } else {
     // ------------------------------------------------------- softmax warps
     const int r = tid;  // row in the tile == TMEM lane
-    const int i = q0 + r;
-    const bool row_ok = i < qend;
-    const int qbr = row_ok ? r / a.Bq : 0;
+    const int slot = r / RH;
+    const int i = q0 + r % RH;
+    const bool row_ok = i < qend && (slot == 0 || has_h1);
+    const int qbr = row_ok ? i / a.Bq - qb0 : 0;
+    const int bh_row = b * a.Hq + (slot == 0 ? h0 : h1);
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const float sl2 = a.scale_log2;
     // running max of the raw scores (the scale is positive, so the max of the
@@ -589,7 +623,7 @@ __global__ void __launch_bounds__(kAtThreads, 2)
     if (ok && !*abort_flag) {
       tc_fence_after();
       const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
-      __nv_bfloat16* orow = a.o + (static_cast<int64_t>(bh) * a.N + i) * D;
+      __nv_bfloat16* orow = a.o + (static_cast<int64_t>(bh_row) * a.N + i) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t ov[32];
@@ -613,7 +647,7 @@ __global__ void __launch_bounds__(kAtThreads, 2)
       }
       if (row_ok && a.lse != nullptr) {
         const float lse2 = (l_sum > 0.f) ? m_raw * sl2 + __log2f(l_sum) : -INFINITY;
-        a.lse[static_cast<int64_t>(bh) * a.N + i] = lse2 * 0.69314718055994530942f;
+        a.lse[static_cast<int64_t>(bh_row) * a.N + i] = lse2 * 0.69314718055994530942f;
       }
     }
   }

@@ -18,6 +18,7 @@
 #include "../../include/ssa.h"
 #include "attend.cuh"
 #include "common.cuh"
+#include "consensus.cuh"
 #include "pool.cuh"
 #include "route.cuh"
 #include "route_tc.cuh"
@@ -102,6 +103,11 @@ ssa_status validate(const ssa_params* p) {
   if (!(p->scale >= 0.f) || !std::isfinite(p->scale))
     return fail(SSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if (p->wait_timeout_us < 0) return fail(SSA_ERR_INVALID_ARG, "wait_timeout_us must be >= 0");
+  if (p->consensus != 0 && p->consensus != 1)
+    return fail(SSA_ERR_INVALID_ARG, "consensus must be 0 or 1");
+  if (p->consensus && (p->Hq / p->Hkv) * p->top_k > ssa::kConsMaxVotes)
+    return fail(SSA_ERR_UNSUPPORTED, "consensus routing needs (Hq / Hkv) * top_k <= %d",
+                ssa::kConsMaxVotes);
   const int64_t nb = p->N / p->block_k;
   if (nb >= (1 << 23)) return fail(SSA_ERR_UNSUPPORTED, "N / block_k must be below 2^23");
   const int64_t rows = static_cast<int64_t>(p->B) * p->Hq * p->N;
@@ -268,6 +274,16 @@ ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksu
   return SSA_OK;
 }
 
+// Query heads per attend CTA.  Consensus lists are shared by a KV group, so
+// two heads of the group fill one 128-row tile (64 rows each) and every chunk
+// serves all rows.  SSA_PACK=1 forces one head per tile (the tests run both).
+int attend_pack(const ssa_params* p) {
+  if (!p->consensus || p->Hq / p->Hkv < 2) return 1;
+  const char* env = std::getenv("SSA_PACK");
+  if (env != nullptr && std::string(env) == "1") return 1;
+  return 2;
+}
+
 template <int D>
 cudaError_t launch_attend_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const ssa::AttendArgs& a, int n_ctas, cudaStream_t stream) {
@@ -286,8 +302,11 @@ ssa_status launch_attend(const ssa_params* p, const void* q, const void* k, cons
   ssa_status s = get_encoder();
   if (s != SSA_OK) return s;
   CUtensorMap tq, tk, tv;
+  const int pack = attend_pack(p);
   const uint32_t kv_rows = static_cast<uint32_t>(p->block_k < 64 ? p->block_k : 64);
-  if ((s = make_map(&tq, q, static_cast<int64_t>(p->B) * p->Hq, p->N, p->D, 128)) != SSA_OK) return s;
+  const uint32_t q_rows = static_cast<uint32_t>(ssa::kAtQT / pack);
+  if ((s = make_map(&tq, q, static_cast<int64_t>(p->B) * p->Hq, p->N, p->D, q_rows)) != SSA_OK)
+    return s;
   if ((s = make_map(&tk, k, static_cast<int64_t>(p->B) * p->Hkv, p->N, p->D, kv_rows)) != SSA_OK)
     return s;
   if ((s = make_map(&tv, v, static_cast<int64_t>(p->B) * p->Hkv, p->N, p->D, kv_rows)) != SSA_OK)
@@ -307,11 +326,16 @@ ssa_status launch_attend(const ssa_params* p, const void* q, const void* k, cons
   a.top_k = p->top_k;
   a.window = p->window;
   a.causal = p->causal;
-  a.n_qtiles = (p->N + ssa::kAtQT - 1) / ssa::kAtQT;
+  a.idx_heads = p->consensus ? p->Hkv : p->Hq;
+  a.pack = pack;
+  a.n_qtiles = (p->N + static_cast<int32_t>(q_rows) - 1) / static_cast<int32_t>(q_rows);
   const float scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
   a.scale_log2 = scale * 1.4426950408889634f;
   a.timeout_ns = timeout_ns(p);
-  const int64_t n_ctas = static_cast<int64_t>(p->B) * p->Hq * a.n_qtiles;
+  const int64_t head_tiles = pack == 1 ? static_cast<int64_t>(p->B) * p->Hq
+                                       : static_cast<int64_t>(p->B) * p->Hkv *
+                                             ((p->Hq / p->Hkv + 1) / 2);
+  const int64_t n_ctas = head_tiles * a.n_qtiles;
   if (n_ctas > 0x7FFFFFFF) return fail(SSA_ERR_UNSUPPORTED, "too many query tiles");
   const cudaError_t e =
       p->D == 64 ? launch_attend_t<64>(tq, tk, tv, a, static_cast<int>(n_ctas), stream)
@@ -320,8 +344,31 @@ ssa_status launch_attend(const ssa_params* p, const void* q, const void* k, cons
   return SSA_OK;
 }
 
+ssa_status launch_consensus(const ssa_params* p, const int32_t* idx, const int32_t* cnt,
+                            int32_t* idx_kv, int32_t* cnt_kv, cudaStream_t stream) {
+  ssa::ConsensusArgs a;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.idx_kv = idx_kv;
+  a.cnt_kv = cnt_kv;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.NQB = p->N / p->block_q;
+  a.NB = p->N / p->block_k;
+  a.top_k = p->top_k;
+  a.n_rows = static_cast<int64_t>(p->B) * p->Hkv * a.NQB;
+  const int64_t grid = (a.n_rows + ssa::kConsWarps - 1) / ssa::kConsWarps;
+  if (grid > 0x7FFFFFFF) return fail(SSA_ERR_UNSUPPORTED, "too many query blocks");
+  ssa::consensus_kernel<<<static_cast<unsigned>(grid), ssa::kConsThreads, 0, stream>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "consensus_kernel launch");
+  return SSA_OK;
+}
+
+// Workspace of ssa_forward: K and Q summaries, the per-head routed lists and
+// counts, and (consensus routing only) the per-group lists and counts.
 struct WsLayout {
-  size_t ksum, qsum, idx, cnt, total;
+  size_t ksum, qsum, idx, cnt, idx_kv, cnt_kv, total;
 };
 
 WsLayout ws_layout(const ssa_params* p) {
@@ -331,11 +378,15 @@ WsLayout ws_layout(const ssa_params* p) {
   const size_t qs = static_cast<size_t>(p->B) * p->Hq * nqb * p->D * sizeof(float);
   const size_t ix = static_cast<size_t>(p->B) * p->Hq * nqb * p->top_k * sizeof(int32_t);
   const size_t cn = static_cast<size_t>(p->B) * p->Hq * nqb * sizeof(int32_t);
+  const size_t g = static_cast<size_t>(p->Hq / p->Hkv);
+  const size_t ixk = p->consensus ? ix / g : 0, cnk = p->consensus ? cn / g : 0;
   w.ksum = 0;
   w.qsum = align256(ks);
   w.idx = w.qsum + align256(qs);
   w.cnt = w.idx + align256(ix);
-  w.total = w.cnt + align256(cn);
+  w.idx_kv = w.cnt + align256(cn);
+  w.cnt_kv = w.idx_kv + align256(ixk);
+  w.total = w.cnt_kv + align256(cnk);
   return w;
 }
 
@@ -374,6 +425,22 @@ ssa_status ssa_route(const ssa_params* p, const float* qsum, const float* ksum, 
   return s == SSA_OK ? ok() : s;
 }
 
+ssa_status ssa_route_consensus(const ssa_params* p, const int32_t* idx, const int32_t* cnt,
+                               int32_t* idx_kv, int32_t* cnt_kv, ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if ((p->Hq / p->Hkv) * p->top_k > ssa::kConsMaxVotes)
+    return fail(SSA_ERR_UNSUPPORTED, "consensus routing needs (Hq / Hkv) * top_k <= %d",
+                ssa::kConsMaxVotes);
+  if (cnt == nullptr || cnt_kv == nullptr || (p->top_k > 0 && (idx == nullptr || idx_kv == nullptr)))
+    return fail(SSA_ERR_INVALID_ARG, "cnt, cnt_kv (and idx, idx_kv when top_k > 0) must be non-NULL");
+  if (!aligned16(cnt) || !aligned16(cnt_kv) || (idx && !aligned16(idx)) ||
+      (idx_kv && !aligned16(idx_kv)))
+    return fail(SSA_ERR_INVALID_ARG, "routing buffers must be 16-byte aligned");
+  s = launch_consensus(p, idx, cnt, idx_kv, cnt_kv, static_cast<cudaStream_t>(stream));
+  return s == SSA_OK ? ok() : s;
+}
+
 ssa_status ssa_attend(const ssa_params* p, const void* q, const void* k, const void* v,
                       const int32_t* idx, const int32_t* cnt, void* o, float* lse,
                       ssa_stream_t stream) {
@@ -404,13 +471,25 @@ ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* ksum = reinterpret_cast<float*>(ws + w.ksum);
   float* qsum = reinterpret_cast<float*>(ws + w.qsum);
-  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + w.idx);
-  int32_t* cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(ws + w.cnt);
+  // the lists attend reads: per head, or per KV group with consensus routing;
+  // the caller's idx_out / cnt_out receive them when given
+  int32_t* idx_h = reinterpret_cast<int32_t*>(ws + w.idx);
+  int32_t* cnt_h = reinterpret_cast<int32_t*>(ws + w.cnt);
+  int32_t* idx_a = p->consensus ? reinterpret_cast<int32_t*>(ws + w.idx_kv) : idx_h;
+  int32_t* cnt_a = p->consensus ? reinterpret_cast<int32_t*>(ws + w.cnt_kv) : cnt_h;
+  if (idx_out) idx_a = idx_out;
+  if (cnt_out) cnt_a = cnt_out;
+  if (!p->consensus) {
+    idx_h = idx_a;
+    cnt_h = cnt_a;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = launch_pool(p, k, p->Hkv, p->block_k, ksum, q, p->Hq, p->block_q, qsum, st)) != SSA_OK)
     return s;
-  if ((s = launch_route(p, qsum, ksum, idx, cnt, st)) != SSA_OK) return s;
-  if ((s = launch_attend(p, q, k, v, idx, cnt, o, lse, st)) != SSA_OK) return s;
+  if ((s = launch_route(p, qsum, ksum, idx_h, cnt_h, st)) != SSA_OK) return s;
+  if (p->consensus && (s = launch_consensus(p, idx_h, cnt_h, idx_a, cnt_a, st)) != SSA_OK)
+    return s;
+  if ((s = launch_attend(p, q, k, v, idx_a, cnt_a, o, lse, st)) != SSA_OK) return s;
   return ok();
 }
 

@@ -15,7 +15,8 @@ import torch
 
 __all__ = [
     "Params", "SsaError", "lib", "make_params", "params_of", "workspace_size", "block_summary",
-    "route", "attend", "forward", "forward_host", "check_error", "probe_wait_timeout",
+    "route", "route_consensus", "attend", "forward", "forward_host", "check_error",
+    "probe_wait_timeout",
     "declared_functions", "LIB_PATH", "HEADER_PATH",
 ]
 
@@ -40,7 +41,7 @@ class Params(ctypes.Structure):
         ("N", ctypes.c_int32), ("D", ctypes.c_int32), ("block_k", ctypes.c_int32),
         ("block_q", ctypes.c_int32), ("top_k", ctypes.c_int32), ("window", ctypes.c_int32),
         ("causal", ctypes.c_int32), ("scale", ctypes.c_float),
-        ("wait_timeout_us", ctypes.c_int32),
+        ("wait_timeout_us", ctypes.c_int32), ("consensus", ctypes.c_int32),
     ]
 
     @property
@@ -51,17 +52,23 @@ class Params(ctypes.Structure):
     def n_qblocks(self) -> int:
         return self.N // self.block_q
 
+    @property
+    def list_heads(self) -> int:
+        """Heads the attended lists span: Hkv with consensus routing, else Hq."""
+        return self.Hkv if self.consensus else self.Hq
+
 
 def make_params(B, Hq, Hkv, N, D, block_k, block_q, top_k, window, causal, scale=0.0,
-                wait_timeout_us=0) -> Params:
+                wait_timeout_us=0, consensus=False) -> Params:
     return Params(B, Hq, Hkv, N, D, block_k, block_q, top_k, window, int(bool(causal)),
-                  float(scale), wait_timeout_us)
+                  float(scale), wait_timeout_us, int(bool(consensus)))
 
 
 def params_of(w, **over) -> Params:
     """Params from any object with the workload field names."""
     f = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=w.N, D=w.D, block_k=w.block_k, block_q=w.block_q,
-             top_k=w.top_k, window=w.window, causal=w.causal, scale=getattr(w, "scale", 0.0))
+             top_k=w.top_k, window=w.window, causal=w.causal, scale=getattr(w, "scale", 0.0),
+             consensus=getattr(w, "consensus", False))
     f.update(over)
     return make_params(**f)
 
@@ -84,6 +91,7 @@ def lib() -> ctypes.CDLL:
         "ssa_workspace_size": (sz, [P]),
         "ssa_block_summary": (i32, [P, vp, i32, i32, vp, vp]),
         "ssa_route": (i32, [P, vp, vp, vp, vp, vp]),
+        "ssa_route_consensus": (i32, [P, vp, vp, vp, vp, vp]),
         "ssa_attend": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ssa_forward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_check_error": (i32, [vp]),
@@ -156,13 +164,27 @@ def route(qsum: torch.Tensor, ksum: torch.Tensor, p: Params):
     return idx, cnt
 
 
+def route_consensus(idx: torch.Tensor, cnt: torch.Tensor, p: Params):
+    """Per-group consensus lists from per-head lists:
+    (idx_kv int32 [B, Hkv, NQB, top_k], cnt_kv int32 [B, Hkv, NQB])."""
+    _need(idx, torch.int32, (p.B, p.Hq, p.n_qblocks, p.top_k), "idx")
+    _need(cnt, torch.int32, (p.B, p.Hq, p.n_qblocks), "cnt")
+    dev = cnt.device
+    idx_kv = torch.empty((p.B, p.Hkv, p.n_qblocks, p.top_k), dtype=torch.int32, device=dev)
+    cnt_kv = torch.empty((p.B, p.Hkv, p.n_qblocks), dtype=torch.int32, device=dev)
+    _check(lib().ssa_route_consensus(ctypes.byref(p), _ptr(idx) if p.top_k else None, _ptr(cnt),
+                                     _ptr(idx_kv) if p.top_k else None, _ptr(cnt_kv), _stream()))
+    return idx_kv, cnt_kv
+
+
 def attend(q, k, v, idx, cnt, p: Params, with_lse: bool = True):
-    """(o bf16 [B, Hq, N, D], lse fp32 [B, Hq, N] or None)."""
+    """(o bf16 [B, Hq, N, D], lse fp32 [B, Hq, N] or None).  idx/cnt span Hq
+    heads, or Hkv groups with ``p.consensus``."""
     _need(q, torch.bfloat16, (p.B, p.Hq, p.N, p.D), "q")
     _need(k, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "k")
     _need(v, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "v")
-    _need(idx, torch.int32, (p.B, p.Hq, p.n_qblocks, p.top_k), "idx")
-    _need(cnt, torch.int32, (p.B, p.Hq, p.n_qblocks), "cnt")
+    _need(idx, torch.int32, (p.B, p.list_heads, p.n_qblocks, p.top_k), "idx")
+    _need(cnt, torch.int32, (p.B, p.list_heads, p.n_qblocks), "cnt")
     o = torch.empty_like(q)
     lse = torch.empty((p.B, p.Hq, p.N), dtype=torch.float32, device=q.device) if with_lse else None
     _check(lib().ssa_attend(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
@@ -175,7 +197,8 @@ def forward(q, k, v, p: Params, workspace: torch.Tensor | None = None, with_lse:
             out: torch.Tensor | None = None, lse_out: torch.Tensor | None = None,
             idx_out: torch.Tensor | None = None, cnt_out: torch.Tensor | None = None):
     """Whole path in one library call.  Returns (o, lse, idx, cnt); idx/cnt are
-    the caller's ``idx_out``/``cnt_out`` if given, else fresh tensors."""
+    the lists attend used (per KV group with ``p.consensus``), in the caller's
+    ``idx_out``/``cnt_out`` if given, else in fresh tensors."""
     _need(q, torch.bfloat16, (p.B, p.Hq, p.N, p.D), "q")
     _need(k, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "k")
     _need(v, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "v")
@@ -187,9 +210,11 @@ def forward(q, k, v, p: Params, workspace: torch.Tensor | None = None, with_lse:
     lse = lse_out if lse_out is not None else (
         torch.empty((p.B, p.Hq, p.N), dtype=torch.float32, device=dev) if with_lse else None)
     idx = idx_out if idx_out is not None else torch.empty(
-        (p.B, p.Hq, p.n_qblocks, max(p.top_k, 0)), dtype=torch.int32, device=dev)
+        (p.B, p.list_heads, p.n_qblocks, max(p.top_k, 0)), dtype=torch.int32, device=dev)
     cnt = cnt_out if cnt_out is not None else torch.empty(
-        (p.B, p.Hq, p.n_qblocks), dtype=torch.int32, device=dev)
+        (p.B, p.list_heads, p.n_qblocks), dtype=torch.int32, device=dev)
+    _need(idx, torch.int32, (p.B, p.list_heads, p.n_qblocks, max(p.top_k, 0)), "idx_out")
+    _need(cnt, torch.int32, (p.B, p.list_heads, p.n_qblocks), "cnt_out")
     _check(lib().ssa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                              _ptr(idx) if p.top_k else None, _ptr(cnt), _ptr(workspace),
                              workspace.numel(), _stream()))
@@ -213,7 +238,9 @@ def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
     device on one copy stream, each head's forward (one ``ssa_forward`` on the
     head's slice, B = Hq = Hkv = 1) runs on the compute stream as soon as its
     inputs have landed, and its O returns on a second copy stream while later
-    heads are still arriving or computing.  ``dev_bufs`` may hold
+    heads are still arriving or computing.  With consensus routing the heads
+    of a group depend on one another, so the unit is the (batch, KV head)
+    group (Hq = g, Hkv = 1).  ``dev_bufs`` may hold
     preallocated device tensors and streams to reuse between calls.  The call
     returns once all work is queued; the caller's current stream waits for it.
     """
@@ -224,8 +251,10 @@ def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
             d[name] = torch.empty(src.shape, dtype=src.dtype, device=dev)
     if "o" not in d:
         d["o"] = torch.empty(q_host.shape, dtype=torch.bfloat16, device=dev)
-    sub = make_params(1, 1, 1, p.N, p.D, p.block_k, p.block_q, p.top_k, p.window, p.causal,
-                      p.scale, p.wait_timeout_us)
+    grp = p.Hq // p.Hkv
+    unit = grp if p.consensus else 1          # query heads per sub-problem
+    sub = make_params(1, unit, 1, p.N, p.D, p.block_k, p.block_q, p.top_k, p.window, p.causal,
+                      p.scale, p.wait_timeout_us, p.consensus)
     if "ws" not in d:
         d["ws"] = torch.empty(workspace_size(sub), dtype=torch.uint8, device=dev)
     if "streams" not in d:
@@ -234,7 +263,6 @@ def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
     compute = torch.cuda.current_stream(dev)
     s_in.wait_stream(compute)       # buffers may still be read by earlier work
     s_out.wait_stream(compute)
-    grp = p.Hq // p.Hkv
     q, k, v, o = d["q"], d["k"], d["v"], d["o"]
     row = p.N * p.D * 2             # bytes of one head
     for b in range(p.B):
@@ -242,9 +270,10 @@ def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
             with torch.cuda.stream(s_in):
                 k[b, g].copy_(k_host[b, g], non_blocking=True)
                 v[b, g].copy_(v_host[b, g], non_blocking=True)
-            for h in range(g * grp, (g + 1) * grp):
+            for h in range(g * grp, (g + 1) * grp, unit):
+                hs = slice(h, h + unit)
                 with torch.cuda.stream(s_in):
-                    q[b, h].copy_(q_host[b, h], non_blocking=True)
+                    q[b, hs].copy_(q_host[b, hs], non_blocking=True)
                     ready = torch.cuda.Event()
                     ready.record(s_in)
                 compute.wait_event(ready)
@@ -257,7 +286,7 @@ def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
                 done.record(compute)
                 s_out.wait_event(done)
                 with torch.cuda.stream(s_out):
-                    o_host[b, h].copy_(o[b, h], non_blocking=True)
+                    o_host[b, hs].copy_(o[b, hs], non_blocking=True)
     compute.wait_stream(s_out)
     compute.wait_stream(s_in)
     return o_host

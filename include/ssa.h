@@ -67,6 +67,10 @@ typedef struct {
   int32_t causal;          /* 1 causal (requires W >= 1); 0 non-causal (W = 0, k >= 1) */
   float scale;             /* softmax scale; 0 -> 1/sqrt(D)                    */
   int32_t wait_timeout_us; /* bound on every device-side wait; 0 -> 2 s        */
+  int32_t consensus;       /* 0: each query head attends over its own routed
+                              blocks; 1: the query heads of a KV group share
+                              one consensus list (ssa_route_consensus);
+                              requires (Hq / Hkv) * top_k <= 512            */
 } ssa_params;
 
 /* Bytes of device workspace ssa_forward needs for these parameters:
@@ -99,6 +103,26 @@ ssa_status ssa_block_summary(const ssa_params* p, const void* x, int32_t H,
 ssa_status ssa_route(const ssa_params* p, const float* qsum, const float* ksum,
                      int32_t* idx, int32_t* cnt, ssa_stream_t stream);
 
+/* GQA-shared consensus route (jonsmirl/ssa README, "Complete 10M transformer
+ * result": one route formed across heads by consensus, carrying the blocks
+ * with the most votes; "Mathematical status": a highest-count reservoir keeps
+ * the items the per-head selectors voted for most often).  Every query head
+ * of a KV group votes once for each block of its own list; the group keeps
+ * the first min(top_k, #voted blocks) blocks in the order (votes descending,
+ * block index ascending) -- the method's lower-index tie rule.
+ *   idx/cnt        per-head lists as written by ssa_route: int32
+ *                  [B, Hq, N/Bq, top_k] and [B, Hq, N/Bq] (device)
+ *   idx_kv/cnt_kv  int32 [B, Hkv, N/Bq, top_k] and [B, Hkv, N/Bq] (device,
+ *                  out): the group's blocks ascending, padded with -1, and
+ *                  their count.  KV head kv's group is query heads
+ *                  kv*g .. kv*g + g - 1, g = Hq / Hkv.
+ * Requires (Hq / Hkv) * top_k <= 512 (SSA_ERR_UNSUPPORTED otherwise).  Lists
+ * with a count outside 0..top_k or a block outside 0..N/Bk-1 are reported
+ * through ssa_check_error (SSA_ERR_DEVICE_CHECK) and the bad entries skipped.
+ * One launch; p->consensus is not consulted. */
+ssa_status ssa_route_consensus(const ssa_params* p, const int32_t* idx, const int32_t* cnt,
+                               int32_t* idx_kv, int32_t* cnt_kv, ssa_stream_t stream);
+
 /* Attend (step 4; jonsmirl/ssa README, introduction: ordinary softmax over
  * the selected keys; "Mathematical status": the routed set is cut at each
  * query's position).  For query i in query block qb the key set is
@@ -107,7 +131,10 @@ ssa_status ssa_route(const ssa_params* p, const float* qsum, const float* ksum,
  * counted once each; o_i = softmax(scale * q_i . k_j) . v_j over the set.
  *   q, k, v  bf16 (device), layouts above
  *   idx/cnt  as written by ssa_route (any valid lists: ascending, distinct,
- *            admissible, cnt <= top_k)
+ *            admissible, cnt <= top_k); with p->consensus the per-group
+ *            lists of ssa_route_consensus, [B, Hkv, N/Bq, top_k] and
+ *            [B, Hkv, N/Bq], used by every query head of the group (the
+ *            kernel then packs two heads of a group into one tile)
  *   o        bf16 [B, Hq, N, D] (device, out), round-to-nearest-even
  *   lse      fp32 [B, Hq, N] (device, out, may be NULL): natural-log
  *            log-sum-exp of the scaled logits over the key set
@@ -117,9 +144,11 @@ ssa_status ssa_attend(const ssa_params* p, const void* q, const void* k, const v
                       ssa_stream_t stream);
 
 /* The whole path in one call: summaries of K and Q (one launch), routing,
- * attend.  workspace must hold ssa_workspace_size(p) bytes (device, 256-byte
- * aligned).  idx_out / cnt_out (device, may be NULL) receive the routed lists
- * when given; otherwise they live in the workspace.  lse may be NULL. */
+ * (with p->consensus) the consensus route, attend.  workspace must hold
+ * ssa_workspace_size(p) bytes (device, 256-byte aligned).  idx_out / cnt_out
+ * (device, may be NULL) receive the lists attend used when given -- per head
+ * [B, Hq, N/Bq, top_k], or per KV group [B, Hkv, N/Bq, top_k] with
+ * p->consensus; otherwise they live in the workspace.  lse may be NULL. */
 ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const void* v,
                        void* o, float* lse, int32_t* idx_out, int32_t* cnt_out,
                        void* workspace, size_t workspace_bytes, ssa_stream_t stream);

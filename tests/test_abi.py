@@ -45,6 +45,32 @@ def test_workspace_layout(L):
     assert ssa.workspace_size(p) == a(ks) + a(qs) + a(ix) + a(cn)
 
 
+def test_workspace_layout_with_consensus(L):
+    p = _p(consensus=True)
+    ks = 1 * 2 * 512 * 64 * 4
+    qs = 1 * 14 * 512 * 64 * 4
+    ix = 1 * 14 * 512 * 16 * 4
+    cn = 1 * 14 * 512 * 4
+    a = lambda x: (x + 255) // 256 * 256
+    assert ssa.workspace_size(p) == a(ks) + a(qs) + a(ix) + a(cn) + a(ix // 7) + a(cn // 7)
+
+
+def test_consensus_entry_point_rejects_bad_arguments_before_launch(L):
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    f = L.ssa_route_consensus
+    p = _p()
+    assert f(ctypes.byref(p), good, None, good, good, None) == 1
+    assert f(ctypes.byref(p), good, good, good, None, None) == 1
+    assert f(ctypes.byref(p), odd, good, good, good, None) == 1
+    big = _p(Hq=16, Hkv=1, top_k=33)
+    assert f(ctypes.byref(big), good, good, good, good, None) == 2
+    flag = _p()
+    flag.consensus = 2                   # the flag is 0 or 1
+    assert L.ssa_workspace_size(ctypes.byref(flag)) == 0
+    assert f(ctypes.byref(flag), good, good, good, good, None) == 1
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(D=96), 2), (dict(D=32), 2), (dict(Hq=3, Hkv=2), 1), (dict(N=1000), 2),
     (dict(top_k=65), 2), (dict(top_k=-1), 2), (dict(block_k=48), 2), (dict(block_k=256), 2),
@@ -53,6 +79,7 @@ def test_workspace_layout(L):
     (dict(scale=float("nan")), 1), (dict(scale=-1.0), 1), (dict(wait_timeout_us=-5), 1),
     (dict(N=16 * 2 ** 23, block_k=16, block_q=16, B=1, Hq=1, Hkv=1), 2),
     (dict(window=200000, block_k=16, block_q=16), 2),
+    (dict(consensus=True, Hq=16, Hkv=1, top_k=33), 2),
 ])
 def test_invalid_params_are_rejected_before_launch(L, kw, status):
     p = _p(**kw)
