@@ -51,6 +51,12 @@ __device__ __forceinline__ uint64_t route_key(float s, int c) {
   return (static_cast<uint64_t>(hi) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(c));
 }
 
+// the score a key was made from (inverse of route_key's orderable mapping)
+__device__ __forceinline__ float key_score(uint64_t key) {
+  const uint32_t hi = static_cast<uint32_t>(key >> 32);
+  return __uint_as_float((hi & 0x80000000u) ? (hi & 0x7FFFFFFFu) : ~hi);
+}
+
 __device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
 __device__ __forceinline__ uint64_t umin64(uint64_t a, uint64_t b) { return a < b ? a : b; }
 
@@ -170,17 +176,51 @@ __device__ __forceinline__ void warp_sort_asc_i32(int (&a)[R], int lane) {
   }
 }
 
+// shared-memory bytes of route_kernel<D, R, RT>
+template <int D, int R, int RT>
+__host__ __device__ constexpr size_t route_smem_bytes() {
+  return static_cast<size_t>(D * RT + D * kRouteCands + RT * (kRouteCands + 1)) * 4 +
+         static_cast<size_t>(RT) * (32 * R + 1) * 8 + static_cast<size_t>(RT) * 4;
+}
+
+// admissible key blocks of query block qb: 0 .. limit-1
+__device__ __forceinline__ int route_row_limit(const RouteArgs& a, int qb) {
+  return a.causal ? min(a.NB, static_cast<int>((static_cast<int64_t>(qb) * a.Bq) / a.Bk)) : a.NB;
+}
+
+// this thread's share of the key-summary tile starting at block c0: float4
+// j of the thread is element i = tid + 256 j, i.e. block c0 + i % 64,
+// columns 4 (i / 64) .. 4 (i / 64) + 3
+template <int D, int NPRE>
+__device__ __forceinline__ void route_load_tile(float4 (&pre)[NPRE], const float* ksrc, int c0,
+                                                int NB, int tid) {
+#pragma unroll
+  for (int j = 0; j < NPRE; ++j) {
+    const int i = tid + kRouteThreads * j;
+    const int c = i % kRouteCands, d4 = i / kRouteCands;
+    pre[j] = (c0 + c < NB)
+                 ? *reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(c0 + c) * D + d4 * 4)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
 // RT query blocks per CTA (64, or 16 when 64 would leave SMs idle)
 template <int D, int R, int RT>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a) {
   constexpr int kRouteRows = RT;
+  constexpr int SC_LD = kRouteCands + 1;
+  constexpr int ROWS_PER_WARP = kRouteRows / (kRouteThreads / 32);
+  constexpr int RPT = kRouteRows / 16;      // score rows per thread
+  constexpr int NPRE = (kRouteCands * D / 4) / kRouteThreads;  // float4 per thread per tile
   extern __shared__ __align__(16) float rsm[];
   float* qsT = rsm;                         // [D][RT]   query summaries, transposed
   float* ksT = qsT + D * kRouteRows;        // [D][64]   key summaries, transposed
   float* sc = ksT + D * kRouteCands;        // [RT][65]  score tile
-  constexpr int SC_LD = kRouteCands + 1;
-  constexpr int ROWS_PER_WARP = kRouteRows / (kRouteThreads / 32);
-  constexpr int RPT = kRouteRows / 16;      // score rows per thread
+  // per-row top lists (element e = lane + 32 r of row `row` at
+  // lst[(row * R + r) * 32 + lane], descending), the k-th key, and its score
+  uint64_t* lst = reinterpret_cast<uint64_t*>(sc + kRouteRows * SC_LD);
+  uint64_t* thr_s = lst + kRouteRows * R * 32;
+  float* thrf_s = reinterpret_cast<float*>(thr_s + kRouteRows);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.y;
@@ -190,14 +230,17 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
                           : static_cast<int>(blockIdx.x);
   const int qb0 = rt * kRouteRows;
   const int qb_last = min(qb0 + kRouteRows - 1, a.NQB - 1);
-  const int lim_max =
-      a.top_k == 0 ? 0
-      : a.causal   ? min(a.NB, static_cast<int>((static_cast<int64_t>(qb_last) * a.Bq) / a.Bk))
-                   : a.NB;
+  const int lim_max = a.top_k == 0 ? 0 : route_row_limit(a, qb_last);
   const int n_tiles = (lim_max + kRouteCands - 1) / kRouteCands;
 
   const float* qsrc = a.qsum + static_cast<int64_t>(bh) * a.NQB * D;
   const float* ksrc = a.ksum + static_cast<int64_t>(bkv) * a.NB * D;
+
+  // key-summary tiles go global -> registers one tile ahead, then registers
+  // -> shared memory (transposed) at the top of the next iteration, so the
+  // L2 latency of tile t+1 hides behind the scoring and selection of tile t
+  float4 pre[NPRE];
+  if (n_tiles > 0) route_load_tile<D, NPRE>(pre, ksrc, 0, a.NB, tid);
 
   // query summaries of this row tile, transposed (consecutive threads take
   // consecutive rows so the shared-memory stores do not conflict)
@@ -211,35 +254,28 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     qsT[(d4 * 4 + 2) * kRouteRows + r] = v.z;
     qsT[(d4 * 4 + 3) * kRouteRows + r] = v.w;
   }
-
-  uint64_t list[ROWS_PER_WARP][R];
-  uint64_t thr[ROWS_PER_WARP];
-  int lim[ROWS_PER_WARP];
-#pragma unroll
-  for (int rr = 0; rr < ROWS_PER_WARP; ++rr) {
-#pragma unroll
-    for (int r = 0; r < R; ++r) list[rr][r] = 0ull;
-    thr[rr] = 0ull;
-    const int qb = qb0 + warp * ROWS_PER_WARP + rr;
-    lim[rr] = a.causal ? min(a.NB, static_cast<int>((static_cast<int64_t>(qb) * a.Bq) / a.Bk))
-                       : a.NB;
-    if (qb >= a.NQB) lim[rr] = 0;
+  for (int i = tid; i < kRouteRows * R * 32; i += kRouteThreads) lst[i] = 0ull;
+  for (int i = tid; i < kRouteRows; i += kRouteThreads) {
+    thr_s[i] = 0ull;
+    thrf_s[i] = -INFINITY;
   }
 
   const int ty = tid / 16, tx = tid % 16;
   for (int tile = 0; tile < n_tiles; ++tile) {
     const int c0 = tile * kRouteCands;
-    for (int i = tid; i < kRouteCands * (D / 4); i += kRouteThreads) {
+#pragma unroll
+    for (int j = 0; j < NPRE; ++j) {
+      const int i = tid + kRouteThreads * j;
       const int c = i % kRouteCands, d4 = i / kRouteCands;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + c < a.NB)
-        v = *reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(c0 + c) * D + d4 * 4);
-      ksT[(d4 * 4 + 0) * kRouteCands + c] = v.x;
-      ksT[(d4 * 4 + 1) * kRouteCands + c] = v.y;
-      ksT[(d4 * 4 + 2) * kRouteCands + c] = v.z;
-      ksT[(d4 * 4 + 3) * kRouteCands + c] = v.w;
+      ksT[(d4 * 4 + 0) * kRouteCands + c] = pre[j].x;
+      ksT[(d4 * 4 + 1) * kRouteCands + c] = pre[j].y;
+      ksT[(d4 * 4 + 2) * kRouteCands + c] = pre[j].z;
+      ksT[(d4 * 4 + 3) * kRouteCands + c] = pre[j].w;
     }
+    // the tile is staged, and every warp has finished the previous tile's
+    // selection (it read the score tile that is about to be overwritten)
     __syncthreads();
+    if (tile + 1 < n_tiles) route_load_tile<D, NPRE>(pre, ksrc, c0 + kRouteCands, a.NB, tid);
 
     float acc[RPT][4];
 #pragma unroll
@@ -269,35 +305,54 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
       for (int j = 0; j < 4; ++j) sc[(ty * RPT + i) * SC_LD + tx * 4 + j] = acc[i][j];
     __syncthreads();
 
-#pragma unroll
+    // selection: a row's 64 candidates are first compared, as floats, with
+    // the score of its current k-th key; only when one reaches it is the
+    // row's list brought into registers and the candidates offered as
+    // 64-bit keys (an equal score is settled there by the block index)
+#pragma unroll 1
     for (int rr = 0; rr < ROWS_PER_WARP; ++rr) {
       const int row = warp * ROWS_PER_WARP + rr;
-      if (c0 < lim[rr]) {
+      const int qb = qb0 + row;
+      if (qb >= a.NQB) continue;
+      const int lim = route_row_limit(a, qb);
+      if (c0 >= lim) continue;
+      const float tf = thrf_s[row];
+      const int ca = c0 + lane, cb = c0 + 32 + lane;
+      const float sa = sc[row * SC_LD + lane], sb = sc[row * SC_LD + 32 + lane];
+      const bool pa = ca < lim && sa >= tf;
+      const bool pb = cb < lim && sb >= tf;
+      if (!__any_sync(0xffffffffu, pa || pb)) continue;
+      uint64_t v[R];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int cl = half * 32 + lane;
-          const int c = c0 + cl;
-          const uint64_t key = (c < lim[rr]) ? route_key(sc[row * SC_LD + cl], c) : 0ull;
-          list_offer<R>(list[rr], thr[rr], key, a.top_k, lane);
-        }
+      for (int r = 0; r < R; ++r) v[r] = lst[(row * R + r) * 32 + lane];
+      uint64_t thr = thr_s[row];
+      list_offer<R>(v, thr, pa ? route_key(sa, ca) : 0ull, a.top_k, lane);
+      list_offer<R>(v, thr, pb ? route_key(sb, cb) : 0ull, a.top_k, lane);
+#pragma unroll
+      for (int r = 0; r < R; ++r) lst[(row * R + r) * 32 + lane] = v[r];
+      __syncwarp();
+      if (lane == 0) {
+        thr_s[row] = thr;
+        thrf_s[row] = thr != 0ull ? key_score(thr) : -INFINITY;
       }
+      __syncwarp();
     }
-    __syncthreads();
   }
 
   // epilogue: the first top_k keys, as block indices in ascending order
-#pragma unroll
+#pragma unroll 1
   for (int rr = 0; rr < ROWS_PER_WARP; ++rr) {
-    const int qb = qb0 + warp * ROWS_PER_WARP + rr;
+    const int row = warp * ROWS_PER_WARP + rr;
+    const int qb = qb0 + row;
     if (qb >= a.NQB) continue;
     int vals[R];
     int n_valid = 0;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int e = lane + 32 * r;
-      const bool ok = e < a.top_k && list[rr][r] != 0ull;
-      vals[r] = ok ? static_cast<int>(~static_cast<uint32_t>(list[rr][r] & 0xFFFFFFFFull))
-                   : 0x7FFFFFFF;
+      const uint64_t key = lst[(row * R + r) * 32 + lane];
+      const bool ok = e < a.top_k && key != 0ull;
+      vals[r] = ok ? static_cast<int>(~static_cast<uint32_t>(key & 0xFFFFFFFFull)) : 0x7FFFFFFF;
       n_valid += __popc(__ballot_sync(0xffffffffu, ok));
     }
     warp_sort_asc_i32<R>(vals, lane);

@@ -109,11 +109,6 @@ __device__ __forceinline__ void sorted_insert(T (&arr)[KM], T v) {
   arr[0] = v > arr[0] ? v : arr[0];
 }
 
-__device__ __forceinline__ float key_score(uint64_t key) {
-  const uint32_t hi = static_cast<uint32_t>(key >> 32);
-  return __uint_as_float((hi & 0x80000000u) ? (hi & 0x7FFFFFFFu) : ~hi);
-}
-
 template <int D, int KM>
 __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     route_tc_kernel(const RouteArgs a) {

@@ -192,7 +192,7 @@ ssa_status launch_pool(const ssa_params* p, const void* x0, int32_t H0, int32_t 
 template <int D, int R, int RT>
 cudaError_t launch_route_t(ssa::RouteArgs a, int B, cudaStream_t stream) {
   a.n_row_tiles = (a.NQB + RT - 1) / RT;
-  const size_t smem = static_cast<size_t>(D * RT + D * 64 + RT * 65) * sizeof(float);
+  const size_t smem = ssa::route_smem_bytes<D, R, RT>();
   cudaError_t e = cudaFuncSetAttribute(ssa::route_kernel<D, R, RT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -232,9 +232,10 @@ cudaError_t launch_route_rt(const ssa::RouteArgs& a, int B, cudaStream_t stream)
 }
 
 // The tensor-core router ranks exactly like the fp32 one (see route_tc.cuh).
-// Measured on B200 it wins once the score matrix is large (1M tokens: 6.6 vs
-// 10.6 ms) and loses on small ones (its per-tile steps are latency-bound), so
-// it takes problems with at least 2^26 (query block, key block) pairs.
+// Measured on B200 it wins once its grid of 128-query-block tiles fills the
+// GPU and the score matrix is not small (1M tokens: 6.5 vs 12.4 ms; 16K
+// image tokens, 32 heads: 0.35 vs 0.41 ms) and loses when its grid is a
+// fraction of the SMs (32K tokens, 14 heads: 56 CTAs, 0.35 vs 0.07 ms).
 // SSA_ROUTER=fp32 / tc forces one form (the tests run both and compare).
 bool use_tc_router(const ssa_params* p) {
   const char* env = std::getenv("SSA_ROUTER");
@@ -242,7 +243,8 @@ bool use_tc_router(const ssa_params* p) {
   if (p->top_k == 0 || nb > 65535) return false;  // queued candidates are 16-bit offsets
   if (env != nullptr && std::string(env) == "fp32") return false;
   if (env != nullptr && std::string(env) == "tc") return true;
-  return nb * nqb >= (static_cast<int64_t>(1) << 26);
+  const int64_t tc_ctas = static_cast<int64_t>(p->B) * p->Hq * ((nqb + ssa::kRtcRows - 1) / ssa::kRtcRows);
+  return tc_ctas >= 148 && nb * nqb >= (static_cast<int64_t>(1) << 20);
 }
 
 ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksum, int32_t* idx,
