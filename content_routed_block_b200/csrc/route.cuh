@@ -8,6 +8,10 @@
 // deterministic index order is needed to name one top set).  The selected
 // blocks are written in ascending order, padded with -1, with their count.
 //
+// Two selection schemes share the scoring below: route_rows_kernel (top_k <=
+// 32, at the end of this file) keeps a per-thread register list; the
+// warp-list route_kernel serves 32 < top_k <= 64.
+//
 // Design (sm_100a):
 //  * One CTA owns 64 consecutive query blocks of one (b, head) and streams
 //    the key summaries of its KV head in tiles of 64 blocks through shared
@@ -363,6 +367,206 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
       if (e < a.top_k) dst[e] = e < n_valid ? vals[r] : -1;
     }
     if (lane == 0) a.cnt[static_cast<int64_t>(bh) * a.NQB + qb] = n_valid;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Thread-per-row form (top_k <= 32).  The same tiles and the same fp32 scores
+// (sequential FMA over d) as route_kernel, but the selection is per thread:
+// row r of the tile is split among TPR = 256 / RT consecutive threads, each
+// of which keeps the top KM (>= top_k) keys of its candidates in registers,
+// sorted descending.  A candidate first meets a float filter (its score
+// against the score of the thread's KM-th key); only a survivor becomes a
+// 64-bit key and is inserted.  At the end the TPR lists of a row are merged
+// pairwise with shuffles (bitonic merge of two sorted lists keeps the top
+// KM of their union), so every thread of the row holds the row's top KM.
+// ---------------------------------------------------------------------------
+template <int D, int KM, int RT>
+__host__ __device__ constexpr size_t route_rows_smem_bytes() {
+  return static_cast<size_t>(D * RT + D * kRouteCands + RT * (kRouteCands + kRouteThreads / RT)) * 4;
+}
+
+// insert v into a descending array (the smallest falls off the end)
+template <int KM>
+__device__ __forceinline__ void route_sorted_insert(uint64_t (&arr)[KM], uint64_t v) {
+#pragma unroll
+  for (int j = KM - 1; j > 0; --j) arr[j] = (v > arr[j - 1]) ? arr[j - 1] : (v > arr[j] ? v : arr[j]);
+  arr[0] = v > arr[0] ? v : arr[0];
+}
+
+// keep in `a` the top KM of a U b, where a and b are sorted descending and b
+// is the list of lane ^ mask: max(a[i], b[KM-1-i]) is a bitonic sequence
+// holding the top KM, which a bitonic clean-up sorts descending
+template <int KM>
+__device__ __forceinline__ void route_merge_partner(uint64_t (&a)[KM], int mask) {
+  uint64_t b[KM];
+#pragma unroll
+  for (int i = 0; i < KM; ++i) b[i] = __shfl_xor_sync(0xffffffffu, a[i], mask);
+#pragma unroll
+  for (int i = 0; i < KM; ++i) a[i] = umax64(a[i], b[KM - 1 - i]);
+#pragma unroll
+  for (int j = KM / 2; j > 0; j >>= 1) {
+#pragma unroll
+    for (int i = 0; i < KM; ++i) {
+      if ((i & j) == 0) {
+        const uint64_t x = a[i], y = a[i + j];
+        a[i] = umax64(x, y);
+        a[i + j] = umin64(x, y);
+      }
+    }
+  }
+}
+
+template <int D, int KM, int RT>
+__global__ void __launch_bounds__(kRouteThreads) route_rows_kernel(const RouteArgs a) {
+  constexpr int TPR = kRouteThreads / RT;           // threads per row
+  constexpr int CPT = kRouteCands / TPR;            // candidates per thread per tile
+  constexpr int SC_LD = kRouteCands + TPR;          // each thread's span padded by one
+  constexpr int RPT = RT / 16;                      // score rows per thread (FMA tile)
+  constexpr int NPRE = (kRouteCands * D / 4) / kRouteThreads;
+  static_assert(TPR >= 2 && TPR <= 16 && CPT <= 32, "tile shape");
+  extern __shared__ __align__(16) float rsm[];
+  float* qsT = rsm;                   // [D][RT]
+  float* ksT = qsT + D * RT;          // [D][64]
+  float* sc = ksT + D * kRouteCands;  // [RT][SC_LD]: candidate c of the tile at
+                                      // (c / CPT) * (CPT + 1) + c % CPT
+
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / a.Hq, h = bh % a.Hq;
+  const int bkv = b * a.Hkv + h / (a.Hq / a.Hkv);
+  const int rt = a.causal ? (a.n_row_tiles - 1 - static_cast<int>(blockIdx.x))
+                          : static_cast<int>(blockIdx.x);
+  const int qb0 = rt * RT;
+  const int qb_last = min(qb0 + RT - 1, a.NQB - 1);
+  const int lim_max = a.top_k == 0 ? 0 : route_row_limit(a, qb_last);
+  const int n_tiles = (lim_max + kRouteCands - 1) / kRouteCands;
+  const float* qsrc = a.qsum + static_cast<int64_t>(bh) * a.NQB * D;
+  const float* ksrc = a.ksum + static_cast<int64_t>(bkv) * a.NB * D;
+
+  float4 pre[NPRE];
+  if (n_tiles > 0) route_load_tile<D, NPRE>(pre, ksrc, 0, a.NB, tid);
+  for (int i = tid; i < RT * (D / 4); i += kRouteThreads) {
+    const int r = i % RT, d4 = i / RT;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (qb0 + r < a.NQB)
+      v = *reinterpret_cast<const float4*>(qsrc + static_cast<int64_t>(qb0 + r) * D + d4 * 4);
+    qsT[(d4 * 4 + 0) * RT + r] = v.x;
+    qsT[(d4 * 4 + 1) * RT + r] = v.y;
+    qsT[(d4 * 4 + 2) * RT + r] = v.z;
+    qsT[(d4 * 4 + 3) * RT + r] = v.w;
+  }
+
+  // selection state of this thread: row `row`, candidates part * CPT ..
+  const int row = tid / TPR, part = tid % TPR;
+  const int qb = qb0 + row;
+  const int lim = (qb < a.NQB && a.top_k > 0) ? route_row_limit(a, qb) : 0;
+  uint64_t keys[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) keys[j] = 0ull;
+  float thr_f = -INFINITY;  // score of keys[KM-1] once the list is full
+
+  const int ty = tid / 16, tx = tid % 16;
+  for (int tile = 0; tile < n_tiles; ++tile) {
+    const int c0 = tile * kRouteCands;
+#pragma unroll
+    for (int j = 0; j < NPRE; ++j) {
+      const int i = tid + kRouteThreads * j;
+      const int c = i % kRouteCands, d4 = i / kRouteCands;
+      ksT[(d4 * 4 + 0) * kRouteCands + c] = pre[j].x;
+      ksT[(d4 * 4 + 1) * kRouteCands + c] = pre[j].y;
+      ksT[(d4 * 4 + 2) * kRouteCands + c] = pre[j].z;
+      ksT[(d4 * 4 + 3) * kRouteCands + c] = pre[j].w;
+    }
+    __syncthreads();
+    if (tile + 1 < n_tiles) route_load_tile<D, NPRE>(pre, ksrc, c0 + kRouteCands, a.NB, tid);
+
+    float acc[RPT][4];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+    for (int d = 0; d < D; ++d) {
+      const float4 kb = *reinterpret_cast<const float4*>(ksT + d * kRouteCands + tx * 4);
+      const float kv[4] = {kb.x, kb.y, kb.z, kb.w};
+      float qv[RPT];
+      if constexpr (RPT % 4 == 0) {
+#pragma unroll
+        for (int i4 = 0; i4 < RPT / 4; ++i4) {
+          const float4 qa = *reinterpret_cast<const float4*>(qsT + d * RT + ty * RPT + i4 * 4);
+          qv[i4 * 4 + 0] = qa.x; qv[i4 * 4 + 1] = qa.y; qv[i4 * 4 + 2] = qa.z; qv[i4 * 4 + 3] = qa.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) qv[i] = qsT[d * RT + ty * RPT + i];
+      }
+#pragma unroll
+      for (int i = 0; i < RPT; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qv[i], kv[j], acc[i][j]);
+    }
+    {
+      const int cl = tx * 4;  // 4 candidates in one thread span (CPT >= 4)
+      const int pos = (cl / CPT) * (CPT + 1) + cl % CPT;
+#pragma unroll
+      for (int i = 0; i < RPT; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sc[(ty * RPT + i) * SC_LD + pos + j] = acc[i][j];
+    }
+    __syncthreads();
+
+    // selection over this thread's CPT candidates
+    const int cb = c0 + part * CPT;
+    if (cb < lim) {
+      const float* srow = sc + row * SC_LD + part * (CPT + 1);
+      uint32_t m = 0u;
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) m |= ((cb + j < lim) && srow[j] >= thr_f) ? (1u << j) : 0u;
+      while (m) {
+        const int j = __ffs(m) - 1;
+        m &= m - 1;
+        const uint64_t key = route_key(srow[j], cb + j);
+        if (key > keys[KM - 1]) {
+          route_sorted_insert<KM>(keys, key);
+          if (keys[KM - 1] != 0ull) thr_f = key_score(keys[KM - 1]);
+        }
+      }
+    }
+    // the next iteration's __syncthreads (after staging) keeps the score
+    // tile alive until every thread has read it
+  }
+
+  // merge the TPR partial lists of each row (consecutive lanes)
+#pragma unroll
+  for (int mask = 1; mask < TPR; mask <<= 1) route_merge_partner<KM>(keys, mask);
+
+  if (part == 0 && qb < a.NQB) {
+    const int k = a.top_k;
+    int sel[KM];
+    int n = 0;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      const bool real = j < k && keys[j] != 0ull;
+      sel[j] = real ? static_cast<int>(~static_cast<uint32_t>(keys[j] & 0xFFFFFFFFull)) : 0x7FFFFFFF;
+      n += real ? 1 : 0;
+    }
+#pragma unroll
+    for (int x = 1; x < KM; ++x) {
+#pragma unroll
+      for (int y = x; y > 0; --y) {
+        const int lo = min(sel[y - 1], sel[y]), hi = max(sel[y - 1], sel[y]);
+        sel[y - 1] = lo;
+        sel[y] = hi;
+      }
+    }
+    if (k > 0) {
+      int32_t* dst = a.idx + (static_cast<int64_t>(bh) * a.NQB + qb) * k;
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (j < k) dst[j] = j < n ? sel[j] : -1;
+    }
+    a.cnt[static_cast<int64_t>(bh) * a.NQB + qb] = n;
   }
 }
 

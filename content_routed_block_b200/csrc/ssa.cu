@@ -231,11 +231,41 @@ cudaError_t launch_route_rt(const ssa::RouteArgs& a, int B, cudaStream_t stream)
   return launch_route_t<D, R, 64>(a, B, stream);
 }
 
+template <int D, int KM, int RT>
+cudaError_t launch_route_rows_t(ssa::RouteArgs a, int B, cudaStream_t stream) {
+  a.n_row_tiles = (a.NQB + RT - 1) / RT;
+  const size_t smem = ssa::route_rows_smem_bytes<D, KM, RT>();
+  cudaError_t e = cudaFuncSetAttribute(ssa::route_rows_kernel<D, KM, RT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.n_row_tiles, B * a.Hq);
+  ssa::route_rows_kernel<D, KM, RT><<<grid, ssa::kRouteThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int KM>
+cudaError_t launch_route_rows_km(const ssa::RouteArgs& a, int B, cudaStream_t stream) {
+  const int64_t ctas64 = static_cast<int64_t>(B) * a.Hq * ((a.NQB + 63) / 64);
+  if (ctas64 < 2 * 148) return launch_route_rows_t<D, KM, 16>(a, B, stream);
+  return launch_route_rows_t<D, KM, 64>(a, B, stream);
+}
+
+// fp32 router: thread-per-row selection for top_k <= 32, warp lists beyond
+template <int D>
+cudaError_t launch_route_fp32(const ssa::RouteArgs& a, int B, cudaStream_t stream) {
+  if (a.top_k <= 8) return launch_route_rows_km<D, 8>(a, B, stream);
+  if (a.top_k <= 16) return launch_route_rows_km<D, 16>(a, B, stream);
+  if (a.top_k <= 32) return launch_route_rows_km<D, 32>(a, B, stream);
+  return launch_route_rt<D, 2>(a, B, stream);
+}
+
 // The tensor-core router ranks exactly like the fp32 one (see route_tc.cuh).
-// Measured on B200 it wins once its grid of 128-query-block tiles fills the
-// GPU and the score matrix is not small (1M tokens: 6.5 vs 12.4 ms; 16K
-// image tokens, 32 heads: 0.35 vs 0.41 ms) and loses when its grid is a
-// fraction of the SMs (32K tokens, 14 heads: 56 CTAs, 0.35 vs 0.07 ms).
+// Measured on B200 (fp32 form = thread-per-row selection): it wins once the
+// score matrix is large (1M tokens: 6.5 vs 10.3 ms) and loses on smaller ones
+// (16K image tokens, 32 heads: 0.35 vs 0.27 ms; 32K tokens: 0.35 vs 0.07 ms),
+// where its per-tile steps are latency-bound, so it takes problems with at
+// least 2^26 (query block, key block) pairs per head.
 // SSA_ROUTER=fp32 / tc forces one form (the tests run both and compare).
 bool use_tc_router(const ssa_params* p) {
   const char* env = std::getenv("SSA_ROUTER");
@@ -243,8 +273,7 @@ bool use_tc_router(const ssa_params* p) {
   if (p->top_k == 0 || nb > 65535) return false;  // queued candidates are 16-bit offsets
   if (env != nullptr && std::string(env) == "fp32") return false;
   if (env != nullptr && std::string(env) == "tc") return true;
-  const int64_t tc_ctas = static_cast<int64_t>(p->B) * p->Hq * ((nqb + ssa::kRtcRows - 1) / ssa::kRtcRows);
-  return tc_ctas >= 148 && nb * nqb >= (static_cast<int64_t>(1) << 20);
+  return nb * nqb >= (static_cast<int64_t>(1) << 26);
 }
 
 ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksum, int32_t* idx,
@@ -267,11 +296,9 @@ ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksu
   cudaError_t e;
   if (use_tc_router(p)) {
     e = p->D == 64 ? launch_route_tc<64>(a, p->B, stream) : launch_route_tc<128>(a, p->B, stream);
-  } else if (p->D == 64)
-    e = p->top_k <= 32 ? launch_route_rt<64, 1>(a, p->B, stream) : launch_route_rt<64, 2>(a, p->B, stream);
-  else
-    e = p->top_k <= 32 ? launch_route_rt<128, 1>(a, p->B, stream)
-                       : launch_route_rt<128, 2>(a, p->B, stream);
+  } else {
+    e = p->D == 64 ? launch_route_fp32<64>(a, p->B, stream) : launch_route_fp32<128>(a, p->B, stream);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "route_kernel launch");
   return SSA_OK;
 }
