@@ -66,6 +66,7 @@ class Workload:
     needles: int = 64          # needles only
     needle_gap: int = 4096     # needles only: minimum query-after-key distance
     consensus: bool = False    # one route per (batch, KV head, query block), voted by its heads
+    beta: float = 0.0          # weight of the second-cumulant routing term
 
     @property
     def n_kblocks(self) -> int:

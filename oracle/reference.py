@@ -23,7 +23,11 @@ non-causal variant):
    that end at or before the block's first query, (c+1)*Bk <= qb*Bq, so no
    summary averages a future key; non-causal -- every key block.
 5. Score s_c = <qbar, mu_c> (unscaled: a positive scale does not change the
-   ranking).
+   ranking).  With the second-cumulant weight beta != 0 (SSA's full score
+   r_c(q) = <q, mu_c> + (beta/2) q^T Sigma_c q), a query block scores by the
+   mean of its queries' scores: s_c = <qbar, mu_c> + (beta/2) tr(Sigma_c Q2),
+   Sigma_c the population covariance of block c's keys and Q2 the mean of
+   q_i q_i^T over the block's queries (``block_scores``).
 6. Selection: the first min(top_k, |A|) admissible blocks in the order
    (score descending, block index ascending) -- ties go to the lower index --
    stored ascending by block index, padded with -1, with their count.
@@ -58,6 +62,7 @@ __all__ = [
     "RouteResult", "key_set", "attend_masked_dense", "attend_gathered", "forward",
     "near_tie_rows", "acceptable_selections", "route_row",
     "consensus_row", "route_consensus", "expand_consensus",
+    "block_covariance", "block_second_moment", "block_scores",
 ]
 
 NEAR_TIE_REL = 1e-4   # relative score gap under which two blocks count as tied
@@ -78,6 +83,7 @@ class Params:
     causal: bool
     scale: float = 0.0          # 0 -> 1/sqrt(D)
     consensus: bool = False     # GQA-shared (consensus) routing, see route_consensus
+    beta: float = 0.0           # weight of the second-cumulant score term, see block_scores
 
     @property
     def group(self) -> int:
@@ -100,7 +106,7 @@ class Params:
         """Build from any object with the same field names (e.g. a workload)."""
         return Params(w.B, w.Hq, w.Hkv, w.N, w.D, w.block_k, w.block_q, w.top_k,
                       w.window, bool(w.causal), getattr(w, "scale", 0.0),
-                      bool(getattr(w, "consensus", False)))
+                      bool(getattr(w, "consensus", False)), float(getattr(w, "beta", 0.0)))
 
 
 def upcast_bf16(u16: np.ndarray) -> np.ndarray:
@@ -143,6 +149,46 @@ def admissible_blocks(qb: int, p: Params) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# second-cumulant summaries (the beta term of the routing score)
+# --------------------------------------------------------------------------
+def block_covariance(x: np.ndarray, block: int) -> np.ndarray:
+    """Second cumulant of every block of ``block`` rows of ``x[..., N, D]``:
+    Sigma_c = (1/block) sum_t (x_t - mu_c)(x_t - mu_c)^T, the population
+    covariance of the block's keys.  Returns [..., N/block, D, D].
+
+    jonsmirl/ssa README, "Algorithm and complexity": the second-cumulant
+    routing score r_c(q) = <q, mu_c> + (beta/2) q^T Sigma_c q."""
+    n, d = x.shape[-2], x.shape[-1]
+    if n % block:
+        raise ValueError("sequence length must be a multiple of the block size")
+    xb = x.reshape(*x.shape[:-2], n // block, block, d)
+    c = xb - xb.mean(axis=-2, keepdims=True)
+    return np.einsum("...td,...te->...de", c, c) / block
+
+
+def block_second_moment(x: np.ndarray, block: int) -> np.ndarray:
+    """(1/block) sum_t x_t x_t^T for every block of ``block`` rows:
+    [..., N/block, D, D].  Averaging q^T Sigma q over a query block's queries
+    gives tr(Sigma Q2) with Q2 this moment."""
+    n, d = x.shape[-2], x.shape[-1]
+    if n % block:
+        raise ValueError("sequence length must be a multiple of the block size")
+    xb = x.reshape(*x.shape[:-2], n // block, block, d)
+    return np.einsum("...td,...te->...de", xb, xb) / block
+
+
+def block_scores(qbar, mu, cand, beta: float = 0.0, q2=None, sigma=None) -> np.ndarray:
+    """Routing scores of the candidate blocks ``cand`` for one query block:
+    s_c = <qbar, mu_c> + (beta/2) tr(Sigma_c Q2), the mean over the block's
+    queries of SSA's r_c(q_i) = <q_i, mu_c> + (beta/2) q_i^T Sigma_c q_i
+    (both terms are linear in q q^T).  With beta = 0 only the means enter."""
+    s = mu[cand] @ qbar
+    if beta != 0.0:
+        s = s + 0.5 * beta * np.einsum("cde,de->c", sigma[cand], q2)
+    return s
+
+
+# --------------------------------------------------------------------------
 # steps 5-6: scores and top-k
 # --------------------------------------------------------------------------
 @dataclass
@@ -153,13 +199,15 @@ class RouteResult:
     next: np.ndarray       # float64 [B, Hq, NQB]: (k+1)-th best score (nan if none)
 
 
-def route_row(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, top_k: int):
-    """Select from candidate blocks ``cand`` for one query-block summary.
+def route_row(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, top_k: int,
+              beta: float = 0.0, q2=None, sigma=None):
+    """Select from candidate blocks ``cand`` for one query-block summary
+    (scores from ``block_scores``; ``q2``/``sigma`` only when beta != 0).
 
     Returns (selected ascending, k-th score, (k+1)-th score)."""
     if len(cand) == 0 or top_k == 0:
         return np.zeros(0, dtype=np.int64), math.nan, math.nan
-    s = mu[cand] @ qbar
+    s = block_scores(qbar, mu, cand, beta, q2, sigma)
     # order: score descending, then block index ascending (lower index wins a tie)
     order = np.lexsort((cand, -s))
     take = min(top_k, len(cand))
@@ -169,13 +217,16 @@ def route_row(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, top_k: int):
     return chosen, kth, nxt
 
 
-def route(qsum: np.ndarray, ksum: np.ndarray, p: Params, rows=None) -> RouteResult:
+def route(qsum: np.ndarray, ksum: np.ndarray, p: Params, rows=None, qm2=None,
+          kcov=None) -> RouteResult:
     """Top-k routing for every (b, query head, query block).
 
     ``qsum`` [B, Hq, NQB, D] and ``ksum`` [B, Hkv, NB, D] are block summaries
-    (float64).  ``rows`` optionally restricts the work to a list of
-    (b, h, qb) triples; the arrays keep their full shape and rows not listed
-    stay at idx = -1, cnt = 0, scores nan."""
+    (float64); with ``p.beta`` != 0 also ``qm2`` [B, Hq, NQB, D, D]
+    (``block_second_moment`` of Q) and ``kcov`` [B, Hkv, NB, D, D]
+    (``block_covariance`` of K).  ``rows`` optionally restricts the work to a
+    list of (b, h, qb) triples; the arrays keep their full shape and rows not
+    listed stay at idx = -1, cnt = 0, scores nan."""
     nqb = p.n_qblocks
     idx = np.full((p.B, p.Hq, nqb, p.top_k), -1, dtype=np.int32)
     cnt = np.zeros((p.B, p.Hq, nqb), dtype=np.int32)
@@ -185,7 +236,10 @@ def route(qsum: np.ndarray, ksum: np.ndarray, p: Params, rows=None) -> RouteResu
         (b, h, qb) for b in range(p.B) for h in range(p.Hq) for qb in range(nqb)]
     for b, h, qb in todo:
         mu = ksum[b, h // p.group]
-        sel, a, c = route_row(qsum[b, h, qb], mu, admissible_blocks(qb, p), p.top_k)
+        extra = {}
+        if p.beta != 0.0:
+            extra = dict(beta=p.beta, q2=qm2[b, h, qb], sigma=kcov[b, h // p.group])
+        sel, a, c = route_row(qsum[b, h, qb], mu, admissible_blocks(qb, p), p.top_k, **extra)
         idx[b, h, qb, :len(sel)] = sel
         cnt[b, h, qb] = len(sel)
         kth[b, h, qb], nxt[b, h, qb] = a, c
@@ -203,7 +257,8 @@ def near_tie_rows(r: RouteResult, rel: float = NEAR_TIE_REL) -> np.ndarray:
 
 
 def acceptable_selections(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, top_k: int,
-                          rel: float = NEAR_TIE_REL, limit: int = 256) -> list:
+                          rel: float = NEAR_TIE_REL, limit: int = 256, beta: float = 0.0,
+                          q2=None, sigma=None) -> list:
     """Every selection that the near-tie rule accepts, ascending.
 
     Scores are fp64.  Let s_k be the k-th best score.  Blocks whose score is
@@ -214,7 +269,7 @@ def acceptable_selections(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, to
     import itertools
     if len(cand) == 0 or top_k == 0:
         return [np.zeros(0, dtype=np.int64)]
-    s = mu[cand] @ qbar
+    s = block_scores(qbar, mu, cand, beta, q2, sigma)
     order = np.lexsort((cand, -s))
     take = min(top_k, len(cand))
     sk = s[order[take - 1]]
@@ -373,7 +428,11 @@ def forward(q, k, v, p: Params, form: str = "dense"):
     head of a group attends over its group's list."""
     ksum = block_summary(k, p.block_k)
     qsum = block_summary(q, p.block_q)
-    r = route(qsum, ksum, p)
+    if p.beta != 0.0:
+        r = route(qsum, ksum, p, qm2=block_second_moment(q, p.block_q),
+                  kcov=block_covariance(k, p.block_k))
+    else:
+        r = route(qsum, ksum, p)
     attend = attend_masked_dense if form == "dense" else attend_gathered
     if p.consensus:
         idx, cnt = route_consensus(r.idx, r.cnt, p)

@@ -497,3 +497,77 @@ def test_consensus_worked_example_matches_hand_derivation(form):
             assert out["o"][0, int(h), int(i), 1] == pytest.approx(1.0, abs=1e-12)
             n += 1
     assert n == 16
+
+
+# ---------------------------------------------------------------- second-cumulant score
+def test_block_covariance_and_second_moment_match_numpy():
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((2, 3, 48, 5))
+    cov = O.block_covariance(x, 8)
+    m2 = O.block_second_moment(x, 8)
+    for b in range(2):
+        for h in range(3):
+            for c in range(6):
+                xb = x[b, h, c * 8:(c + 1) * 8]
+                np.testing.assert_allclose(cov[b, h, c], np.cov(xb.T, bias=True), atol=1e-13)
+                np.testing.assert_allclose(m2[b, h, c], xb.T @ xb / 8, atol=1e-13)
+    # a block of one row has no spread
+    assert np.abs(O.block_covariance(x, 1)).max() == 0.0
+
+
+def test_second_cumulant_route_matches_hand_derivation():
+    k = np.array([[0, 0], [0, 0], [1, 0], [-1, 0], [0.5, 0], [0.5, 0], [0, 1], [0, 1]],
+                 dtype=np.float64)[None, None]
+    q = np.zeros((1, 1, 8, 2))
+    q[0, 0, 6] = (2.0, 0.0)
+    v = np.stack([np.arange(8.0), np.ones(8)], axis=1)[None, None]
+    n = 0
+    with open(os.path.join(GOLDEN, "second_cumulant_route.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            beta, kk, want = float(parts[0]), int(parts[1]), [int(c) for c in parts[2:]]
+            p = _params(top_k=kk, beta=beta)
+            out = O.forward(q, k, v, p)
+            assert out["idx"][0, 0, 3, :kk].tolist() == want, (beta, kk)
+            n += 1
+    assert n == 9
+
+
+def test_block_score_is_the_mean_of_per_query_scores():
+    # brute force over the block's queries of r_c(q_i) = <q_i, mu_c> + (beta/2) q_i^T Sigma_c q_i
+    rng = np.random.default_rng(32)
+    D, Bk, Bq = 6, 4, 8
+    k = rng.standard_normal((1, 1, 64, D))
+    q = rng.standard_normal((1, 1, 64, D))
+    mu, cov = O.block_summary(k, Bk), O.block_covariance(k, Bk)
+    qbar, qm2 = O.block_summary(q, Bq), O.block_second_moment(q, Bq)
+    cand = np.arange(16)
+    for beta in (0.0, 0.7, -1.3):
+        for qb in range(8):
+            got = O.block_scores(qbar[0, 0, qb], mu[0, 0], cand, beta, qm2[0, 0, qb], cov[0, 0])
+            rows = q[0, 0, qb * Bq:(qb + 1) * Bq]
+            want = np.zeros(16)
+            for c in cand:
+                kc = k[0, 0, c * Bk:(c + 1) * Bk]
+                sig = (kc - kc.mean(0)).T @ (kc - kc.mean(0)) / Bk
+                want[c] = np.mean([qi @ kc.mean(0) + 0.5 * beta * qi @ sig @ qi for qi in rows])
+            np.testing.assert_allclose(got, want, atol=1e-12)
+
+
+def test_second_cumulant_with_zero_beta_or_no_spread_is_the_mean_route():
+    rng = np.random.default_rng(33)
+    p0 = _params(B=1, Hq=2, Hkv=1, N=128, D=4, block_k=8, block_q=8, top_k=3, window=8)
+    q, k, v = rng.standard_normal((1, 2, 128, 4)), rng.standard_normal((1, 1, 128, 4)), \
+        rng.standard_normal((1, 1, 128, 4))
+    base = O.forward(q, k, v, p0)
+    # keys constant inside each block: Sigma_c = 0 for every beta
+    kc = np.repeat(k[:, :, ::8], 8, axis=2)
+    flat0 = O.forward(q, kc, v, p0)
+    flat1 = O.forward(q, kc, v, O.Params(**{**p0.__dict__, "beta": 2.5}))
+    np.testing.assert_array_equal(flat0["idx"], flat1["idx"])
+    # and a nonzero beta moves some selections on spread blocks
+    moved = O.forward(q, k, v, O.Params(**{**p0.__dict__, "beta": 4.0}))
+    assert (moved["idx"] != base["idx"]).any()
