@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--seq-len", type=int, default=0,
                     help="run the chosen workload's recipe at another sequence length "
                          "(e.g. a smaller copy of the million-token workload for profiling)")
+    ap.add_argument("--beta", type=float, default=0.0,
+                    help="weight of the second-cumulant routing term (0: mean summaries only)")
     ap.add_argument("--consensus", action="store_true",
                     help="GQA-shared consensus routing: the query heads of a KV group vote "
                          "and share one list per query block")
@@ -208,7 +210,7 @@ def _cpu_worker(args):
     sys.path.insert(0, ROOT)
     import oracle as O
     from content_routed_block_b200.workloads import CONFIGS, make_inputs
-    cfg, seq_len, consensus, b, h, blocks, seconds = args
+    cfg, seq_len, consensus, beta, b, h, blocks, seconds = args
     w = CONFIGS[cfg]
     if seq_len:
         w = w.with_(N=seq_len)
@@ -217,22 +219,28 @@ def _cpu_worker(args):
     # every head of the KV group, which vote on one shared list
     heads = list(range((h // g) * g, (h // g + 1) * g)) if consensus else [h]
     x = make_inputs(w, q_heads=heads, kv_heads=[h // g])
-    sub = w.with_(Hq=len(heads), Hkv=1, B=1, consensus=consensus)
+    sub = w.with_(Hq=len(heads), Hkv=1, B=1, consensus=consensus, beta=beta)
     p = O.Params.of(sub)
     q = O.upcast_bf16(x["q"][b:b + 1])           # the requested heads, in order
     k = O.upcast_bf16(x["k"][b:b + 1])
     v = O.upcast_bf16(x["v"][b:b + 1])
     t0 = time.perf_counter()
     ksum = O.block_summary(k, p.block_k)
+    kcov = O.block_covariance(k[0, 0], p.block_k) if p.beta else None
     done = 0
     nh = len(heads)
     idx = np.full((1, nh, p.n_qblocks, p.top_k), -1, np.int32)
     cnt = np.zeros((1, nh, p.n_qblocks), np.int32)
     for qb in blocks:
         for j in range(nh):
-            qbar = O.block_summary(q[:, j:j + 1, qb * p.block_q:(qb + 1) * p.block_q],
-                                   p.block_q)[0, 0, 0]
-            sel, _, _ = O.route_row(qbar, ksum[0, 0], O.admissible_blocks(qb, p), p.top_k)
+            rows = q[:, j:j + 1, qb * p.block_q:(qb + 1) * p.block_q]
+            qbar = O.block_summary(rows, p.block_q)[0, 0, 0]
+            extra = {}
+            if p.beta:
+                extra = dict(beta=p.beta, q2=O.block_second_moment(rows, p.block_q)[0, 0, 0],
+                             sigma=kcov)
+            sel, _, _ = O.route_row(qbar, ksum[0, 0], O.admissible_blocks(qb, p), p.top_k,
+                                    **extra)
             idx[0, j, qb, :len(sel)] = sel
             cnt[0, j, qb] = len(sel)
         if consensus:
@@ -248,11 +256,12 @@ def _cpu_worker(args):
 
 
 class OraclePool:
-    def __init__(self, cfg: int, seq_len: int = 0, consensus: bool = False):
+    def __init__(self, cfg: int, seq_len: int = 0, consensus: bool = False, beta: float = 0.0):
         import multiprocessing as mp
         self.cfg = cfg
         self.seq_len = seq_len
         self.consensus = consensus
+        self.beta = beta
         self.cores = max(1, min(len(os.sched_getaffinity(0)), 64))
         old = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
         for k in old:
@@ -284,7 +293,7 @@ class OraclePool:
             b = c % w.B
             h = (c // w.B) % w.Hq
             blocks = rng.permutation(nqb).tolist()
-            tasks.append((self.cfg, self.seq_len, self.consensus, b, h, blocks, seconds))
+            tasks.append((self.cfg, self.seq_len, self.consensus, self.beta, b, h, blocks, seconds))
         res = self.pool.map(_cpu_worker, tasks)
         blocks = sum(r[0] for r in res)
         wall = max(r[1] for r in res)
@@ -300,7 +309,7 @@ def run_reference(args):
         return
     w = workload_of(args)
     per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
-    pool = OraclePool(args.config, args.seq_len, args.consensus)
+    pool = OraclePool(args.config, args.seq_len, args.consensus, args.beta)
     try:
         for _ in range(args.warmup):
             pool.run(per_step)
@@ -337,6 +346,8 @@ def workload_of(args):
         w = w.with_(N=args.seq_len, name=f"{w.name}@{args.seq_len}")
     if getattr(args, "consensus", False):
         w = w.with_(consensus=True, name=f"{w.name}+consensus")
+    if getattr(args, "beta", 0.0):
+        w = w.with_(beta=float(args.beta), name=f"{w.name}+beta{args.beta:g}")
     return w
 
 
@@ -344,7 +355,8 @@ def workload_config(w, args):
     return {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} D={w.D} "
                         f"Bk={w.block_k} Bq={w.block_q} top_k={w.top_k} W={w.window} "
                         f"{'causal' if w.causal else 'non-causal'} {w.kind}"
-                        f"{' consensus-routed' if w.consensus else ''}",
+                        f"{' consensus-routed' if w.consensus else ''}"
+                        f"{f' second-cumulant beta={w.beta:g}' if w.beta else ''}",
             "global_batch": w.B * args.gpus, "seq_len": w.N, "parallelism": f"replicas{args.gpus}",
             "l2": "flushed between timed steps (256 MiB write)"}
 
@@ -437,8 +449,11 @@ def run_ssa(args):
     # per-kernel split: the same path as separate calls with events between them
     n_split = min(args.steps, 200)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_split)]
-    ks = torch.empty((w.B, w.Hkv, w.N // w.block_k, w.D), dtype=torch.float32, device=dev)
-    qs = torch.empty((w.B, w.Hq, w.N // w.block_q, w.D), dtype=torch.float32, device=dev)
+    F = w.D + w.D * (w.D + 1) // 2 if w.beta else w.D      # summary / feature length
+    ks = torch.empty((w.B, w.Hkv, w.N // w.block_k, F), dtype=torch.float32, device=dev)
+    qs = torch.empty((w.B, w.Hq, w.N // w.block_q, F), dtype=torch.float32, device=dev)
+    sc = (torch.empty((w.B, w.Hq, w.N // w.block_q, w.N // w.block_k), dtype=torch.float32,
+                      device=dev) if w.beta else None)
     L = ssa.lib()
     import ctypes
     st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -448,18 +463,25 @@ def run_ssa(args):
         flush.zero_()
         e = ev[s]
         e[0].record()
-        assert L.ssa_block_summary(pp, P(kd), w.Hkv, w.block_k, P(ks), st) == 0
-        e[1].record()
-        assert L.ssa_block_summary(pp, P(qd), w.Hq, w.block_q, P(qs), st) == 0
+        if w.beta:
+            assert L.ssa_route_features(pp, P(kd), w.Hkv, w.block_k, 0, P(ks), st) == 0
+            e[1].record()
+            assert L.ssa_route_features(pp, P(qd), w.Hq, w.block_q, 1, P(qs), st) == 0
+        else:
+            assert L.ssa_block_summary(pp, P(kd), w.Hkv, w.block_k, P(ks), st) == 0
+            e[1].record()
+            assert L.ssa_block_summary(pp, P(qd), w.Hq, w.block_q, P(qs), st) == 0
         e[2].record()
+        ri, rc = (idx_h, cnt_h) if w.consensus else (idx, cnt)
+        if w.beta:
+            assert L.ssa_route_cumulant(pp, P(qs), P(ks), P(sc), P(ri) if w.top_k else None,
+                                        P(rc), st) == 0
+        else:
+            assert L.ssa_route(pp, P(qs), P(ks), P(ri) if w.top_k else None, P(rc), st) == 0
+        e[3].record()
         if w.consensus:
-            assert L.ssa_route(pp, P(qs), P(ks), P(idx_h) if w.top_k else None, P(cnt_h), st) == 0
-            e[3].record()
             assert L.ssa_route_consensus(pp, P(idx_h) if w.top_k else None, P(cnt_h),
                                          P(idx) if w.top_k else None, P(cnt), st) == 0
-        else:
-            assert L.ssa_route(pp, P(qs), P(ks), P(idx) if w.top_k else None, P(cnt), st) == 0
-            e[3].record()
         e[4].record()
         assert L.ssa_attend(pp, P(qd), P(kd), P(vd), P(idx) if w.top_k else None, P(cnt),
                             P(o), P(lse), st) == 0
@@ -525,7 +547,7 @@ def run_ssa(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        pool = OraclePool(args.config, args.seq_len, args.consensus)
+        pool = OraclePool(args.config, args.seq_len, args.consensus, args.beta)
         try:
             v, nb, wall = pool.run(args.cpu_seconds)
         finally:
@@ -533,7 +555,8 @@ def run_ssa(args):
         cpu = {"value": v, "unit": UNIT, "cores": pool.cores, "kind": "oracle",
                "sample": f"{nb} (query head, query block) units of this workload (each 1/Hq of "
                          f"the work of {w.block_q} tokens), whole path (summaries, routing"
-                         f"{', consensus' if w.consensus else ''}, masked-dense attend) in "
+                         f"{', consensus' if w.consensus else ''}"
+                         f"{', second-cumulant scores' if w.beta else ''}, masked-dense attend) in "
                          f"float64, {pool.cores} processes x ~{args.cpu_seconds:.0f} s"}
 
     clocks = sampler.summary()
@@ -550,7 +573,8 @@ def run_ssa(args):
         "selected_tflops": tflops,
         "keys_per_query": work["keys_per_query"],
         "nominal_keys_per_query": work["nominal_keys_per_query"],
-        "kernels_ms": {"pool_k": pool_k_ms, "pool_q": pool_q_ms, "route": route_ms,
+        "kernels_ms": {("features_k" if w.beta else "pool_k"): pool_k_ms,
+                       ("features_q" if w.beta else "pool_q"): pool_q_ms, "route": route_ms,
                        **({"consensus": cons_ms} if w.consensus else {}), "attend": attend_ms},
         "roofline": {"bound": roof["bound"], "kernel": "attend_kernel",
                      "achieved": roof["achieved"], "peak": roof["peak"], "unit": roof["unit"],

@@ -19,6 +19,7 @@
 #include "attend.cuh"
 #include "common.cuh"
 #include "consensus.cuh"
+#include "cumulant.cuh"
 #include "pool.cuh"
 #include "route.cuh"
 #include "route_tc.cuh"
@@ -103,6 +104,7 @@ ssa_status validate(const ssa_params* p) {
   if (!(p->scale >= 0.f) || !std::isfinite(p->scale))
     return fail(SSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if (p->wait_timeout_us < 0) return fail(SSA_ERR_INVALID_ARG, "wait_timeout_us must be >= 0");
+  if (!std::isfinite(p->beta)) return fail(SSA_ERR_INVALID_ARG, "beta must be finite");
   if (p->consensus != 0 && p->consensus != 1)
     return fail(SSA_ERR_INVALID_ARG, "consensus must be 0 or 1");
   if (p->consensus && (p->Hq / p->Hkv) * p->top_k > ssa::kConsMaxVotes)
@@ -373,6 +375,91 @@ ssa_status launch_attend(const ssa_params* p, const void* q, const void* k, cons
   return SSA_OK;
 }
 
+// ------------------------------------------------ second-cumulant routing
+int64_t cum_features(const ssa_params* p) { return p->D + static_cast<int64_t>(p->D) * (p->D + 1) / 2; }
+
+template <int D>
+cudaError_t launch_cum_features_t(const ssa::CumFeatArgs& a, cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(a.block) * D * 4 + D * 4 + D * (D + 1) / 2 * 2;
+  cudaError_t e = cudaFuncSetAttribute(ssa::cumulant_features_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  ssa::cumulant_features_kernel<D><<<static_cast<unsigned>(a.n_blocks), ssa::kCumThreads, smem,
+                                     stream>>>(a);
+  return cudaGetLastError();
+}
+
+ssa_status launch_cum_features(const ssa_params* p, const void* x, int32_t H, int32_t block,
+                               int32_t queries, float* out, cudaStream_t stream) {
+  ssa::CumFeatArgs a;
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.out = out;
+  a.n_blocks = static_cast<int64_t>(p->B) * H * (p->N / block);
+  a.block = block;
+  a.queries = queries;
+  a.half_beta = 0.5f * p->beta;
+  if (a.n_blocks > 0x7FFFFFFF) return fail(SSA_ERR_UNSUPPORTED, "too many blocks");
+  if (a.n_blocks == 0) return SSA_OK;
+  const cudaError_t e = p->D == 64 ? launch_cum_features_t<64>(a, stream)
+                                   : launch_cum_features_t<128>(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cumulant_features_kernel launch");
+  return SSA_OK;
+}
+
+ssa_status launch_cum_route(const ssa_params* p, const float* qf, const float* kf, float* scores,
+                            int32_t* idx, int32_t* cnt, cudaStream_t stream) {
+  ssa::CumScoreArgs sa;
+  sa.qf = qf;
+  sa.kf = kf;
+  sa.scores = scores;
+  sa.Hq = p->Hq;
+  sa.Hkv = p->Hkv;
+  sa.NQB = p->N / p->block_q;
+  sa.NB = p->N / p->block_k;
+  sa.Bq = p->block_q;
+  sa.Bk = p->block_k;
+  sa.causal = p->causal;
+  sa.n_row_tiles = (sa.NQB + ssa::kCumTile - 1) / ssa::kCumTile;
+  sa.n_cand_tiles = (sa.NB + ssa::kCumTile - 1) / ssa::kCumTile;
+  cudaError_t e;
+  if (p->top_k > 0) {
+    const int64_t gx = static_cast<int64_t>(sa.n_row_tiles) * sa.n_cand_tiles;
+    const int64_t gy = static_cast<int64_t>(p->B) * p->Hq;
+    if (gx > 0x7FFFFFFF || gy > 65535) return fail(SSA_ERR_UNSUPPORTED, "score grid too large");
+    dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+    if (p->D == 64)
+      ssa::cumulant_scores_kernel<64><<<grid, ssa::kCumThreads, 0, stream>>>(sa);
+    else
+      ssa::cumulant_scores_kernel<128><<<grid, ssa::kCumThreads, 0, stream>>>(sa);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "cumulant_scores_kernel launch");
+  }
+  ssa::CumSelectArgs c;
+  c.scores = scores;
+  c.idx = idx;
+  c.cnt = cnt;
+  c.NQB = sa.NQB;
+  c.NB = sa.NB;
+  c.Bq = p->block_q;
+  c.Bk = p->block_k;
+  c.top_k = p->top_k;
+  c.causal = p->causal;
+  c.n_rows = static_cast<int64_t>(p->B) * p->Hq * sa.NQB;
+  const int64_t grid = (c.n_rows + 7) / 8;
+  if (grid > 0x7FFFFFFF) return fail(SSA_ERR_UNSUPPORTED, "too many query blocks");
+  const unsigned g = static_cast<unsigned>(grid);
+  if (p->top_k <= 8)
+    ssa::cumulant_select_kernel<8><<<g, ssa::kCumThreads, 0, stream>>>(c);
+  else if (p->top_k <= 16)
+    ssa::cumulant_select_kernel<16><<<g, ssa::kCumThreads, 0, stream>>>(c);
+  else if (p->top_k <= 32)
+    ssa::cumulant_select_kernel<32><<<g, ssa::kCumThreads, 0, stream>>>(c);
+  else
+    ssa::cumulant_select_kernel<64><<<g, ssa::kCumThreads, 0, stream>>>(c);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "cumulant_select_kernel launch");
+  return SSA_OK;
+}
+
 ssa_status launch_consensus(const ssa_params* p, const int32_t* idx, const int32_t* cnt,
                             int32_t* idx_kv, int32_t* cnt_kv, cudaStream_t stream) {
   ssa::ConsensusArgs a;
@@ -397,7 +484,7 @@ ssa_status launch_consensus(const ssa_params* p, const int32_t* idx, const int32
 // Workspace of ssa_forward: K and Q summaries, the per-head routed lists and
 // counts, and (consensus routing only) the per-group lists and counts.
 struct WsLayout {
-  size_t ksum, qsum, idx, cnt, idx_kv, cnt_kv, total;
+  size_t ksum, qsum, idx, cnt, idx_kv, cnt_kv, qf, kf, sc, total;
 };
 
 WsLayout ws_layout(const ssa_params* p) {
@@ -415,7 +502,16 @@ WsLayout ws_layout(const ssa_params* p) {
   w.cnt = w.idx + align256(ix);
   w.idx_kv = w.cnt + align256(cn);
   w.cnt_kv = w.idx_kv + align256(ixk);
-  w.total = w.cnt_kv + align256(cnk);
+  // second-cumulant routing: query and key features, and the score matrix
+  const bool cum = p->beta != 0.0f;
+  const size_t F = static_cast<size_t>(cum_features(p));
+  const size_t qfb = cum ? static_cast<size_t>(p->B) * p->Hq * nqb * F * sizeof(float) : 0;
+  const size_t kfb = cum ? static_cast<size_t>(p->B) * p->Hkv * nb * F * sizeof(float) : 0;
+  const size_t scb = cum ? static_cast<size_t>(p->B) * p->Hq * nqb * nb * sizeof(float) : 0;
+  w.qf = w.cnt_kv + align256(cnk);
+  w.kf = w.qf + align256(qfb);
+  w.sc = w.kf + align256(kfb);
+  w.total = w.sc + align256(scb);
   return w;
 }
 
@@ -446,6 +542,9 @@ ssa_status ssa_route(const ssa_params* p, const float* qsum, const float* ksum, 
                      int32_t* cnt, ssa_stream_t stream) {
   ssa_status s = validate(p);
   if (s != SSA_OK) return s;
+  if (p->beta != 0.0f)
+    return fail(SSA_ERR_INVALID_ARG,
+                "beta != 0: route with ssa_route_features and ssa_route_cumulant");
   if (qsum == nullptr || ksum == nullptr || cnt == nullptr || (p->top_k > 0 && idx == nullptr))
     return fail(SSA_ERR_INVALID_ARG, "qsum, ksum, cnt (and idx when top_k > 0) must be non-NULL");
   if (!aligned16(qsum) || !aligned16(ksum) || !aligned16(cnt) || (idx && !aligned16(idx)))
@@ -467,6 +566,35 @@ ssa_status ssa_route_consensus(const ssa_params* p, const int32_t* idx, const in
       (idx_kv && !aligned16(idx_kv)))
     return fail(SSA_ERR_INVALID_ARG, "routing buffers must be 16-byte aligned");
   s = launch_consensus(p, idx, cnt, idx_kv, cnt_kv, static_cast<cudaStream_t>(stream));
+  return s == SSA_OK ? ok() : s;
+}
+
+ssa_status ssa_route_features(const ssa_params* p, const void* x, int32_t H, int32_t block,
+                              int32_t queries, float* out, ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (x == nullptr || out == nullptr) return fail(SSA_ERR_INVALID_ARG, "x and out must be non-NULL");
+  if (!aligned16(x) || !aligned16(out))
+    return fail(SSA_ERR_INVALID_ARG, "x and out must be 16-byte aligned");
+  if (H < 1) return fail(SSA_ERR_INVALID_ARG, "H must be positive");
+  if (queries != 0 && queries != 1) return fail(SSA_ERR_INVALID_ARG, "queries must be 0 or 1");
+  if (!pow2_in(block, 1, 128) || p->N % block != 0)
+    return fail(SSA_ERR_INVALID_ARG, "block must be a power of two <= 128 dividing N");
+  s = launch_cum_features(p, x, H, block, queries, out, static_cast<cudaStream_t>(stream));
+  return s == SSA_OK ? ok() : s;
+}
+
+ssa_status ssa_route_cumulant(const ssa_params* p, const float* qfeat, const float* kfeat,
+                              float* scores, int32_t* idx, int32_t* cnt, ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (!qfeat || !kfeat || !scores || !cnt || (p->top_k > 0 && !idx))
+    return fail(SSA_ERR_INVALID_ARG,
+                "qfeat, kfeat, scores, cnt (and idx when top_k > 0) must be non-NULL");
+  if (!aligned16(qfeat) || !aligned16(kfeat) || !aligned16(scores) || !aligned16(cnt) ||
+      (idx && !aligned16(idx)))
+    return fail(SSA_ERR_INVALID_ARG, "routing buffers must be 16-byte aligned");
+  s = launch_cum_route(p, qfeat, kfeat, scores, idx, cnt, static_cast<cudaStream_t>(stream));
   return s == SSA_OK ? ok() : s;
 }
 
@@ -513,9 +641,18 @@ ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const 
     cnt_h = cnt_a;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = launch_pool(p, k, p->Hkv, p->block_k, ksum, q, p->Hq, p->block_q, qsum, st)) != SSA_OK)
-    return s;
-  if ((s = launch_route(p, qsum, ksum, idx_h, cnt_h, st)) != SSA_OK) return s;
+  if (p->beta != 0.0f) {
+    float* qf = reinterpret_cast<float*>(ws + w.qf);
+    float* kf = reinterpret_cast<float*>(ws + w.kf);
+    float* sc = reinterpret_cast<float*>(ws + w.sc);
+    if ((s = launch_cum_features(p, k, p->Hkv, p->block_k, 0, kf, st)) != SSA_OK) return s;
+    if ((s = launch_cum_features(p, q, p->Hq, p->block_q, 1, qf, st)) != SSA_OK) return s;
+    if ((s = launch_cum_route(p, qf, kf, sc, idx_h, cnt_h, st)) != SSA_OK) return s;
+  } else {
+    if ((s = launch_pool(p, k, p->Hkv, p->block_k, ksum, q, p->Hq, p->block_q, qsum, st)) != SSA_OK)
+      return s;
+    if ((s = launch_route(p, qsum, ksum, idx_h, cnt_h, st)) != SSA_OK) return s;
+  }
   if (p->consensus && (s = launch_consensus(p, idx_h, cnt_h, idx_a, cnt_a, st)) != SSA_OK)
     return s;
   if ((s = launch_attend(p, q, k, v, idx_a, cnt_a, o, lse, st)) != SSA_OK) return s;

@@ -15,7 +15,8 @@ import torch
 
 __all__ = [
     "Params", "SsaError", "lib", "make_params", "params_of", "workspace_size", "block_summary",
-    "route", "route_consensus", "attend", "forward", "forward_host", "check_error",
+    "route", "route_consensus", "route_features", "route_cumulant", "attend", "forward",
+    "forward_host", "check_error",
     "probe_wait_timeout",
     "declared_functions", "LIB_PATH", "HEADER_PATH",
 ]
@@ -42,6 +43,7 @@ class Params(ctypes.Structure):
         ("block_q", ctypes.c_int32), ("top_k", ctypes.c_int32), ("window", ctypes.c_int32),
         ("causal", ctypes.c_int32), ("scale", ctypes.c_float),
         ("wait_timeout_us", ctypes.c_int32), ("consensus", ctypes.c_int32),
+        ("beta", ctypes.c_float),
     ]
 
     @property
@@ -59,16 +61,16 @@ class Params(ctypes.Structure):
 
 
 def make_params(B, Hq, Hkv, N, D, block_k, block_q, top_k, window, causal, scale=0.0,
-                wait_timeout_us=0, consensus=False) -> Params:
+                wait_timeout_us=0, consensus=False, beta=0.0) -> Params:
     return Params(B, Hq, Hkv, N, D, block_k, block_q, top_k, window, int(bool(causal)),
-                  float(scale), wait_timeout_us, int(bool(consensus)))
+                  float(scale), wait_timeout_us, int(bool(consensus)), float(beta))
 
 
 def params_of(w, **over) -> Params:
     """Params from any object with the workload field names."""
     f = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=w.N, D=w.D, block_k=w.block_k, block_q=w.block_q,
              top_k=w.top_k, window=w.window, causal=w.causal, scale=getattr(w, "scale", 0.0),
-             consensus=getattr(w, "consensus", False))
+             consensus=getattr(w, "consensus", False), beta=getattr(w, "beta", 0.0))
     f.update(over)
     return make_params(**f)
 
@@ -92,6 +94,8 @@ def lib() -> ctypes.CDLL:
         "ssa_block_summary": (i32, [P, vp, i32, i32, vp, vp]),
         "ssa_route": (i32, [P, vp, vp, vp, vp, vp]),
         "ssa_route_consensus": (i32, [P, vp, vp, vp, vp, vp]),
+        "ssa_route_features": (i32, [P, vp, i32, i32, i32, vp, vp]),
+        "ssa_route_cumulant": (i32, [P, vp, vp, vp, vp, vp, vp]),
         "ssa_attend": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ssa_forward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_check_error": (i32, [vp]),
@@ -177,6 +181,33 @@ def route_consensus(idx: torch.Tensor, cnt: torch.Tensor, p: Params):
     return idx_kv, cnt_kv
 
 
+def route_features(x: torch.Tensor, block: int, p: Params, queries: bool) -> torch.Tensor:
+    """Second-cumulant routing features, fp32 [B, H, N/block, D + D(D+1)/2]:
+    [mean | vech(covariance)] of key blocks, or [mean | (beta/2) w . vech(second
+    moment)] of query blocks."""
+    H = x.shape[1]
+    _need(x, torch.bfloat16, (p.B, H, p.N, p.D), "x")
+    F = p.D + p.D * (p.D + 1) // 2
+    out = torch.empty((p.B, H, p.N // block, F), dtype=torch.float32, device=x.device)
+    _check(lib().ssa_route_features(ctypes.byref(p), _ptr(x), H, block, int(bool(queries)),
+                                    _ptr(out), _stream()))
+    return out
+
+
+def route_cumulant(qfeat: torch.Tensor, kfeat: torch.Tensor, p: Params):
+    """Routing on the second-cumulant score: (idx, cnt) as ``route``."""
+    F = p.D + p.D * (p.D + 1) // 2
+    _need(qfeat, torch.float32, (p.B, p.Hq, p.n_qblocks, F), "qfeat")
+    _need(kfeat, torch.float32, (p.B, p.Hkv, p.n_kblocks, F), "kfeat")
+    dev = qfeat.device
+    scores = torch.empty((p.B, p.Hq, p.n_qblocks, p.n_kblocks), dtype=torch.float32, device=dev)
+    idx = torch.empty((p.B, p.Hq, p.n_qblocks, p.top_k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((p.B, p.Hq, p.n_qblocks), dtype=torch.int32, device=dev)
+    _check(lib().ssa_route_cumulant(ctypes.byref(p), _ptr(qfeat), _ptr(kfeat), _ptr(scores),
+                                    _ptr(idx) if p.top_k else None, _ptr(cnt), _stream()))
+    return idx, cnt
+
+
 def attend(q, k, v, idx, cnt, p: Params, with_lse: bool = True):
     """(o bf16 [B, Hq, N, D], lse fp32 [B, Hq, N] or None).  idx/cnt span Hq
     heads, or Hkv groups with ``p.consensus``."""
@@ -254,7 +285,7 @@ def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
     grp = p.Hq // p.Hkv
     unit = grp if p.consensus else 1          # query heads per sub-problem
     sub = make_params(1, unit, 1, p.N, p.D, p.block_k, p.block_q, p.top_k, p.window, p.causal,
-                      p.scale, p.wait_timeout_us, p.consensus)
+                      p.scale, p.wait_timeout_us, p.consensus, p.beta)
     if "ws" not in d:
         d["ws"] = torch.empty(workspace_size(sub), dtype=torch.uint8, device=dev)
     if "streams" not in d:

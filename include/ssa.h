@@ -71,6 +71,10 @@ typedef struct {
                               blocks; 1: the query heads of a KV group share
                               one consensus list (ssa_route_consensus);
                               requires (Hq / Hkv) * top_k <= 512            */
+  float beta;              /* weight of the second-cumulant routing term:
+                              0 ranks by <qbar, mu_c> (ssa_route); otherwise
+                              by <qbar, mu_c> + (beta/2) tr(Sigma_c Q2)
+                              (ssa_route_features + ssa_route_cumulant)     */
 } ssa_params;
 
 /* Bytes of device workspace ssa_forward needs for these parameters:
@@ -99,9 +103,37 @@ ssa_status ssa_block_summary(const ssa_params* p, const void* x, int32_t H,
  * Admissible blocks: causal -- completed blocks ending at or before the
  * query block's first token, (c+1)*Bk <= qb*Bq; non-causal -- all blocks.
  * Scores are fp32 dot products of the summaries; the top_k largest win, ties
- * to the lower block index.  top_k == 0 writes cnt = 0 only.  One launch. */
+ * to the lower block index.  top_k == 0 writes cnt = 0 only.  One launch.
+ * Requires p->beta == 0 (SSA_ERR_INVALID_ARG otherwise). */
 ssa_status ssa_route(const ssa_params* p, const float* qsum, const float* ksum,
                      int32_t* idx, int32_t* cnt, ssa_stream_t stream);
+
+/* Second-cumulant routing features (jonsmirl/ssa README, "Algorithm and
+ * complexity": r_c(q) = <q, mu_c> + (beta/2) q^T Sigma_c q with Sigma_c block
+ * c's second cumulant).  A query block scores by the mean of its queries'
+ * scores, <qbar, mu_c> + (beta/2) tr(Sigma_c Q2), Q2 = mean of q_i q_i^T over
+ * the block, which is one dot product of the feature vectors written here:
+ *   queries == 0 (keys, block = Bk):    [mu_c | vech(Sigma_c)]
+ *   queries == 1 (queries, block = Bq): [qbar | (beta/2) w . vech(Q2)]
+ * vech = the upper triangle d <= e, row by row; w = 1 on the diagonal, 2 off
+ * it; Sigma_c = (1/block) sum (x - mu)(x - mu)^T.
+ *   x    bf16 [B, H, N, D] (device)
+ *   out  fp32 [B, H, N/block, F] (device), F = D + D(D+1)/2 (2144 for D = 64)
+ * block is a power of two <= 128 dividing N.  One launch. */
+ssa_status ssa_route_features(const ssa_params* p, const void* x, int32_t H, int32_t block,
+                              int32_t queries, float* out, ssa_stream_t stream);
+
+/* Routing on the second-cumulant score: s = qfeat . kfeat over the admissible
+ * blocks (fp32), then the top_k of every query block (ties to the lower block
+ * index), listed ascending, padded with -1, with their count -- the same
+ * output as ssa_route.
+ *   qfeat   fp32 [B, Hq, N/Bq, F], kfeat fp32 [B, Hkv, N/Bk, F] from
+ *           ssa_route_features (device)
+ *   scores  fp32 [B, Hq, N/Bq, N/Bk] (device scratch: the score matrix)
+ *   idx/cnt as for ssa_route (device, out)
+ * Two launches. */
+ssa_status ssa_route_cumulant(const ssa_params* p, const float* qfeat, const float* kfeat,
+                              float* scores, int32_t* idx, int32_t* cnt, ssa_stream_t stream);
 
 /* GQA-shared consensus route (jonsmirl/ssa README, "Complete 10M transformer
  * result": one route formed across heads by consensus, carrying the blocks
@@ -143,8 +175,9 @@ ssa_status ssa_attend(const ssa_params* p, const void* q, const void* k, const v
                       const int32_t* idx, const int32_t* cnt, void* o, float* lse,
                       ssa_stream_t stream);
 
-/* The whole path in one call: summaries of K and Q (one launch), routing,
- * (with p->consensus) the consensus route, attend.  workspace must hold
+/* The whole path in one call: summaries of K and Q (one launch) and routing
+ * -- or, with p->beta != 0, the second-cumulant features of K and Q and
+ * ssa_route_cumulant --, (with p->consensus) the consensus route, attend.  workspace must hold
  * ssa_workspace_size(p) bytes (device, 256-byte aligned).  idx_out / cnt_out
  * (device, may be NULL) receive the lists attend used when given -- per head
  * [B, Hq, N/Bq, top_k], or per KV group [B, Hkv, N/Bq, top_k] with

@@ -79,7 +79,7 @@ def test_consensus_entry_point_rejects_bad_arguments_before_launch(L):
     (dict(scale=float("nan")), 1), (dict(scale=-1.0), 1), (dict(wait_timeout_us=-5), 1),
     (dict(N=16 * 2 ** 23, block_k=16, block_q=16, B=1, Hq=1, Hkv=1), 2),
     (dict(window=200000, block_k=16, block_q=16), 2),
-    (dict(consensus=True, Hq=16, Hkv=1, top_k=33), 2),
+    (dict(consensus=True, Hq=16, Hkv=1, top_k=33), 2), (dict(beta=float("inf")), 1),
 ])
 def test_invalid_params_are_rejected_before_launch(L, kw, status):
     p = _p(**kw)
@@ -117,3 +117,27 @@ def test_binding_rejects_wrong_tensors():
     q = torch.zeros(1, 2, 1024, 64, dtype=torch.bfloat16)   # CPU tensor: refused by the binding
     with pytest.raises(ValueError):
         ssa.forward(q, q, q, p)
+
+
+def test_workspace_layout_with_second_cumulant(L):
+    p = _p(beta=0.5)
+    a = lambda x: (x + 255) // 256 * 256
+    ks, qs = 2 * 512 * 64 * 4, 14 * 512 * 64 * 4
+    ix, cn = 14 * 512 * 16 * 4, 14 * 512 * 4
+    F = 64 + 64 * 65 // 2
+    qf, kf, sc = 14 * 512 * F * 4, 2 * 512 * F * 4, 14 * 512 * 512 * 4
+    assert ssa.workspace_size(p) == a(ks) + a(qs) + a(ix) + a(cn) + a(qf) + a(kf) + a(sc)
+
+
+def test_second_cumulant_entry_points_reject_bad_arguments_before_launch(L):
+    good = ctypes.c_void_p(1 << 20)
+    p = _p(beta=1.0)
+    # the mean-only router refuses a nonzero beta
+    assert L.ssa_route(ctypes.byref(p), good, good, good, good, None) == 1
+    f = L.ssa_route_features
+    assert f(ctypes.byref(p), good, 14, 64, 2, good, None) == 1      # queries flag
+    assert f(ctypes.byref(p), good, 14, 256, 1, good, None) == 1     # block too large
+    assert f(ctypes.byref(p), None, 14, 64, 1, good, None) == 1
+    g = L.ssa_route_cumulant
+    assert g(ctypes.byref(p), good, good, None, good, good, None) == 1
+    assert g(ctypes.byref(p), good, good, good, None, good, None) == 1
