@@ -46,24 +46,27 @@ struct CumFeatArgs {
   float half_beta;         // beta / 2 (queries only)
 };
 
-// one CTA per block; dynamic shared memory holds the block as fp32
-// [block][D], its mean, and the (d, e) pair of every vech entry
+// One CTA per block; dynamic shared memory holds the block as fp32 [block][D]
+// and its mean.  The D x D outer-product sum is computed on 4 x 4 register
+// tiles of the upper triangle (tile rows ti <= tile columns tj): per row t of
+// the block a thread reads two float4 and does 16 FMAs.
+template <int D>
+__host__ __device__ constexpr size_t cumulant_features_smem(int block) {
+  return static_cast<size_t>(block) * D * 4 + D * 4;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kCumThreads) cumulant_features_kernel(const CumFeatArgs a) {
   constexpr int F = cumulant_features<D>();
-  constexpr int NV = D * (D + 1) / 2;
+  constexpr int T = D / 4;                  // tiles per side
+  constexpr int NT = T * (T + 1) / 2;       // upper-triangular tiles
   extern __shared__ __align__(16) float cum_x[];
-  float* mean = cum_x + a.block * D;                                 // [D]
-  uint16_t* pair = reinterpret_cast<uint16_t*>(mean + D);             // [NV]: d << 8 | e
+  float* mean = cum_x + a.block * D;        // [D]
   const int64_t blk = blockIdx.x;
   if (blk >= a.n_blocks) return;
   const int tid = threadIdx.x;
   const __nv_bfloat16* src = a.x + blk * a.block * D;
   for (int i = tid; i < a.block * D; i += kCumThreads) cum_x[i] = __bfloat162float(src[i]);
-  if (tid < D) {  // row d of the upper triangle starts at d*D - d(d-1)/2
-    const int off = tid * D - tid * (tid - 1) / 2;
-    for (int e = tid; e < D; ++e) pair[off + e - tid] = static_cast<uint16_t>((tid << 8) | e);
-  }
   __syncthreads();
   const float inv = 1.0f / static_cast<float>(a.block);  // exact: block is a power of two
   if (tid < D) {
@@ -79,13 +82,43 @@ __global__ void __launch_bounds__(kCumThreads) cumulant_features_kernel(const Cu
     for (int i = tid; i < a.block * D; i += kCumThreads) cum_x[i] -= mean[i % D];
     __syncthreads();
   }
-  for (int v = tid; v < NV; v += kCumThreads) {
-    const int d = pair[v] >> 8, e = pair[v] & 0xFF;
-    float s = 0.f;
-    for (int t = 0; t < a.block; ++t) s = fmaf(cum_x[t * D + d], cum_x[t * D + e], s);
-    s *= inv;
-    if (a.queries) s *= a.half_beta * (d == e ? 1.f : 2.f);
-    dst[D + v] = s;
+  for (int u = tid; u < NT; u += kCumThreads) {
+    // tile u -> (ti, tj), ti <= tj: row ti of the tile triangle starts at
+    // ti*T - ti(ti-1)/2
+    int ti = 0, off = 0;
+    while (off + (T - ti) <= u) {
+      off += T - ti;
+      ++ti;
+    }
+    const int tj = ti + (u - off);
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+    for (int t = 0; t < a.block; ++t) {
+      const float4 xa = *reinterpret_cast<const float4*>(cum_x + t * D + 4 * ti);
+      const float4 xb = *reinterpret_cast<const float4*>(cum_x + t * D + 4 * tj);
+      const float va[4] = {xa.x, xa.y, xa.z, xa.w};
+      const float vb[4] = {xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(va[i], vb[j], acc[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int d = 4 * ti + i;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = 4 * tj + j;
+        if (d > e) continue;  // lower half of a diagonal tile
+        float v = acc[i][j] * inv;
+        if (a.queries) v *= a.half_beta * (d == e ? 1.f : 2.f);
+        dst[D + d * D - d * (d - 1) / 2 + (e - d)] = v;
+      }
+    }
   }
 }
 

@@ -380,7 +380,7 @@ int64_t cum_features(const ssa_params* p) { return p->D + static_cast<int64_t>(p
 
 template <int D>
 cudaError_t launch_cum_features_t(const ssa::CumFeatArgs& a, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(a.block) * D * 4 + D * 4 + D * (D + 1) / 2 * 2;
+  const size_t smem = ssa::cumulant_features_smem<D>(a.block);
   cudaError_t e = cudaFuncSetAttribute(ssa::cumulant_features_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
