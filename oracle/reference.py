@@ -62,7 +62,7 @@ __all__ = [
     "RouteResult", "key_set", "attend_masked_dense", "attend_gathered", "forward",
     "near_tie_rows", "acceptable_selections", "route_row",
     "consensus_row", "route_consensus", "expand_consensus",
-    "block_covariance", "block_second_moment", "block_scores",
+    "block_covariance", "block_second_moment", "block_scores", "decode_step",
 ]
 
 NEAR_TIE_REL = 1e-4   # relative score gap under which two blocks count as tied
@@ -416,6 +416,47 @@ def attend_gathered(q, k, v, idx, cnt, p: Params, queries=None):
     if queries is not None:
         return o_out, l_out
     return o_out.reshape(p.B, p.Hq, p.N, dv), l_out.reshape(p.B, p.Hq, p.N)
+
+
+# --------------------------------------------------------------------------
+# decode: one new query per head against the cached keys
+# --------------------------------------------------------------------------
+def decode_step(q, k, v, n_ctx: int, p: Params):
+    """One decode step.  ``q`` [B, Hq, D] is the query at position
+    i = n_ctx - 1 (its own key and value are already the cache's row i);
+    ``k``/``v`` [B, Hkv, >= n_ctx, D] float64 caches.
+
+    The query is its own query block (Bq = 1): it scores the completed key
+    blocks (c+1)*Bk <= i by <q, mu_c> (step 5), keeps the top_k ordered by
+    (score descending, block index ascending) (step 6), and reads exact
+    softmax over the routed blocks' keys united with the window
+    i - W < j <= i, cut at i (steps 7-8) -- the method's steps for one query.
+    Causal only.  Returns (o [B, Hq, Dv], lse [B, Hq], idx [B, Hq, top_k]
+    ascending and -1 padded, cnt [B, Hq])."""
+    if not p.causal:
+        raise ValueError("decode is causal")
+    i = n_ctx - 1
+    nb = i // p.block_k                       # admissible: c < i // Bk
+    mu = block_summary(k[:, :, :nb * p.block_k], p.block_k) if nb else None
+    scale = p.softmax_scale
+    o = np.zeros((p.B, p.Hq, v.shape[-1]))
+    lse = np.zeros((p.B, p.Hq))
+    idx = np.full((p.B, p.Hq, p.top_k), -1, dtype=np.int32)
+    cnt = np.zeros((p.B, p.Hq), dtype=np.int32)
+    for b in range(p.B):
+        for h in range(p.Hq):
+            g = h // p.group
+            if nb:
+                sel, _, _ = route_row(q[b, h], mu[b, g], np.arange(nb), p.top_k)
+            else:
+                sel = np.zeros(0, dtype=np.int64)
+            idx[b, h, :len(sel)] = sel
+            cnt[b, h] = len(sel)
+            ks = key_set(i, sel, p)
+            logits = (k[b, g, ks] @ q[b, h]) * scale
+            o1, l1 = _softmax_read(logits[None, :], v[b, g, ks])
+            o[b, h], lse[b, h] = o1[0], l1[0]
+    return o, lse, idx, cnt
 
 
 def forward(q, k, v, p: Params, form: str = "dense"):

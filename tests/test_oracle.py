@@ -571,3 +571,52 @@ def test_second_cumulant_with_zero_beta_or_no_spread_is_the_mean_route():
     # and a nonzero beta moves some selections on spread blocks
     moved = O.forward(q, k, v, O.Params(**{**p0.__dict__, "beta": 4.0}))
     assert (moved["idx"] != base["idx"]).any()
+
+
+# ---------------------------------------------------------------- decode step
+@pytest.mark.parametrize("kk", [0, 1, 2, 4])
+def test_decode_steps_match_hand_derivation(kk):
+    # in the 4-block example the decode admissible set of every position equals
+    # its query block's, so the hand-derived prefill values hold per step
+    q, k, v = _worked_inputs()
+    E = math.exp(math.sqrt(2.0))
+    want = {i: eval(expr, {"E": E}) for k_, i, expr in _read_worked_golden() if k_ == kk}
+    assert len(want) == (2 if kk == 4 else 8)
+    p = _params(top_k=kk)
+    for i, val in want.items():
+        o, lse, idx, cnt = O.decode_step(q[:, :, i], k, v, i + 1, p)
+        assert o[0, 0, 0] == pytest.approx(val, abs=1e-12), (kk, i)
+        assert o[0, 0, 1] == pytest.approx(1.0, abs=1e-12)
+
+
+def test_decode_step_equals_prefill_with_query_blocks_of_one():
+    rng = np.random.default_rng(41)
+    p = _params(B=2, Hq=4, Hkv=2, N=96, D=8, block_k=8, block_q=1, top_k=3, window=10)
+    q, k, v = _rand((2, 4, 96, 8), 42), _rand((2, 2, 96, 8), 43), _rand((2, 2, 96, 8), 44)
+    full = O.forward(q, k, v, p)                       # masked-dense form, Bq = 1
+    for i in list(range(0, 96, 7)) + [95]:
+        o, lse, idx, cnt = O.decode_step(q[:, :, i], k, v, i + 1, p)
+        np.testing.assert_allclose(o, full["o"][:, :, i], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(lse, full["lse"][:, :, i], atol=1e-12, rtol=0)
+        np.testing.assert_array_equal(idx, full["idx"][:, :, i])
+        # the cache beyond n_ctx is never read
+        k2, v2 = k.copy(), v.copy()
+        k2[:, :, i + 1:] = rng.standard_normal(k2[:, :, i + 1:].shape) * 50
+        v2[:, :, i + 1:] = 7.0
+        o2, _, _, _ = O.decode_step(q[:, :, i], k2, v2, i + 1, p)
+        np.testing.assert_array_equal(o2, o)
+
+
+def test_decode_step_dense_and_sliding_window_limits():
+    N, D, bk = 160, 16, 16
+    q, k, v = _rand((1, 4, N, D), 45), _rand((1, 2, N, D), 46), _rand((1, 2, N, D), 47)
+    i = N - 1
+    dense = _params(B=1, Hq=4, Hkv=2, N=N, D=D, block_k=bk, block_q=1, top_k=N // bk, window=bk)
+    o, _, _, _ = O.decode_step(q[:, :, i], k, v, N, dense)
+    want = _sdpa(q[:, :, i:i + 1], k, v, gqa=True)[:, :, 0]
+    np.testing.assert_allclose(o, want, atol=1e-12, rtol=0)
+    W = 37
+    win = _params(B=1, Hq=4, Hkv=2, N=N, D=D, block_k=bk, block_q=1, top_k=0, window=W)
+    o, _, _, _ = O.decode_step(q[:, :, i], k, v, N, win)
+    want = _sdpa(q[:, :, i:i + 1], k[:, :, i - W + 1:], v[:, :, i - W + 1:], gqa=True)[:, :, 0]
+    np.testing.assert_allclose(o, want, atol=1e-12, rtol=0)
