@@ -60,6 +60,9 @@ def parse_args(argv=None):
     ap.add_argument("--seq-len", type=int, default=0,
                     help="run the chosen workload's recipe at another sequence length "
                          "(e.g. a smaller copy of the million-token workload for profiling)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time one decode step (a query per head at the last position of the "
+                         "workload's full K/V cache) instead of the prefill")
     ap.add_argument("--beta", type=float, default=0.0,
                     help="weight of the second-cumulant routing term (0: mean summaries only)")
     ap.add_argument("--consensus", action="store_true",
@@ -593,8 +596,214 @@ def run_ssa(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------
+# decode: one query per head at the end of the cache
+# ----------------------------------------------------------------------------
+def decode_work(w, cnt_sel, idx_sel):
+    """Algorithmic bytes of one decode step: the block means the router reads
+    (B * Hkv * nb * D * 4) and, per query head, the distinct keys it reads
+    (routed blocks' keys below the window plus the window) as K and V rows,
+    plus q, o and lse.  Also the mean keys per query."""
+    i = w.N - 1
+    nb = i // w.block_k
+    lo = max(0, i - w.window + 1)
+    keys = 0
+    for b in range(w.B):
+        for h in range(w.Hq):
+            n = int(cnt_sel[b, h])
+            far = 0
+            for c in idx_sel[b, h, :n].tolist():
+                start = c * w.block_k
+                far += max(0, min(start + w.block_k, lo) - start)
+            keys += far + (i - lo + 1)
+    summaries = w.B * w.Hkv * nb * w.D * 4
+    kv = keys * w.D * 2 * 2
+    io = w.B * w.Hq * (w.D * 2 * 2 + 4)
+    return {"bytes": summaries + kv + io, "keys_per_query": keys / (w.B * w.Hq),
+            "summary_bytes": summaries, "kv_bytes": kv}
+
+
+def run_decode(args):
+    import numpy as np
+    import torch
+
+    from content_routed_block_b200 import build, ssa
+    from content_routed_block_b200.workloads import make_inputs
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    w = workload_of(args)
+    p = ssa.params_of(w)
+    x = make_inputs(w)
+    n_ctx = w.N
+    qh = torch.from_numpy(np.ascontiguousarray(x["q"][:, :, n_ctx - 1]).view(np.int16)).view(torch.bfloat16)
+    kd, vd = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in "kv")
+    qd = qh.to(dev)
+    ksum0 = ssa.block_summary(kd, w.block_k, p)
+    ksum = ksum0.clone()
+    ws = torch.empty(ssa.decode_workspace_size(p), dtype=torch.uint8, device=dev)
+    o = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        return ssa.decode(qd, kd, vd, n_ctx, ksum, p, workspace=ws, out=o)
+
+    for _ in range(max(3, args.warmup)):
+        _, _, idx, cnt = step()
+    torch.cuda.synchronize()
+    ssa.check_error()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = str(getattr(props, "uuid", "")) or str(local)
+    if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) > 8:
+        gpu_id = "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark("start")
+    for s_ in range(args.steps):
+        flush.zero_()
+        starts[s_].record()
+        step()
+        ends[s_].record()
+    torch.cuda.synchronize()
+    sampler.mark("end")
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    ssa.check_error()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in zip(starts, ends))
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = w.B * world
+    value = tokens / (ms * 1e-3)
+    work = decode_work(w, cnt.cpu().numpy(), idx.cpu().numpy())
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    achieved = work["bytes"] / (ms * 1e-3) / 1e9
+
+    # end to end: the query from pinned host memory in, O back to pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        qp = qh.pin_memory()
+        oh = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16).pin_memory()
+        for _ in range(3):
+            qd.copy_(qp, non_blocking=True)
+            step()
+            oh.copy_(o, non_blocking=True)
+        torch.cuda.synchronize()
+        n_e2e = min(args.steps, 200)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_e2e):
+            qd.copy_(qp, non_blocking=True)
+            step()
+            oh.copy_(o, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        e2e = {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": qp.numel() * 2, "d2h_bytes_per_step": oh.numel() * 2,
+               "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle as O
+        op = O.Params.of(w)
+        q64 = O.upcast_bf16(x["q"][:, :, n_ctx - 1])
+        k64, v64 = O.upcast_bf16(x["k"]), O.upcast_bf16(x["v"])
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            O.decode_step(q64, k64, v64, n_ctx, op)
+            reps += 1
+            if time.perf_counter() - t0 > args.cpu_seconds:
+                break
+        wall = time.perf_counter() - t0
+        cpu = {"value": reps * w.B / wall, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{reps} whole decode steps of this workload (block means of the cache, "
+                         f"routing and the read of every head) in float64 in one process"}
+    clocks = sampler.summary()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    cfg = workload_config(w, args)
+    cfg["workload"] = f"decode at n_ctx={n_ctx}: " + cfg["workload"]
+    cfg["global_batch"] = w.B * world
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ssa", "config": cfg,
+        "keys_per_query": work["keys_per_query"],
+        "roofline": {"bound": "hbm", "kernel": "decode (route + attend + combine)",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "peak_source": f"{peak_kind} hbm_gbs",
+                     "bytes_per_launch": work["bytes"], "summary_bytes": work["summary_bytes"],
+                     "kv_bytes": work["kv_bytes"]},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_decode(args):
+    """The oracle's decode step, timed per step on one host core."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle as O
+    from content_routed_block_b200.workloads import make_inputs
+    w = workload_of(args)
+    x = make_inputs(w)
+    op = O.Params.of(w)
+    n_ctx = w.N
+    q64 = O.upcast_bf16(x["q"][:, :, n_ctx - 1])
+    k64, v64 = O.upcast_bf16(x["k"]), O.upcast_bf16(x["v"])
+    for _ in range(args.warmup):
+        O.decode_step(q64, k64, v64, n_ctx, op)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.decode_step(q64, k64, v64, n_ctx, op)
+        ts.append(time.perf_counter() - t0)
+    sec = statistics.mean(ts)
+    value = w.B / sec
+    cfg = workload_config(w, args)
+    cfg["workload"] = f"decode at n_ctx={n_ctx}: " + cfg["workload"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sec, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} whole decode steps in float64, one process"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.decode:
+        (run_reference_decode if args.impl == "reference" else run_decode)(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -245,7 +245,69 @@ __global__ void __launch_bounds__(kAtThreads, 2)
     }
   }
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 0 && static_cast<int>(misc[1]) <= 32) {
+    // Few routed entries outside the window (the common case, e.g. 2 query
+    // blocks x 16): the whole union list is built in registers, one entry
+    // per lane, in the same order as the general path below.
+    const int nfar = static_cast<int>(misc[1]);
+    int x = lane < nfar ? far[lane] : 0x7FFFFFFF;
+    // ascending bitonic sort across the lanes
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const int y = __shfl_xor_sync(0xffffffffu, x, j);
+        const bool asc = (lane & k) == 0;
+        const bool low = (lane & j) == 0;
+        x = (low == asc) ? min(x, y) : max(x, y);
+      }
+    }
+    // deduplicate: the first lane of each run of one block ORs the routed
+    // bits of the run (at most one entry per query block of the tile: <= 8)
+    const int c = x >> 8;
+    const int prev = __shfl_up_sync(0xffffffffu, x, 1);
+    const bool head = lane < nfar && (lane == 0 || (prev >> 8) != c);
+    int bits = x & 0xFF;
+#pragma unroll
+    for (int d = 1; d < 8; ++d) {
+      const int nb = __shfl_down_sync(0xffffffffu, x, d);
+      if (lane + d < nfar && (nb >> 8) == c) bits |= nb & 0xFF;
+    }
+    const uint32_t hm = __ballot_sync(0xffffffffu, head);
+    const int nf = __popc(hm);
+    if (head) faru[__popc(hm & ((1u << lane) - 1u))] = (c << 8) | bits;
+    __syncwarp();
+    // interleave: class = which softmax warps need the entry; order by
+    // (rank within the class, class), i.e. round-robin over the classes
+    const int e = lane < nf ? faru[lane] : 0;
+    int m = 32 + lane;  // distinct for the empty lanes
+    if (lane < nf) {
+      m = 0;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int i_lo = q0 + (32 * w) % RH;
+        const int lo = i_lo / a.Bq - qb0, hi = min(R - 1, (i_lo + 31) / a.Bq - qb0);
+        const uint32_t qm = (lo < R) ? ((2u << hi) - (1u << lo)) : 0u;
+        m |= ((static_cast<uint32_t>(e) & 0xFFu & qm) != 0u) << w;
+      }
+    }
+    const uint32_t same = __match_any_sync(0xffffffffu, m);
+    const int rank = __popc(same & ((1u << lane) - 1u));
+    uint64_t kv = lane < nf ? ((static_cast<uint64_t>(rank * 16 + m) << 32) | static_cast<uint32_t>(e))
+                            : ~0ull;
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const uint64_t y = __shfl_xor_sync(0xffffffffu, kv, j);
+        const bool asc = (lane & k) == 0;
+        const bool low = (lane & j) == 0;
+        kv = (low == asc) ? (kv < y ? kv : y) : (kv < y ? y : kv);
+      }
+    }
+    if (lane < nf) faru[lane] = static_cast<int>(static_cast<uint32_t>(kv));
+    if (lane == 0) misc[2] = static_cast<uint32_t>(nf);
+  } else if (warp == 0) {
     const int nfar = static_cast<int>(misc[1]);
     int P = 1;
     while (P < nfar) P <<= 1;

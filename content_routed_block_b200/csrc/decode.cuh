@@ -1,0 +1,366 @@
+// Decode: one new query per head against the cached keys.
+//
+// jonsmirl/ssa README, introduction and "Algorithm and complexity", for a
+// single query: the query at position i = n_ctx - 1 is its own query block;
+// it scores the completed key blocks (c+1)*Bk <= i by <q, mu_c>, keeps the
+// top_k (score desc, index asc), and reads exact softmax over the routed
+// blocks' keys united with the window i - W < j <= i, cut at i.
+//
+// B200 design (flash-decoding with routing in front; three launches):
+//  * decode_route_kernel: grid (candidate splits, b * KV head).  One warp per
+//    query head of the group (the group's block means are read once per CTA
+//    and hit L1 for the other heads); lanes take strided candidates and keep
+//    a register top-KM list each, merged by shuffle bitonic merges; lane 0
+//    writes the split's KM keys.  The split holding the newest admissible
+//    block (i / Bk - 1) first recomputes that block's mean from the key cache
+//    into the summary cache, so a caller only has to keep the cache valid for
+//    the blocks before it.
+//  * decode_attend_kernel: grid (key splits, b * head).  Merges the splits'
+//    keys into the top_k, lays the key set out as the routed blocks' keys
+//    below the window followed by the window, and runs an online softmax in
+//    the exp2 domain over its share: 32 keys per warp step with lanes = keys
+//    for q.k, then lanes = dims for p.v.  Writes a partial (m, l, o).
+//  * decode_combine_kernel: merges the key splits' partials, writes O (bf16)
+//    and the natural-log LSE.
+// The work is memory-bound: the block means of the admissible blocks
+// (A * D * 4 bytes per KV head) and the gathered K/V rows (k*Bk + W rows per
+// head).
+#pragma once
+
+#include "common.cuh"
+#include "route.cuh"
+
+namespace ssa {
+
+constexpr int kDecThreads = 256;
+constexpr int kDecMaxSplits = 32;
+
+struct DecodeArgs {
+  const __nv_bfloat16* q;   // [B*Hq, D]
+  const __nv_bfloat16* k;   // [B*Hkv, Ncap, D]
+  const __nv_bfloat16* v;   // [B*Hkv, Ncap, D]
+  float* ksum;              // [B*Hkv, Ncap/Bk, D] (in / out)
+  uint64_t* part_keys;      // [B*Hq, S, KM]
+  float* part_attn;         // [B*Hq, KS, D + 2]: m, l, o
+  __nv_bfloat16* o;         // [B*Hq, D]
+  float* lse;               // [B*Hq] or null
+  int32_t* idx;             // [B*Hq, top_k] or null
+  int32_t* cnt;             // [B*Hq] or null
+  int32_t Hq, Hkv, Ncap, Bk, top_k, window;
+  int32_t i;                // query position (n_ctx - 1)
+  int32_t nb;               // admissible blocks: i / Bk
+  int32_t S, cands_per_split, KS;
+  float scale_log2;
+};
+
+// dynamic shared memory of decode_route_kernel: the group's queries and the
+// split's scores for every head of the group
+template <int D>
+__host__ __device__ constexpr size_t decode_route_smem(int g, int cands) {
+  return static_cast<size_t>(g) * D * 4 + static_cast<size_t>(g) * cands * 4;
+}
+
+template <int D, int KM>
+__global__ void __launch_bounds__(kDecThreads) decode_route_kernel(const DecodeArgs a) {
+  constexpr int LPR = D / 4;        // lanes per block-mean row (one float4 each)
+  constexpr int RPI = 32 / LPR;     // rows per warp step
+  constexpr int NW = kDecThreads / 32;
+  extern __shared__ __align__(16) float dec_smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int s = blockIdx.x, bkv = blockIdx.y;
+  const int g = a.Hq / a.Hkv;
+  const int b = bkv / a.Hkv, kv = bkv % a.Hkv;
+  const int c0 = s * a.cands_per_split, c1 = min(a.nb, c0 + a.cands_per_split);
+  const int nc = max(0, c1 - c0);
+  float* qs = dec_smem;                       // [g][D]
+  float* sc = dec_smem + g * D;               // [g][cands_per_split]
+  float* ksum = a.ksum + static_cast<int64_t>(bkv) * (a.Ncap / a.Bk) * D;
+  // the newest admissible block's mean (its last key is i - 1 or earlier)
+  const int c_new = a.nb - 1;
+  if (c_new >= c0 && c_new < c1 && tid < D) {
+    const __nv_bfloat16* src = a.k + (static_cast<int64_t>(bkv) * a.Ncap + c_new * a.Bk) * D + tid;
+    float acc = 0.f;
+    for (int t = 0; t < a.Bk; ++t) acc += __bfloat162float(src[static_cast<int64_t>(t) * D]);
+    ksum[static_cast<int64_t>(c_new) * D + tid] = acc * (1.0f / static_cast<float>(a.Bk));
+  }
+  for (int e = tid; e < g * D; e += kDecThreads)
+    qs[e] = __bfloat162float(a.q[(static_cast<int64_t>(b) * a.Hq + kv * g) * D + e]);
+  __syncthreads();
+
+  // 1. scores of every head for the split's candidates: a row is read once,
+  //    coalesced (LPR lanes x float4), and dotted with all g queries
+  const int sub = lane / LPR, part = lane % LPR;
+  for (int r0 = warp * RPI; r0 < nc; r0 += NW * RPI) {
+    const int r = r0 + sub;
+    const bool ok = r < nc;
+    float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (ok) m = reinterpret_cast<const float4*>(ksum + static_cast<int64_t>(c0 + r) * D)[part];
+    for (int j = 0; j < g; ++j) {
+      const float4 qv = reinterpret_cast<const float4*>(qs + j * D)[part];
+      float acc = qv.x * m.x;
+      acc = fmaf(qv.y, m.y, acc);
+      acc = fmaf(qv.z, m.z, acc);
+      acc = fmaf(qv.w, m.w, acc);
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (ok && part == 0) sc[j * a.cands_per_split + r] = acc;
+    }
+  }
+  __syncthreads();
+
+  // 2. per head, the top KM of the split: a lower bound L from the lanes'
+  //    maxima (the KM-th largest of them is reached by >= KM candidates)
+  //    admits few candidates into the per-lane register lists
+  for (int j = warp; j < g; j += NW) {
+    const int bh = b * a.Hq + kv * g + j;
+    const float* sj = sc + j * a.cands_per_split;
+    float lmax = -INFINITY;
+    for (int r = lane; r < nc; r += 32) lmax = fmaxf(lmax, sj[r]);
+    float L = -INFINITY;
+    if (KM <= 32) {
+      // descending bitonic sort of the 32 lane maxima
+      float x = lmax;
+#pragma unroll
+      for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+          const float y = __shfl_xor_sync(0xffffffffu, x, jj);
+          const bool desc_block = (lane & k) == 0;
+          const bool low = (lane & jj) == 0;
+          x = (low == desc_block) ? fmaxf(x, y) : fminf(x, y);
+        }
+      }
+      L = __shfl_sync(0xffffffffu, x, KM - 1);
+    }
+    uint64_t keys[KM];
+#pragma unroll
+    for (int e = 0; e < KM; ++e) keys[e] = 0ull;
+    if (a.top_k > 0) {
+      for (int r = lane; r < nc; r += 32) {
+        const float v = sj[r];
+        if (v >= L) {
+          const uint64_t key = route_key(v, c0 + r);
+          if (key > keys[KM - 1]) route_sorted_insert<KM>(keys, key);
+        }
+      }
+    }
+#pragma unroll
+    for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);
+    if (lane == 0) {
+      uint64_t* dst = a.part_keys + (static_cast<int64_t>(bh) * a.S + s) * KM;
+#pragma unroll
+      for (int e = 0; e < KM; ++e) dst[e] = keys[e];
+    }
+  }
+}
+
+template <int D, int KM>
+__global__ void __launch_bounds__(kDecThreads) decode_attend_kernel(const DecodeArgs a) {
+  constexpr int NW = kDecThreads / 32;
+  constexpr int DL = D / 32;  // dims per lane in the p.v step
+  extern __shared__ __align__(16) uint4 dec_vstage[];  // [NW][32 keys][D/8]: a warp's V rows
+  __shared__ __align__(16) float qs[D];
+  __shared__ int sel[64];
+  __shared__ int seg_off[65];
+  __shared__ int n_sel_s;
+  __shared__ float wm[NW], wl[NW];
+  __shared__ __align__(16) float wo[NW][D];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int x = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.Hq, h = bh % a.Hq;
+  const int bkv = b * a.Hkv + h / (a.Hq / a.Hkv);
+  const int i = a.i;
+  const int lo = max(0, i - a.window + 1);
+
+  for (int d = tid; d < D; d += kDecThreads) qs[d] = __bfloat162float(a.q[static_cast<int64_t>(bh) * D + d]);
+  // 1. merge the splits' keys (warp 0) and list the selection ascending
+  if (warp == 0) {
+    uint64_t keys[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) keys[j] = 0ull;
+    // lane l holds split l's list (already sorted descending; S <= 32), and
+    // the shuffle bitonic merges keep the top KM of all of them
+    if (lane < a.S) {
+      const uint64_t* src = a.part_keys + (static_cast<int64_t>(bh) * a.S + lane) * KM;
+#pragma unroll
+      for (int j = 0; j < KM; ++j) keys[j] = src[j];
+    }
+#pragma unroll
+    for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);
+    if (lane == 0) {
+      int v[KM];
+      int n = 0;
+#pragma unroll
+      for (int j = 0; j < KM; ++j) {
+        const bool real = j < a.top_k && keys[j] != 0ull;
+        v[j] = real ? static_cast<int>(~static_cast<uint32_t>(keys[j] & 0xFFFFFFFFull)) : 0x7FFFFFFF;
+        n += real ? 1 : 0;
+      }
+#pragma unroll
+      for (int p = 1; p < KM; ++p) {
+#pragma unroll
+        for (int y = p; y > 0; --y) {
+          const int l0 = min(v[y - 1], v[y]), h0 = max(v[y - 1], v[y]);
+          v[y - 1] = l0;
+          v[y] = h0;
+        }
+      }
+      // far segments: the part of each routed block below the window
+      int off = 0;
+#pragma unroll
+      for (int j = 0; j < KM; ++j) {
+        if (j < n) {
+          sel[j] = v[j];
+          seg_off[j] = off;
+          const int start = v[j] * a.Bk;
+          off += max(0, min(start + a.Bk, lo) - start);
+        }
+      }
+      seg_off[n] = off;
+      n_sel_s = n;
+      if (x == 0) {
+        if (a.cnt != nullptr) a.cnt[bh] = n;
+        if (a.idx != nullptr) {
+#pragma unroll
+          for (int j = 0; j < KM; ++j)
+            if (j < a.top_k) a.idx[static_cast<int64_t>(bh) * a.top_k + j] = j < n ? v[j] : -1;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int n_sel = n_sel_s;
+  const int far_total = seg_off[n_sel];
+  const int L = far_total + (i - lo + 1);
+  const int p0 = static_cast<int>((static_cast<int64_t>(L) * x) / a.KS);
+  const int p1 = static_cast<int>((static_cast<int64_t>(L) * (x + 1)) / a.KS);
+
+  // 2. online softmax over key positions p0..p1-1 (lanes = keys for q.k)
+  const __nv_bfloat16* kb = a.k + static_cast<int64_t>(bkv) * a.Ncap * D;
+  const __nv_bfloat16* vb = a.v + static_cast<int64_t>(bkv) * a.Ncap * D;
+  float m = -INFINITY, l = 0.f;
+  float o[DL];
+#pragma unroll
+  for (int d = 0; d < DL; ++d) o[d] = 0.f;
+  for (int base = p0 + warp * 32; base < p1; base += NW * 32) {
+    const int pos = base + lane;
+    const bool valid = pos < p1;
+    int j = 0;
+    if (valid) {
+      if (pos < far_total) {
+        int seg = 0;
+        while (seg + 1 < n_sel && seg_off[seg + 1] <= pos) ++seg;
+        j = sel[seg] * a.Bk + (pos - seg_off[seg]);
+      } else {
+        j = lo + (pos - far_total);
+      }
+    }
+    float sc = -INFINITY;
+    uint4* vst = dec_vstage + (warp * 32 + lane) * (D / 8);
+    if (valid) {
+      // this lane's V row goes to the warp's stage now, so that all 32 rows
+      // are in flight at once
+      const uint4* vr = reinterpret_cast<const uint4*>(vb + static_cast<int64_t>(j) * D);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) vst[c] = vr[c];
+      const uint4* kr = reinterpret_cast<const uint4*>(kb + static_cast<int64_t>(j) * D);
+      float acc = 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 u = kr[c];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          acc = fmaf(qs[8 * c + 2 * t], __uint_as_float(w[t] << 16), acc);
+          acc = fmaf(qs[8 * c + 2 * t + 1], __uint_as_float(w[t] & 0xFFFF0000u), acc);
+        }
+      }
+      sc = acc * a.scale_log2;
+    }
+    float bm = sc;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+    const float m_new = fmaxf(m, bm);
+    const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
+    const float pk = valid ? exp2f(sc - m_new) : 0.f;
+    float ps = pk;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+    l = l * alpha + ps;
+#pragma unroll
+    for (int d = 0; d < DL; ++d) o[d] *= alpha;
+    m = m_new;
+    // p.v with lanes = dims from the staged rows: key t, dims lane + 32 d
+    __syncwarp();
+    const int nk = min(32, p1 - base);
+    const __nv_bfloat16* vs = reinterpret_cast<const __nv_bfloat16*>(dec_vstage + warp * 32 * (D / 8));
+    for (int t = 0; t < nk; ++t) {
+      const float pt = __shfl_sync(0xffffffffu, pk, t);
+#pragma unroll
+      for (int d = 0; d < DL; ++d) o[d] = fmaf(pt, __bfloat162float(vs[t * D + lane + 32 * d]), o[d]);
+    }
+    __syncwarp();  // the stage is rewritten by the next step
+  }
+  // 3. combine the warps, write the split's partial
+  if (lane == 0) {
+    wm[warp] = m;
+    wl[warp] = l;
+  }
+#pragma unroll
+  for (int d = 0; d < DL; ++d) wo[warp][lane + 32 * d] = o[d];
+  __syncthreads();
+  if (warp == 0) {
+    float M = -INFINITY;
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, wm[w]);
+    float Lsum = 0.f;
+    float oo[DL];
+#pragma unroll
+    for (int d = 0; d < DL; ++d) oo[d] = 0.f;
+    for (int w = 0; w < NW; ++w) {
+      const float f = (wm[w] == -INFINITY) ? 0.f : exp2f(wm[w] - M);
+      Lsum += wl[w] * f;
+#pragma unroll
+      for (int d = 0; d < DL; ++d) oo[d] += wo[w][lane + 32 * d] * f;
+    }
+    float* dst = a.part_attn + (static_cast<int64_t>(bh) * a.KS + x) * (D + 2);
+    if (lane == 0) {
+      dst[0] = M;
+      dst[1] = Lsum;
+    }
+#pragma unroll
+    for (int d = 0; d < DL; ++d) dst[2 + lane + 32 * d] = oo[d];
+  }
+}
+
+template <int D>
+__host__ __device__ constexpr size_t decode_attend_smem() {
+  return static_cast<size_t>(kDecThreads / 32) * 32 * D * 2;
+}
+
+template <int D>
+__global__ void __launch_bounds__(32) decode_combine_kernel(const DecodeArgs a) {
+  constexpr int DL = D / 32;
+  const int bh = blockIdx.x, lane = threadIdx.x;
+  const float* src = a.part_attn + static_cast<int64_t>(bh) * a.KS * (D + 2);
+  float M = -INFINITY;
+  for (int x = 0; x < a.KS; ++x) M = fmaxf(M, src[x * (D + 2)]);
+  float L = 0.f;
+  float o[DL];
+#pragma unroll
+  for (int d = 0; d < DL; ++d) o[d] = 0.f;
+  for (int x = 0; x < a.KS; ++x) {
+    const float mx = src[x * (D + 2)];
+    const float f = (mx == -INFINITY) ? 0.f : exp2f(mx - M);
+    L += src[x * (D + 2) + 1] * f;
+#pragma unroll
+    for (int d = 0; d < DL; ++d) o[d] += src[x * (D + 2) + 2 + lane + 32 * d] * f;
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int d = 0; d < DL; ++d)
+    a.o[static_cast<int64_t>(bh) * D + lane + 32 * d] = __float2bfloat16_rn(o[d] * inv);
+  if (lane == 0 && a.lse != nullptr)
+    a.lse[bh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
+}
+
+}  // namespace ssa

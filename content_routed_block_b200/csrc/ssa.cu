@@ -12,6 +12,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <mutex>
 #include <string>
 
@@ -20,6 +21,7 @@
 #include "common.cuh"
 #include "consensus.cuh"
 #include "cumulant.cuh"
+#include "decode.cuh"
 #include "pool.cuh"
 #include "route.cuh"
 #include "route_tc.cuh"
@@ -515,6 +517,55 @@ WsLayout ws_layout(const ssa_params* p) {
   return w;
 }
 
+// ------------------------------------------------------------------ decode
+int decode_km(int32_t top_k) { return top_k <= 8 ? 8 : top_k <= 16 ? 16 : top_k <= 32 ? 32 : 64; }
+
+size_t decode_ws_bytes(const ssa_params* p) {
+  const size_t heads = static_cast<size_t>(p->B) * p->Hq;
+  return align256(heads * ssa::kDecMaxSplits * decode_km(p->top_k) * sizeof(uint64_t)) +
+         align256(heads * ssa::kDecMaxSplits * (p->D + 2) * sizeof(float));
+}
+
+ssa_status validate_decode(const ssa_params* p) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (!p->causal) return fail(SSA_ERR_INVALID_ARG, "decode is causal (causal must be 1)");
+  if (p->consensus) return fail(SSA_ERR_UNSUPPORTED, "decode routes per head (consensus must be 0)");
+  if (p->beta != 0.0f) return fail(SSA_ERR_UNSUPPORTED, "decode ranks by block means (beta must be 0)");
+  if (static_cast<int64_t>(p->B) * p->Hq > 65535)
+    return fail(SSA_ERR_UNSUPPORTED, "decode needs B * Hq <= 65535");
+  return SSA_OK;
+}
+
+template <int D, int KM>
+cudaError_t launch_decode_t(const ssa::DecodeArgs& a, int B, cudaStream_t stream) {
+  const size_t rs = ssa::decode_route_smem<D>(a.Hq / a.Hkv, a.cands_per_split);
+  cudaError_t e = cudaFuncSetAttribute(ssa::decode_route_kernel<D, KM>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(rs));
+  if (e != cudaSuccess) return e;
+  ssa::decode_route_kernel<D, KM><<<dim3(a.S, B * a.Hkv), ssa::kDecThreads, rs, stream>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t as = ssa::decode_attend_smem<D>();
+  e = cudaFuncSetAttribute(ssa::decode_attend_kernel<D, KM>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(as));
+  if (e != cudaSuccess) return e;
+  ssa::decode_attend_kernel<D, KM><<<dim3(a.KS, B * a.Hq), ssa::kDecThreads, as, stream>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  ssa::decode_combine_kernel<D><<<B * a.Hq, 32, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_decode_d(const ssa::DecodeArgs& a, int B, cudaStream_t stream) {
+  switch (decode_km(a.top_k)) {
+    case 8: return launch_decode_t<D, 8>(a, B, stream);
+    case 16: return launch_decode_t<D, 16>(a, B, stream);
+    case 32: return launch_decode_t<D, 32>(a, B, stream);
+    default: return launch_decode_t<D, 64>(a, B, stream);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -699,6 +750,76 @@ ssa_status ssa_forward_static(const ssa_params* p, const void* q, const void* k,
   // nothing has to be cleared between calls.
   return ssa_forward(p, q, k, v, o, lse, idx_out, cnt_out, scratch, ssa::kStaticScratchBytes,
                      stream);
+}
+
+size_t ssa_decode_workspace_size(const ssa_params* p) {
+  if (validate_decode(p) != SSA_OK) return 0;
+  return decode_ws_bytes(p);
+}
+
+ssa_status ssa_decode(const ssa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                      int32_t n_ctx, float* ksum_cache, void* o, float* lse, int32_t* idx_out,
+                      int32_t* cnt_out, void* workspace, size_t workspace_bytes,
+                      ssa_stream_t stream) {
+  ssa_status s = validate_decode(p);
+  if (s != SSA_OK) return s;
+  if (!q || !k_cache || !v_cache || !ksum_cache || !o)
+    return fail(SSA_ERR_INVALID_ARG, "q, k_cache, v_cache, ksum_cache and o must be non-NULL");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(ksum_cache) ||
+      !aligned16(o) || (lse && !aligned16(lse)) || (idx_out && !aligned16(idx_out)) ||
+      (cnt_out && !aligned16(cnt_out)))
+    return fail(SSA_ERR_INVALID_ARG, "all buffers must be 16-byte aligned");
+  if (n_ctx < 1 || n_ctx > p->N)
+    return fail(SSA_ERR_INVALID_ARG, "n_ctx must be in 1..N (the cache capacity)");
+  const size_t need = decode_ws_bytes(p);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(SSA_ERR_WORKSPACE, "decode workspace needs %zu bytes", need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  ssa::DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k_cache);
+  a.v = static_cast<const __nv_bfloat16*>(v_cache);
+  a.ksum = ksum_cache;
+  const size_t heads = static_cast<size_t>(p->B) * p->Hq;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.part_keys = reinterpret_cast<uint64_t*>(ws);
+  a.part_attn = reinterpret_cast<float*>(
+      ws + align256(heads * ssa::kDecMaxSplits * decode_km(p->top_k) * sizeof(uint64_t)));
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.idx = idx_out;
+  a.cnt = cnt_out;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.Ncap = p->N;
+  a.Bk = p->block_k;
+  a.top_k = p->top_k;
+  a.window = p->window;
+  a.i = n_ctx - 1;
+  a.nb = a.i / p->block_k;
+  // about two CTAs per SM in each phase; a route split scans >= 32 blocks
+  // (one per lane) and a key split >= 256 keys (32 per warp)
+  const int64_t want_s = (2 * 148 + static_cast<int64_t>(p->B) * p->Hkv - 1) /
+                         (static_cast<int64_t>(p->B) * p->Hkv);
+  int64_t S = std::min<int64_t>(std::min<int64_t>(ssa::kDecMaxSplits, want_s), (a.nb + 31) / 32);
+  S = std::max<int64_t>(S, 1);
+  a.cands_per_split = static_cast<int32_t>(std::max<int64_t>(1, (a.nb + S - 1) / S));
+  const size_t route_smem = p->D == 64 ? ssa::decode_route_smem<64>(p->Hq / p->Hkv, a.cands_per_split)
+                                       : ssa::decode_route_smem<128>(p->Hq / p->Hkv, a.cands_per_split);
+  if (route_smem > 200 * 1024)
+    return fail(SSA_ERR_UNSUPPORTED, "decode: too many key blocks per routing split for shared memory");
+  a.S = static_cast<int32_t>(S);
+  const int64_t lmax = static_cast<int64_t>(p->top_k) * p->block_k + p->window;
+  const int64_t want_ks = (2 * 148 + static_cast<int64_t>(heads) - 1) / static_cast<int64_t>(heads);
+  int64_t KS = std::min<int64_t>(std::min<int64_t>(ssa::kDecMaxSplits, want_ks), (lmax + 255) / 256);
+  a.KS = static_cast<int32_t>(std::max<int64_t>(KS, 1));
+  const float scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = p->D == 64 ? launch_decode_d<64>(a, p->B, st) : launch_decode_d<128>(a, p->B, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernels launch");
+  return ok();
 }
 
 ssa_status ssa_check_error(ssa_stream_t stream) {

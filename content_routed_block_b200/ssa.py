@@ -16,7 +16,7 @@ import torch
 __all__ = [
     "Params", "SsaError", "lib", "make_params", "params_of", "workspace_size", "block_summary",
     "route", "route_consensus", "route_features", "route_cumulant", "attend", "forward",
-    "forward_host", "check_error",
+    "forward_host", "decode", "decode_workspace_size", "check_error",
     "probe_wait_timeout",
     "declared_functions", "LIB_PATH", "HEADER_PATH",
 ]
@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
         "ssa_route_cumulant": (i32, [P, vp, vp, vp, vp, vp, vp]),
         "ssa_attend": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ssa_forward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ssa_decode_workspace_size": (sz, [P]),
+        "ssa_decode": (i32, [P, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_check_error": (i32, [vp]),
         "ssa_probe_wait_timeout": (i32, [i32, vp]),
         "ssa_status_string": (ctypes.c_char_p, [i32]),
@@ -321,6 +323,34 @@ def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
     compute.wait_stream(s_out)
     compute.wait_stream(s_in)
     return o_host
+
+
+def decode_workspace_size(p: Params) -> int:
+    return int(lib().ssa_decode_workspace_size(ctypes.byref(p)))
+
+
+def decode(q, k_cache, v_cache, n_ctx: int, ksum_cache, p: Params,
+           workspace: torch.Tensor | None = None, with_lse: bool = True, out=None):
+    """One decode step.  q bf16 [B, Hq, D] (the queries at position n_ctx-1);
+    k_cache / v_cache bf16 [B, Hkv, N, D] with N = p.N the capacity;
+    ksum_cache fp32 [B, Hkv, N/Bk, D], updated in place (the block that
+    becomes admissible at this step).  Returns (o, lse, idx, cnt)."""
+    _need(q, torch.bfloat16, (p.B, p.Hq, p.D), "q")
+    _need(k_cache, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "k_cache")
+    _need(v_cache, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "v_cache")
+    _need(ksum_cache, torch.float32, (p.B, p.Hkv, p.n_kblocks, p.D), "ksum_cache")
+    dev = q.device
+    ws = decode_workspace_size(p)
+    if workspace is None or workspace.numel() < ws:
+        workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)
+    o = out if out is not None else torch.empty((p.B, p.Hq, p.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((p.B, p.Hq), dtype=torch.float32, device=dev) if with_lse else None
+    idx = torch.empty((p.B, p.Hq, max(p.top_k, 1)), dtype=torch.int32, device=dev)
+    cnt = torch.empty((p.B, p.Hq), dtype=torch.int32, device=dev)
+    _check(lib().ssa_decode(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache), int(n_ctx),
+                            _ptr(ksum_cache), _ptr(o), _ptr(lse), _ptr(idx) if p.top_k else None,
+                            _ptr(cnt), _ptr(workspace), workspace.numel(), _stream()))
+    return o, lse, idx[..., :p.top_k], cnt
 
 
 def check_error(stream=None):

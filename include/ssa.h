@@ -211,6 +211,35 @@ ssa_status ssa_forward_static(const ssa_params* p, const void* q, const void* k,
                               void* o, float* lse, int32_t* idx_out, int32_t* cnt_out,
                               ssa_stream_t stream);
 
+/* Bytes of device workspace ssa_decode needs for these parameters (0 if they
+ * are invalid for decode). */
+size_t ssa_decode_workspace_size(const ssa_params* p);
+
+/* One decode step (jonsmirl/ssa README, introduction and "Algorithm and
+ * complexity", for a single query): the query of every (b, query head) at
+ * position i = n_ctx - 1 is its own query block.  It scores the completed
+ * key blocks (c+1)*Bk <= i by <q, mu_c> (fp32), keeps the top_k (ties to the
+ * lower block index), and reads exact softmax over the routed blocks' keys
+ * united with the window i - W < j <= i (each key once).
+ *   p          p->N is the cache capacity (a multiple of Bk); causal = 1,
+ *              consensus = 0, beta = 0; block_q is not used
+ *   q          bf16 [B, Hq, D] (device): the new queries
+ *   k_cache,   bf16 [B, Hkv, N, D] (device): rows 0 .. n_ctx-1 valid, row
+ *   v_cache    n_ctx - 1 holding the new token's key and value
+ *   ksum_cache fp32 [B, Hkv, N/Bk, D] (device, in/out): block means.  Rows
+ *              c < i/Bk - 1 must hold them on entry (ssa_block_summary over
+ *              the prefilled cache, then earlier decode steps); the call
+ *              writes row i/Bk - 1, the block that becomes admissible at i.
+ *   o          bf16 [B, Hq, D] (device, out); lse fp32 [B, Hq] (nullable)
+ *   idx_out    int32 [B, Hq, top_k] (nullable): the selection, ascending,
+ *              -1 padded; cnt_out int32 [B, Hq] (nullable)
+ *   workspace  ssa_decode_workspace_size(p) bytes (device, 256-byte aligned)
+ * Three launches (routing splits, attend splits, combine). */
+ssa_status ssa_decode(const ssa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                      int32_t n_ctx, float* ksum_cache, void* o, float* lse, int32_t* idx_out,
+                      int32_t* cnt_out, void* workspace, size_t workspace_bytes,
+                      ssa_stream_t stream);
+
 /* Synchronise the stream, then read and clear this device's error word.
  * Returns SSA_OK, SSA_ERR_TIMEOUT, SSA_ERR_DEVICE_CHECK or SSA_ERR_CUDA. */
 ssa_status ssa_check_error(ssa_stream_t stream);

@@ -63,6 +63,7 @@ __all__ = [
     "near_tie_rows", "acceptable_selections", "route_row",
     "consensus_row", "route_consensus", "expand_consensus",
     "block_covariance", "block_second_moment", "block_scores", "decode_step",
+    "decode_attend",
 ]
 
 NEAR_TIE_REL = 1e-4   # relative score gap under which two blocks count as tied
@@ -452,11 +453,19 @@ def decode_step(q, k, v, n_ctx: int, p: Params):
                 sel = np.zeros(0, dtype=np.int64)
             idx[b, h, :len(sel)] = sel
             cnt[b, h] = len(sel)
-            ks = key_set(i, sel, p)
-            logits = (k[b, g, ks] @ q[b, h]) * scale
-            o1, l1 = _softmax_read(logits[None, :], v[b, g, ks])
-            o[b, h], lse[b, h] = o1[0], l1[0]
+            o[b, h], lse[b, h] = decode_attend(q[b, h], k[b, g], v[b, g], i, sel, p)
     return o, lse, idx, cnt
+
+
+def decode_attend(q, k, v, i: int, sel, p: Params):
+    """The read of one decode query: exact softmax of ``q`` [D] over the keys
+    of the selected blocks ``sel`` united with the window i - W < j <= i
+    (``key_set``), against one head's caches ``k``/``v`` [>= i+1, D].
+    Returns (o [Dv], lse)."""
+    ks = key_set(i, np.asarray(sel, dtype=np.int64), p)
+    logits = (k[ks] @ q) * p.softmax_scale
+    o1, l1 = _softmax_read(logits[None, :], v[ks])
+    return o1[0], l1[0]
 
 
 def forward(q, k, v, p: Params, form: str = "dense"):

@@ -141,3 +141,23 @@ def test_second_cumulant_entry_points_reject_bad_arguments_before_launch(L):
     g = L.ssa_route_cumulant
     assert g(ctypes.byref(p), good, good, None, good, good, None) == 1
     assert g(ctypes.byref(p), good, good, good, None, good, None) == 1
+
+
+def test_decode_entry_point_rejects_bad_arguments_before_launch(L):
+    good = ctypes.c_void_p(1 << 20)
+    p = _p()
+    ws = L.ssa_decode_workspace_size(ctypes.byref(p))
+    assert ws > 0
+    f = L.ssa_decode
+    args = lambda n, w=good, wb=ws: (ctypes.byref(p), good, good, good, n, good, good, None, None,
+                                     None, w, wb, None)
+    assert f(*args(0)) == 1                       # n_ctx below 1
+    assert f(*args(32769)) == 1                   # n_ctx above the capacity
+    assert f(*args(100, wb=ws - 1)) == 3          # workspace too small
+    assert f(*args(100, w=ctypes.c_void_p((1 << 20) + 16))) == 1
+    for kw, status in ((dict(causal=False, window=0), 1), (dict(consensus=True), 2),
+                       (dict(beta=0.5), 2)):
+        bad = _p(**kw)
+        assert L.ssa_decode_workspace_size(ctypes.byref(bad)) == 0
+        assert f(ctypes.byref(bad), good, good, good, 100, good, good, None, None, None, good,
+                 ws, None) == status
