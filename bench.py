@@ -590,7 +590,9 @@ def run_ssa(args):
                      "path_frac_of_roofline": t_roof / (ms * 1e-3)},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (4 if w.consensus else 3) * args.steps,
+        # per forward: pool (K and Q in one launch) + route + attend, or with
+        # beta: two feature launches + scores + select + attend; +1 consensus
+        "gpu_launches": ((5 if w.beta else 3) + (1 if w.consensus else 0)) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -173,6 +173,17 @@ __global__ void __launch_bounds__(kAtThreads, 2)
     nwin = (qend - 1) / a.Bk - wlo + 1;
   }
 
+  // this thread's first routed entry, loaded before the set-up so that the
+  // load latency overlaps the barrier and TMEM set-up (reading the entry
+  // past the row's count stays inside the row: rows are top_k long)
+  const int total = R * a.top_k;
+  int pre_n = 0, pre_c = -1;
+  if (tid < total) {
+    const int64_t row = static_cast<int64_t>(ibh) * a.NQB + qb0 + tid / a.top_k;
+    pre_n = a.cnt[row];
+    pre_c = a.idx[row * a.top_k + tid % a.top_k];
+  }
+
   // ---------------------------------------------------------------- setup
   if (tid == 0) {
     mbar_init(bar_q, 1);
@@ -219,17 +230,16 @@ __global__ void __launch_bounds__(kAtThreads, 2)
 
   // ------------------------------------------ union of routed and window blocks
   {
-    const int total = R * a.top_k;
     for (int t = tid; t < total; t += kAtThreads) {
       const int r = t / a.top_k, e = t % a.top_k;
       const int64_t row = static_cast<int64_t>(ibh) * a.NQB + qb0 + r;
-      int n = a.cnt[row];
+      int n = (t == tid) ? pre_n : a.cnt[row];
       if (n > a.top_k || n < 0) {
         record_error(kErrCheck, kSiteIdx);
         n = min(max(n, 0), a.top_k);
       }
       if (e >= n) continue;
-      const int c = a.idx[row * a.top_k + e];
+      const int c = (t == tid) ? pre_c : a.idx[row * a.top_k + e];
       if (c < 0 || c >= a.NB) {
         record_error(kErrCheck, kSiteIdx);
         continue;
@@ -245,7 +255,8 @@ __global__ void __launch_bounds__(kAtThreads, 2)
     }
   }
   __syncthreads();
-  if (warp == 0 && static_cast<int>(misc[1]) <= 32) {
+  const int G = (a.Bk < kAtKT) ? kAtKT / a.Bk : 1;           // blocks per chunk
+  if (warp == 0 && static_cast<int>(misc[1]) <= 32 && G == 1) {
     // Few routed entries outside the window (the common case, e.g. 2 query
     // blocks x 16): the whole union list is built in registers, one entry
     // per lane, in the same order as the general path below.
@@ -378,15 +389,19 @@ __global__ void __launch_bounds__(kAtThreads, 2)
 #pragma unroll
         for (int bkt = 0; bkt < 16; ++bkt) bc[bkt] += __popc(__ballot_sync(0xffffffffu, m == bkt));
       }
-      // round-robin position: entries of round r follow all entries of
-      // earlier rounds, and within a round go by class
+      // Position.  With one block per chunk (Bk >= 64): round-robin over the
+      // classes, so that chunks exclusive to different warps alternate.
+      // With G blocks per chunk (Bk < 64): class by class, so that a chunk's
+      // blocks mostly serve one warp and the other warps skip it (measured
+      // on 16-key blocks: 0.360 ms against 0.395 ms for the round-robin and
+      // 0.425 ms for class-pure chunks padded with masked slots).
       int seen[16];
 #pragma unroll
       for (int bkt = 0; bkt < 16; ++bkt) seen[bkt] = 0;
       for (int i0 = 0; i0 < nf; i0 += 32) {
         const int e = i0 + lane;
         const int m = (e < nf) ? wmask(e) : -1;
-        int rank = 0;
+        int rank = 0;  // index of the entry within its class, in block order
 #pragma unroll
         for (int bkt = 0; bkt < 16; ++bkt) {
           const uint32_t bm = __ballot_sync(0xffffffffu, m == bkt);
@@ -395,8 +410,14 @@ __global__ void __launch_bounds__(kAtThreads, 2)
         }
         if (e < nf) {
           int pos = 0;
+          if (G == 1) {
 #pragma unroll
-          for (int bkt = 0; bkt < 16; ++bkt) pos += min(bc[bkt], rank) + ((bkt < m && bc[bkt] > rank) ? 1 : 0);
+            for (int bkt = 0; bkt < 16; ++bkt) pos += min(bc[bkt], rank) + ((bkt < m && bc[bkt] > rank) ? 1 : 0);
+          } else {
+#pragma unroll
+            for (int bkt = 0; bkt < 16; ++bkt) pos += (bkt < m) ? bc[bkt] : 0;
+            pos += rank;
+          }
           far[pos] = faru[e];
         }
       }
@@ -409,7 +430,6 @@ __global__ void __launch_bounds__(kAtThreads, 2)
 
   const int nf = static_cast<int>(misc[2]);
   const int n_entries = nf + nwin;
-  const int G = (a.Bk < kAtKT) ? kAtKT / a.Bk : 1;           // blocks per chunk
   const int SUBS = (a.Bk > kAtKT) ? a.Bk / kAtKT : 1;        // chunks per block
   const int T = (a.Bk >= kAtKT) ? n_entries * SUBS : (n_entries + G - 1) / G;
   int issued = 0;  // chunks the producer has put in flight

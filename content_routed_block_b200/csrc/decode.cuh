@@ -33,7 +33,7 @@
 namespace ssa {
 
 constexpr int kDecThreads = 256;
-constexpr int kDecMaxSplits = 32;
+constexpr int kDecMaxSplits = 128;
 
 struct DecodeArgs {
   const __nv_bfloat16* q;   // [B*Hq, D]
@@ -61,7 +61,7 @@ __host__ __device__ constexpr size_t decode_route_smem(int g, int cands) {
 }
 
 template <int D, int KM>
-__global__ void __launch_bounds__(kDecThreads) decode_route_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, (KM <= 16) ? 2 : 1) decode_route_kernel(const DecodeArgs a) {
   constexpr int LPR = D / 4;        // lanes per block-mean row (one float4 each)
   constexpr int RPI = 32 / LPR;     // rows per warp step
   constexpr int NW = kDecThreads / 32;
@@ -75,13 +75,26 @@ __global__ void __launch_bounds__(kDecThreads) decode_route_kernel(const DecodeA
   float* qs = dec_smem;                       // [g][D]
   float* sc = dec_smem + g * D;               // [g][cands_per_split]
   float* ksum = a.ksum + static_cast<int64_t>(bkv) * (a.Ncap / a.Bk) * D;
-  // the newest admissible block's mean (its last key is i - 1 or earlier)
+  // the newest admissible block's mean (its last key is i - 1 or earlier):
+  // thread t sums rows t / D, t / D + 256 / D, ... of column t % D (the loads
+  // are independent and unrolled), then D threads add the row phases
   const int c_new = a.nb - 1;
-  if (c_new >= c0 && c_new < c1 && tid < D) {
-    const __nv_bfloat16* src = a.k + (static_cast<int64_t>(bkv) * a.Ncap + c_new * a.Bk) * D + tid;
+  if (c_new >= c0 && c_new < c1) {  // uniform over the CTA
+    constexpr int RPH = kDecThreads / D;
+    __shared__ float red[RPH][D];
+    const int d = tid % D, rp = tid / D;
+    const __nv_bfloat16* src = a.k + (static_cast<int64_t>(bkv) * a.Ncap + c_new * a.Bk) * D + d;
     float acc = 0.f;
-    for (int t = 0; t < a.Bk; ++t) acc += __bfloat162float(src[static_cast<int64_t>(t) * D]);
-    ksum[static_cast<int64_t>(c_new) * D + tid] = acc * (1.0f / static_cast<float>(a.Bk));
+#pragma unroll 8
+    for (int t = rp; t < a.Bk; t += RPH) acc += __bfloat162float(src[static_cast<int64_t>(t) * D]);
+    red[rp][d] = acc;
+    __syncthreads();
+    if (tid < D) {
+      float sum = 0.f;
+#pragma unroll
+      for (int r = 0; r < RPH; ++r) sum += red[r][tid];
+      ksum[static_cast<int64_t>(c_new) * D + tid] = sum * (1.0f / static_cast<float>(a.Bk));
+    }
   }
   for (int e = tid; e < g * D; e += kDecThreads)
     qs[e] = __bfloat162float(a.q[(static_cast<int64_t>(b) * a.Hq + kv * g) * D + e]);
@@ -89,21 +102,30 @@ __global__ void __launch_bounds__(kDecThreads) decode_route_kernel(const DecodeA
 
   // 1. scores of every head for the split's candidates: a row is read once,
   //    coalesced (LPR lanes x float4), and dotted with all g queries
+  //    (four rows' loads are issued before any is used)
+  constexpr int UN = 4;
   const int sub = lane / LPR, part = lane % LPR;
-  for (int r0 = warp * RPI; r0 < nc; r0 += NW * RPI) {
-    const int r = r0 + sub;
-    const bool ok = r < nc;
-    float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (ok) m = reinterpret_cast<const float4*>(ksum + static_cast<int64_t>(c0 + r) * D)[part];
-    for (int j = 0; j < g; ++j) {
-      const float4 qv = reinterpret_cast<const float4*>(qs + j * D)[part];
-      float acc = qv.x * m.x;
-      acc = fmaf(qv.y, m.y, acc);
-      acc = fmaf(qv.z, m.z, acc);
-      acc = fmaf(qv.w, m.w, acc);
+  for (int r0 = warp * RPI * UN; r0 < nc; r0 += NW * RPI * UN) {
+    float4 m[UN];
 #pragma unroll
-      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (ok && part == 0) sc[j * a.cands_per_split + r] = acc;
+    for (int u = 0; u < UN; ++u) {
+      const int r = r0 + u * RPI + sub;
+      m[u] = r < nc ? reinterpret_cast<const float4*>(ksum + static_cast<int64_t>(c0 + r) * D)[part]
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < UN; ++u) {
+      const int r = r0 + u * RPI + sub;
+      for (int j = 0; j < g; ++j) {
+        const float4 qv = reinterpret_cast<const float4*>(qs + j * D)[part];
+        float acc = qv.x * m[u].x;
+        acc = fmaf(qv.y, m[u].y, acc);
+        acc = fmaf(qv.z, m[u].z, acc);
+        acc = fmaf(qv.w, m[u].w, acc);
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (r < nc && part == 0) sc[j * a.cands_per_split + r] = acc;
+      }
     }
   }
   __syncthreads();
@@ -178,12 +200,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_attend_kernel(const Decode
     uint64_t keys[KM];
 #pragma unroll
     for (int j = 0; j < KM; ++j) keys[j] = 0ull;
-    // lane l holds split l's list (already sorted descending; S <= 32), and
-    // the shuffle bitonic merges keep the top KM of all of them
-    if (lane < a.S) {
-      const uint64_t* src = a.part_keys + (static_cast<int64_t>(bh) * a.S + lane) * KM;
+    // lane l folds splits l, l + 32, ... (each sorted descending) into its
+    // list with in-register bitonic merges; the shuffle merges then keep the
+    // top KM of all of them
+    for (int sp = lane; sp < a.S; sp += 32) {
+      const uint64_t* src = a.part_keys + (static_cast<int64_t>(bh) * a.S + sp) * KM;
+      uint64_t other[KM];
 #pragma unroll
-      for (int j = 0; j < KM; ++j) keys[j] = src[j];
+      for (int j = 0; j < KM; ++j) other[j] = src[j];
+      route_merge_lists<KM>(keys, other);
     }
 #pragma unroll
     for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);

@@ -417,6 +417,24 @@ __device__ __forceinline__ void route_merge_partner(uint64_t (&a)[KM], int mask)
   }
 }
 
+// keep in `a` the top KM of a U b, both sorted descending (b in registers)
+template <int KM>
+__device__ __forceinline__ void route_merge_lists(uint64_t (&a)[KM], const uint64_t (&b)[KM]) {
+#pragma unroll
+  for (int i = 0; i < KM; ++i) a[i] = umax64(a[i], b[KM - 1 - i]);
+#pragma unroll
+  for (int j = KM / 2; j > 0; j >>= 1) {
+#pragma unroll
+    for (int i = 0; i < KM; ++i) {
+      if ((i & j) == 0) {
+        const uint64_t x = a[i], y = a[i + j];
+        a[i] = umax64(x, y);
+        a[i + j] = umin64(x, y);
+      }
+    }
+  }
+}
+
 template <int D, int KM, int RT>
 __global__ void __launch_bounds__(kRouteThreads) route_rows_kernel(const RouteArgs a) {
   constexpr int TPR = kRouteThreads / RT;           // threads per row

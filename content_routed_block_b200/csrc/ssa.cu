@@ -799,7 +799,7 @@ ssa_status ssa_decode(const ssa_params* p, const void* q, const void* k_cache, c
   a.i = n_ctx - 1;
   a.nb = a.i / p->block_k;
   // about two CTAs per SM in each phase; a route split scans >= 32 blocks
-  // (one per lane) and a key split >= 256 keys (32 per warp)
+  // and a key split >= 256 keys (32 per warp)
   const int64_t want_s = (2 * 148 + static_cast<int64_t>(p->B) * p->Hkv - 1) /
                          (static_cast<int64_t>(p->B) * p->Hkv);
   int64_t S = std::min<int64_t>(std::min<int64_t>(ssa::kDecMaxSplits, want_s), (a.nb + 31) / 32);
