@@ -153,6 +153,30 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # algorithmic work of one forward (from the routed lists)
 # ----------------------------------------------------------------------------
+# ----------------------------------------------------------------------------
+# replicas over ranks: every rank runs the whole workload on its own GPU
+# ----------------------------------------------------------------------------
+def max_over_ranks(x: float, world: int, dev) -> float:
+    """The largest of every rank's ``x`` (a per-step time): the job is as
+    slow as its slowest replica.  ``dev`` is the device of the process
+    group's backend (a CUDA device under NCCL, the CPU under gloo)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(tokens_per_rank: int, world: int, ms: float):
+    """Whole-job tokens per step and tokens/s when each of ``world`` ranks
+    processes ``tokens_per_rank`` tokens per step and the step takes ``ms``
+    (the max over ranks): weak scaling, no exchange between replicas."""
+    tokens = tokens_per_rank * world
+    return tokens, tokens / (ms * 1e-3)
+
+
 def algorithmic_work(w, idx, cnt):
     """Mean distinct keys per query (|S_i|), selected-key flops, and the attend
     kernel's algorithmic bytes: per routed list (a query block of a query head;
@@ -441,13 +465,8 @@ def run_ssa(args):
     sampler.stop()
     ssa.check_error()
     times = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    ms = statistics.mean(times)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    tokens = w.B * w.N * world
-    value = tokens / (ms * 1e-3)
+    ms = max_over_ranks(statistics.mean(times), world, dev)
+    tokens, value = replica_throughput(w.B * w.N, world, ms)
 
     # per-kernel split: the same path as separate calls with events between them
     n_split = min(args.steps, 200)
@@ -539,11 +558,7 @@ def run_ssa(args):
             ssa.forward_host(qh, kh, vh, p, oh, device=dev, dev_bufs=bufs)
         e1.record()
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
         e2e = {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": oh.numel() * oh.element_size(), "ms_per_step": e2e_ms}
@@ -689,13 +704,8 @@ def run_decode(args):
         dist.barrier()
     sampler.stop()
     ssa.check_error()
-    ms = statistics.mean(a.elapsed_time(b) for a, b in zip(starts, ends))
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    tokens = w.B * world
-    value = tokens / (ms * 1e-3)
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(starts, ends)), world, dev)
+    tokens, value = replica_throughput(w.B, world, ms)
     work = decode_work(w, cnt.cpu().numpy(), idx.cpu().numpy())
     peaks, peak_kind = load_peaks()
     hbm = float(peaks["hbm_gbs"])

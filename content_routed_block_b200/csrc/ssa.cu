@@ -248,11 +248,39 @@ cudaError_t launch_route_rows_t(ssa::RouteArgs a, int B, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Row tile: a larger tile reuses each key-summary tile over more query
+// blocks, which pays as long as the grid keeps most SMs busy.  Measured on
+// B200 (route ms for RT = 16 / 32 / 64 / 128): 32K tokens x 14 heads
+// 0.067 / 0.072 / 0.064 / 0.089; 8K tokens x 64 heads 0.044 / 0.031 / 0.027 /
+// 0.038; 16K non-causal x 32 heads 0.536 / 0.340 / 0.265 / 0.208.  Rule: the
+// largest tile whose grid has at least two thirds as many CTAs as SMs.
+// SSA_ROUTE_RT=16|32|64|128 forces one (a tuning hook).
 template <int D, int KM>
 cudaError_t launch_route_rows_km(const ssa::RouteArgs& a, int B, cudaStream_t stream) {
-  const int64_t ctas64 = static_cast<int64_t>(B) * a.Hq * ((a.NQB + 63) / 64);
-  if (ctas64 < 2 * 148) return launch_route_rows_t<D, KM, 16>(a, B, stream);
-  return launch_route_rows_t<D, KM, 64>(a, B, stream);
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  int rt = 16;
+  for (const int cand : {128, 64, 32, 16}) {
+    const int64_t ctas = static_cast<int64_t>(B) * a.Hq * ((a.NQB + cand - 1) / cand);
+    if (3 * ctas >= 2 * static_cast<int64_t>(sms)) {
+      rt = cand;
+      break;
+    }
+  }
+  if (const char* force = std::getenv("SSA_ROUTE_RT")) {
+    const int f = std::atoi(force);
+    if (f == 16 || f == 32 || f == 64 || f == 128) rt = f;
+  }
+  switch (rt) {
+    case 128: return launch_route_rows_t<D, KM, 128>(a, B, stream);
+    case 64: return launch_route_rows_t<D, KM, 64>(a, B, stream);
+    case 32: return launch_route_rows_t<D, KM, 32>(a, B, stream);
+    default: return launch_route_rows_t<D, KM, 16>(a, B, stream);
+  }
 }
 
 // fp32 router: thread-per-row selection for top_k <= 32, warp lists beyond
