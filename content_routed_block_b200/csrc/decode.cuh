@@ -212,7 +212,52 @@ __global__ void __launch_bounds__(kDecThreads) decode_attend_kernel(const Decode
     }
 #pragma unroll
     for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);
-    if (lane == 0) {
+    if constexpr (KM <= 32) {
+      // every lane now holds the top KM; lane j takes entry j (j < top_k), the
+      // warp sorts the block indices ascending and scans the far-segment
+      // lengths (the part of each routed block below the window)
+      int n = 0;
+      uint64_t mine = 0ull;
+#pragma unroll
+      for (int j = 0; j < KM; ++j) {
+        const bool real = j < a.top_k && keys[j] != 0ull;
+        n += real ? 1 : 0;
+        if (j == lane) mine = real ? keys[j] : 0ull;
+      }
+      int c = mine != 0ull ? static_cast<int>(~static_cast<uint32_t>(mine & 0xFFFFFFFFull)) : 0x7FFFFFFF;
+#pragma unroll
+      for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+          const int y = __shfl_xor_sync(0xffffffffu, c, jj);
+          const bool asc = (lane & k) == 0;
+          const bool low = (lane & jj) == 0;
+          c = (low == asc) ? min(c, y) : max(c, y);
+        }
+      }
+      // KM <= 32 here: lanes 0..n-1 hold the selection ascending
+      const int start = c * a.Bk;
+      int len = lane < n ? max(0, min(start + a.Bk, lo) - start) : 0;
+      int incl = len;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (lane < n) {
+        sel[lane] = c;
+        seg_off[lane] = incl - len;
+      }
+      if (lane == n - 1 || (n == 0 && lane == 0)) {
+        seg_off[n] = n ? incl : 0;
+        n_sel_s = n;
+      }
+      if (x == 0) {
+        if (a.cnt != nullptr && lane == 0) a.cnt[bh] = n;
+        if (a.idx != nullptr && lane < a.top_k) a.idx[static_cast<int64_t>(bh) * a.top_k + lane] = lane < n ? c : -1;
+      }
+    } else if (lane == 0) {
+      // top_k > 32: one lane lists the selection
       int v[KM];
       int n = 0;
 #pragma unroll
@@ -230,7 +275,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_attend_kernel(const Decode
           v[y] = h0;
         }
       }
-      // far segments: the part of each routed block below the window
       int off = 0;
 #pragma unroll
       for (int j = 0; j < KM; ++j) {
