@@ -10,11 +10,11 @@
 // with -1, with their count.
 //
 // One warp per (b, KV head, query block).  The g*top_k votes (at most
-// kConsMaxVotes) go to the warp's shared-memory slab, a bitonic sort brings
-// equal blocks together, each run's length is its vote count, and a second
-// sort on the key (votes << 23 | (2^23 - 1 - block)) ranks the runs; the
-// winners are sorted once more by block index.  The work is a few hundred
-// shared-memory operations per query block, negligible beside the router.
+// kConsMaxVotes) are sorted in registers (bitonic: register exchanges and
+// shuffles), which brings equal blocks together; each run's length is its
+// vote count (read from one shared-memory copy); a second sort on the key
+// (votes << 23 | (2^23 - 1 - block)) ranks the runs, and the winners are
+// sorted once more by block index.
 #pragma once
 
 #include "common.cuh"
@@ -34,29 +34,46 @@ struct ConsensusArgs {
   int64_t n_rows;      // B * Hkv * NQB
 };
 
-// bitonic sort of x[0..P) (P a power of two >= 32) by one warp, ascending or
-// descending, through shared memory
-__device__ __forceinline__ void cons_warp_sort(uint32_t* x, int P, bool descending, int lane) {
-  for (int k = 2; k <= P; k <<= 1) {
+// bitonic sort of 32*R values held as element e = lane + 32 r in registers
+// (r-th register of lane `lane`), ascending; partners at distance >= 32 sit
+// in the same lane, the others are reached by shuffles
+template <int R, typename T>
+__device__ __forceinline__ void cons_sort_regs(T (&x)[R], int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32 * R; k <<= 1) {
+#pragma unroll
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = lane; i < P; i += 32) {
-        const int l = i ^ j;
-        if (l > i) {
-          const uint32_t u = x[i], w = x[l];
-          const bool up = (((i & k) == 0) != descending);
-          if ((u > w) == up) {
-            x[i] = w;
-            x[l] = u;
+      if (j >= 32) {
+        const int jr = j >> 5;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int pr = r ^ jr;
+          if (pr > r) {
+            const bool asc = ((lane + 32 * r) & k) == 0;
+            const T lo = x[r] < x[pr] ? x[r] : x[pr], hi = x[r] < x[pr] ? x[pr] : x[r];
+            x[r] = asc ? lo : hi;
+            x[pr] = asc ? hi : lo;
           }
         }
+      } else {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const T y = __shfl_xor_sync(0xffffffffu, x[r], j);
+          const bool asc = ((lane + 32 * r) & k) == 0;
+          const bool low = (lane & j) == 0;
+          x[r] = (low == asc) ? (x[r] < y ? x[r] : y) : (x[r] < y ? y : x[r]);
+        }
       }
-      __syncwarp();
     }
   }
 }
 
+// R = P / 32 entries per lane, P = the vote count g*top_k rounded up to a
+// power of two (>= 32)
+template <int R>
 __global__ void __launch_bounds__(kConsThreads) consensus_kernel(const ConsensusArgs a) {
-  __shared__ uint32_t slab[kConsWarps][kConsMaxVotes];
+  constexpr int P = 32 * R;
+  __shared__ uint32_t slab[kConsWarps][P];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kConsWarps + warp;
   if (row >= a.n_rows) return;  // warp-uniform
@@ -66,13 +83,14 @@ __global__ void __launch_bounds__(kConsThreads) consensus_kernel(const Consensus
   const int qb = static_cast<int>(row % a.NQB);
   const int b = static_cast<int>(bkv / a.Hkv), kv = static_cast<int>(bkv % a.Hkv);
   const int E = g * k;
-  int P = 32;
-  while (P < E) P <<= 1;
   uint32_t* x = slab[warp];
   constexpr uint32_t kEmpty = 0xFFFFFFFFu;
 
   // 1. the group's votes: entry e is head (e / k)'s (e % k)-th block
-  for (int e = lane; e < P; e += 32) {
+  uint32_t v[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = lane + 32 * r;
     uint32_t val = kEmpty;
     if (e < E) {
       const int j = e / k, t = e % k;
@@ -90,61 +108,55 @@ __global__ void __launch_bounds__(kConsThreads) consensus_kernel(const Consensus
           record_error(kErrCheck, kSiteCons);
       }
     }
-    x[e] = val;
+    v[r] = val;
   }
-  __syncwarp();
-  cons_warp_sort(x, P, false, lane);
+  cons_sort_regs<R>(v, lane);
 
   // 2. one key per distinct block (at the first entry of its run):
   //    votes << 23 | (2^23 - 1 - block); 0 elsewhere.  Blocks are < 2^23
   //    (checked by the host) and votes <= P <= 512 < 2^9.
-  constexpr int kMaxPer = kConsMaxVotes / 32;
-  uint32_t key[kMaxPer];
 #pragma unroll
-  for (int s = 0; s < kMaxPer; ++s) {
-    const int e = lane + 32 * s;
-    key[s] = 0u;
-    if (e < P) {
-      const uint32_t c = x[e];
-      if (c != kEmpty && (e == 0 || x[e - 1] != c)) {
-        uint32_t votes = 1;
-        while (e + static_cast<int>(votes) < P && x[e + votes] == c) ++votes;
-        key[s] = (votes << 23) | (0x7FFFFFu - c);
-      }
+  for (int r = 0; r < R; ++r) x[lane + 32 * r] = v[r];
+  __syncwarp();
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = lane + 32 * r;
+    const uint32_t c = v[r];
+    uint32_t key = 0u;
+    if (c != kEmpty && (e == 0 || x[e - 1] != c)) {
+      uint32_t votes = 1;
+      while (e + static_cast<int>(votes) < P && x[e + votes] == c) ++votes;
+      key = (votes << 23) | (0x7FFFFFu - c);
     }
+    v[r] = ~key;  // ascending sort of ~key == descending sort of key
   }
-  __syncwarp();
-#pragma unroll
-  for (int s = 0; s < kMaxPer; ++s) {
-    const int e = lane + 32 * s;
-    if (e < P) x[e] = key[s];
-  }
-  __syncwarp();
-  cons_warp_sort(x, P, true, lane);
+  cons_sort_regs<R>(v, lane);
 
-  // 3. the first min(k, #runs) keys win; list their blocks ascending
-  int P2 = 32;
-  while (P2 < k) P2 <<= 1;  // k <= 64, so P2 <= 64 <= P
-  uint32_t win[2];
+  // 3. the first min(k, #runs) keys win; list their blocks ascending.  The
+  //    winners are elements 0 .. k-1 (k <= 64: registers 0 and 1).
+  uint32_t w[2];
   int n_win = 0;
 #pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    const int e = lane + 32 * s;
-    const uint32_t kk = (e < P2) ? x[e] : 0u;
+  for (int r = 0; r < 2; ++r) {
+    const uint32_t kk = (r < R) ? ~v[r] : 0u;
+    const int e = lane + 32 * r;
     const bool real = e < k && kk != 0u;
-    win[s] = real ? (0x7FFFFFu - (kk & 0x7FFFFFu)) : kEmpty;
+    w[r] = real ? (0x7FFFFFu - (kk & 0x7FFFFFu)) : kEmpty;
     n_win += __popc(__ballot_sync(0xffffffffu, real));
   }
-  __syncwarp();
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    const int e = lane + 32 * s;
-    if (e < P2) x[e] = win[s];
+  if (k > 32) {
+    cons_sort_regs<2>(w, lane);
+  } else {
+    uint32_t w1[1] = {w[0]};
+    cons_sort_regs<1>(w1, lane);
+    w[0] = w1[0];
   }
-  __syncwarp();
-  cons_warp_sort(x, P2, false, lane);
   int32_t* dst = a.idx_kv + (bkv * a.NQB + qb) * k;
-  for (int e = lane; e < k; e += 32) dst[e] = e < n_win ? static_cast<int32_t>(x[e]) : -1;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int e = lane + 32 * r;
+    if (e < k) dst[e] = e < n_win ? static_cast<int32_t>(w[r]) : -1;
+  }
   if (lane == 0) a.cnt_kv[bkv * a.NQB + qb] = n_win;
 }
 

@@ -505,7 +505,16 @@ ssa_status launch_consensus(const ssa_params* p, const int32_t* idx, const int32
   a.n_rows = static_cast<int64_t>(p->B) * p->Hkv * a.NQB;
   const int64_t grid = (a.n_rows + ssa::kConsWarps - 1) / ssa::kConsWarps;
   if (grid > 0x7FFFFFFF) return fail(SSA_ERR_UNSUPPORTED, "too many query blocks");
-  ssa::consensus_kernel<<<static_cast<unsigned>(grid), ssa::kConsThreads, 0, stream>>>(a);
+  int P = 32;
+  while (P < (p->Hq / p->Hkv) * p->top_k) P <<= 1;
+  const unsigned gr = static_cast<unsigned>(grid);
+  switch (P) {
+    case 32: ssa::consensus_kernel<1><<<gr, ssa::kConsThreads, 0, stream>>>(a); break;
+    case 64: ssa::consensus_kernel<2><<<gr, ssa::kConsThreads, 0, stream>>>(a); break;
+    case 128: ssa::consensus_kernel<4><<<gr, ssa::kConsThreads, 0, stream>>>(a); break;
+    case 256: ssa::consensus_kernel<8><<<gr, ssa::kConsThreads, 0, stream>>>(a); break;
+    default: ssa::consensus_kernel<16><<<gr, ssa::kConsThreads, 0, stream>>>(a); break;
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "consensus_kernel launch");
   return SSA_OK;
