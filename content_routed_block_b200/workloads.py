@@ -67,6 +67,8 @@ class Workload:
     needle_gap: int = 4096     # needles only: minimum query-after-key distance
     consensus: bool = False    # one route per (batch, KV head, query block), voted by its heads
     beta: float = 0.0          # weight of the second-cumulant routing term
+    tree_fanout: int = 0       # two-level routing: key blocks per super-block (0: flat)
+    tree_beam: int = 0         # two-level routing: super-blocks kept per query block
 
     @property
     def n_kblocks(self) -> int:

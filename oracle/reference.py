@@ -37,6 +37,11 @@ non-causal variant):
    -- one list per (b, KV head, query block) that all of the group's heads
    use ("Complete 10M transformer result": a cross-head consensus route
    carrying the highest-vote blocks).
+6c. (Optional, ``Params.tree_fanout``) two-level fixed-beam routing: the
+   blocks are grouped F at a time into super-blocks summarised by their key
+   means; a query block keeps its best tree_beam complete admissible
+   super-blocks (step 6's order) and selects its top_k blocks (step 6) among
+   their children and the frontier blocks (``route_tree_row``).
 7. Key set of query i as a SET: the keys of its query block's selected blocks
    united with the local causal window {j : i - W < j <= i} and cut at i
    (causal); only the selected blocks' keys (non-causal).  A key that is both
@@ -63,7 +68,8 @@ __all__ = [
     "near_tie_rows", "acceptable_selections", "route_row",
     "consensus_row", "route_consensus", "expand_consensus",
     "block_covariance", "block_second_moment", "block_scores", "decode_step",
-    "decode_attend",
+    "decode_attend", "tree_summary", "tree_candidates", "route_tree_row",
+    "acceptable_tree_selections",
 ]
 
 NEAR_TIE_REL = 1e-4   # relative score gap under which two blocks count as tied
@@ -85,6 +91,8 @@ class Params:
     scale: float = 0.0          # 0 -> 1/sqrt(D)
     consensus: bool = False     # GQA-shared (consensus) routing, see route_consensus
     beta: float = 0.0           # weight of the second-cumulant score term, see block_scores
+    tree_fanout: int = 0        # two-level routing: key blocks per super-block (0: flat)
+    tree_beam: int = 0          # super-blocks kept at the upper level, see route_tree_row
 
     @property
     def group(self) -> int:
@@ -107,7 +115,8 @@ class Params:
         """Build from any object with the same field names (e.g. a workload)."""
         return Params(w.B, w.Hq, w.Hkv, w.N, w.D, w.block_k, w.block_q, w.top_k,
                       w.window, bool(w.causal), getattr(w, "scale", 0.0),
-                      bool(getattr(w, "consensus", False)), float(getattr(w, "beta", 0.0)))
+                      bool(getattr(w, "consensus", False)), float(getattr(w, "beta", 0.0)),
+                      int(getattr(w, "tree_fanout", 0)), int(getattr(w, "tree_beam", 0)))
 
 
 def upcast_bf16(u16: np.ndarray) -> np.ndarray:
@@ -198,6 +207,8 @@ class RouteResult:
     cnt: np.ndarray        # int32 [B, Hq, NQB]
     kth: np.ndarray        # float64 [B, Hq, NQB]: k-th best score (nan if none)
     next: np.ndarray       # float64 [B, Hq, NQB]: (k+1)-th best score (nan if none)
+    sup_idx: np.ndarray = None   # tree form: int32 [B, Hq, NQB, tree_beam] kept super-blocks
+    sup_cnt: np.ndarray = None   # tree form: int32 [B, Hq, NQB]
 
 
 def route_row(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, top_k: int,
@@ -219,31 +230,49 @@ def route_row(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, top_k: int,
 
 
 def route(qsum: np.ndarray, ksum: np.ndarray, p: Params, rows=None, qm2=None,
-          kcov=None) -> RouteResult:
+          kcov=None, ksum2=None) -> RouteResult:
     """Top-k routing for every (b, query head, query block).
 
     ``qsum`` [B, Hq, NQB, D] and ``ksum`` [B, Hkv, NB, D] are block summaries
     (float64); with ``p.beta`` != 0 also ``qm2`` [B, Hq, NQB, D, D]
     (``block_second_moment`` of Q) and ``kcov`` [B, Hkv, NB, D, D]
-    (``block_covariance`` of K).  ``rows`` optionally restricts the work to a
-    list of (b, h, qb) triples; the arrays keep their full shape and rows not
-    listed stay at idx = -1, cnt = 0, scores nan."""
+    (``block_covariance`` of K); with ``p.tree_fanout`` > 0 (two-level form,
+    ``route_tree_row``) also ``ksum2`` [B, Hkv, NS, D] (``tree_summary``).
+    ``rows`` optionally restricts the work to a list of (b, h, qb) triples;
+    the arrays keep their full shape and rows not listed stay at idx = -1,
+    cnt = 0, scores nan."""
     nqb = p.n_qblocks
     idx = np.full((p.B, p.Hq, nqb, p.top_k), -1, dtype=np.int32)
     cnt = np.zeros((p.B, p.Hq, nqb), dtype=np.int32)
     kth = np.full((p.B, p.Hq, nqb), math.nan)
     nxt = np.full((p.B, p.Hq, nqb), math.nan)
+    tree = p.tree_fanout > 0
+    if tree:
+        if p.beta != 0.0:
+            raise ValueError("the two-level form scores by block means only (beta = 0)")
+        if ksum2 is None:
+            raise ValueError("the two-level form needs the super-block summaries ksum2")
+        sup_idx = np.full((p.B, p.Hq, nqb, p.tree_beam), -1, dtype=np.int32)
+        sup_cnt = np.zeros((p.B, p.Hq, nqb), dtype=np.int32)
     todo = rows if rows is not None else [
         (b, h, qb) for b in range(p.B) for h in range(p.Hq) for qb in range(nqb)]
     for b, h, qb in todo:
         mu = ksum[b, h // p.group]
-        extra = {}
-        if p.beta != 0.0:
-            extra = dict(beta=p.beta, q2=qm2[b, h, qb], sigma=kcov[b, h // p.group])
-        sel, a, c = route_row(qsum[b, h, qb], mu, admissible_blocks(qb, p), p.top_k, **extra)
+        if tree:
+            sup, sel, a, c = route_tree_row(qsum[b, h, qb], mu, ksum2[b, h // p.group],
+                                            len(admissible_blocks(qb, p)), p)
+            sup_idx[b, h, qb, :len(sup)] = sup
+            sup_cnt[b, h, qb] = len(sup)
+        else:
+            extra = {}
+            if p.beta != 0.0:
+                extra = dict(beta=p.beta, q2=qm2[b, h, qb], sigma=kcov[b, h // p.group])
+            sel, a, c = route_row(qsum[b, h, qb], mu, admissible_blocks(qb, p), p.top_k, **extra)
         idx[b, h, qb, :len(sel)] = sel
         cnt[b, h, qb] = len(sel)
         kth[b, h, qb], nxt[b, h, qb] = a, c
+    if tree:
+        return RouteResult(idx, cnt, kth, nxt, sup_idx, sup_cnt)
     return RouteResult(idx, cnt, kth, nxt)
 
 
@@ -283,6 +312,69 @@ def acceptable_selections(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, to
         out.append(np.sort(np.concatenate([sure, np.array(combo, dtype=sure.dtype)])))
         if len(out) >= limit:
             break
+    return out
+
+
+# --------------------------------------------------------------------------
+# steps 5-6, two-level form (optional): fixed-beam tree routing
+# --------------------------------------------------------------------------
+# jonsmirl/ssa README, "Algorithm and complexity": a hierarchical router with
+# a fixed block size and a fixed budget approaches linear routing work on
+# benign geometry, where a flat router scans every block; the measured 10M
+# tree uses fanout 16.  "Mathematical status": fixed-beam routing is not an
+# exact selector (its retrieval quality is an empirical matter).  Here the
+# tree has two levels: super-block S covers the F key blocks S*F .. S*F+F-1
+# and is summarised by the mean of its F*Bk keys; a query block scores the
+# super-blocks like blocks (step 5), keeps the best tree_beam of them
+# (step 6's order), and then selects its top_k blocks (step 6) among the
+# children of the kept super-blocks plus the frontier -- the admissible
+# blocks of the one super-block that is not yet completely admissible.  With
+# every super-block kept this is the flat selection.
+def tree_summary(k: np.ndarray, block_k: int, fanout: int) -> np.ndarray:
+    """Super-block summaries of ``k[..., N, D]``: the mean of the F*Bk keys
+    of every complete super-block (N // (F*Bk) of them), [..., NS, D]."""
+    span = fanout * block_k
+    ns = k.shape[-2] // span
+    return block_summary(k[..., :ns * span, :], span)
+
+
+def tree_candidates(sup, n_adm: int, fanout: int) -> np.ndarray:
+    """Blocks scored at the lower level: the ``fanout`` children of every
+    kept super-block ``sup``, then the frontier blocks (admissible blocks
+    0 .. n_adm-1 past the last complete admissible super-block)."""
+    ns = n_adm // fanout
+    kids = (np.asarray(sup, dtype=np.int64)[:, None] * fanout
+            + np.arange(fanout, dtype=np.int64)[None, :]).ravel()
+    return np.concatenate([kids, np.arange(ns * fanout, n_adm, dtype=np.int64)])
+
+
+def route_tree_row(qbar: np.ndarray, mu: np.ndarray, mu2: np.ndarray, n_adm: int, p: Params):
+    """Two-level selection for one query-block summary.  The admissible key
+    blocks are 0 .. n_adm-1 (step 4); the complete admissible super-blocks
+    are 0 .. n_adm // F - 1.  Returns (kept super-blocks ascending, selected
+    blocks ascending, k-th score, (k+1)-th score) -- the scores of the lower
+    level, among its candidates."""
+    F = p.tree_fanout
+    sup, _, _ = route_row(qbar, mu2, np.arange(n_adm // F, dtype=np.int64), p.tree_beam)
+    sel, kth, nxt = route_row(qbar, mu, tree_candidates(sup, n_adm, F), p.top_k)
+    return sup, sel, kth, nxt
+
+
+def acceptable_tree_selections(qbar: np.ndarray, mu: np.ndarray, mu2: np.ndarray, n_adm: int,
+                               p: Params, rel: float = NEAR_TIE_REL, limit: int = 256) -> list:
+    """Every (kept super-blocks, selected blocks) pair that the near-tie rule
+    accepts at both levels: any super-block set ``acceptable_selections``
+    accepts at the upper level, each followed by any selection it accepts
+    among that set's candidates.  At most ``limit`` pairs."""
+    F = p.tree_fanout
+    out = []
+    for sup in acceptable_selections(qbar, mu2, np.arange(n_adm // F, dtype=np.int64),
+                                     p.tree_beam, rel, limit):
+        for sel in acceptable_selections(qbar, mu, tree_candidates(sup, n_adm, F), p.top_k,
+                                         rel, limit):
+            out.append((sup, sel))
+            if len(out) >= limit:
+                return out
     return out
 
 
@@ -478,9 +570,13 @@ def forward(q, k, v, p: Params, form: str = "dense"):
     head of a group attends over its group's list."""
     ksum = block_summary(k, p.block_k)
     qsum = block_summary(q, p.block_q)
+    ksum2 = None
     if p.beta != 0.0:
         r = route(qsum, ksum, p, qm2=block_second_moment(q, p.block_q),
                   kcov=block_covariance(k, p.block_k))
+    elif p.tree_fanout > 0:
+        ksum2 = tree_summary(k, p.block_k, p.tree_fanout)
+        r = route(qsum, ksum, p, ksum2=ksum2)
     else:
         r = route(qsum, ksum, p)
     attend = attend_masked_dense if form == "dense" else attend_gathered
@@ -491,4 +587,4 @@ def forward(q, k, v, p: Params, form: str = "dense"):
         idx, cnt = r.idx, r.cnt
         o, lse = attend(q, k, v, idx, cnt, p)
     return {"o": o, "lse": lse, "idx": idx, "cnt": cnt, "route": r,
-            "qsum": qsum, "ksum": ksum}
+            "qsum": qsum, "ksum": ksum, "ksum2": ksum2}

@@ -620,3 +620,161 @@ def test_decode_step_dense_and_sliding_window_limits():
     o, _, _, _ = O.decode_step(q[:, :, i], k, v, N, win)
     want = _sdpa(q[:, :, i:i + 1], k[:, :, i - W + 1:], v[:, :, i - W + 1:], gqa=True)[:, :, 0]
     np.testing.assert_allclose(o, want, atol=1e-12, rtol=0)
+
+
+# ---------------------------------------------------------------- two-level (tree) routing
+def _tree_worked_inputs():
+    k = np.array([[1, 0], [1, 0], [4, 0], [-4, 0], [0, 1], [0, 0], [2, 0], [0, 0]],
+                 dtype=np.float64)[None, None]
+    q = np.tile(np.array([[1.0, 0.0]]), (8, 1))[None, None]
+    return q, k
+
+
+def _lst(tok):
+    return [] if tok == "-" else [int(x) for x in tok.split(",")]
+
+
+def test_tree_route_matches_hand_derivation():
+    q, k = _tree_worked_inputs()
+    ksum = O.block_summary(k, 1)
+    qsum = O.block_summary(q, 1)
+    ksum2 = O.tree_summary(k, 1, 2)
+    assert ksum2[0, 0].tolist() == [[1, 0], [0, 0], [0, 0.5], [1, 0]]
+    n = 0
+    with open(os.path.join(GOLDEN, "tree_route.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            causal, qb, beam, kk, sup, sel = line.split()
+            causal = bool(int(causal))
+            p = _params(N=8, block_k=1, block_q=1, top_k=int(kk), causal=causal,
+                        window=1 if causal else 0, tree_fanout=2, tree_beam=int(beam))
+            r = O.route(qsum, ksum, p, rows=[(0, 0, int(qb))], ksum2=ksum2)
+            row = (0, 0, int(qb))
+            assert r.sup_idx[row][:r.sup_cnt[row]].tolist() == _lst(sup), line
+            assert r.idx[row][:r.cnt[row]].tolist() == _lst(sel), line
+            n += 1
+    assert n == 10
+
+
+def test_tree_summary_is_the_mean_of_its_child_block_means():
+    rng = np.random.default_rng(41)
+    k = rng.standard_normal((2, 3, 16 * 22, 5))          # 22 blocks of 16: 5 super-blocks of 4
+    got = O.tree_summary(k, 16, 4)
+    assert got.shape == (2, 3, 5, 5)
+    mu = O.block_summary(k, 16)
+    for s in range(5):
+        np.testing.assert_allclose(got[:, :, s], mu[:, :, 4 * s:4 * s + 4].mean(axis=2),
+                                   atol=1e-14)
+        np.testing.assert_allclose(got[:, :, s], k[:, :, 64 * s:64 * s + 64].mean(axis=2),
+                                   atol=1e-14)
+
+
+def _tree_case(causal, N=16 * 22, D=6, bk=16, F=4, beam=2, top_k=3, Hq=2, Hkv=1, seed=43):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, Hq, N, D))
+    k = rng.standard_normal((1, Hkv, N, D)) + rng.standard_normal((1, Hkv, N // bk, 1, D)).repeat(
+        bk, axis=2).reshape(1, Hkv, N, D)
+    p = _params(Hq=Hq, Hkv=Hkv, N=N, D=D, block_k=bk, block_q=bk, top_k=top_k, causal=causal,
+                window=bk if causal else 0, tree_fanout=F, tree_beam=beam)
+    return p, q, k
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_tree_keeping_every_super_block_is_the_flat_route(causal):
+    p, q, k = _tree_case(causal, beam=64, top_k=4)
+    ksum, qsum = O.block_summary(k, p.block_k), O.block_summary(q, p.block_q)
+    tree = O.route(qsum, ksum, p, ksum2=O.tree_summary(k, p.block_k, p.tree_fanout))
+    flat = O.route(qsum, ksum, O.Params(**{**p.__dict__, "tree_fanout": 0, "tree_beam": 0}))
+    np.testing.assert_array_equal(tree.idx, flat.idx)
+    np.testing.assert_array_equal(tree.cnt, flat.cnt)
+    assert (tree.cnt > 0).any()
+
+
+def test_tree_with_fanout_one_keeps_the_flat_top_k():
+    p, q, k = _tree_case(True, F=1, beam=5, top_k=3)
+    ksum, qsum = O.block_summary(k, p.block_k), O.block_summary(q, p.block_q)
+    tree = O.route(qsum, ksum, p, ksum2=O.tree_summary(k, p.block_k, 1))
+    flat = O.route(qsum, ksum, O.Params(**{**p.__dict__, "tree_fanout": 0, "tree_beam": 0}))
+    np.testing.assert_array_equal(tree.idx, flat.idx)
+    # the upper level alone is the flat top-beam
+    flat5 = O.route(qsum, ksum, O.Params(**{**p.__dict__, "tree_fanout": 0, "tree_beam": 0,
+                                            "top_k": 5}))
+    np.testing.assert_array_equal(tree.sup_idx, flat5.idx)
+
+
+def _top_set_brute(keys_of, items, m):
+    """The one m-subset of ``items`` whose every member's (score, -index) key
+    beats every non-member's, found by enumerating all m-subsets."""
+    import itertools
+    found = []
+    for sub in itertools.combinations(items, m):
+        rest = [c for c in items if c not in sub]
+        if all(keys_of(a) > keys_of(b) for a in sub for b in rest):
+            found.append(sorted(sub))
+    assert len(found) == 1
+    return found[0]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_tree_route_matches_brute_force_on_tiny_integer_inputs(causal):
+    from fractions import Fraction
+    rng = np.random.default_rng(47 + causal)
+    bk, F, N, D, beam, top_k = 4, 2, 52, 3, 2, 3            # 13 blocks: 6 super-blocks + 1
+    # small integers: exact in float64 and full of exact ties
+    k = rng.integers(-2, 3, size=(1, 1, N, D)).astype(np.float64)
+    q = rng.integers(-2, 3, size=(1, 1, N, D)).astype(np.float64)
+    p = _params(N=N, D=D, block_k=bk, block_q=bk, top_k=top_k, causal=causal,
+                window=bk if causal else 0, tree_fanout=F, tree_beam=beam)
+    r = O.route(O.block_summary(q, bk), O.block_summary(k, bk), p,
+                ksum2=O.tree_summary(k, bk, F))
+    kk, qq = k[0, 0].astype(int).tolist(), q[0, 0].astype(int).tolist()
+
+    def mean_rows(x, lo, hi):
+        return [Fraction(sum(x[t][d] for t in range(lo, hi)), hi - lo) for d in range(D)]
+
+    nb = N // bk
+    for qb in range(N // bk):
+        qbar = mean_rows(qq, qb * bk, qb * bk + bk)
+        n_adm = min(qb, nb) if causal else nb             # Bq = Bk: c + 1 <= qb
+        score_blk = lambda c: sum(a * b for a, b in zip(qbar, mean_rows(kk, c * bk, c * bk + bk)))
+        score_sup = lambda s: sum(a * b for a, b in
+                                  zip(qbar, mean_rows(kk, s * F * bk, (s + 1) * F * bk)))
+        sups = list(range(n_adm // F))
+        kept = _top_set_brute(lambda s: (score_sup(s), -s), sups, min(beam, len(sups)))
+        cand = [s * F + j for s in kept for j in range(F)] + list(range(len(sups) * F, n_adm))
+        sel = _top_set_brute(lambda c: (score_blk(c), -c), cand, min(top_k, len(cand)))
+        assert r.sup_idx[0, 0, qb][:r.sup_cnt[0, 0, qb]].tolist() == kept, qb
+        assert r.idx[0, 0, qb][:r.cnt[0, 0, qb]].tolist() == sel, qb
+
+
+def test_tree_acceptable_selections_hold_the_route_and_its_tie_alternatives():
+    q, k = _tree_worked_inputs()
+    p = _params(N=8, block_k=1, block_q=1, top_k=2, causal=False, window=0, tree_fanout=2,
+                tree_beam=1)
+    mu, mu2 = O.block_summary(k, 1)[0, 0], O.tree_summary(k, 1, 2)[0, 0]
+    qbar = np.array([1.0, 0.0])
+    acc = [(a.tolist(), b.tolist()) for a, b in O.acceptable_tree_selections(qbar, mu, mu2, 8, p)]
+    # S0 and S3 tie exactly: both beams are acceptable; inside S0, blocks 0
+    # and 1 are both taken; inside S3, block 6 and then 7 (score 0, alone)
+    assert ([0], [0, 1]) in acc and ([3], [6, 7]) in acc
+    assert len(acc) == 2
+    sup, sel, _, _ = O.route_tree_row(qbar, mu, mu2, 8, p)
+    assert (sup.tolist(), sel.tolist()) == ([0], [0, 1])
+
+
+def test_tree_forward_attends_over_the_tree_selection():
+    p, q, k = _tree_case(True, N=16 * 12, beam=1, top_k=2)
+    v = np.random.default_rng(5).standard_normal(k.shape)
+    out = O.forward(q, k, v, p)
+    r = out["route"]
+    assert r.sup_idx is not None and out["ksum2"].shape[2] == 3
+    o2, l2 = O.attend_gathered(q, k, v, r.idx, r.cnt, p)
+    np.testing.assert_allclose(out["o"], o2, atol=1e-12)
+    np.testing.assert_allclose(out["lse"], l2, atol=1e-12)
+    # every selected block is a candidate of the row's kept super-blocks
+    for qb in range(p.n_qblocks):
+        n_adm = len(O.admissible_blocks(qb, p))
+        cand = O.tree_candidates(r.sup_idx[0, 0, qb][:r.sup_cnt[0, 0, qb]], n_adm, p.tree_fanout)
+        assert set(r.idx[0, 0, qb][:r.cnt[0, 0, qb]].tolist()) <= set(cand.tolist())
