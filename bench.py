@@ -65,6 +65,10 @@ def parse_args(argv=None):
                          "workload's full K/V cache) instead of the prefill")
     ap.add_argument("--beta", type=float, default=0.0,
                     help="weight of the second-cumulant routing term (0: mean summaries only)")
+    ap.add_argument("--tree-fanout", type=int, default=0,
+                    help="two-level (fixed-beam tree) routing: key blocks per super-block")
+    ap.add_argument("--tree-beam", type=int, default=0,
+                    help="two-level routing: super-blocks kept per query block (default top_k)")
     ap.add_argument("--consensus", action="store_true",
                     help="GQA-shared consensus routing: the query heads of a KV group vote "
                          "and share one list per query block")
@@ -237,7 +241,7 @@ def _cpu_worker(args):
     sys.path.insert(0, ROOT)
     import oracle as O
     from content_routed_block_b200.workloads import CONFIGS, make_inputs
-    cfg, seq_len, consensus, beta, b, h, blocks, seconds = args
+    cfg, seq_len, consensus, beta, tree, b, h, blocks, seconds = args
     w = CONFIGS[cfg]
     if seq_len:
         w = w.with_(N=seq_len)
@@ -246,7 +250,8 @@ def _cpu_worker(args):
     # every head of the KV group, which vote on one shared list
     heads = list(range((h // g) * g, (h // g + 1) * g)) if consensus else [h]
     x = make_inputs(w, q_heads=heads, kv_heads=[h // g])
-    sub = w.with_(Hq=len(heads), Hkv=1, B=1, consensus=consensus, beta=beta)
+    sub = w.with_(Hq=len(heads), Hkv=1, B=1, consensus=consensus, beta=beta,
+                  tree_fanout=tree[0], tree_beam=tree[1])
     p = O.Params.of(sub)
     q = O.upcast_bf16(x["q"][b:b + 1])           # the requested heads, in order
     k = O.upcast_bf16(x["k"][b:b + 1])
@@ -254,6 +259,7 @@ def _cpu_worker(args):
     t0 = time.perf_counter()
     ksum = O.block_summary(k, p.block_k)
     kcov = O.block_covariance(k[0, 0], p.block_k) if p.beta else None
+    ksum2 = O.tree_summary(k, p.block_k, p.tree_fanout) if p.tree_fanout else None
     done = 0
     nh = len(heads)
     idx = np.full((1, nh, p.n_qblocks, p.top_k), -1, np.int32)
@@ -266,8 +272,12 @@ def _cpu_worker(args):
             if p.beta:
                 extra = dict(beta=p.beta, q2=O.block_second_moment(rows, p.block_q)[0, 0, 0],
                              sigma=kcov)
-            sel, _, _ = O.route_row(qbar, ksum[0, 0], O.admissible_blocks(qb, p), p.top_k,
-                                    **extra)
+            if p.tree_fanout:
+                _, sel, _, _ = O.route_tree_row(qbar, ksum[0, 0], ksum2[0, 0],
+                                                len(O.admissible_blocks(qb, p)), p)
+            else:
+                sel, _, _ = O.route_row(qbar, ksum[0, 0], O.admissible_blocks(qb, p), p.top_k,
+                                        **extra)
             idx[0, j, qb, :len(sel)] = sel
             cnt[0, j, qb] = len(sel)
         if consensus:
@@ -283,12 +293,14 @@ def _cpu_worker(args):
 
 
 class OraclePool:
-    def __init__(self, cfg: int, seq_len: int = 0, consensus: bool = False, beta: float = 0.0):
+    def __init__(self, cfg: int, seq_len: int = 0, consensus: bool = False, beta: float = 0.0,
+                 tree=(0, 0)):
         import multiprocessing as mp
         self.cfg = cfg
         self.seq_len = seq_len
         self.consensus = consensus
         self.beta = beta
+        self.tree = tuple(tree)
         self.cores = max(1, min(len(os.sched_getaffinity(0)), 64))
         old = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
         for k in old:
@@ -320,7 +332,8 @@ class OraclePool:
             b = c % w.B
             h = (c // w.B) % w.Hq
             blocks = rng.permutation(nqb).tolist()
-            tasks.append((self.cfg, self.seq_len, self.consensus, self.beta, b, h, blocks, seconds))
+            tasks.append((self.cfg, self.seq_len, self.consensus, self.beta, self.tree, b, h,
+                          blocks, seconds))
         res = self.pool.map(_cpu_worker, tasks)
         blocks = sum(r[0] for r in res)
         wall = max(r[1] for r in res)
@@ -336,7 +349,7 @@ def run_reference(args):
         return
     w = workload_of(args)
     per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
-    pool = OraclePool(args.config, args.seq_len, args.consensus, args.beta)
+    pool = OraclePool(args.config, args.seq_len, args.consensus, args.beta, tree_of(w))
     try:
         for _ in range(args.warmup):
             pool.run(per_step)
@@ -375,7 +388,15 @@ def workload_of(args):
         w = w.with_(consensus=True, name=f"{w.name}+consensus")
     if getattr(args, "beta", 0.0):
         w = w.with_(beta=float(args.beta), name=f"{w.name}+beta{args.beta:g}")
+    if getattr(args, "tree_fanout", 0):
+        beam = args.tree_beam or w.top_k
+        w = w.with_(tree_fanout=args.tree_fanout, tree_beam=beam,
+                    name=f"{w.name}+tree{args.tree_fanout}x{beam}")
     return w
+
+
+def tree_of(w):
+    return (int(getattr(w, "tree_fanout", 0)), int(getattr(w, "tree_beam", 0)))
 
 
 def workload_config(w, args):
@@ -383,7 +404,8 @@ def workload_config(w, args):
                         f"Bk={w.block_k} Bq={w.block_q} top_k={w.top_k} W={w.window} "
                         f"{'causal' if w.causal else 'non-causal'} {w.kind}"
                         f"{' consensus-routed' if w.consensus else ''}"
-                        f"{f' second-cumulant beta={w.beta:g}' if w.beta else ''}",
+                        f"{f' second-cumulant beta={w.beta:g}' if w.beta else ''}"
+                        f"{f' two-level routing fanout={w.tree_fanout} beam={w.tree_beam}' if w.tree_fanout else ''}",
             "global_batch": w.B * args.gpus, "seq_len": w.N, "parallelism": f"replicas{args.gpus}",
             "l2": "flushed between timed steps (256 MiB write)"}
 
@@ -470,12 +492,19 @@ def run_ssa(args):
 
     # per-kernel split: the same path as separate calls with events between them
     n_split = min(args.steps, 200)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_split)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(n_split)]
     F = w.D + w.D * (w.D + 1) // 2 if w.beta else w.D      # summary / feature length
     ks = torch.empty((w.B, w.Hkv, w.N // w.block_k, F), dtype=torch.float32, device=dev)
     qs = torch.empty((w.B, w.Hq, w.N // w.block_q, F), dtype=torch.float32, device=dev)
     sc = (torch.empty((w.B, w.Hq, w.N // w.block_q, w.N // w.block_k), dtype=torch.float32,
                       device=dev) if w.beta else None)
+    tree = w.tree_fanout > 0
+    if tree:
+        ks2 = torch.empty((w.B, w.Hkv, (w.N // w.block_k) // w.tree_fanout, w.D),
+                          dtype=torch.float32, device=dev)
+        sup = torch.empty((w.B, w.Hq, w.N // w.block_q, w.tree_beam), dtype=torch.int32,
+                          device=dev)
+        supc = torch.empty((w.B, w.Hq, w.N // w.block_q), dtype=torch.int32, device=dev)
     L = ssa.lib()
     import ctypes
     st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -494,24 +523,41 @@ def run_ssa(args):
             e[1].record()
             assert L.ssa_block_summary(pp, P(qd), w.Hq, w.block_q, P(qs), st) == 0
         e[2].record()
+        if tree:
+            assert L.ssa_tree_summary(pp, P(ks), P(ks2), st) == 0
+        e[3].record()
         ri, rc = (idx_h, cnt_h) if w.consensus else (idx, cnt)
         if w.beta:
             assert L.ssa_route_cumulant(pp, P(qs), P(ks), P(sc), P(ri) if w.top_k else None,
                                         P(rc), st) == 0
+        elif tree:
+            assert L.ssa_route_tree(pp, P(qs), P(ks), P(ks2), P(sup), P(supc),
+                                    P(ri) if w.top_k else None, P(rc), st) == 0
         else:
             assert L.ssa_route(pp, P(qs), P(ks), P(ri) if w.top_k else None, P(rc), st) == 0
-        e[3].record()
+        e[4].record()
         if w.consensus:
             assert L.ssa_route_consensus(pp, P(idx_h) if w.top_k else None, P(cnt_h),
                                          P(idx) if w.top_k else None, P(cnt), st) == 0
-        e[4].record()
+        e[5].record()
         assert L.ssa_attend(pp, P(qd), P(kd), P(vd), P(idx) if w.top_k else None, P(cnt),
                             P(o), P(lse), st) == 0
-        e[5].record()
+        e[6].record()
     torch.cuda.synchronize()
     ssa.check_error()
     seg = lambda i: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(n_split))  # noqa: E731
-    pool_k_ms, pool_q_ms, route_ms, cons_ms, attend_ms = seg(0), seg(1), seg(2), seg(3), seg(4)
+    pool_k_ms, pool_q_ms, tree_pool_ms = seg(0), seg(1), seg(2)
+    route_ms, cons_ms, attend_ms = seg(3), seg(4), seg(5)
+    # two-level routing: share of the flat route's per-head selections that
+    # the tree route also selects, on the same summaries (outside the timing)
+    tree_recall = None
+    if tree and w.top_k:
+        flat_p = ssa.params_of(w, tree_fanout=0, tree_beam=0, consensus=False)
+        fi, fc = ssa.route(qs, ks, flat_p)
+        ti = (idx_h if w.consensus else idx).cpu().numpy().reshape(-1, w.top_k)
+        fi = fi.cpu().numpy().reshape(-1, w.top_k)
+        hit = ((fi[:, :, None] == ti[:, None, :]) & (fi[:, :, None] >= 0)).any(axis=2)
+        tree_recall = float(hit.sum() / max(1, int(fc.sum().item())))
 
     work = algorithmic_work(w, idx.cpu().numpy(), cnt.cpu().numpy())
     peaks, peak_kind = load_peaks()
@@ -536,7 +582,8 @@ def run_ssa(args):
         with open(TRAFFIC_FILE) as f:
             tr = json.load(f)
         if tr.get("kernel_hash") == kernel_source_hash():
-            key = f"{args.config}{'c' if w.consensus else ''}" + (f"@{args.seq_len}" if args.seq_len else "")
+            key = (f"{args.config}{'c' if w.consensus else ''}{'t' if tree else ''}"
+                   + (f"@{args.seq_len}" if args.seq_len else ""))
             traffic = tr.get("bytes_per_launch", {}).get(key)
 
     # end to end through the public call, from pinned host memory
@@ -565,7 +612,7 @@ def run_ssa(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        pool = OraclePool(args.config, args.seq_len, args.consensus, args.beta)
+        pool = OraclePool(args.config, args.seq_len, args.consensus, args.beta, tree_of(w))
         try:
             v, nb, wall = pool.run(args.cpu_seconds)
         finally:
@@ -592,8 +639,10 @@ def run_ssa(args):
         "keys_per_query": work["keys_per_query"],
         "nominal_keys_per_query": work["nominal_keys_per_query"],
         "kernels_ms": {("features_k" if w.beta else "pool_k"): pool_k_ms,
-                       ("features_q" if w.beta else "pool_q"): pool_q_ms, "route": route_ms,
+                       ("features_q" if w.beta else "pool_q"): pool_q_ms,
+                       **({"tree_pool": tree_pool_ms} if tree else {}), "route": route_ms,
                        **({"consensus": cons_ms} if w.consensus else {}), "attend": attend_ms},
+        **({"tree_recall_of_flat_route": tree_recall} if tree else {}),
         "roofline": {"bound": roof["bound"], "kernel": "attend_kernel",
                      "achieved": roof["achieved"], "peak": roof["peak"], "unit": roof["unit"],
                      "frac": roof["achieved"] / roof["peak"], "traffic": traffic,
@@ -605,9 +654,10 @@ def run_ssa(args):
                      "path_frac_of_roofline": t_roof / (ms * 1e-3)},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        # per forward: pool (K and Q in one launch) + route + attend, or with
-        # beta: two feature launches + scores + select + attend; +1 consensus
-        "gpu_launches": ((5 if w.beta else 3) + (1 if w.consensus else 0)) * args.steps,
+        # per forward: pool (K and Q in one launch) + route + attend; with
+        # beta: two feature launches + scores + select + attend; two-level:
+        # pool + super-block pool + upper route + select + attend; +1 consensus
+        "gpu_launches": ((5 if (w.beta or tree) else 3) + (1 if w.consensus else 0)) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

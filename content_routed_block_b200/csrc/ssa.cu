@@ -25,6 +25,7 @@
 #include "pool.cuh"
 #include "route.cuh"
 #include "route_tc.cuh"
+#include "tree.cuh"
 
 namespace ssa {
 __global__ void probe_wait_kernel(uint64_t timeout_ns) {
@@ -53,7 +54,7 @@ static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 namespace {
 
-constexpr int32_t kVersion = 1;
+constexpr int32_t kVersion = 2;
 thread_local std::string g_msg;
 
 ssa_status fail(ssa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
@@ -114,6 +115,17 @@ ssa_status validate(const ssa_params* p) {
                 ssa::kConsMaxVotes);
   const int64_t nb = p->N / p->block_k;
   if (nb >= (1 << 23)) return fail(SSA_ERR_UNSUPPORTED, "N / block_k must be below 2^23");
+  if (p->tree_fanout != 0) {
+    if (!pow2_in(p->tree_fanout, 1, 256) || p->tree_fanout > nb)
+      return fail(SSA_ERR_UNSUPPORTED,
+                  "tree_fanout must be 0 or a power of two in [1, 256] and at most N / block_k");
+    if (p->tree_beam < 1 || p->tree_beam > ssa::kTreeMaxBeam)
+      return fail(SSA_ERR_UNSUPPORTED, "tree_beam must be in 1..%d", ssa::kTreeMaxBeam);
+    if (p->beta != 0.0f)
+      return fail(SSA_ERR_UNSUPPORTED, "two-level routing ranks by block means (beta must be 0)");
+  } else if (p->tree_beam != 0) {
+    return fail(SSA_ERR_INVALID_ARG, "tree_beam must be 0 without tree_fanout");
+  }
   const int64_t rows = static_cast<int64_t>(p->B) * p->Hq * p->N;
   if (rows > (static_cast<int64_t>(1) << 31) - 1)
     return fail(SSA_ERR_UNSUPPORTED, "B * Hq * N must fit in int32");
@@ -335,6 +347,89 @@ ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksu
   return SSA_OK;
 }
 
+// ------------------------------------------------------------ two-level route
+ssa_status launch_tree_pool(const ssa_params* p, const float* ksum, float* ksum2,
+                            cudaStream_t stream) {
+  const int32_t nb = p->N / p->block_k, ns = nb / p->tree_fanout;
+  ssa::TreePoolArgs a{ksum, ksum2, static_cast<int64_t>(p->B) * p->Hkv * ns, nb, ns,
+                      p->tree_fanout, 1.0f / static_cast<float>(p->tree_fanout)};
+  const int64_t threads = a.n_nodes * (p->D / 4);
+  const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
+  if (grid > 0) {
+    if (p->D == 64)
+      ssa::tree_pool_kernel<64><<<grid, 256, 0, stream>>>(a);
+    else
+      ssa::tree_pool_kernel<128><<<grid, 256, 0, stream>>>(a);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "tree_pool_kernel launch");
+  return SSA_OK;
+}
+
+template <int D, int KM>
+cudaError_t launch_tree_select_t(const ssa::TreeSelectArgs& a, cudaStream_t stream) {
+  const int64_t grid = (a.n_rows + ssa::kTreeWarps - 1) / ssa::kTreeWarps;
+  ssa::tree_select_kernel<D, KM><<<static_cast<unsigned>(grid), ssa::kTreeThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_tree_select_d(const ssa::TreeSelectArgs& a, cudaStream_t stream) {
+  if (a.top_k <= 8) return launch_tree_select_t<D, 8>(a, stream);
+  if (a.top_k <= 16) return launch_tree_select_t<D, 16>(a, stream);
+  if (a.top_k <= 32) return launch_tree_select_t<D, 32>(a, stream);
+  return launch_tree_select_t<D, 64>(a, stream);
+}
+
+// upper level: the flat router over the super-block summaries (block F*Bk,
+// top tree_beam); lower level: tree_select_kernel
+ssa_status launch_route_tree(const ssa_params* p, const float* qsum, const float* ksum,
+                             const float* ksum2, int32_t* sup_idx, int32_t* sup_cnt, int32_t* idx,
+                             int32_t* cnt, cudaStream_t stream) {
+  const int32_t nb = p->N / p->block_k;
+  ssa::RouteArgs u;
+  u.qsum = qsum;
+  u.ksum = ksum2;
+  u.idx = sup_idx;
+  u.cnt = sup_cnt;
+  u.Hq = p->Hq;
+  u.Hkv = p->Hkv;
+  u.NQB = p->N / p->block_q;
+  u.NB = nb / p->tree_fanout;
+  u.Bq = p->block_q;
+  u.Bk = p->block_k * p->tree_fanout;
+  u.top_k = p->tree_beam;
+  u.causal = p->causal;
+  u.n_row_tiles = 0;
+  u.timeout_ns = timeout_ns(p);
+  cudaError_t e = p->D == 64 ? launch_route_fp32<64>(u, p->B, stream)
+                             : launch_route_fp32<128>(u, p->B, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tree upper-level route launch");
+  ssa::TreeSelectArgs a;
+  a.qsum = qsum;
+  a.ksum = ksum;
+  a.sup_idx = sup_idx;
+  a.sup_cnt = sup_cnt;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.NQB = p->N / p->block_q;
+  a.NB = nb;
+  a.Bq = p->block_q;
+  a.Bk = p->block_k;
+  a.top_k = p->top_k;
+  a.causal = p->causal;
+  int lf = 0;
+  while ((1 << lf) < p->tree_fanout) ++lf;
+  a.log2_f = lf;
+  a.beam = p->tree_beam;
+  a.n_rows = static_cast<int64_t>(p->B) * p->Hq * a.NQB;
+  e = p->D == 64 ? launch_tree_select_d<64>(a, stream) : launch_tree_select_d<128>(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tree_select_kernel launch");
+  return SSA_OK;
+}
+
 // Query heads per attend CTA.  Consensus lists are shared by a KV group, so
 // two heads of the group fill one 128-row tile (64 rows each) and every chunk
 // serves all rows.  SSA_PACK=1 forces one head per tile (the tests run both).
@@ -523,7 +618,7 @@ ssa_status launch_consensus(const ssa_params* p, const int32_t* idx, const int32
 // Workspace of ssa_forward: K and Q summaries, the per-head routed lists and
 // counts, and (consensus routing only) the per-group lists and counts.
 struct WsLayout {
-  size_t ksum, qsum, idx, cnt, idx_kv, cnt_kv, qf, kf, sc, total;
+  size_t ksum, qsum, idx, cnt, idx_kv, cnt_kv, qf, kf, sc, ksum2, sup_idx, sup_cnt, total;
 };
 
 WsLayout ws_layout(const ssa_params* p) {
@@ -550,7 +645,16 @@ WsLayout ws_layout(const ssa_params* p) {
   w.qf = w.cnt_kv + align256(cnk);
   w.kf = w.qf + align256(qfb);
   w.sc = w.kf + align256(kfb);
-  w.total = w.sc + align256(scb);
+  // two-level routing: super-block summaries and the kept super-blocks
+  const bool tree = p->tree_fanout > 0;
+  const size_t ns = tree ? nb / p->tree_fanout : 0;
+  const size_t k2b = static_cast<size_t>(p->B) * p->Hkv * ns * p->D * sizeof(float);
+  const size_t s2b = tree ? static_cast<size_t>(p->B) * p->Hq * nqb * p->tree_beam * sizeof(int32_t) : 0;
+  const size_t c2b = tree ? cn : 0;
+  w.ksum2 = w.sc + align256(scb);
+  w.sup_idx = w.ksum2 + align256(k2b);
+  w.sup_cnt = w.sup_idx + align256(s2b);
+  w.total = w.sup_cnt + align256(c2b);
   return w;
 }
 
@@ -569,6 +673,8 @@ ssa_status validate_decode(const ssa_params* p) {
   if (!p->causal) return fail(SSA_ERR_INVALID_ARG, "decode is causal (causal must be 1)");
   if (p->consensus) return fail(SSA_ERR_UNSUPPORTED, "decode routes per head (consensus must be 0)");
   if (p->beta != 0.0f) return fail(SSA_ERR_UNSUPPORTED, "decode ranks by block means (beta must be 0)");
+  if (p->tree_fanout != 0)
+    return fail(SSA_ERR_UNSUPPORTED, "decode routes over the flat block list (tree_fanout must be 0)");
   if (static_cast<int64_t>(p->B) * p->Hq > 65535)
     return fail(SSA_ERR_UNSUPPORTED, "decode needs B * Hq <= 65535");
   return SSA_OK;
@@ -638,6 +744,36 @@ ssa_status ssa_route(const ssa_params* p, const float* qsum, const float* ksum, 
   if (!aligned16(qsum) || !aligned16(ksum) || !aligned16(cnt) || (idx && !aligned16(idx)))
     return fail(SSA_ERR_INVALID_ARG, "routing buffers must be 16-byte aligned");
   s = launch_route(p, qsum, ksum, idx, cnt, static_cast<cudaStream_t>(stream));
+  return s == SSA_OK ? ok() : s;
+}
+
+ssa_status ssa_tree_summary(const ssa_params* p, const float* ksum, float* ksum2,
+                            ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (p->tree_fanout < 1) return fail(SSA_ERR_INVALID_ARG, "tree_fanout must be >= 1");
+  if (ksum == nullptr || ksum2 == nullptr)
+    return fail(SSA_ERR_INVALID_ARG, "ksum and ksum2 must be non-NULL");
+  if (!aligned16(ksum) || !aligned16(ksum2))
+    return fail(SSA_ERR_INVALID_ARG, "ksum and ksum2 must be 16-byte aligned");
+  s = launch_tree_pool(p, ksum, ksum2, static_cast<cudaStream_t>(stream));
+  return s == SSA_OK ? ok() : s;
+}
+
+ssa_status ssa_route_tree(const ssa_params* p, const float* qsum, const float* ksum,
+                          const float* ksum2, int32_t* sup_idx, int32_t* sup_cnt, int32_t* idx,
+                          int32_t* cnt, ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (p->tree_fanout < 1) return fail(SSA_ERR_INVALID_ARG, "tree_fanout must be >= 1");
+  if (!qsum || !ksum || !ksum2 || !sup_idx || !sup_cnt || !cnt || (p->top_k > 0 && !idx))
+    return fail(SSA_ERR_INVALID_ARG,
+                "qsum, ksum, ksum2, sup_idx, sup_cnt, cnt (and idx when top_k > 0) must be non-NULL");
+  if (!aligned16(qsum) || !aligned16(ksum) || !aligned16(ksum2) || !aligned16(sup_idx) ||
+      !aligned16(sup_cnt) || !aligned16(cnt) || (idx && !aligned16(idx)))
+    return fail(SSA_ERR_INVALID_ARG, "routing buffers must be 16-byte aligned");
+  s = launch_route_tree(p, qsum, ksum, ksum2, sup_idx, sup_cnt, idx, cnt,
+                        static_cast<cudaStream_t>(stream));
   return s == SSA_OK ? ok() : s;
 }
 
@@ -739,7 +875,17 @@ ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const 
   } else {
     if ((s = launch_pool(p, k, p->Hkv, p->block_k, ksum, q, p->Hq, p->block_q, qsum, st)) != SSA_OK)
       return s;
-    if ((s = launch_route(p, qsum, ksum, idx_h, cnt_h, st)) != SSA_OK) return s;
+    if (p->tree_fanout > 0) {
+      float* ksum2 = reinterpret_cast<float*>(ws + w.ksum2);
+      int32_t* sup_idx = reinterpret_cast<int32_t*>(ws + w.sup_idx);
+      int32_t* sup_cnt = reinterpret_cast<int32_t*>(ws + w.sup_cnt);
+      if ((s = launch_tree_pool(p, ksum, ksum2, st)) != SSA_OK) return s;
+      if ((s = launch_route_tree(p, qsum, ksum, ksum2, sup_idx, sup_cnt, idx_h, cnt_h, st)) !=
+          SSA_OK)
+        return s;
+    } else if ((s = launch_route(p, qsum, ksum, idx_h, cnt_h, st)) != SSA_OK) {
+      return s;
+    }
   }
   if (p->consensus && (s = launch_consensus(p, idx_h, cnt_h, idx_a, cnt_a, st)) != SSA_OK)
     return s;

@@ -15,7 +15,8 @@ import torch
 
 __all__ = [
     "Params", "SsaError", "lib", "make_params", "params_of", "workspace_size", "block_summary",
-    "route", "route_consensus", "route_features", "route_cumulant", "attend", "forward",
+    "route", "route_consensus", "route_features", "route_cumulant", "tree_summary", "route_tree",
+    "attend", "forward",
     "forward_host", "decode", "decode_workspace_size", "check_error",
     "probe_wait_timeout",
     "declared_functions", "LIB_PATH", "HEADER_PATH",
@@ -43,7 +44,7 @@ class Params(ctypes.Structure):
         ("block_q", ctypes.c_int32), ("top_k", ctypes.c_int32), ("window", ctypes.c_int32),
         ("causal", ctypes.c_int32), ("scale", ctypes.c_float),
         ("wait_timeout_us", ctypes.c_int32), ("consensus", ctypes.c_int32),
-        ("beta", ctypes.c_float),
+        ("beta", ctypes.c_float), ("tree_fanout", ctypes.c_int32), ("tree_beam", ctypes.c_int32),
     ]
 
     @property
@@ -61,16 +62,19 @@ class Params(ctypes.Structure):
 
 
 def make_params(B, Hq, Hkv, N, D, block_k, block_q, top_k, window, causal, scale=0.0,
-                wait_timeout_us=0, consensus=False, beta=0.0) -> Params:
+                wait_timeout_us=0, consensus=False, beta=0.0, tree_fanout=0,
+                tree_beam=0) -> Params:
     return Params(B, Hq, Hkv, N, D, block_k, block_q, top_k, window, int(bool(causal)),
-                  float(scale), wait_timeout_us, int(bool(consensus)), float(beta))
+                  float(scale), wait_timeout_us, int(bool(consensus)), float(beta),
+                  int(tree_fanout), int(tree_beam))
 
 
 def params_of(w, **over) -> Params:
     """Params from any object with the workload field names."""
     f = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=w.N, D=w.D, block_k=w.block_k, block_q=w.block_q,
              top_k=w.top_k, window=w.window, causal=w.causal, scale=getattr(w, "scale", 0.0),
-             consensus=getattr(w, "consensus", False), beta=getattr(w, "beta", 0.0))
+             consensus=getattr(w, "consensus", False), beta=getattr(w, "beta", 0.0),
+             tree_fanout=getattr(w, "tree_fanout", 0), tree_beam=getattr(w, "tree_beam", 0))
     f.update(over)
     return make_params(**f)
 
@@ -94,6 +98,8 @@ def lib() -> ctypes.CDLL:
         "ssa_block_summary": (i32, [P, vp, i32, i32, vp, vp]),
         "ssa_route": (i32, [P, vp, vp, vp, vp, vp]),
         "ssa_route_consensus": (i32, [P, vp, vp, vp, vp, vp]),
+        "ssa_tree_summary": (i32, [P, vp, vp, vp]),
+        "ssa_route_tree": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ssa_route_features": (i32, [P, vp, i32, i32, i32, vp, vp]),
         "ssa_route_cumulant": (i32, [P, vp, vp, vp, vp, vp, vp]),
         "ssa_attend": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
@@ -168,6 +174,32 @@ def route(qsum: torch.Tensor, ksum: torch.Tensor, p: Params):
     _check(lib().ssa_route(ctypes.byref(p), _ptr(qsum), _ptr(ksum),
                            _ptr(idx) if p.top_k else None, _ptr(cnt), _stream()))
     return idx, cnt
+
+
+def tree_summary(ksum: torch.Tensor, p: Params) -> torch.Tensor:
+    """Super-block means fp32 [B, Hkv, (N/Bk) // tree_fanout, D] from block means."""
+    _need(ksum, torch.float32, (p.B, p.Hkv, p.n_kblocks, p.D), "ksum")
+    ns = p.n_kblocks // max(p.tree_fanout, 1)
+    out = torch.empty((p.B, p.Hkv, ns, p.D), dtype=torch.float32, device=ksum.device)
+    _check(lib().ssa_tree_summary(ctypes.byref(p), _ptr(ksum), _ptr(out), _stream()))
+    return out
+
+
+def route_tree(qsum: torch.Tensor, ksum: torch.Tensor, ksum2: torch.Tensor, p: Params):
+    """Two-level routing: (sup_idx int32 [B, Hq, NQB, tree_beam], sup_cnt int32
+    [B, Hq, NQB], idx int32 [B, Hq, NQB, top_k], cnt int32 [B, Hq, NQB])."""
+    _need(qsum, torch.float32, (p.B, p.Hq, p.n_qblocks, p.D), "qsum")
+    _need(ksum, torch.float32, (p.B, p.Hkv, p.n_kblocks, p.D), "ksum")
+    _need(ksum2, torch.float32, (p.B, p.Hkv, p.n_kblocks // max(p.tree_fanout, 1), p.D), "ksum2")
+    dev = qsum.device
+    sup_idx = torch.empty((p.B, p.Hq, p.n_qblocks, p.tree_beam), dtype=torch.int32, device=dev)
+    sup_cnt = torch.empty((p.B, p.Hq, p.n_qblocks), dtype=torch.int32, device=dev)
+    idx = torch.empty((p.B, p.Hq, p.n_qblocks, p.top_k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((p.B, p.Hq, p.n_qblocks), dtype=torch.int32, device=dev)
+    _check(lib().ssa_route_tree(ctypes.byref(p), _ptr(qsum), _ptr(ksum), _ptr(ksum2),
+                                _ptr(sup_idx), _ptr(sup_cnt), _ptr(idx) if p.top_k else None,
+                                _ptr(cnt), _stream()))
+    return sup_idx, sup_cnt, idx, cnt
 
 
 def route_consensus(idx: torch.Tensor, cnt: torch.Tensor, p: Params):
@@ -287,7 +319,7 @@ def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
     grp = p.Hq // p.Hkv
     unit = grp if p.consensus else 1          # query heads per sub-problem
     sub = make_params(1, unit, 1, p.N, p.D, p.block_k, p.block_q, p.top_k, p.window, p.causal,
-                      p.scale, p.wait_timeout_us, p.consensus, p.beta)
+                      p.scale, p.wait_timeout_us, p.consensus, p.beta, p.tree_fanout, p.tree_beam)
     if "ws" not in d:
         d["ws"] = torch.empty(workspace_size(sub), dtype=torch.uint8, device=dev)
     if "streams" not in d:

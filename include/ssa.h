@@ -75,11 +75,19 @@ typedef struct {
                               0 ranks by <qbar, mu_c> (ssa_route); otherwise
                               by <qbar, mu_c> + (beta/2) tr(Sigma_c Q2)
                               (ssa_route_features + ssa_route_cumulant)     */
+  int32_t tree_fanout;     /* 0: flat routing (every admissible block scored).
+                              F > 0: two-level routing (ssa_route_tree) with
+                              F key blocks per super-block; a power of two in
+                              [1, 256], at most N/Bk; requires beta == 0    */
+  int32_t tree_beam;       /* two-level routing: super-blocks kept per query
+                              block, 1..64 (0 when tree_fanout == 0)        */
 } ssa_params;
 
 /* Bytes of device workspace ssa_forward needs for these parameters:
- * K summaries, Q summaries, the routed index list and counts, each 256-byte
- * aligned.  Returns 0 if the parameters are invalid. */
+ * K summaries, Q summaries, the routed index list and counts (plus the
+ * consensus lists, the second-cumulant features and scores, or the
+ * super-block summaries and kept super-blocks, when those options are on),
+ * each 256-byte aligned.  Returns 0 if the parameters are invalid. */
 size_t ssa_workspace_size(const ssa_params* p);
 
 /* Block summary (step 1 of the path; jonsmirl/ssa README, "Algorithm and
@@ -135,6 +143,46 @@ ssa_status ssa_route_features(const ssa_params* p, const void* x, int32_t H, int
 ssa_status ssa_route_cumulant(const ssa_params* p, const float* qfeat, const float* kfeat,
                               float* scores, int32_t* idx, int32_t* cnt, ssa_stream_t stream);
 
+/* Super-block summaries for two-level routing (jonsmirl/ssa README,
+ * "Algorithm and complexity": a hierarchical router in place of the flat
+ * block scan; the measured tree has fanout 16).  Super-block S covers key
+ * blocks S*F .. S*F+F-1, F = p->tree_fanout, and is summarised by the mean of
+ * its F*Bk keys, computed as the fp32 mean of its children's means (exact in
+ * real arithmetic: every block has Bk keys).
+ *   ksum   fp32 [B, Hkv, N/Bk, D] block means (device), from ssa_block_summary
+ *   ksum2  fp32 [B, Hkv, NS, D] (device, out), NS = (N/Bk) / F complete
+ *          super-blocks (a trailing partial super-block has no summary)
+ * Requires p->tree_fanout >= 1.  One launch. */
+ssa_status ssa_tree_summary(const ssa_params* p, const float* ksum, float* ksum2,
+                            ssa_stream_t stream);
+
+/* Two-level (fixed-beam tree) routing (jonsmirl/ssa README, "Algorithm and
+ * complexity"; "Mathematical status": fixed-beam routing is not an exact
+ * selector -- a block whose super-block is not kept is never scored).  For
+ * query block qb with admissible blocks 0 .. A-1 (the rule of ssa_route):
+ *   1. the complete admissible super-blocks 0 .. A/F - 1 are scored by
+ *      <qbar, super-block mean> (fp32) and the best tree_beam are kept,
+ *      ties to the lower index -- the flat router on ksum2 with block F*Bk;
+ *   2. the candidates are the F children of every kept super-block and the
+ *      frontier blocks (A/F)*F .. A-1; the top_k of them by <qbar, mu_c>
+ *      (fp32), ties to the lower index, are selected.
+ * With tree_beam >= A/F every block is a candidate and the result is
+ * ssa_route's.
+ *   qsum, ksum      as for ssa_route (device)
+ *   ksum2           from ssa_tree_summary (device)
+ *   sup_idx/sup_cnt int32 [B, Hq, N/Bq, tree_beam] and [B, Hq, N/Bq]
+ *                   (device, out): the kept super-blocks ascending, padded
+ *                   with -1, and their count min(tree_beam, A/F)
+ *   idx/cnt         as for ssa_route (device, out)
+ * Requires p->tree_fanout >= 1 and p->beta == 0.  The lower level checks
+ * the upper level's lists as it reads them (count within min(tree_beam, A/F),
+ * super-blocks ascending and complete); a failed check is reported through
+ * ssa_check_error (SSA_ERR_DEVICE_CHECK) and the bad entry contributes no
+ * candidates.  Two launches. */
+ssa_status ssa_route_tree(const ssa_params* p, const float* qsum, const float* ksum,
+                          const float* ksum2, int32_t* sup_idx, int32_t* sup_cnt, int32_t* idx,
+                          int32_t* cnt, ssa_stream_t stream);
+
 /* GQA-shared consensus route (jonsmirl/ssa README, "Complete 10M transformer
  * result": one route formed across heads by consensus, carrying the blocks
  * with the most votes; "Mathematical status": a highest-count reservoir keeps
@@ -177,7 +225,8 @@ ssa_status ssa_attend(const ssa_params* p, const void* q, const void* k, const v
 
 /* The whole path in one call: summaries of K and Q (one launch) and routing
  * -- or, with p->beta != 0, the second-cumulant features of K and Q and
- * ssa_route_cumulant --, (with p->consensus) the consensus route, attend.  workspace must hold
+ * ssa_route_cumulant --, or, with p->tree_fanout > 0, the super-block
+ * summaries and ssa_route_tree --, (with p->consensus) the consensus route, attend.  workspace must hold
  * ssa_workspace_size(p) bytes (device, 256-byte aligned).  idx_out / cnt_out
  * (device, may be NULL) receive the lists attend used when given -- per head
  * [B, Hq, N/Bq, top_k], or per KV group [B, Hkv, N/Bq, top_k] with

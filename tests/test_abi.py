@@ -22,7 +22,7 @@ def test_every_declared_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.ssa_version() == 1
+    assert L.ssa_version() == 2
     for s in range(7):
         assert L.ssa_status_string(s).decode() not in ("", "unknown status")
     assert L.ssa_status_string(99).decode() == "unknown status"
@@ -161,3 +161,45 @@ def test_decode_entry_point_rejects_bad_arguments_before_launch(L):
         assert L.ssa_decode_workspace_size(ctypes.byref(bad)) == 0
         assert f(ctypes.byref(bad), good, good, good, 100, good, good, None, None, None, good,
                  ws, None) == status
+
+
+def test_workspace_layout_with_tree_routing(L):
+    p = _p(tree_fanout=16, tree_beam=8)
+    a = lambda x: (x + 255) // 256 * 256
+    ks, qs = 2 * 512 * 64 * 4, 14 * 512 * 64 * 4
+    ix, cn = 14 * 512 * 16 * 4, 14 * 512 * 4
+    k2, s2 = 2 * 32 * 64 * 4, 14 * 512 * 8 * 4
+    assert ssa.workspace_size(p) == a(ks) + a(qs) + a(ix) + a(cn) + a(k2) + a(s2) + a(cn)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(tree_fanout=3, tree_beam=4), 2),          # not a power of two
+    (dict(tree_fanout=512, tree_beam=4), 2),        # above 256
+    (dict(N=1024, tree_fanout=32, tree_beam=4), 2),  # more than N/Bk = 16 blocks
+    (dict(tree_fanout=16, tree_beam=0), 2), (dict(tree_fanout=16, tree_beam=65), 2),
+    (dict(tree_fanout=16, tree_beam=4, beta=0.5), 2),
+    (dict(tree_beam=4), 1),                         # a beam without a tree
+])
+def test_invalid_tree_params_are_rejected_before_launch(L, kw, status):
+    p = _p(**kw)
+    assert L.ssa_workspace_size(ctypes.byref(p)) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.ssa_forward(ctypes.byref(p), fake, fake, fake, fake, None, None, None, fake,
+                         1 << 40, None) == status
+
+
+def test_tree_entry_points_reject_bad_arguments_before_launch(L):
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    flat = _p()
+    p = _p(tree_fanout=16, tree_beam=4)
+    assert L.ssa_tree_summary(ctypes.byref(flat), good, good, None) == 1     # no tree
+    assert L.ssa_tree_summary(ctypes.byref(p), None, good, None) == 1
+    assert L.ssa_tree_summary(ctypes.byref(p), good, odd, None) == 1
+    f = L.ssa_route_tree
+    assert f(ctypes.byref(flat), good, good, good, good, good, good, good, None) == 1
+    assert f(ctypes.byref(p), good, good, None, good, good, good, good, None) == 1
+    assert f(ctypes.byref(p), good, good, good, good, None, good, good, None) == 1
+    assert f(ctypes.byref(p), good, good, good, odd, good, good, good, None) == 1
+    # decode keeps the flat block list
+    assert L.ssa_decode_workspace_size(ctypes.byref(p)) == 0

@@ -27,8 +27,9 @@ def _inputs(w, seed):
     return [to_dev(x[n]) for n in "qkv"]
 
 
-@pytest.mark.parametrize("kw", [dict(), dict(consensus=True), dict(beta=0.5)],
-                         ids=["per-head", "consensus", "second-cumulant"])
+@pytest.mark.parametrize("kw", [dict(), dict(consensus=True), dict(beta=0.5),
+                                dict(tree_fanout=4, tree_beam=2)],
+                         ids=["per-head", "consensus", "second-cumulant", "two-level"])
 def test_forward_replays_in_a_cuda_graph(kw):
     w = Workload("graph", B=1, Hq=4, Hkv=2, N=2048, D=64, block_k=64, block_q=64, top_k=6,
                  window=128, causal=True, kind="clustered", centres=16, seed=3, **kw)
