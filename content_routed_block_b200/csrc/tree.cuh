@@ -18,13 +18,14 @@
 //  * the upper level is the flat router (route.cuh) run on the super-block
 //    summaries with block F*Bk and top_k = beam: its admissibility rule
 //    (S+1)*F*Bk <= qb*Bq is exactly "S is complete and admissible".
-//  * tree_select_kernel: one warp per query block.  Lane l scores candidates
-//    l, l+32, ... (fp32 dot products, the block summary read as float4) and
-//    keeps its top KM in registers as route.cuh's 64-bit keys; five shuffle
-//    merges leave the row's top KM in every lane.  The CTA's eight warps
-//    take eight consecutive query blocks of one head, whose kept
-//    super-blocks mostly coincide, so the children's summaries are re-read
-//    from L1.
+//  * tree_select_kernel: one warp per query block.  Candidates go 32 at a
+//    time, 16 per half-warp: each candidate's summary row is read coalesced
+//    (16 lanes x float4), 16 independent loads per lane, and a shuffle
+//    reduce-scatter leaves lane l with candidate e0 + l's fp32 score, which
+//    it keeps in its register top-KM list (route.cuh's 64-bit keys); five
+//    shuffle merges leave the row's top KM in every lane.  The CTA's eight warps take eight consecutive query
+//    blocks of one head, whose kept super-blocks mostly coincide, so the
+//    children's summaries are re-read from L1.
 #pragma once
 
 #include "common.cuh"
@@ -122,38 +123,94 @@ __global__ void __launch_bounds__(kTreeThreads) tree_select_kernel(const TreeSel
   const int n_kids = n2 << a.log2_f;
   const int n_cand = a.top_k == 0 ? 0 : n_kids + (n_adm - (ns << a.log2_f));
   const float* kbase = a.ksum + bkv * a.NB * D;
-  const float4* q4 = reinterpret_cast<const float4*>(qs[warp]);
+  // candidate e -> key block (-1: a child of a rejected super-block)
+  auto block_of = [&](int e) -> int {
+    if (e >= n_kids) return (ns << a.log2_f) + (e - n_kids);
+    const int s = sup_s[warp][e >> a.log2_f];
+    return s < 0 ? -1 : (s << a.log2_f) + (e & (F - 1));
+  };
+  // Candidates go 32 at a time, 16 per half-warp: lane hl of half h reads
+  // columns 4hl .. 4hl+3 (+64 i) of the rows of candidates e0 + 16h + j,
+  // j = 0..15 (each row read coalesced by the half-warp, all 16 loads
+  // independent), and forms 16 partial dot products with its slice of qbar.
+  // A reduce-scatter over the half-warp (8 + 4 + 2 + 1 shuffles) then leaves
+  // lane hl holding the full product of candidate j = hl, i.e. lane l holds
+  // candidate e0 + l.
+  constexpr int QV = D / 64;
+  const int half = lane >> 4, hl = lane & 15;
+  float4 qv[QV];
+#pragma unroll
+  for (int i = 0; i < QV; ++i) qv[i] = reinterpret_cast<const float4*>(qs[warp])[hl + 16 * i];
   uint64_t keys[KM];
 #pragma unroll
   for (int j = 0; j < KM; ++j) keys[j] = 0ull;
   float thr_f = -INFINITY;
-  for (int e = lane; e < n_cand; e += 32) {
-    int c;
-    if (e < n_kids) {
-      const int s = sup_s[warp][e >> a.log2_f];
-      if (s < 0) continue;
-      c = (s << a.log2_f) + (e & (F - 1));
-    } else {
-      c = (ns << a.log2_f) + (e - n_kids);
-    }
-    const float4* k4 = reinterpret_cast<const float4*>(kbase + static_cast<int64_t>(c) * D);
-    float acc0 = 0.f, acc1 = 0.f;
+  // With F >= 16 a half's 16 candidates (e0 + 16h is a multiple of 16, and
+  // so are n_kids and every super-block's first child) are 16 consecutive
+  // blocks of one kept super-block, or of the frontier: one base row serves
+  // all of them.  Smaller fanouts map every candidate separately.
+  const bool contiguous = F >= 16;
+  for (int e0 = 0; e0 < n_cand; e0 += 32) {  // warp-uniform
+    float p[16];
+    if (contiguous) {
+      const int eh = e0 + 16 * half;
+      const int nh = min(16, n_cand - eh);   // candidates of this half (may be <= 0)
+      const int c0 = nh > 0 ? block_of(eh) : -1;
+      const float4* k4 =
+          reinterpret_cast<const float4*>(kbase + static_cast<int64_t>(max(c0, 0)) * D) + hl;
 #pragma unroll
-    for (int i = 0; i < D / 4; i += 2) {
-      const float4 x0 = __ldg(k4 + i), y0 = q4[i];
-      const float4 x1 = __ldg(k4 + i + 1), y1 = q4[i + 1];
-      acc0 = fmaf(x0.x, y0.x, acc0);
-      acc0 = fmaf(x0.y, y0.y, acc0);
-      acc0 = fmaf(x0.z, y0.z, acc0);
-      acc0 = fmaf(x0.w, y0.w, acc0);
-      acc1 = fmaf(x1.x, y1.x, acc1);
-      acc1 = fmaf(x1.y, y1.y, acc1);
-      acc1 = fmaf(x1.z, y1.z, acc1);
-      acc1 = fmaf(x1.w, y1.w, acc1);
+      for (int j = 0; j < 16; ++j) {
+        float part = 0.f;
+        if (c0 >= 0 && j < nh) {
+#pragma unroll
+          for (int i = 0; i < QV; ++i) {
+            const float4 x = __ldg(k4 + j * (D / 4) + 16 * i);
+            part = fmaf(x.x, qv[i].x, part);
+            part = fmaf(x.y, qv[i].y, part);
+            part = fmaf(x.z, qv[i].z, part);
+            part = fmaf(x.w, qv[i].w, part);
+          }
+        }
+        p[j] = part;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int e = e0 + 16 * half + j;
+        const int c = e < n_cand ? block_of(e) : -1;
+        float part = 0.f;
+        if (c >= 0) {
+          const float4* k4 =
+              reinterpret_cast<const float4*>(kbase + static_cast<int64_t>(c) * D) + hl;
+#pragma unroll
+          for (int i = 0; i < QV; ++i) {
+            const float4 x = __ldg(k4 + 16 * i);
+            part = fmaf(x.x, qv[i].x, part);
+            part = fmaf(x.y, qv[i].y, part);
+            part = fmaf(x.z, qv[i].z, part);
+            part = fmaf(x.w, qv[i].w, part);
+          }
+        }
+        p[j] = part;
+      }
     }
-    const float v = acc0 + acc1;
-    if (v >= thr_f) {
-      const uint64_t key = route_key(v, c);
+    // reduce-scatter: at offset m a lane keeps the half of its candidates
+    // whose bit m matches its own lane bit and adds its partner's partials
+#pragma unroll
+    for (int m = 8; m > 0; m >>= 1) {
+      const bool up = (hl & m) != 0;
+#pragma unroll
+      for (int i = 0; i < m; ++i) {
+        const float send = up ? p[i] : p[i + m];
+        const float keep = up ? p[i + m] : p[i];
+        p[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+      }
+    }
+    const float mine = p[0];
+    const int e = e0 + lane;
+    const int c = e < n_cand ? block_of(e) : -1;
+    if (c >= 0 && mine >= thr_f) {
+      const uint64_t key = route_key(mine, c);
       if (key > keys[KM - 1]) {
         route_sorted_insert<KM>(keys, key);
         if (keys[KM - 1] != 0ull) thr_f = key_score(keys[KM - 1]);
@@ -163,26 +220,40 @@ __global__ void __launch_bounds__(kTreeThreads) tree_select_kernel(const TreeSel
 #pragma unroll
   for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);
 
-  // every lane now holds the row's top KM keys, best first; lane j writes
-  // the j-th smallest selected block index (rank by counting)
+  // every lane now holds the row's top KM keys, best first; the selected
+  // blocks are written ascending
   const int k = a.top_k;
   int n = 0;
 #pragma unroll
   for (int j = 0; j < KM; ++j) n += (j < k && keys[j] != 0ull) ? 1 : 0;
   if (k > 0) {
     int32_t* dst = a.idx + row * k;
+    if (KM <= 32) {
+      // lane j takes the j-th selected block; a shuffle bitonic sort of
+      // (2^32 - 1 - block) descending lists the blocks ascending, the empty
+      // lanes (key 0) last
+      uint64_t mine_key = 0ull;
 #pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      if (j >= n) continue;
-      const int cj = static_cast<int>(~static_cast<uint32_t>(keys[j] & 0xFFFFFFFFull));
-      // rank of block cj among the n selected blocks
-      int rank = 0;
+      for (int j = 0; j < KM; ++j)
+        if (j == lane && j < n)
+          mine_key = 0xFFFFFFFFull - (~static_cast<uint32_t>(keys[j] & 0xFFFFFFFFull));
+      mine_key = warp_sort_desc(mine_key, lane);
+      if (lane < k) dst[lane] = lane < n ? static_cast<int>(0xFFFFFFFFull - mine_key) : -1;
+    } else {
+      // rank by counting
 #pragma unroll
-      for (int i = 0; i < KM; ++i)
-        if (i < n && static_cast<int>(~static_cast<uint32_t>(keys[i] & 0xFFFFFFFFull)) < cj) ++rank;
-      if ((j & 31) == lane) dst[rank] = cj;
+      for (int j = 0; j < KM; ++j) {
+        if (j >= n) continue;
+        const int cj = static_cast<int>(~static_cast<uint32_t>(keys[j] & 0xFFFFFFFFull));
+        int rank = 0;
+#pragma unroll
+        for (int i = 0; i < KM; ++i)
+          if (i < n && static_cast<int>(~static_cast<uint32_t>(keys[i] & 0xFFFFFFFFull)) < cj)
+            ++rank;
+        if ((j & 31) == lane) dst[rank] = cj;
+      }
+      for (int j = n + lane; j < k; j += 32) dst[j] = -1;
     }
-    for (int j = n + lane; j < k; j += 32) dst[j] = -1;
   }
   if (lane == 0) a.cnt[row] = n;
 }
