@@ -69,7 +69,7 @@ __all__ = [
     "consensus_row", "route_consensus", "expand_consensus",
     "block_covariance", "block_second_moment", "block_scores", "decode_step",
     "decode_attend", "tree_summary", "tree_candidates", "route_tree_row",
-    "acceptable_tree_selections",
+    "acceptable_tree_selections", "attend_backward",
 ]
 
 NEAR_TIE_REL = 1e-4   # relative score gap under which two blocks count as tied
@@ -486,6 +486,54 @@ def attend_masked_dense(q, k, v, idx, cnt, p: Params, blocks=None):
     o = o_out.reshape(p.B, p.Hq, p.N, dv)
     lse = l_out.reshape(p.B, p.Hq, p.N)
     return o, lse
+
+
+def attend_backward(q, k, v, do, idx, cnt, p: Params, blocks=None):
+    """Gradients of step 8 with the selection held fixed: the routed lists are
+    a discrete choice and carry no gradient; within a row's key set the read
+    is ordinary softmax attention (jonsmirl/ssa README, introduction).
+
+    For query i with key set S_i, logits l_ij = scale <q_i, k_j>, weights
+    P_ij = softmax_j(l_i), read o_i = sum_j P_ij v_j and an upstream gradient
+    g_i = dL/do_i:
+        dL/dv_j += P_ij g_i
+        dP_ij    = <g_i, v_j>
+        dl_ij    = P_ij (dP_ij - sum_m P_im dP_im)      (softmax derivative)
+        dL/dq_i  = scale sum_j dl_ij k_j
+        dL/dk_j += scale dl_ij q_i
+    Query head h reads KV head h // g, so a KV head's gradients sum over its
+    group.  ``do`` [B, Hq, N, D] float64.  Returns (dq [B, Hq, N, D], dk, dv
+    [B, Hkv, N, D]).  ``blocks`` optionally restricts the sum to the listed
+    (b, h, qb) query blocks: dq is then filled on their rows only and dk/dv
+    hold only their contributions."""
+    scale = p.softmax_scale
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dvv = np.zeros_like(v)
+    todo = blocks if blocks is not None else [
+        (b, h, qb) for b in range(p.B) for h in range(p.Hq) for qb in range(p.n_qblocks)]
+    jpos = np.arange(p.N)
+    jblk = jpos // p.block_k
+    for b, h, qb in todo:
+        g = h // p.group
+        rows = np.arange(qb * p.block_q, (qb + 1) * p.block_q)
+        routed = np.zeros(p.n_kblocks, dtype=bool)
+        routed[idx[b, h, qb, :cnt[b, h, qb]]] = True
+        allow = np.broadcast_to(routed[jblk][None, :], (len(rows), p.N)).copy()
+        if p.causal:
+            allow |= jpos[None, :] > rows[:, None] - p.window
+            allow &= jpos[None, :] <= rows[:, None]
+        logits = np.where(allow, (q[b, h, rows] @ k[b, g].T) * scale, -np.inf)
+        m = logits.max(axis=-1, keepdims=True)
+        w = np.exp(logits - m)
+        P = w / w.sum(axis=-1, keepdims=True)                  # [Bq, N], 0 off the key sets
+        gi = do[b, h, rows]
+        dP = gi @ v[b, g].T
+        dl = P * (dP - (P * dP).sum(axis=-1, keepdims=True))
+        dq[b, h, rows] = scale * (dl @ k[b, g])
+        dk[b, g] += scale * (dl.T @ q[b, h, rows])
+        dvv[b, g] += P.T @ gi
+    return dq, dk, dvv
 
 
 def attend_gathered(q, k, v, idx, cnt, p: Params, queries=None):

@@ -778,3 +778,117 @@ def test_tree_forward_attends_over_the_tree_selection():
         n_adm = len(O.admissible_blocks(qb, p))
         cand = O.tree_candidates(r.sup_idx[0, 0, qb][:r.sup_cnt[0, 0, qb]], n_adm, p.tree_fanout)
         assert set(r.idx[0, 0, qb][:r.cnt[0, 0, qb]].tolist()) <= set(cand.tolist())
+
+
+# ---------------------------------------------------------------- backward (fixed selection)
+def _bwd_case(causal, seed=61, B=1, Hq=4, Hkv=2, N=96, D=5, bk=8, top_k=3, W=10):
+    rng = np.random.default_rng(seed)
+    p = _params(B=B, Hq=Hq, Hkv=Hkv, N=N, D=D, block_k=bk, block_q=bk, top_k=top_k,
+                causal=causal, window=W if causal else 0)
+    q = rng.standard_normal((B, Hq, N, D))
+    k = rng.standard_normal((B, Hkv, N, D))
+    v = rng.standard_normal((B, Hkv, N, D))
+    do = rng.standard_normal((B, Hq, N, D))
+    r = O.route(O.block_summary(q, bk), O.block_summary(k, bk), p)
+    return p, q, k, v, do, r.idx, r.cnt
+
+
+def _torch_masked_attention(p, q, k, v, idx, cnt):
+    """The read as a torch graph: the allowed (query, key) pairs built here
+    from the lists and the window, a -inf mask, softmax, weights @ V."""
+    B, Hq, N, D = q.shape
+    g = p.Hq // p.Hkv
+    allow = torch.zeros((B, Hq, N, N), dtype=torch.bool)
+    for b in range(B):
+        for h in range(Hq):
+            for qb in range(N // p.block_q):
+                r0, r1 = qb * p.block_q, (qb + 1) * p.block_q
+                for c in idx[b, h, qb, :cnt[b, h, qb]]:
+                    allow[b, h, r0:r1, c * p.block_k:(c + 1) * p.block_k] = True
+    i = torch.arange(N)[:, None]
+    j = torch.arange(N)[None, :]
+    if p.causal:
+        allow |= ((j > i - p.window) & (j <= i))[None, None]
+        allow &= (j <= i)[None, None]
+    kk = k.repeat_interleave(g, dim=1)
+    vv = v.repeat_interleave(g, dim=1)
+    s = (q @ kk.transpose(-1, -2)) * p.softmax_scale
+    s = s.masked_fill(~allow, float("-inf"))
+    return torch.softmax(s, dim=-1) @ vv
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_backward_matches_torch_autograd(causal):
+    p, q, k, v, do, idx, cnt = _bwd_case(causal)
+    dq, dk, dv = O.attend_backward(q, k, v, do, idx, cnt, p)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    o = _torch_masked_attention(p, tq, tk, tv, idx, cnt)
+    o.backward(torch.tensor(do))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-11)
+    # the forward of that graph is the oracle's read
+    o_ref, _ = O.attend_masked_dense(q, k, v, idx, cnt, p)
+    np.testing.assert_allclose(o.detach().numpy(), o_ref, atol=1e-12)
+
+
+def test_backward_dense_case_matches_sdpa_autograd():
+    # every block routed and W >= Bq: the read is dense causal GQA attention
+    p, q, k, v, do, _, _ = _bwd_case(True, top_k=12, W=8)
+    r = O.route(O.block_summary(q, 8), O.block_summary(k, 8), p)
+    dq, dk, dv = O.attend_backward(q, k, v, do, r.idx, r.cnt, p)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    o = F.scaled_dot_product_attention(tq, tk.repeat_interleave(2, dim=1),
+                                       tv.repeat_interleave(2, dim=1), is_causal=True)
+    o.backward(torch.tensor(do))
+    for got, t in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(got, t.grad.numpy(), atol=1e-11)
+
+
+def test_backward_matches_central_differences():
+    p, q, k, v, do, idx, cnt = _bwd_case(True, N=48, Hq=2, Hkv=1, D=3, bk=8, top_k=2, W=6,
+                                         seed=67)
+    dq, dk, dv = O.attend_backward(q, k, v, do, idx, cnt, p)
+
+    def loss(q_, k_, v_):
+        o, _ = O.attend_masked_dense(q_, k_, v_, idx, cnt, p)
+        return float((o * do).sum())
+
+    rng = np.random.default_rng(3)
+    eps = 1e-6
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(6):
+            pos = tuple(int(rng.integers(n)) for n in x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[pos] += eps
+            xm[pos] -= eps
+            args = {"q": (q, k, v), "k": (q, k, v), "v": (q, k, v)}[name]
+            a_p = [xp if t is x else t for t in args]
+            a_m = [xm if t is x else t for t in args]
+            fd = (loss(*a_p) - loss(*a_m)) / (2 * eps)
+            assert fd == pytest.approx(grad[pos], abs=2e-7), (name, pos)
+
+
+def test_backward_shift_invariants():
+    # a common shift of every key adds the same logit to a row: no change,
+    # so the key gradients of a KV head sum to zero; a common shift of every
+    # value shifts every read by it, so the value gradients of a KV head sum
+    # to the upstream gradients of its query heads
+    p, q, k, v, do, idx, cnt = _bwd_case(True, seed=71)
+    _, dk, dv = O.attend_backward(q, k, v, do, idx, cnt, p)
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-11)
+    g = p.group
+    for kv in range(p.Hkv):
+        want = do[:, kv * g:(kv + 1) * g].sum(axis=(1, 2))
+        np.testing.assert_allclose(dv[:, kv].sum(axis=1), want, atol=1e-11)
+
+
+def test_backward_restricted_to_blocks_sums_to_the_whole():
+    p, q, k, v, do, idx, cnt = _bwd_case(True, seed=73)
+    dq, dk, dv = O.attend_backward(q, k, v, do, idx, cnt, p)
+    blocks = [(0, h, qb) for h in range(p.Hq) for qb in range(p.n_qblocks)]
+    a = O.attend_backward(q, k, v, do, idx, cnt, p, blocks=blocks[::2])
+    b = O.attend_backward(q, k, v, do, idx, cnt, p, blocks=blocks[1::2])
+    np.testing.assert_allclose(a[0] + b[0], dq, atol=1e-12)
+    np.testing.assert_allclose(a[1] + b[1], dk, atol=1e-12)
+    np.testing.assert_allclose(a[2] + b[2], dv, atol=1e-12)
