@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--seq-len", type=int, default=0,
                     help="run the chosen workload's recipe at another sequence length "
                          "(e.g. a smaller copy of the million-token workload for profiling)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward of the read (lists held fixed) instead of the forward")
     ap.add_argument("--decode", action="store_true",
                     help="time one decode step (a query per head at the last position of the "
                          "workload's full K/V cache) instead of the prefill")
@@ -826,6 +828,153 @@ def run_decode(args):
     print(json.dumps(line), flush=True)
 
 
+def run_backward(args):
+    """The backward of the read (lists held fixed) after one forward: a step
+    is one ssa_attend_backward over the whole workload."""
+    import numpy as np
+    import torch
+
+    from content_routed_block_b200 import build, ssa
+    from content_routed_block_b200.workloads import make_inputs, to_bf16_bits
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    w = workload_of(args)
+    p = ssa.params_of(w)
+    x = make_inputs(w)
+    qd, kd, vd = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in "qkv")
+    g16 = to_bf16_bits(np.random.default_rng(w.seed + 1000).standard_normal(
+        (w.B, w.Hq, w.N, w.D)).astype(np.float32))
+    gh = torch.from_numpy(g16.view(np.int16)).view(torch.bfloat16)
+    gd = gh.to(dev)
+    o, lse, idx, cnt = ssa.forward(qd, kd, vd, p)
+    outs = (torch.empty((w.B, w.Hq, w.N, w.D), dtype=torch.float32, device=dev),
+            torch.empty((w.B, w.Hkv, w.N, w.D), dtype=torch.float32, device=dev),
+            torch.empty((w.B, w.Hkv, w.N, w.D), dtype=torch.float32, device=dev))
+    ws = torch.empty(max(ssa.lib().ssa_backward_workspace_size(__import__("ctypes").byref(p)), 1),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        ssa.backward(qd, kd, vd, o, lse, gd, idx, cnt, p, workspace=ws, out=outs)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    ssa.check_error()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = str(getattr(props, "uuid", "")) or str(local)
+    if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) > 8:
+        gpu_id = "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark("start")
+    for s_ in range(args.steps):
+        flush.zero_()
+        starts[s_].record()
+        step()
+        ends[s_].record()
+    torch.cuda.synchronize()
+    sampler.mark("end")
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    ssa.check_error()
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(starts, ends)), world, dev)
+    tokens, value = replica_throughput(w.B * w.N, world, ms)
+    work = algorithmic_work(w, idx.cpu().numpy(), cnt.cpu().numpy())
+    pairs = work["keys_per_query"] * w.B * w.Hq * w.N
+    flops = 10.0 * w.D * pairs            # S, dP, dq, dk, dv: 2 D flops each per (query, key) pair
+    achieved = flops / (ms * 1e-3) / 1e12
+    fma_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        gp = gh.pin_memory()
+        host_out = [torch.empty(t.shape, dtype=torch.float32).pin_memory() for t in outs]
+        for _ in range(3):
+            gd.copy_(gp, non_blocking=True)
+            step()
+            for hh, dd in zip(host_out, outs):
+                hh.copy_(dd, non_blocking=True)
+        torch.cuda.synchronize()
+        n_e2e = min(args.steps, 20)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_e2e):
+            gd.copy_(gp, non_blocking=True)
+            step()
+            for hh, dd in zip(host_out, outs):
+                hh.copy_(dd, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
+        e2e = {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": gp.numel() * 2,
+               "d2h_bytes_per_step": sum(t.numel() * 4 for t in host_out), "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle as O
+        op = O.Params.of(w)
+        q64, k64, v64 = (O.upcast_bf16(x[n]) for n in "qkv")
+        g64 = O.upcast_bf16(g16)
+        r = O.route(O.block_summary(q64, w.block_q), O.block_summary(k64, w.block_k), op,
+                    rows=[(0, 0, qb) for qb in range(op.n_qblocks)])
+        rng = np.random.default_rng(0)
+        t0 = time.perf_counter()
+        units = 0
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            qb = int(rng.integers(op.n_qblocks))
+            O.attend_backward(q64, k64, v64, g64, r.idx, r.cnt, op, blocks=[(0, 0, qb)])
+            units += 1
+        wall = time.perf_counter() - t0
+        cpu = {"value": units * w.block_q / w.Hq / wall, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{units} (query head, query block) units of this workload's backward "
+                         f"(the oracle's fp64 masked-dense gradients; one unit is 1/Hq of the "
+                         f"work of {w.block_q} tokens) in one process, ~{args.cpu_seconds:.0f} s"}
+    clocks = sampler.summary()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    cfg = workload_config(w, args)
+    cfg["workload"] = "backward (lists held fixed): " + cfg["workload"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ssa", "config": cfg,
+        "keys_per_query": work["keys_per_query"],
+        "roofline": {"bound": "alu", "kernel": "bwd_kernel (CUDA-core fp32 FMA)",
+                     "achieved": achieved, "peak": fma_peak, "unit": "TFLOP/s",
+                     "frac": achieved / fma_peak, "traffic": None,
+                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz",
+                     "flops_per_launch": flops},
+        "cpu_baseline": cpu, "e2e": e2e,
+        # per step: two memsets (dk, dv), the delta kernel and the gradient kernel
+        "gpu_launches": 2 * args.steps, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference_decode(args):
     """The oracle's decode step, timed per step on one host core."""
     if int(os.environ.get("RANK", "0")) != 0:
@@ -861,10 +1010,61 @@ def run_reference_decode(args):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_backward(args):
+    """The oracle's backward, a bounded sample per step on one host core."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import numpy as np
+    import oracle as O
+    from content_routed_block_b200.workloads import make_inputs, to_bf16_bits
+    w = workload_of(args)
+    op = O.Params.of(w)
+    x = make_inputs(w, q_heads=[0], kv_heads=[0])
+    q64, k64, v64 = (O.upcast_bf16(x[n]) for n in "qkv")
+    g64 = O.upcast_bf16(to_bf16_bits(np.random.default_rng(w.seed + 1000).standard_normal(
+        (1, 1, w.N, w.D)).astype(np.float32)))
+    sub = O.Params.of(w.with_(B=1, Hq=1, Hkv=1))
+    r = O.route(O.block_summary(q64[:1], w.block_q), O.block_summary(k64[:1], w.block_k), sub)
+    per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
+    rng = np.random.default_rng(0)
+    vals, units_all = [], 0
+    t_all = time.time()
+    for s_ in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        units = 0
+        while time.perf_counter() - t0 < per_step:
+            O.attend_backward(q64[:1], k64[:1], v64[:1], g64, r.idx, r.cnt, sub,
+                              blocks=[(0, 0, int(rng.integers(sub.n_qblocks)))])
+            units += 1
+        if s_ >= args.warmup:
+            vals.append(units * w.block_q / w.Hq / (time.perf_counter() - t0))
+            units_all += units
+    wall = time.time() - t_all
+    value = statistics.mean(vals)
+    sample = (f"{units_all} (query head, query block) units of this workload's backward over "
+              f"{args.steps} steps, ~{per_step:.1f} s each, one process; one unit is 1/Hq of the "
+              f"work of {w.block_q} tokens")
+    cfg = workload_config(w, args)
+    cfg["workload"] = "backward (lists held fixed): " + cfg["workload"]
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * wall / max(1, args.steps + args.warmup), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": cfg,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.decode:
         (run_reference_decode if args.impl == "reference" else run_decode)(args)
+        return
+    if args.backward:
+        (run_reference_backward if args.impl == "reference" else run_backward)(args)
         return
     if args.impl == "reference":
         run_reference(args)

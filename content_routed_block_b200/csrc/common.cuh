@@ -22,7 +22,7 @@ enum : uint32_t {
 enum : uint32_t {
   kSiteProbe = 1,
   kSiteQFull = 10, kSiteKvEmpty, kSiteKvFull, kSiteSFull, kSitePFull, kSitePvDone,
-  kSiteDrain, kSiteMma, kSiteListCap = 30, kSiteIdx, kSiteCons, kSiteTree,
+  kSiteDrain, kSiteMma, kSiteListCap = 30, kSiteIdx, kSiteCons, kSiteTree, kSiteBwd,
 };
 
 // the library is a single translation unit, so the word is defined here

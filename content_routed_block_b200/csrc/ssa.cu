@@ -18,6 +18,7 @@
 
 #include "../../include/ssa.h"
 #include "attend.cuh"
+#include "backward.cuh"
 #include "common.cuh"
 #include "consensus.cuh"
 #include "cumulant.cuh"
@@ -428,6 +429,25 @@ ssa_status launch_route_tree(const ssa_params* p, const float* qsum, const float
   e = p->D == 64 ? launch_tree_select_d<64>(a, stream) : launch_tree_select_d<128>(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "tree_select_kernel launch");
   return SSA_OK;
+}
+
+// ------------------------------------------------------------------ backward
+size_t bwd_ws_bytes(const ssa_params* p) {
+  return align256(static_cast<size_t>(p->B) * p->Hq * p->N * sizeof(float));
+}
+
+template <int D>
+cudaError_t launch_backward_d(const ssa::BwdArgs& a, int B, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(B) * a.Hq * a.N;
+  ssa::bwd_delta_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(a, rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = ssa::bwd_smem_bytes<D>();
+  e = cudaFuncSetAttribute(ssa::bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  ssa::bwd_kernel<D><<<dim3(a.N / a.RT, B * a.Hq), ssa::kBwdThreads, smem, stream>>>(a);
+  return cudaGetLastError();
 }
 
 // Query heads per attend CTA.  Consensus lists are shared by a KV group, so
@@ -933,6 +953,66 @@ ssa_status ssa_forward_static(const ssa_params* p, const void* q, const void* k,
   // nothing has to be cleared between calls.
   return ssa_forward(p, q, k, v, o, lse, idx_out, cnt_out, scratch, ssa::kStaticScratchBytes,
                      stream);
+}
+
+size_t ssa_backward_workspace_size(const ssa_params* p) {
+  if (validate(p) != SSA_OK) return 0;
+  return bwd_ws_bytes(p);
+}
+
+ssa_status ssa_attend_backward(const ssa_params* p, const void* q, const void* k, const void* v,
+                               const void* o, const float* lse, const void* d_o,
+                               const int32_t* idx, const int32_t* cnt, float* dq, float* dk,
+                               float* dv, void* workspace, size_t workspace_bytes,
+                               ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (!q || !k || !v || !o || !lse || !d_o || !cnt || !dq || !dk || !dv || (p->top_k > 0 && !idx))
+    return fail(SSA_ERR_INVALID_ARG,
+                "q, k, v, o, lse, d_o, cnt, dq, dk, dv (and idx when top_k > 0) must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(d_o) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(SSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  const size_t need = bwd_ws_bytes(p);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(SSA_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t kv_bytes = static_cast<size_t>(p->B) * p->Hkv * p->N * p->D * sizeof(float);
+  cudaError_t e = cudaMemsetAsync(dk, 0, kv_bytes, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clear dk / dv");
+  ssa::BwdArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.o = static_cast<const __nv_bfloat16*>(o);
+  a.d_o = static_cast<const __nv_bfloat16*>(d_o);
+  a.lse = lse;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.delta = static_cast<float*>(workspace);
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.N = p->N;
+  a.Bq = p->block_q;
+  a.Bk = p->block_k;
+  a.top_k = p->top_k;
+  a.window = p->window;
+  a.causal = p->causal;
+  a.list_heads = p->consensus ? p->Hkv : p->Hq;
+  a.NQB = p->N / p->block_q;
+  a.NB = p->N / p->block_k;
+  a.RT = std::min(p->block_q, ssa::kBwdRows);
+  a.CK = std::min(p->block_k, ssa::kBwdKeys);
+  a.scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
+  e = p->D == 64 ? launch_backward_d<64>(a, p->B, st) : launch_backward_d<128>(a, p->B, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  return ok();
 }
 
 size_t ssa_decode_workspace_size(const ssa_params* p) {

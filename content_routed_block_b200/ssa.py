@@ -17,7 +17,7 @@ __all__ = [
     "Params", "SsaError", "lib", "make_params", "params_of", "workspace_size", "block_summary",
     "route", "route_consensus", "route_features", "route_cumulant", "tree_summary", "route_tree",
     "attend", "forward",
-    "forward_host", "decode", "decode_workspace_size", "check_error",
+    "forward_host", "backward", "decode", "decode_workspace_size", "check_error",
     "probe_wait_timeout",
     "declared_functions", "LIB_PATH", "HEADER_PATH",
 ]
@@ -104,6 +104,8 @@ def lib() -> ctypes.CDLL:
         "ssa_route_cumulant": (i32, [P, vp, vp, vp, vp, vp, vp]),
         "ssa_attend": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ssa_forward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ssa_backward_workspace_size": (sz, [P]),
+        "ssa_attend_backward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_decode_workspace_size": (sz, [P]),
         "ssa_decode": (i32, [P, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_check_error": (i32, [vp]),
@@ -355,6 +357,34 @@ def forward_host(q_host, k_host, v_host, p: Params, o_host: torch.Tensor,
     compute.wait_stream(s_out)
     compute.wait_stream(s_in)
     return o_host
+
+
+def backward(q, k, v, o, lse, d_o, idx, cnt, p: Params, workspace: torch.Tensor | None = None,
+             out=None):
+    """Gradients of the read with the lists held fixed: (dq fp32 [B, Hq, N, D],
+    dk fp32 [B, Hkv, N, D], dv fp32 [B, Hkv, N, D]).  ``o``/``lse``/``idx``/
+    ``cnt`` are the forward's outputs; ``out`` may hold preallocated (dq, dk, dv)."""
+    for t, name in ((q, "q"), (o, "o"), (d_o, "d_o")):
+        _need(t, torch.bfloat16, (p.B, p.Hq, p.N, p.D), name)
+    _need(k, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "k")
+    _need(v, torch.bfloat16, (p.B, p.Hkv, p.N, p.D), "v")
+    _need(lse, torch.float32, (p.B, p.Hq, p.N), "lse")
+    _need(idx, torch.int32, (p.B, p.list_heads, p.n_qblocks, max(p.top_k, 0)), "idx")
+    _need(cnt, torch.int32, (p.B, p.list_heads, p.n_qblocks), "cnt")
+    dev = q.device
+    ws = lib().ssa_backward_workspace_size(ctypes.byref(p))
+    if workspace is None or workspace.numel() < ws:
+        workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = (torch.empty((p.B, p.Hq, p.N, p.D), dtype=torch.float32, device=dev),
+               torch.empty((p.B, p.Hkv, p.N, p.D), dtype=torch.float32, device=dev),
+               torch.empty((p.B, p.Hkv, p.N, p.D), dtype=torch.float32, device=dev))
+    dq, dk, dv = out
+    _check(lib().ssa_attend_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                     _ptr(lse), _ptr(d_o), _ptr(idx) if p.top_k else None,
+                                     _ptr(cnt), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                     workspace.numel(), _stream()))
+    return dq, dk, dv
 
 
 def decode_workspace_size(p: Params) -> int:

@@ -260,6 +260,37 @@ ssa_status ssa_forward_static(const ssa_params* p, const void* q, const void* k,
                               void* o, float* lse, int32_t* idx_out, int32_t* cnt_out,
                               ssa_stream_t stream);
 
+/* Bytes of device workspace ssa_attend_backward needs (0 if the parameters
+ * are invalid): one fp32 per query row. */
+size_t ssa_backward_workspace_size(const ssa_params* p);
+
+/* Backward of the read with the selection held fixed (jonsmirl/ssa README,
+ * introduction: within a query's key set the read is ordinary softmax
+ * attention; the routed lists are a discrete choice and pass no gradient).
+ * For query i with key set S_i (the set ssa_attend reads), P_ij =
+ * exp(scale q_i . k_j - lse_i) and upstream gradient g_i = dL/do_i:
+ *   dv_j += P_ij g_i;  dS_ij = P_ij (g_i . v_j - delta_i), delta_i = g_i . o_i;
+ *   dq_i = scale sum_j dS_ij k_j;  dk_j += scale dS_ij q_i.
+ * A KV head's dk / dv sum over the query heads of its group.
+ *   q, k, v, o  bf16 (device): the forward's inputs and output
+ *   lse         fp32 [B, Hq, N] (device): the forward's log-sum-exp
+ *   d_o         bf16 [B, Hq, N, D] (device): the upstream gradient
+ *   idx/cnt     the lists the forward read (per head, or per KV group with
+ *               p->consensus), as for ssa_attend
+ *   dq          fp32 [B, Hq, N, D] (device, out)
+ *   dk, dv      fp32 [B, Hkv, N, D] (device, out; cleared by the call, then
+ *               accumulated with atomic adds, so their summation order -- and
+ *               the last bits -- can vary from run to run)
+ *   workspace   ssa_backward_workspace_size(p) bytes (device, 256-byte aligned)
+ * List entries that are out of range, not ascending or not admissible are
+ * reported through ssa_check_error (SSA_ERR_DEVICE_CHECK) and skipped.  Two
+ * memsets and two launches (delta, then the gradients). */
+ssa_status ssa_attend_backward(const ssa_params* p, const void* q, const void* k, const void* v,
+                               const void* o, const float* lse, const void* d_o,
+                               const int32_t* idx, const int32_t* cnt, float* dq, float* dk,
+                               float* dv, void* workspace, size_t workspace_bytes,
+                               ssa_stream_t stream);
+
 /* Bytes of device workspace ssa_decode needs for these parameters (0 if they
  * are invalid for decode). */
 size_t ssa_decode_workspace_size(const ssa_params* p);
