@@ -12,16 +12,19 @@
 // First form, on the CUDA cores:
 //  * bwd_delta_kernel: delta_i = <g_i, o_i> in fp32, one warp per row.
 //  * bwd_kernel<D>: one CTA per (b, query head, tile of RT = min(Bq, 64)
-//    query rows).  The tile walks the same key set as the forward: the key
-//    blocks of its window range (mask j <= i and (j > i - W or the block is
-//    routed)), then the routed blocks before that range (every key visible).
-//    Per chunk of CK = min(Bk, 64) keys, K and V are staged in shared memory
-//    (fp32, rows padded by one word), each thread scores 4 rows x 1 key
-//    (S and dP over D), writes P and dS to shared memory, then accumulates
-//    dq in registers (4 rows x 1 column per task) and the chunk's dk and dv
-//    (1 key x 4 columns per task) which it adds to global fp32 with
-//    vector (float4) atomic reductions: many query tiles of a KV group read
-//    the same key.
+//    query rows; 32 for D = 128).  The tile walks the same key set as the
+//    forward: the key blocks of its window range (mask j <= i and
+//    (j > i - W or the block is routed)), then the routed blocks before that
+//    range (every key visible).  Per chunk of CK = min(Bk, 64) keys, K and V
+//    are staged in shared memory as fp32, and the five products run as 4 x 4
+//    register outer products fed by float4 shared-memory loads (each operand
+//    kept in the layout its product reads: Q, g, K also transposed, dS both
+//    ways):
+//      S, dP  (4 rows x 4 keys over D)  -> P and dS in shared memory
+//      dq    += dS K   (4 rows x 4 columns over the chunk's keys, registers)
+//      dk, dv  = scale dS^T Q, P^T g (4 keys x 4 columns over the rows),
+//    and dk, dv go to global fp32 with float4 atomic reductions: many query
+//    tiles of a KV group read the same key.
 #pragma once
 
 #include "common.cuh"
@@ -29,7 +32,6 @@
 namespace ssa {
 
 constexpr int kBwdThreads = 256;
-constexpr int kBwdRows = 64;   // query rows per CTA (at most)
 constexpr int kBwdKeys = 64;   // keys per chunk (at most)
 
 struct BwdArgs {
@@ -69,28 +71,56 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdArgs a, int64_t
   if (lane == 0) a.delta[row] = s;
 }
 
+// Rows per CTA at most: 64 for D = 64, 32 for D = 128 (shared memory).
+template <int D>
+__host__ __device__ constexpr int bwd_rows() { return D == 64 ? 64 : 32; }
+
+// Shared-memory layout (fp32; transposed arrays padded by 4 words per row,
+// which keeps float4 alignment):
+//   QT, GT [D][RTM+4]   queries / upstream gradients, transposed
+//   QR, GR [RTM][D]     the same, row-major
+//   KT, VT [D][CK+4]    the chunk's keys / values, transposed
+//   KR     [CK][D]      the chunk's keys, row-major
+//   PM, SM [RTM][CK+4]  P and dS
+//   ST     [CK][RTM+4]  dS transposed
+//   lse, delta [RTM]; the list [64]
+template <int D>
+struct BwdLayout {
+  static constexpr int RTM = bwd_rows<D>();
+  static constexpr int CK = kBwdKeys;
+  static constexpr int LQ = RTM + 4, LK = CK + 4;
+  static constexpr int QT = 0, GT = QT + D * LQ, QR = GT + D * LQ, GR = QR + RTM * D;
+  static constexpr int KT = GR + RTM * D, VT = KT + D * LK, KR = VT + D * LK;
+  static constexpr int PM = KR + CK * D, SM = PM + RTM * LK, ST = SM + RTM * LK;
+  static constexpr int LSE = ST + CK * LQ, DEL = LSE + RTM, LIST = DEL + RTM;
+  static constexpr int TOTAL = LIST + 64;
+};
+
 template <int D>
 __host__ __device__ constexpr size_t bwd_smem_bytes() {
-  // Q, dO [RT][D]; K, V [CK][D+1]; P, dS [RT][CK+1]; lse, delta [RT]; list
-  return static_cast<size_t>(2 * kBwdRows * D + 2 * kBwdKeys * (D + 1) +
-                             2 * kBwdRows * (kBwdKeys + 1) + 2 * kBwdRows) * 4 + 64 * 4;
+  return static_cast<size_t>(BwdLayout<D>::TOTAL) * 4;
 }
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads) bwd_kernel(const BwdArgs a) {
+  using L = BwdLayout<D>;
   extern __shared__ __align__(16) float bsm[];
   const int RT = a.RT, CK = a.CK;
-  float* Qs = bsm;                          // [RT][D]
-  float* Gs = Qs + kBwdRows * D;            // [RT][D]   upstream gradient
-  float* Ks = Gs + kBwdRows * D;            // [CK][D+1]
-  float* Vs = Ks + kBwdKeys * (D + 1);      // [CK][D+1]
-  float* Ps = Vs + kBwdKeys * (D + 1);      // [RT][CK+1]
-  float* Ss = Ps + kBwdRows * (kBwdKeys + 1);  // [RT][CK+1] dS
-  float* lse_s = Ss + kBwdRows * (kBwdKeys + 1);
-  float* del_s = lse_s + kBwdRows;
-  int* list_s = reinterpret_cast<int*>(del_s + kBwdRows);  // [top_k <= 64]
+  float* QT = bsm + L::QT;
+  float* GT = bsm + L::GT;
+  float* QR = bsm + L::QR;
+  float* GR = bsm + L::GR;
+  float* KT = bsm + L::KT;
+  float* VT = bsm + L::VT;
+  float* KR = bsm + L::KR;
+  float* PM = bsm + L::PM;
+  float* SM = bsm + L::SM;
+  float* ST = bsm + L::ST;
+  float* lse_s = bsm + L::LSE;
+  float* del_s = bsm + L::DEL;
+  int* list_s = reinterpret_cast<int*>(bsm + L::LIST);
+  constexpr int LQ = L::LQ, LK = L::LK;
   const int tid = threadIdx.x;
-  const int PD = D + 1, PK = CK + 1;
 
   const int64_t bh = blockIdx.y;                    // b * Hq + h
   const int b = static_cast<int>(bh / a.Hq), h = static_cast<int>(bh % a.Hq);
@@ -103,15 +133,18 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_kernel(const BwdArgs a) {
   const float l2e = 1.4426950408889634f;
   const float sl2 = a.scale * l2e;
 
-  // the tile's query rows and upstream gradients (fp32), LSE and delta
+  // the tile's query rows and upstream gradients (fp32, both layouts)
   const int64_t qoff = (bh * a.N + i0) * D;
   for (int t = tid; t < RT * D / 2; t += kBwdThreads) {
     const float2 x = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.q + qoff)[t]);
     const float2 y = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.d_o + qoff)[t]);
-    Qs[2 * t] = x.x;
-    Qs[2 * t + 1] = x.y;
-    Gs[2 * t] = y.x;
-    Gs[2 * t + 1] = y.y;
+    const int i = (2 * t) / D, d = (2 * t) % D;
+    reinterpret_cast<float2*>(QR + i * D + d)[0] = x;
+    reinterpret_cast<float2*>(GR + i * D + d)[0] = y;
+    QT[d * LQ + i] = x.x;
+    QT[(d + 1) * LQ + i] = x.y;
+    GT[d * LQ + i] = y.x;
+    GT[(d + 1) * LQ + i] = y.y;
   }
   for (int t = tid; t < RT; t += kBwdThreads) {
     lse_s[t] = a.lse[bh * a.N + i0 + t] * l2e;
@@ -136,13 +169,15 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_kernel(const BwdArgs a) {
   }
   __syncthreads();
 
-  // dq accumulators: task u = tid + 256 r covers rows 4 (u / D) .. +3, column u % D
-  constexpr int QT = (kBwdRows / 4) * D / kBwdThreads;  // tasks per thread at RT = 64
-  float acc[QT][4];
+  // dq tile of this thread: rows 4 rq .. +3, columns 4 cq .. +3
+  const int n_qtiles = (RT / 4) * (D / 4);
+  const bool has_q = tid < n_qtiles;
+  const int cq = tid % (D / 4), rq = tid / (D / 4);
+  float dq[4][4];
 #pragma unroll
-  for (int r = 0; r < QT; ++r)
+  for (int e = 0; e < 4; ++e)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[r][e] = 0.f;
+    for (int f = 0; f < 4; ++f) dq[e][f] = 0.f;
 
   // blocks to visit: causal -- the window range [wlo, whi], then routed
   // blocks below wlo; non-causal -- the routed blocks
@@ -154,6 +189,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_kernel(const BwdArgs a) {
   if (a.causal)
     while (below < n && list_s[below] >= 0 && list_s[below] < wlo) ++below;  // uniform
   const int n_visit = a.causal ? n_win + below : n;
+  const int n_stiles = (RT / 4) * (CK / 4);
+  const int n_ktiles = (CK / 4) * (D / 4);
 
   for (int vi = 0; vi < n_visit; ++vi) {
     int c;
@@ -176,93 +213,122 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_kernel(const BwdArgs a) {
     if (c < 0) continue;  // a rejected list entry (uniform)
     for (int ch = 0; ch < chunks_per_block; ++ch) {
       const int j0 = c * a.Bk + ch * CK;
-      __syncthreads();  // the previous chunk's K, V, P, dS are no longer read
+      __syncthreads();  // the previous chunk's arrays are no longer read
       const int64_t koff = (bkv * a.N + j0) * D;
       for (int t = tid; t < CK * D / 2; t += kBwdThreads) {
         const float2 x = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.k + koff)[t]);
         const float2 y = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(a.v + koff)[t]);
         const int jj = (2 * t) / D, d = (2 * t) % D;
-        Ks[jj * PD + d] = x.x;
-        Ks[jj * PD + d + 1] = x.y;
-        Vs[jj * PD + d] = y.x;
-        Vs[jj * PD + d + 1] = y.y;
+        reinterpret_cast<float2*>(KR + jj * D + d)[0] = x;
+        KT[d * LK + jj] = x.x;
+        KT[(d + 1) * LK + jj] = x.y;
+        VT[d * LK + jj] = y.x;
+        VT[(d + 1) * LK + jj] = y.y;
       }
       __syncthreads();
-      // phase 1: P and dS, 4 rows x 1 key per task
-      for (int u = tid; u < (RT / 4) * CK; u += kBwdThreads) {
-        const int ig = u / CK, jj = u % CK;
-        const int j = j0 + jj;
-        float s[4] = {0.f, 0.f, 0.f, 0.f}, dp[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int d = 0; d < D; ++d) {
-          const float kx = Ks[jj * PD + d], vx = Vs[jj * PD + d];
+      // phase 1: S and dP for rows 4 rs .. +3 x keys 4 ks .. +3, then P, dS
+      for (int u = tid; u < n_stiles; u += kBwdThreads) {
+        const int ks = u % (CK / 4), rs = u / (CK / 4);
+        float sv[4][4], dp[4][4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            s[e] = fmaf(Qs[(4 * ig + e) * D + d], kx, s[e]);
-            dp[e] = fmaf(Gs[(4 * ig + e) * D + d], vx, dp[e]);
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+          for (int f = 0; f < 4; ++f) sv[e][f] = dp[e][f] = 0.f;
+#pragma unroll 4
+        for (int d = 0; d < D; ++d) {
+          const float4 qx = *reinterpret_cast<const float4*>(QT + d * LQ + 4 * rs);
+          const float4 kx = *reinterpret_cast<const float4*>(KT + d * LK + 4 * ks);
+          const float4 gx = *reinterpret_cast<const float4*>(GT + d * LQ + 4 * rs);
+          const float4 vx = *reinterpret_cast<const float4*>(VT + d * LK + 4 * ks);
+          const float qa[4] = {qx.x, qx.y, qx.z, qx.w}, ka[4] = {kx.x, kx.y, kx.z, kx.w};
+          const float ga[4] = {gx.x, gx.y, gx.z, gx.w}, va[4] = {vx.x, vx.y, vx.z, vx.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+              sv[e][f] = fmaf(qa[e], ka[f], sv[e][f]);
+              dp[e][f] = fmaf(ga[e], va[f], dp[e][f]);
+            }
+        }
+        float pt[4][4], st[4][4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * rs + e;
+          const int pos = i0 + i;
+#pragma unroll
+          for (int f = 0; f < 4; ++f) {
+            const int j = j0 + 4 * ks + f;
+            const bool ok = full || (j <= pos && (j > pos - a.window || routed_c));
+            const float p = ok ? exp2f(fmaf(sv[e][f], sl2, -lse_s[i])) : 0.f;
+            pt[e][f] = p;
+            st[e][f] = p * (dp[e][f] - del_s[i]);
           }
+          *reinterpret_cast<float4*>(PM + i * LK + 4 * ks) = make_float4(pt[e][0], pt[e][1], pt[e][2], pt[e][3]);
+          *reinterpret_cast<float4*>(SM + i * LK + 4 * ks) = make_float4(st[e][0], st[e][1], st[e][2], st[e][3]);
+        }
+#pragma unroll
+        for (int f = 0; f < 4; ++f)
+          *reinterpret_cast<float4*>(ST + (4 * ks + f) * LQ + 4 * rs) =
+              make_float4(st[0][f], st[1][f], st[2][f], st[3][f]);
+      }
+      __syncthreads();
+      // phase 2a: dq += dS K over the chunk's keys (rows 4 rq.., columns 4 cq..)
+      if (has_q) {
+#pragma unroll 4
+        for (int jj = 0; jj < CK; ++jj) {
+          const float4 sx = *reinterpret_cast<const float4*>(ST + jj * LQ + 4 * rq);
+          const float4 kx = *reinterpret_cast<const float4*>(KR + jj * D + 4 * cq);
+          const float sa[4] = {sx.x, sx.y, sx.z, sx.w}, ka[4] = {kx.x, kx.y, kx.z, kx.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int f = 0; f < 4; ++f) dq[e][f] = fmaf(sa[e], ka[f], dq[e][f]);
+        }
+      }
+      // phase 2b: the chunk's dk = scale dS^T Q and dv = P^T G (keys 4 kk..,
+      // columns 4 ck..), added to global memory with float4 atomics
+      for (int u = tid; u < n_ktiles; u += kBwdThreads) {
+        const int ck = u % (D / 4), kk = u / (D / 4);
+        float gk[4][4], gv[4][4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+          for (int f = 0; f < 4; ++f) gk[e][f] = gv[e][f] = 0.f;
+#pragma unroll 2
+        for (int i = 0; i < RT; ++i) {
+          const float4 sx = *reinterpret_cast<const float4*>(SM + i * LK + 4 * kk);
+          const float4 px = *reinterpret_cast<const float4*>(PM + i * LK + 4 * kk);
+          const float4 qx = *reinterpret_cast<const float4*>(QR + i * D + 4 * ck);
+          const float4 gx = *reinterpret_cast<const float4*>(GR + i * D + 4 * ck);
+          const float sa[4] = {sx.x, sx.y, sx.z, sx.w}, pa[4] = {px.x, px.y, px.z, px.w};
+          const float qa[4] = {qx.x, qx.y, qx.z, qx.w}, ga[4] = {gx.x, gx.y, gx.z, gx.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+              gk[e][f] = fmaf(sa[e], qa[f], gk[e][f]);
+              gv[e][f] = fmaf(pa[e], ga[f], gv[e][f]);
+            }
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int i = 4 * ig + e;
-          const int pos = i0 + i;
-          const bool ok = full || (j <= pos && (j > pos - a.window || routed_c));
-          const float p = ok ? exp2f(fmaf(s[e], sl2, -lse_s[i])) : 0.f;
-          Ps[i * PK + jj] = p;
-          Ss[i * PK + jj] = p * (dp[e] - del_s[i]);
+          const int64_t off = (bkv * a.N + j0 + 4 * kk + e) * D + 4 * ck;
+          atomicAdd(reinterpret_cast<float4*>(a.dk + off),
+                    make_float4(gk[e][0] * a.scale, gk[e][1] * a.scale, gk[e][2] * a.scale,
+                                gk[e][3] * a.scale));
+          atomicAdd(reinterpret_cast<float4*>(a.dv + off),
+                    make_float4(gv[e][0], gv[e][1], gv[e][2], gv[e][3]));
         }
-      }
-      __syncthreads();
-      // phase 2a: dq += dS K (4 rows x 1 column per task)
-#pragma unroll
-      for (int r = 0; r < QT; ++r) {
-        const int u = tid + kBwdThreads * r;
-        if (u < (RT / 4) * D) {
-          const int ig = u / D, d = u % D;
-          for (int jj = 0; jj < CK; ++jj) {
-            const float kx = Ks[jj * PD + d];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(Ss[(4 * ig + e) * PK + jj], kx, acc[r][e]);
-          }
-        }
-      }
-      // phase 2b: the chunk's dk (dS^T Q) and dv (P^T dO), 1 key x 4 columns
-      for (int u = tid; u < CK * (D / 4); u += kBwdThreads) {
-        const int jj = u / (D / 4), d4 = u % (D / 4);
-        float4 gk = make_float4(0.f, 0.f, 0.f, 0.f), gv = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int i = 0; i < RT; ++i) {
-          const float ds = Ss[i * PK + jj], p = Ps[i * PK + jj];
-          const float4 qx = reinterpret_cast<const float4*>(Qs + i * D)[d4];
-          const float4 gx = reinterpret_cast<const float4*>(Gs + i * D)[d4];
-          gk.x = fmaf(ds, qx.x, gk.x);
-          gk.y = fmaf(ds, qx.y, gk.y);
-          gk.z = fmaf(ds, qx.z, gk.z);
-          gk.w = fmaf(ds, qx.w, gk.w);
-          gv.x = fmaf(p, gx.x, gv.x);
-          gv.y = fmaf(p, gx.y, gv.y);
-          gv.z = fmaf(p, gx.z, gv.z);
-          gv.w = fmaf(p, gx.w, gv.w);
-        }
-        gk.x *= a.scale;
-        gk.y *= a.scale;
-        gk.z *= a.scale;
-        gk.w *= a.scale;
-        const int64_t off = (bkv * a.N + j0 + jj) * D + 4 * d4;
-        atomicAdd(reinterpret_cast<float4*>(a.dk + off), gk);
-        atomicAdd(reinterpret_cast<float4*>(a.dv + off), gv);
       }
     }
   }
   // dq of the tile's rows
+  if (has_q) {
 #pragma unroll
-  for (int r = 0; r < QT; ++r) {
-    const int u = tid + kBwdThreads * r;
-    if (u < (RT / 4) * D) {
-      const int ig = u / D, d = u % D;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        a.dq[(bh * a.N + i0 + 4 * ig + e) * D + d] = acc[r][e] * a.scale;
-    }
+    for (int e = 0; e < 4; ++e)
+      *reinterpret_cast<float4*>(a.dq + (bh * a.N + i0 + 4 * rq + e) * D + 4 * cq) =
+          make_float4(dq[e][0] * a.scale, dq[e][1] * a.scale, dq[e][2] * a.scale,
+                      dq[e][3] * a.scale);
   }
 }
 
