@@ -9,22 +9,23 @@
 // with delta_i = <g_i, o_i> = sum_j P_ij dP_ij (the forward's output and
 // log-sum-exp are reused, so no second pass over the keys is needed).
 //
-// First form, on the CUDA cores:
+// On the CUDA cores:
 //  * bwd_delta_kernel: delta_i = <g_i, o_i> in fp32, one warp per row.
-//  * bwd_kernel<D>: one CTA per (b, query head, tile of RT = min(Bq, 64)
-//    query rows; 32 for D = 128).  The tile walks the same key set as the
+//  * bwd_kernel<D>: one CTA per (b, query head, tile of RT query rows: up to
+//    64 for D = 64, 32 for D = 128).  The tile walks the same key set as the
 //    forward: the key blocks of its window range (mask j <= i and
 //    (j > i - W or the block is routed)), then the routed blocks before that
-//    range (every key visible).  Per chunk of CK = min(Bk, 64) keys, K and V
-//    are staged in shared memory as fp32, and the five products run as 4 x 4
-//    register outer products fed by float4 shared-memory loads (each operand
-//    kept in the layout its product reads: Q, g, K also transposed, dS both
-//    ways):
-//      S, dP  (4 rows x 4 keys over D)  -> P and dS in shared memory
-//      dq    += dS K   (4 rows x 4 columns over the chunk's keys, registers)
-//      dk, dv  = scale dS^T Q, P^T g (4 keys x 4 columns over the rows),
-//    and dk, dv go to global fp32 with float4 atomic reductions: many query
-//    tiles of a KV group read the same key.
+//    range (every key visible).  Per chunk of CK keys (up to 32 for D = 64,
+//    64 for D = 128), K and V are staged in shared memory as fp32, and the
+//    five products run as register outer products fed by vector
+//    shared-memory loads, each operand kept in the layout its product reads
+//    (Q, g and K also transposed):
+//      S, dP  (2 rows x 4 keys over D)     -> P and dS in shared memory
+//      dq    += dS K  (4 rows x 4 columns, 4 keys per step, registers)
+//      dk, dv  = scale dS^T Q, P^T g  (4 keys x TC columns over the rows),
+//    and dk, dv go to global fp32 with vector atomic reductions: many query
+//    tiles of a KV group read the same key.  For D = 64 the shared memory
+//    (113 KB) and registers allow two CTAs per SM.
 #pragma once
 
 #include "common.cuh"
@@ -32,7 +33,6 @@
 namespace ssa {
 
 constexpr int kBwdThreads = 256;
-constexpr int kBwdKeys = 64;   // keys per chunk (at most)
 
 struct BwdArgs {
   const __nv_bfloat16* q;    // [B*Hq, N, D]
@@ -71,28 +71,33 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdArgs a, int64_t
   if (lane == 0) a.delta[row] = s;
 }
 
-// Rows per CTA at most: 64 for D = 64, 32 for D = 128 (shared memory).
+// Tile shape per head dimension: rows per CTA, keys per chunk, and the
+// column width of the dk/dv micro-tiles, chosen so that every phase has 256
+// micro-tiles and (for D = 64) two CTAs fit on an SM.
 template <int D>
 __host__ __device__ constexpr int bwd_rows() { return D == 64 ? 64 : 32; }
+template <int D>
+__host__ __device__ constexpr int bwd_keys() { return D == 64 ? 32 : 64; }
+template <int D>
+__host__ __device__ constexpr int bwd_kcols() { return D == 64 ? 2 : 4; }
 
 // Shared-memory layout (fp32; transposed arrays padded by 4 words per row,
 // which keeps float4 alignment):
 //   QT, GT [D][RTM+4]   queries / upstream gradients, transposed
 //   QR, GR [RTM][D]     the same, row-major
-//   KT, VT [D][CK+4]    the chunk's keys / values, transposed
-//   KR     [CK][D]      the chunk's keys, row-major
-//   PM, SM [RTM][CK+4]  P and dS
-//   ST     [CK][RTM+4]  dS transposed
+//   KT, VT [D][CKM+4]   the chunk's keys / values, transposed
+//   KR     [CKM][D]     the chunk's keys, row-major
+//   PM, SM [RTM][CKM+4] P and dS
 //   lse, delta [RTM]; the list [64]
 template <int D>
 struct BwdLayout {
   static constexpr int RTM = bwd_rows<D>();
-  static constexpr int CK = kBwdKeys;
-  static constexpr int LQ = RTM + 4, LK = CK + 4;
+  static constexpr int CKM = bwd_keys<D>();
+  static constexpr int LQ = RTM + 4, LK = CKM + 4;
   static constexpr int QT = 0, GT = QT + D * LQ, QR = GT + D * LQ, GR = QR + RTM * D;
   static constexpr int KT = GR + RTM * D, VT = KT + D * LK, KR = VT + D * LK;
-  static constexpr int PM = KR + CK * D, SM = PM + RTM * LK, ST = SM + RTM * LK;
-  static constexpr int LSE = ST + CK * LQ, DEL = LSE + RTM, LIST = DEL + RTM;
+  static constexpr int PM = KR + CKM * D, SM = PM + RTM * LK;
+  static constexpr int LSE = SM + RTM * LK, DEL = LSE + RTM, LIST = DEL + RTM;
   static constexpr int TOTAL = LIST + 64;
 };
 
@@ -101,9 +106,28 @@ __host__ __device__ constexpr size_t bwd_smem_bytes() {
   return static_cast<size_t>(BwdLayout<D>::TOTAL) * 4;
 }
 
+template <int N>
+struct BwdVec;
+template <>
+struct BwdVec<2> {
+  using T = float2;
+  __device__ static void to(const T& v, float (&a)[2]) { a[0] = v.x; a[1] = v.y; }
+  __device__ static T make(const float (&a)[2]) { return make_float2(a[0], a[1]); }
+};
+template <>
+struct BwdVec<4> {
+  using T = float4;
+  __device__ static void to(const T& v, float (&a)[4]) {
+    a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w;
+  }
+  __device__ static T make(const float (&a)[4]) { return make_float4(a[0], a[1], a[2], a[3]); }
+};
+
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads) bwd_kernel(const BwdArgs a) {
+__global__ void __launch_bounds__(kBwdThreads, D == 64 ? 2 : 1) bwd_kernel(const BwdArgs a) {
   using L = BwdLayout<D>;
+  constexpr int TC = bwd_kcols<D>();   // dk/dv micro-tile columns
+  using VC = BwdVec<TC>;
   extern __shared__ __align__(16) float bsm[];
   const int RT = a.RT, CK = a.CK;
   float* QT = bsm + L::QT;
@@ -115,7 +139,6 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_kernel(const BwdArgs a) {
   float* KR = bsm + L::KR;
   float* PM = bsm + L::PM;
   float* SM = bsm + L::SM;
-  float* ST = bsm + L::ST;
   float* lse_s = bsm + L::LSE;
   float* del_s = bsm + L::DEL;
   int* list_s = reinterpret_cast<int*>(bsm + L::LIST);
@@ -189,8 +212,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_kernel(const BwdArgs a) {
   if (a.causal)
     while (below < n && list_s[below] >= 0 && list_s[below] < wlo) ++below;  // uniform
   const int n_visit = a.causal ? n_win + below : n;
-  const int n_stiles = (RT / 4) * (CK / 4);
-  const int n_ktiles = (CK / 4) * (D / 4);
+  const int n_stiles = (RT / 2) * (CK / 4);       // phase 1: 2 rows x 4 keys
+  const int n_ktiles = (CK / 4) * (D / TC);       // phase 2b: 4 keys x TC columns
 
   for (int vi = 0; vi < n_visit; ++vi) {
     int c;
@@ -226,98 +249,99 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_kernel(const BwdArgs a) {
         VT[(d + 1) * LK + jj] = y.y;
       }
       __syncthreads();
-      // phase 1: S and dP for rows 4 rs .. +3 x keys 4 ks .. +3, then P, dS
+      // phase 1: S and dP for rows 2 rs, 2 rs + 1 x keys 4 ks .. +3, then P, dS
       for (int u = tid; u < n_stiles; u += kBwdThreads) {
         const int ks = u % (CK / 4), rs = u / (CK / 4);
-        float sv[4][4], dp[4][4];
+        float sv[2][4], dp[2][4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
+        for (int e = 0; e < 2; ++e)
 #pragma unroll
           for (int f = 0; f < 4; ++f) sv[e][f] = dp[e][f] = 0.f;
 #pragma unroll 4
         for (int d = 0; d < D; ++d) {
-          const float4 qx = *reinterpret_cast<const float4*>(QT + d * LQ + 4 * rs);
+          const float2 qx = *reinterpret_cast<const float2*>(QT + d * LQ + 2 * rs);
+          const float2 gx = *reinterpret_cast<const float2*>(GT + d * LQ + 2 * rs);
           const float4 kx = *reinterpret_cast<const float4*>(KT + d * LK + 4 * ks);
-          const float4 gx = *reinterpret_cast<const float4*>(GT + d * LQ + 4 * rs);
           const float4 vx = *reinterpret_cast<const float4*>(VT + d * LK + 4 * ks);
-          const float qa[4] = {qx.x, qx.y, qx.z, qx.w}, ka[4] = {kx.x, kx.y, kx.z, kx.w};
-          const float ga[4] = {gx.x, gx.y, gx.z, gx.w}, va[4] = {vx.x, vx.y, vx.z, vx.w};
+          const float qa[2] = {qx.x, qx.y}, ga[2] = {gx.x, gx.y};
+          const float ka[4] = {kx.x, kx.y, kx.z, kx.w}, va[4] = {vx.x, vx.y, vx.z, vx.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
+          for (int e = 0; e < 2; ++e)
 #pragma unroll
             for (int f = 0; f < 4; ++f) {
               sv[e][f] = fmaf(qa[e], ka[f], sv[e][f]);
               dp[e][f] = fmaf(ga[e], va[f], dp[e][f]);
             }
         }
-        float pt[4][4], st[4][4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 4 * rs + e;
+        for (int e = 0; e < 2; ++e) {
+          const int i = 2 * rs + e;
           const int pos = i0 + i;
+          float pt[4], st[4];
 #pragma unroll
           for (int f = 0; f < 4; ++f) {
             const int j = j0 + 4 * ks + f;
             const bool ok = full || (j <= pos && (j > pos - a.window || routed_c));
             const float p = ok ? exp2f(fmaf(sv[e][f], sl2, -lse_s[i])) : 0.f;
-            pt[e][f] = p;
-            st[e][f] = p * (dp[e][f] - del_s[i]);
+            pt[f] = p;
+            st[f] = p * (dp[e][f] - del_s[i]);
           }
-          *reinterpret_cast<float4*>(PM + i * LK + 4 * ks) = make_float4(pt[e][0], pt[e][1], pt[e][2], pt[e][3]);
-          *reinterpret_cast<float4*>(SM + i * LK + 4 * ks) = make_float4(st[e][0], st[e][1], st[e][2], st[e][3]);
+          *reinterpret_cast<float4*>(PM + i * LK + 4 * ks) = make_float4(pt[0], pt[1], pt[2], pt[3]);
+          *reinterpret_cast<float4*>(SM + i * LK + 4 * ks) = make_float4(st[0], st[1], st[2], st[3]);
         }
-#pragma unroll
-        for (int f = 0; f < 4; ++f)
-          *reinterpret_cast<float4*>(ST + (4 * ks + f) * LQ + 4 * rs) =
-              make_float4(st[0][f], st[1][f], st[2][f], st[3][f]);
       }
       __syncthreads();
-      // phase 2a: dq += dS K over the chunk's keys (rows 4 rq.., columns 4 cq..)
+      // phase 2a: dq += dS K over the chunk's keys, 4 keys at a time (rows
+      // 4 rq.., columns 4 cq..)
       if (has_q) {
-#pragma unroll 4
-        for (int jj = 0; jj < CK; ++jj) {
-          const float4 sx = *reinterpret_cast<const float4*>(ST + jj * LQ + 4 * rq);
-          const float4 kx = *reinterpret_cast<const float4*>(KR + jj * D + 4 * cq);
-          const float sa[4] = {sx.x, sx.y, sx.z, sx.w}, ka[4] = {kx.x, kx.y, kx.z, kx.w};
+#pragma unroll 2
+        for (int jj = 0; jj < CK; jj += 4) {
+          float sa[4][4], ka[4][4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
+            BwdVec<4>::to(*reinterpret_cast<const float4*>(SM + (4 * rq + e) * LK + jj), sa[e]);
 #pragma unroll
-            for (int f = 0; f < 4; ++f) dq[e][f] = fmaf(sa[e], ka[f], dq[e][f]);
+          for (int g = 0; g < 4; ++g)
+            BwdVec<4>::to(*reinterpret_cast<const float4*>(KR + (jj + g) * D + 4 * cq), ka[g]);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+              for (int f = 0; f < 4; ++f) dq[e][f] = fmaf(sa[e][g], ka[g][f], dq[e][f]);
         }
       }
-      // phase 2b: the chunk's dk = scale dS^T Q and dv = P^T G (keys 4 kk..,
-      // columns 4 ck..), added to global memory with float4 atomics
+      // phase 2b: the chunk's dk = scale dS^T Q and dv = P^T g (keys 4 kk..,
+      // columns TC ck..), added to global memory with vector atomics
       for (int u = tid; u < n_ktiles; u += kBwdThreads) {
-        const int ck = u % (D / 4), kk = u / (D / 4);
-        float gk[4][4], gv[4][4];
+        const int ck = u % (D / TC), kk = u / (D / TC);
+        float gk[4][TC], gv[4][TC];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
 #pragma unroll
-          for (int f = 0; f < 4; ++f) gk[e][f] = gv[e][f] = 0.f;
+          for (int f = 0; f < TC; ++f) gk[e][f] = gv[e][f] = 0.f;
 #pragma unroll 2
         for (int i = 0; i < RT; ++i) {
-          const float4 sx = *reinterpret_cast<const float4*>(SM + i * LK + 4 * kk);
-          const float4 px = *reinterpret_cast<const float4*>(PM + i * LK + 4 * kk);
-          const float4 qx = *reinterpret_cast<const float4*>(QR + i * D + 4 * ck);
-          const float4 gx = *reinterpret_cast<const float4*>(GR + i * D + 4 * ck);
-          const float sa[4] = {sx.x, sx.y, sx.z, sx.w}, pa[4] = {px.x, px.y, px.z, px.w};
-          const float qa[4] = {qx.x, qx.y, qx.z, qx.w}, ga[4] = {gx.x, gx.y, gx.z, gx.w};
+          float sa[4], pa[4], qa[TC], ga[TC];
+          BwdVec<4>::to(*reinterpret_cast<const float4*>(SM + i * LK + 4 * kk), sa);
+          BwdVec<4>::to(*reinterpret_cast<const float4*>(PM + i * LK + 4 * kk), pa);
+          VC::to(*reinterpret_cast<const typename VC::T*>(QR + i * D + TC * ck), qa);
+          VC::to(*reinterpret_cast<const typename VC::T*>(GR + i * D + TC * ck), ga);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
 #pragma unroll
-            for (int f = 0; f < 4; ++f) {
+            for (int f = 0; f < TC; ++f) {
               gk[e][f] = fmaf(sa[e], qa[f], gk[e][f]);
               gv[e][f] = fmaf(pa[e], ga[f], gv[e][f]);
             }
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int64_t off = (bkv * a.N + j0 + 4 * kk + e) * D + 4 * ck;
-          atomicAdd(reinterpret_cast<float4*>(a.dk + off),
-                    make_float4(gk[e][0] * a.scale, gk[e][1] * a.scale, gk[e][2] * a.scale,
-                                gk[e][3] * a.scale));
-          atomicAdd(reinterpret_cast<float4*>(a.dv + off),
-                    make_float4(gv[e][0], gv[e][1], gv[e][2], gv[e][3]));
+          const int64_t off = (bkv * a.N + j0 + 4 * kk + e) * D + TC * ck;
+#pragma unroll
+          for (int f = 0; f < TC; ++f) gk[e][f] *= a.scale;
+          atomicAdd(reinterpret_cast<typename VC::T*>(a.dk + off), VC::make(gk[e]));
+          atomicAdd(reinterpret_cast<typename VC::T*>(a.dv + off), VC::make(gv[e]));
         }
       }
     }

@@ -1008,7 +1008,7 @@ ssa_status ssa_attend_backward(const ssa_params* p, const void* q, const void* k
   a.NQB = p->N / p->block_q;
   a.NB = p->N / p->block_k;
   a.RT = std::min(p->block_q, p->D == 64 ? ssa::bwd_rows<64>() : ssa::bwd_rows<128>());
-  a.CK = std::min(p->block_k, ssa::kBwdKeys);
+  a.CK = std::min(p->block_k, p->D == 64 ? ssa::bwd_keys<64>() : ssa::bwd_keys<128>());
   a.scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
   e = p->D == 64 ? launch_backward_d<64>(a, p->B, st) : launch_backward_d<128>(a, p->B, st);
   if (e != cudaSuccess) return cuda_fail(e, "backward launch");
