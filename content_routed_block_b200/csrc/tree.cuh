@@ -22,8 +22,10 @@
 //    time, 16 per half-warp: each candidate's summary row is read coalesced
 //    (16 lanes x float4), 16 independent loads per lane, and a shuffle
 //    reduce-scatter leaves lane l with candidate e0 + l's fp32 score, which
-//    it keeps in its register top-KM list (route.cuh's 64-bit keys); five
-//    shuffle merges leave the row's top KM in every lane.  The CTA's eight warps take eight consecutive query
+//    it keeps in its register top-KM list (route.cuh's 64-bit keys).  The
+//    k-th largest lane maximum bounds the row's k-th key from below; the few
+//    list entries above it are sorted by the warp (butterfly merges of the
+//    lane lists when more than 64 survive, or k > 32).  The CTA's eight warps take eight consecutive query
 //    blocks of one head, whose kept super-blocks mostly coincide, so the
 //    children's summaries are re-read from L1.
 #pragma once
@@ -88,6 +90,7 @@ template <int D, int KM>
 __global__ void __launch_bounds__(kTreeThreads) tree_select_kernel(const TreeSelectArgs a) {
   __shared__ __align__(16) float qs[kTreeWarps][D];
   __shared__ int32_t sup_s[kTreeWarps][kTreeMaxBeam];
+  __shared__ uint64_t surv[kTreeWarps][64];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kTreeWarps + warp;
   if (row >= a.n_rows) return;  // warp-uniform
@@ -217,30 +220,76 @@ __global__ void __launch_bounds__(kTreeThreads) tree_select_kernel(const TreeSel
       }
     }
   }
-#pragma unroll
-  for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);
-
-  // every lane now holds the row's top KM keys, best first; the selected
-  // blocks are written ascending
   const int k = a.top_k;
   int n = 0;
+  if (KM <= 32) {
+    // The row's top k from the 32 lane lists.  The k-th largest lane maximum
+    // T is a lower bound on the row's k-th key (k lanes hold a key >= T), so
+    // only list entries >= T can be selected.  When at most 64 survive they
+    // are sorted directly (two warp sorts and a bitonic merge keep the top
+    // 32); otherwise five butterfly merges of the lane lists.  Either way
+    // lane j ends with the row's j-th best key (0 = none).
+    uint64_t best = 0ull;
+    bool done = false;
+    if (k > 0) {
+      const uint64_t lane_max = warp_sort_desc(keys[0], lane);
+      const uint64_t T = __shfl_sync(0xffffffffu, lane_max, k - 1);
+      if (T != 0ull) {
+        int mine = 0;
 #pragma unroll
-  for (int j = 0; j < KM; ++j) n += (j < k && keys[j] != 0ull) ? 1 : 0;
-  if (k > 0) {
-    int32_t* dst = a.idx + row * k;
-    if (KM <= 32) {
-      // lane j takes the j-th selected block; a shuffle bitonic sort of
-      // (2^32 - 1 - block) descending lists the blocks ascending, the empty
-      // lanes (key 0) last
-      uint64_t mine_key = 0ull;
+        for (int j = 0; j < KM; ++j) mine += keys[j] >= T ? 1 : 0;
+        int incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        if (total <= 64) {  // warp-uniform
+          uint64_t* buf = surv[warp];
+          const int pos = incl - mine;  // the lane's survivors are its first `mine` entries
+#pragma unroll
+          for (int j = 0; j < KM; ++j)
+            if (j < mine) buf[pos + j] = keys[j];
+          __syncwarp();
+          uint64_t v0 = lane < total ? buf[lane] : 0ull;
+          uint64_t v1 = lane + 32 < total ? buf[lane + 32] : 0ull;
+          __syncwarp();
+          v0 = warp_sort_desc(v0, lane);
+          v1 = warp_sort_desc(v1, lane);
+          uint64_t r = umax64(v0, __shfl_sync(0xffffffffu, v1, 31 - lane));
+#pragma unroll
+          for (int j = 16; j > 0; j >>= 1) {
+            const uint64_t y = __shfl_xor_sync(0xffffffffu, r, j);
+            r = (lane & j) ? umin64(r, y) : umax64(r, y);
+          }
+          best = r;
+          done = true;
+        }
+      }
+    }
+    if (!done) {
+#pragma unroll
+      for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);
 #pragma unroll
       for (int j = 0; j < KM; ++j)
-        if (j == lane && j < n)
-          mine_key = 0xFFFFFFFFull - (~static_cast<uint32_t>(keys[j] & 0xFFFFFFFFull));
-      mine_key = warp_sort_desc(mine_key, lane);
-      if (lane < k) dst[lane] = lane < n ? static_cast<int>(0xFFFFFFFFull - mine_key) : -1;
-    } else {
-      // rank by counting
+        if (j == lane) best = keys[j];
+    }
+    n = __popc(__ballot_sync(0xffffffffu, lane < k && best != 0ull));
+    if (k > 0) {
+      // the selected blocks ascending: sort (2^32 - 1 - block) descending
+      uint64_t key = lane < n ? 0xFFFFFFFFull - (~static_cast<uint32_t>(best & 0xFFFFFFFFull)) : 0ull;
+      key = warp_sort_desc(key, lane);
+      if (lane < k) a.idx[row * k + lane] = lane < n ? static_cast<int>(0xFFFFFFFFull - key) : -1;
+    }
+  } else {
+#pragma unroll
+    for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);
+    // every lane holds the row's top KM keys, best first; rank by counting
+#pragma unroll
+    for (int j = 0; j < KM; ++j) n += (j < k && keys[j] != 0ull) ? 1 : 0;
+    if (k > 0) {
+      int32_t* dst = a.idx + row * k;
 #pragma unroll
       for (int j = 0; j < KM; ++j) {
         if (j >= n) continue;
