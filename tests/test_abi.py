@@ -203,3 +203,31 @@ def test_tree_entry_points_reject_bad_arguments_before_launch(L):
     assert f(ctypes.byref(p), good, good, good, odd, good, good, good, None) == 1
     # decode keeps the flat block list
     assert L.ssa_decode_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_backward_entry_point_rejects_bad_arguments_before_launch(L):
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    p = _p()
+    ws = L.ssa_backward_workspace_size(ctypes.byref(p))
+    assert ws == (1 * 14 * 32768 * 4 + 255) // 256 * 256      # one fp32 per query row
+    f = L.ssa_attend_backward
+
+    def call(**over):
+        args = dict(q=good, k=good, v=good, o=good, lse=good, d_o=good, idx=good, cnt=good,
+                    dq=good, dk=good, dv=good, ws=good, wsb=ws)
+        args.update(over)
+        return f(ctypes.byref(p), args["q"], args["k"], args["v"], args["o"], args["lse"],
+                 args["d_o"], args["idx"], args["cnt"], args["dq"], args["dk"], args["dv"],
+                 args["ws"], args["wsb"], None)
+
+    for name in ("q", "o", "lse", "d_o", "cnt", "dq", "dk", "dv", "idx"):
+        assert call(**{name: None}) == 1, name
+    assert call(dk=odd) == 1
+    assert call(wsb=ws - 1) == 3
+    assert call(ws=None) == 3
+    assert call(ws=ctypes.c_void_p((1 << 20) + 16)) == 1
+    bad = _p(D=96)
+    assert L.ssa_backward_workspace_size(ctypes.byref(bad)) == 0
+    assert f(ctypes.byref(bad), good, good, good, good, good, good, good, good, good, good, good,
+             good, ws, None) == 2
