@@ -22,7 +22,7 @@
 //    walked in chunks of 64 keys (one or more whole blocks, or a 64-row slice
 //    of a larger block), so every key block is fetched once per CTA.
 //  * Warp 4 (one lane) gathers each chunk's K and V rows with tiled TMA loads
-//    (one box per block, no multicast) into a 128-byte-swizzled ring of
+//    (one box per block, each CTA fetching its own) into a 128-byte-swizzled ring of
 //    STAGES stages; Q (128 x D) is loaded once.
 //  * Warp 5 (one lane) issues tcgen05.mma: S = Q K^T (M=128, N=64, fp32 in
 //    TMEM, two S buffers) and O += P V (A = P read from TMEM, B = V as an
