@@ -231,3 +231,21 @@ def test_backward_entry_point_rejects_bad_arguments_before_launch(L):
     assert L.ssa_backward_workspace_size(ctypes.byref(bad)) == 0
     assert f(ctypes.byref(bad), good, good, good, good, good, good, good, good, good, good, good,
              good, ws, None) == 2
+
+
+def test_binding_checks_backward_and_tree_tensors_before_calling():
+    import torch
+    p = _p(N=1024, Hq=2, Hkv=1, top_k=4, window=128)
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)          # CPU: refused  # noqa: E731
+    q, k = bf(1, 2, 1024, 64), bf(1, 1, 1024, 64)
+    lse = torch.zeros(1, 2, 1024)
+    idx = torch.zeros(1, 2, 16, 4, dtype=torch.int32)
+    cnt = torch.zeros(1, 2, 16, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        ssa.backward(q, k, k, q, lse, q, idx, cnt, p)                # host tensors
+    t = _p(N=1024, Hq=2, Hkv=1, top_k=4, window=128, tree_fanout=4, tree_beam=2)
+    ksum = torch.zeros(1, 1, 16, 64)
+    with pytest.raises(ValueError):
+        ssa.tree_summary(ksum, t)
+    with pytest.raises(ValueError):
+        ssa.route_tree(torch.zeros(1, 2, 16, 64), ksum, torch.zeros(1, 1, 3, 64), t)
