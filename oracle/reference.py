@@ -69,7 +69,8 @@ __all__ = [
     "consensus_row", "route_consensus", "expand_consensus",
     "block_covariance", "block_second_moment", "block_scores", "decode_step",
     "decode_attend", "tree_summary", "tree_candidates", "route_tree_row",
-    "acceptable_tree_selections", "attend_backward",
+    "acceptable_tree_selections", "attend_backward", "route_flat_all",
+    "attend_gathered_blocks",
 ]
 
 NEAR_TIE_REL = 1e-4   # relative score gap under which two blocks count as tied
@@ -220,6 +221,8 @@ def route_row(qbar: np.ndarray, mu: np.ndarray, cand: np.ndarray, top_k: int,
     if len(cand) == 0 or top_k == 0:
         return np.zeros(0, dtype=np.int64), math.nan, math.nan
     s = block_scores(qbar, mu, cand, beta, q2, sigma)
+    if not np.isfinite(s).all():
+        raise ValueError("non-finite routing scores: the route is defined for finite inputs")
     # order: score descending, then block index ascending (lower index wins a tie)
     order = np.lexsort((cand, -s))
     take = min(top_k, len(cand))
@@ -273,6 +276,85 @@ def route(qsum: np.ndarray, ksum: np.ndarray, p: Params, rows=None, qm2=None,
         kth[b, h, qb], nxt[b, h, qb] = a, c
     if tree:
         return RouteResult(idx, cnt, kth, nxt, sup_idx, sup_cnt)
+    return RouteResult(idx, cnt, kth, nxt)
+
+
+def route_flat_all(qsum: np.ndarray, ksum: np.ndarray, p: Params, heads=None,
+                   chunk: int = 1024) -> RouteResult:
+    """Steps 5-6 for every query block at once: the flat mean-score route
+    (beta = 0, no two-level form) of ``route``, written with whole-array
+    operations so that it finishes at a million tokens.
+
+    Same steps, same order: the scores of a (b, head) are one float64 product
+    qsum @ ksum^T (``chunk`` query blocks at a time), the columns a query
+    block may not route to (step 4) are excluded, and each row keeps the
+    first min(top_k, |A|) admissible blocks in the order (score descending,
+    block index ascending).  Selecting that prefix needs no sort: with s_k the
+    row's k-th largest score, it is every block scoring above s_k plus the
+    lowest-indexed blocks scoring exactly s_k until k are taken.  ``heads``
+    optionally restricts the work to a list of (b, h) pairs (the other rows
+    stay at idx = -1, cnt = 0, scores nan).  Returns the same RouteResult as
+    ``route``."""
+    if p.beta != 0.0 or p.tree_fanout > 0:
+        raise ValueError("route_flat_all is the flat mean-score route (beta = 0, no tree)")
+    nqb, nb, k = p.n_qblocks, p.n_kblocks, p.top_k
+    idx = np.full((p.B, p.Hq, nqb, k), -1, dtype=np.int32)
+    cnt = np.zeros((p.B, p.Hq, nqb), dtype=np.int32)
+    kth = np.full((p.B, p.Hq, nqb), math.nan)
+    nxt = np.full((p.B, p.Hq, nqb), math.nan)
+    if k == 0:
+        return RouteResult(idx, cnt, kth, nxt)
+    if not (np.isfinite(qsum).all() and np.isfinite(ksum).all()):
+        raise ValueError("non-finite summaries: the route is defined for finite inputs only")
+    qb_all = np.arange(nqb)
+    if p.causal:
+        n_adm_all = np.minimum((qb_all * p.block_q) // p.block_k, nb)    # step 4
+    else:
+        n_adm_all = np.full(nqb, nb)
+    todo = heads if heads is not None else [(b, h) for b in range(p.B) for h in range(p.Hq)]
+    for b, h in todo:
+        mu = ksum[b, h // p.group]
+        for r0 in range(0, nqb, chunk):
+            rows = qb_all[r0:r0 + chunk]
+            n_adm = n_adm_all[rows]
+            ncol = int(n_adm.max())
+            if ncol == 0:
+                continue
+            s = qsum[b, h, rows] @ mu[:ncol].T                            # step 5
+            col = np.arange(ncol)
+            valid = col[None, :] < n_adm[:, None]
+            sm = np.where(valid, s, -np.inf)
+            take = np.minimum(k, n_adm)
+            # k-th and (k+1)-th largest admissible score of each row
+            # (descending order = ascending order of the negated scores)
+            neg = -sm
+            kk = min(k, ncol)
+            kths = [kk - 1] + ([kk] if kk < ncol else [])
+            part = np.partition(neg, kths, axis=1)
+            s_k = -part[:, kk - 1]
+            s_k1 = -part[:, kk] if kk < ncol else np.full(len(rows), -np.inf)
+            # rows with fewer admissible blocks than k take all of them: their
+            # last taken score is the row's smallest admissible score
+            short = n_adm <= k
+            if short.any():
+                smallest = np.where(valid, s, np.inf).min(axis=1)
+                s_k = np.where(short, smallest, s_k)
+                s_k1 = np.where(short, -np.inf, s_k1)
+            above = valid & (sm > s_k[:, None])
+            tied = valid & (sm == s_k[:, None])
+            need = take - above.sum(axis=1)
+            chosen = above | (tied & (np.cumsum(tied, axis=1) <= need[:, None]))   # step 6
+            # write each row's chosen blocks ascending (np.nonzero walks rows in
+            # order and each row's columns ascending)
+            rr, cc = np.nonzero(chosen)
+            counts = chosen.sum(axis=1)
+            pos = np.arange(len(rr)) - (np.cumsum(counts) - counts)[rr]
+            idx[b, h, rows[rr], pos] = cc
+            cnt[b, h, rows] = counts
+            has = take > 0
+            kth[b, h, rows[has]] = s_k[has]
+            full = has & ~short
+            nxt[b, h, rows[full]] = s_k1[full]
     return RouteResult(idx, cnt, kth, nxt)
 
 
@@ -557,6 +639,42 @@ def attend_gathered(q, k, v, idx, cnt, p: Params, queries=None):
     if queries is not None:
         return o_out, l_out
     return o_out.reshape(p.B, p.Hq, p.N, dv), l_out.reshape(p.B, p.Hq, p.N)
+
+
+def attend_gathered_blocks(q, k, v, idx, cnt, p: Params, blocks):
+    """Gathered form, one query block at a time: for each listed (b, h, qb)
+    the logits are taken only over the keys any of the block's queries can
+    see -- the selected blocks' keys and, causal, the window span
+    [qb*Bq - W + 1, (qb+1)*Bq - 1] -- and each row keeps exactly its own key
+    set (step 7, the same mask as ``attend_masked_dense``); softmax as in
+    ``_softmax_read``.  Keys outside every
+    row's set would only add exp(-inf) = 0 terms, so this is step 8 on the
+    columns where it can be non-zero, which makes sampled rows of a
+    million-token sequence cheap.  Returns ([len(blocks), Bq, Dv],
+    [len(blocks), Bq])."""
+    scale = p.softmax_scale
+    dv = v.shape[-1]
+    o_out = np.zeros((len(blocks), p.block_q, dv))
+    l_out = np.zeros((len(blocks), p.block_q))
+    for t, (b, h, qb) in enumerate(blocks):
+        g = h // p.group
+        sel = np.asarray(idx[b, h, qb, :cnt[b, h, qb]], dtype=np.int64)
+        rows = np.arange(qb * p.block_q, (qb + 1) * p.block_q)
+        cols = (sel[:, None] * p.block_k + np.arange(p.block_k)[None, :]).ravel()
+        if p.causal:
+            cols = np.union1d(cols, np.arange(max(0, rows[0] - p.window + 1), rows[-1] + 1))
+        else:
+            cols = np.unique(cols)
+        # step 7 on these columns, as in the masked-dense form: a routed key,
+        # or (causal) a window key i - W < j, and never a key after i
+        routed = np.isin(cols, (sel[:, None] * p.block_k + np.arange(p.block_k)[None, :]).ravel())
+        allow = np.broadcast_to(routed[None, :], (len(rows), len(cols))).copy()
+        if p.causal:
+            allow |= cols[None, :] > rows[:, None] - p.window
+            allow &= cols[None, :] <= rows[:, None]
+        logits = np.where(allow, (q[b, h, rows] @ k[b, g, cols].T) * scale, -np.inf)
+        o_out[t], l_out[t] = _softmax_read(logits, v[b, g, cols])
+    return o_out, l_out
 
 
 # --------------------------------------------------------------------------

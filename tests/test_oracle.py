@@ -171,6 +171,56 @@ def test_route_brute_force_tiny():
         assert sorted(best) == r.idx[0, 0, qb, :n].tolist()
 
 
+@pytest.mark.parametrize("causal,bq,bk,k,chunk", [
+    (True, 4, 2, 3, 5), (False, 4, 2, 3, 7), (True, 2, 4, 5, 3), (True, 4, 4, 40, 4),
+    (False, 2, 2, 1, 100), (True, 8, 2, 6, 2)])
+def test_route_flat_all_equals_the_per_row_route(causal, bq, bk, k, chunk):
+    # integer entries make exact ties frequent; chunks smaller than the row
+    # count cross chunk boundaries; k = 40 exceeds every row's admissible set
+    rng = np.random.default_rng(11)
+    p = _params(B=2, Hq=4, Hkv=2, N=64, D=3, block_k=bk, block_q=bq, top_k=k,
+                window=0 if not causal else 3, causal=causal)
+    q = rng.integers(-1, 2, size=(2, 4, 64, 3)).astype(np.float64)
+    kk = rng.integers(-1, 2, size=(2, 2, 64, 3)).astype(np.float64)
+    qs, ks = O.block_summary(q, bq), O.block_summary(kk, bk)
+    a = O.route(qs, ks, p)
+    b = O.route_flat_all(qs, ks, p, chunk=chunk)
+    np.testing.assert_array_equal(a.idx, b.idx)
+    np.testing.assert_array_equal(a.cnt, b.cnt)
+    np.testing.assert_array_equal(a.kth, b.kth)
+    np.testing.assert_array_equal(a.next, b.next)
+    _route_property_check(qs, ks, b, p)
+
+
+def test_route_flat_all_brute_force_and_restriction():
+    # independent of the per-row route: for every row, the selection is the
+    # first top_k of a full Python sort of (-score, index); restricted to one
+    # (b, head) the other heads stay empty
+    rng = np.random.default_rng(4)
+    p = _params(B=1, Hq=3, Hkv=1, N=96, D=4, block_k=4, block_q=4, top_k=4, window=2)
+    q = rng.integers(-2, 3, size=(1, 3, 96, 4)).astype(np.float64)
+    kk = rng.integers(-2, 3, size=(1, 1, 96, 4)).astype(np.float64)
+    qs, ks = O.block_summary(q, 4), O.block_summary(kk, 4)
+    r = O.route_flat_all(qs, ks, p, chunk=8)
+    for h in range(3):
+        for qb in range(p.n_qblocks):
+            cand = [(-float(ks[0, 0, c] @ qs[0, h, qb]), c) for c in range(qb)]
+            want = sorted(c for _, c in sorted(cand)[:4])
+            assert r.idx[0, h, qb, :r.cnt[0, h, qb]].tolist() == want
+    only = O.route_flat_all(qs, ks, p, heads=[(0, 1)])
+    np.testing.assert_array_equal(only.idx[0, 1], r.idx[0, 1])
+    assert (only.cnt[0, 0] == 0).all() and (only.idx[0, 2] == -1).all()
+
+
+def test_route_flat_all_rejects_non_finite_summaries():
+    p = _params(N=16, D=2, block_k=2, block_q=2, top_k=2, window=2)
+    qs = np.zeros((1, 1, 8, 2))
+    ks = np.zeros((1, 1, 8, 2))
+    ks[0, 0, 3, 1] = np.nan
+    with pytest.raises(ValueError):
+        O.route_flat_all(qs, ks, p)
+
+
 # ---------------------------------------------------------------- attend: special cases
 def _rand(shape, seed):
     return np.random.default_rng(seed).standard_normal(shape)
@@ -332,6 +382,22 @@ def test_masked_dense_and_gathered_forms_agree():
     b = O.forward(q, k, v, p, form="gathered")
     np.testing.assert_allclose(a["o"], b["o"], atol=1e-12, rtol=0)
     np.testing.assert_allclose(a["lse"], b["lse"], atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("causal,bq,bk,W", [(True, 32, 16, 23), (True, 16, 32, 40),
+                                            (False, 16, 16, 0), (True, 16, 16, 1)])
+def test_block_gathered_form_agrees_with_masked_dense(causal, bq, bk, W):
+    N, D = 192, 16
+    p = _params(B=2, Hq=4, Hkv=2, N=N, D=D, block_k=bk, block_q=bq, top_k=3, window=W,
+                causal=causal)
+    q, k, v = _rand((2, 4, N, D), 51), _rand((2, 2, N, D), 52), _rand((2, 2, N, D), 53)
+    r = O.forward(q, k, v, p, form="dense")
+    blocks = [(b, h, qb) for b in range(2) for h in range(4) for qb in range(N // bq)]
+    o, l = O.attend_gathered_blocks(q, k, v, r["idx"], r["cnt"], p, blocks)
+    o_ref = np.stack([r["o"][b, h, qb * bq:(qb + 1) * bq] for b, h, qb in blocks])
+    l_ref = np.stack([r["lse"][b, h, qb * bq:(qb + 1) * bq] for b, h, qb in blocks])
+    np.testing.assert_allclose(o, o_ref, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(l, l_ref, atol=1e-12, rtol=0)
 
 
 def test_lse_against_dense_logsumexp():
