@@ -5,17 +5,25 @@
 
 A step is one pass of the whole path (K/Q block summaries, routing, fused
 attend) over one batch of the synthetic workload, inputs resident in HBM.
-Default workload: the GQA clustered-key prefill (1 x 14/2 heads, N = 32768,
-D = 64, Bk = Bq = 64, top-k 16, W = 512).  Prints one JSON line on rank 0.
+Default workload: the long GQA clustered-key prefill (1 x 14/2 heads,
+N = 1,048,576, D = 64, Bk = Bq = 64, top-k 16, W = 1024), the largest
+workload that fits one GPU; --config 2 is the 32K-token prefill.  Prints one
+JSON line on rank 0.
 
 * value     whole-job prefill tokens/s (device time, CUDA events per step,
             L2 flushed between steps by a 256 MiB write outside the events)
-* e2e       the same metric through the public call from pinned host buffers
-            (H2D of Q, K, V and D2H of O inside the timed region)
+* e2e       the same metric through the public host-memory call
+            (ssa.forward_host: pinned Q, K, V streamed to the device per KV
+            group and query head on two copy streams, one ssa_forward per
+            query head, O streamed back; all copies inside the timed region)
 * roofline  the attend kernel: algorithmic gathered bytes (distinct routed +
             window key blocks of every query block, K and V, plus the Q read
             and O / LSE writes) per launch / its event-timed duration, against
             the measured HBM copy bandwidth
+* ceilings  secondary ceilings of the attend kernel: the measured
+            ex2.approx rate (exponentials of the softmax), the compulsory bytes
+            (Q, K, V read once, O and LSE written once), the bf16 tensor peak
+* warm_l2   the same step without the L2 flush between steps
 * cpu_baseline  the float64 oracle on the host cores over a bounded sample
 
 With --gpus N > 1 (torchrun) every rank runs an independent replica of the
@@ -51,9 +59,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=5, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ssa", choices=["ssa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -265,6 +273,9 @@ def _cpu_worker(args):
     q = O.upcast_bf16(x["q"][b:b + 1])           # the requested heads, in order
     k = O.upcast_bf16(x["k"][b:b + 1])
     v = O.upcast_bf16(x["v"][b:b + 1])
+    # masked-dense read up to 32K tokens; beyond, the block-gathered form of
+    # the same read (its [Bq, N] slab would be 512 MB per block at 1M tokens)
+    attend = O.attend_masked_dense if w.N <= 32768 else O.attend_gathered_blocks
     t0 = time.perf_counter()
     ksum = O.block_summary(k, p.block_k)
     kcov = O.block_covariance(k[0, 0], p.block_k) if p.beta else None
@@ -294,7 +305,7 @@ def _cpu_worker(args):
             idx[0, :, qb] = -1
             idx[0, :, qb, :len(shared)] = shared
             cnt[0, :, qb] = len(shared)
-        O.attend_masked_dense(q, k, v, idx, cnt, p, blocks=[(0, j, qb) for j in range(nh)])
+        attend(q, k, v, idx, cnt, p, blocks=[(0, j, qb) for j in range(nh)])
         done += nh
         if time.perf_counter() - t0 > seconds:
             break
@@ -557,6 +568,36 @@ def run_ssa(args):
     seg = lambda i: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(n_split))  # noqa: E731
     pool_k_ms, pool_q_ms, tree_pool_ms = seg(0), seg(1), seg(2)
     route_ms, cons_ms, attend_ms = seg(3), seg(4), seg(5)
+
+    # the same step without the L2 flush (inputs and lists may stay in L2)
+    n_warm = min(args.steps, 100)
+    wev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_warm)]
+    for _ in range(3):
+        step()
+    for a, z in wev:
+        a.record()
+        step()
+        z.record()
+    torch.cuda.synchronize()
+    warm_ms = max_over_ranks(statistics.mean(a.elapsed_time(z) for a, z in wev), world, dev)
+    ssa.check_error()
+
+    # exponential rate of the softmax's ex2.approx on this GPU (a ceiling of
+    # the attend kernel): 8 CTAs of 256 threads per SM, 8 chains per thread
+    sink = torch.zeros(1, dtype=torch.float32, device=dev)
+    n_sm = props.multi_processor_count
+    ex2_ctas, ex2_iters = 8 * n_sm, 4096
+    for _ in range(2):
+        ssa.probe_ex2_rate(ex2_ctas, ex2_iters, sink)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record()
+    for _ in range(5):
+        ssa.probe_ex2_rate(ex2_ctas, ex2_iters, sink)
+    x1.record()
+    torch.cuda.synchronize()
+    ssa.check_error()
+    ex2_rate = 5 * ex2_ctas * 256 * ex2_iters * 8 / (x0.elapsed_time(x1) * 1e-3)
     # two-level routing: share of the flat route's per-head selections that
     # the tree route also selects, on the same summaries (outside the timing)
     tree_recall = None
@@ -586,7 +627,7 @@ def run_ssa(args):
     else:
         roof = {"bound": "tensor", "achieved": attend_tflops, "peak": tensor, "unit": "TFLOP/s",
                 "peak_source": f"{peak_kind} bf16_tflops (burst)"}
-    traffic = None
+    traffic, ncu = None, None
     if os.path.exists(TRAFFIC_FILE):
         with open(TRAFFIC_FILE) as f:
             tr = json.load(f)
@@ -594,6 +635,23 @@ def run_ssa(args):
             key = (f"{args.config}{'c' if w.consensus else ''}{'t' if tree else ''}"
                    + (f"@{args.seq_len}" if args.seq_len else ""))
             traffic = tr.get("bytes_per_launch", {}).get(key)
+            ncu = tr.get("pipes", {}).get(key)
+    # secondary ceilings of the attend kernel: exponentials (one per key a
+    # query reads) at the measured ex2 rate, the compulsory bytes (Q, K, V
+    # read once; O and LSE written once) over HBM, and the bf16 tensor peak
+    exps = w.B * w.Hq * w.N * work["keys_per_query"]
+    compulsory = (w.B * w.Hq * w.N * w.D * 2 * 2 + 2 * w.B * w.Hkv * w.N * w.D * 2
+                  + w.B * w.Hq * w.N * 4)
+    ceilings = {
+        "exp": {"exps_per_launch": exps, "measured_ex2_per_s": ex2_rate,
+                "ms": exps / ex2_rate * 1e3, "frac": exps / ex2_rate * 1e3 / attend_ms},
+        "compulsory_bytes": {"bytes_per_launch": compulsory, "ms": compulsory / (hbm * 1e9) * 1e3,
+                             "frac": compulsory / (hbm * 1e9) * 1e3 / attend_ms},
+        "tensor": {"flops_per_launch": work["flops"], "ms": t_tensor * 1e3,
+                   "frac": t_tensor * 1e3 / attend_ms},
+        "gathered_bytes": {"bytes_per_launch": work["attend_bytes"], "ms": t_hbm * 1e3,
+                           "frac": t_hbm * 1e3 / attend_ms},
+    }
 
     # end to end through the public call, from pinned host memory
     e2e = None
@@ -617,7 +675,11 @@ def run_ssa(args):
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
         e2e = {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": oh.numel() * oh.element_size(), "ms_per_step": e2e_ms}
+               "d2h_bytes_per_step": oh.numel() * oh.element_size(), "ms_per_step": e2e_ms,
+               "call": "ssa.forward_host: per-head streamed call (each KV group's K, V and "
+                       "each query head's Q copied from pinned host memory on a copy stream, "
+                       "one ssa_forward per query head as its inputs land, O copied back on a "
+                       "second copy stream)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -630,7 +692,8 @@ def run_ssa(args):
                "sample": f"{nb} (query head, query block) units of this workload (each 1/Hq of "
                          f"the work of {w.block_q} tokens), whole path (summaries, routing"
                          f"{', consensus' if w.consensus else ''}"
-                         f"{', second-cumulant scores' if w.beta else ''}, masked-dense attend) in "
+                         f"{', second-cumulant scores' if w.beta else ''}, "
+                         f"{'masked-dense' if w.N <= 32768 else 'block-gathered'} attend) in "
                          f"float64, {pool.cores} processes x ~{args.cpu_seconds:.0f} s"}
 
     clocks = sampler.summary()
@@ -656,11 +719,25 @@ def run_ssa(args):
                      "achieved": roof["achieved"], "peak": roof["peak"], "unit": roof["unit"],
                      "frac": roof["achieved"] / roof["peak"], "traffic": traffic,
                      "peak_source": roof["peak_source"],
+                     "frac_basis": ("algorithmic gathered bytes (distinct routed and window key "
+                                    "blocks of every routed list x Bk rows x K and V, plus the "
+                                    "Q read and O/LSE writes) over the attend kernel's event "
+                                    "time, against the measured HBM copy bandwidth; most of "
+                                    "these bytes are served from L2, see dram_frac"
+                                    if roof["bound"] == "hbm" else
+                                    "selected-key bf16 flops over the attend kernel's event "
+                                    "time, against the measured bf16 burst peak"),
+                     "dram_frac": (traffic / (attend_ms * 1e-3) / 1e9 / hbm
+                                   if traffic else None),
+                     "ncu_pipes": ncu,
                      "bytes_per_launch": work["attend_bytes"],
                      "hbm_frac": work["attend_bytes"] / (attend_ms * 1e-3) / 1e9 / hbm,
                      "attend_tflops": attend_tflops,
                      "attend_tensor_frac": attend_tflops / float(peaks["bf16_tflops"]),
                      "path_frac_of_roofline": t_roof / (ms * 1e-3)},
+        "ceilings": ceilings,
+        "warm_l2": {"ms_per_step": warm_ms, "value": tokens / (warm_ms * 1e-3),
+                    "note": "same step, no L2 flush between steps"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         # per forward: pool (K and Q in one launch) + route + attend; with

@@ -23,6 +23,7 @@ enum : uint32_t {
   kSiteProbe = 1,
   kSiteQFull = 10, kSiteKvEmpty, kSiteKvFull, kSiteSFull, kSitePFull, kSitePvDone,
   kSiteDrain, kSiteMma, kSiteListCap = 30, kSiteIdx, kSiteCons, kSiteTree, kSiteBwd,
+  kSitePool,
 };
 
 // the library is a single translation unit, so the word is defined here

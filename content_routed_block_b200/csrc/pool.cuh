@@ -74,6 +74,13 @@ __global__ void __launch_bounds__(256) block_mean_kernel(PoolJob j0, PoolJob j1,
 #pragma unroll
     for (int k = 0; k < 8; ++k) a[k] += __shfl_xor_sync(0xffffffffu, a[k], off);
   if (rs == 0) {
+    // Non-finite inputs are outside the method's domain: a NaN or infinite
+    // summary would give NaN routing scores, which rank nowhere.  Report it
+    // through the error word (the summary is still written).
+    bool finite = true;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) finite = finite && isfinite(a[k]);
+    if (!finite) record_error(kErrCheck, kSitePool);
     float4* dst = reinterpret_cast<float4*>(out + blk * D + g * 8);
     dst[0] = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
     dst[1] = make_float4(a[4] * inv, a[5] * inv, a[6] * inv, a[7] * inv);

@@ -8,15 +8,28 @@
 // key block) pair with fp32 FMAs costs NQB*NB*D*2 flops (240 GFLOP at a
 // million tokens), so this kernel ranks in two passes over tensor-core scores:
 //
-//  scores  each fp32 summary x is split into bf16 parts x = x_hi + x_lo + r
-//          (x_hi = bf16(x), x_lo = bf16(x - x_hi), |r| <= u^2 |x|, u = 2^-9)
-//          and sa_c = q_hi.mu_hi + q_hi.mu_lo + q_lo.mu_hi (three MMAs into
-//          one fp32 TMEM accumulator, M = 128 query blocks, N = 128 key
-//          blocks).  The dropped terms are below 3.1 u^2 sum_d |q_d mu_d| and
-//          the fp32 accumulation of 3*D products adds at most 3D 2^-23 of the
-//          same sum: 3.5e-5 (D = 64) or 5.8e-5 (D = 128) times ||qbar|| ||mu_c||.
-//          E_c = eps ||qbar|| ||mu_c|| with eps = 2^-13 (D = 64) or 2^-12
-//          (D = 128) bounds |sa_c - s_c| with a margin of 3.5x or more.
+//  scores  each fp32 summary x is split into bf16 parts x = x_hi + x_lo + r:
+//          x_hi = bf16(x), x_lo = bf16(x - x_hi) (the difference is exact in
+//          fp32).  bf16 rounds to nearest with an 8-bit significand, so with
+//          u = 2^-8: |x - x_hi| <= u|x|, |x_lo| <= u(1+u)|x|, |r| <= u^2 |x|
+//          (for |x| >= 2^-118; below that the parts' absolute errors are
+//          under 2^-134).  sa_c = q_hi.mu_hi + q_hi.mu_lo + q_lo.mu_hi is three
+//          MMAs into one fp32 TMEM accumulator (M = 128 query blocks, N = 128
+//          key blocks).  Error of sa_c against s_c, the fp32 score the FMA
+//          router computes (sequential fmaf over d), in units of
+//          S = sum_d |q_d mu_d| <= ||qbar|| ||mu_c||:
+//            dropped terms q_lo.mu_lo + q_hi.r + r.mu_hi + O(u^3):
+//              <= u^2 (3 + 6u) S = 4.61e-5 S;
+//            the tensor core's fp32 accumulation of the 3D exact bf16
+//              products, assumed only faithful (each addition within one
+//              fp32 ulp, 2^-23 relative, i.e. truncation allowed):
+//              <= 3D 2^-23 (1 + 4u) S = 2.33e-5 S (D = 64), 4.65e-5 S (128);
+//            the fp32 score itself (sequential fmaf, round to nearest):
+//              <= D 2^-24 S = 0.38e-5 S (D = 64), 0.76e-5 S (128).
+//          Total 7.3e-5 S (D = 64) and 1.00e-4 S (D = 128).  The kernel uses
+//          E_c = eps ||qbar|| ||mu_c|| with eps = 2^-12 (D = 64) or 2^-11
+//          (D = 128), margins of 3.3x and 4.9x over those bounds (1.001 on
+//          each fp32 norm covers the norms' own rounding).
 //  pass 1  L = the k-th largest of the per-32-column maxima of the lower
 //          bounds sa_c - E_c.  Each maximum is the lower bound of a distinct
 //          candidate, so at least k candidates have s_c >= L.
@@ -27,9 +40,9 @@
 //          keys: orderable score bits << 32 | ~block).  The filter starts at L
 //          and rises to the current exact k-th score once k are known.  Every
 //          member of the true top-k passes the filter, so the result equals
-//          the fp32 top-k exactly.  (The filter is widened by
-//          eps/2 ||qbar|| max_c ||mu_c||, covering the fp32 rounding of the
-//          rescored values themselves, ~2^-18 of the same product.)
+//          the fp32 top-k exactly.  (The filter is also lowered by
+//          eps/2 ||qbar|| max_c ||mu_c||, which covers the fp32 rounding of
+//          the bounds sa_c - E_c themselves, at most an ulp of the score.)
 //
 // One CTA owns 128 query blocks of one (b, head): thread r = row r = TMEM
 // lane r runs the per-row tests straight out of TMEM; all 256 threads split
@@ -46,7 +59,7 @@ constexpr int kRtcThreads = 256;
 constexpr int kRtcNT = 128;               // key blocks per MMA (N)
 // error-bound factor of the split tensor-core scores (see above)
 template <int D>
-__host__ __device__ constexpr float rtc_eps() { return D == 64 ? 1.2207031e-4f : 2.4414062e-4f; }
+__host__ __device__ constexpr float rtc_eps() { return D == 64 ? 2.4414062e-4f : 4.8828125e-4f; }
 constexpr int kRtcCap = 32;               // queued candidates per row before a flush
 
 template <int D>
@@ -300,7 +313,7 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
   uint64_t keys[KM];
 #pragma unroll
   for (int j = 0; j < KM; ++j) keys[j] = (j < KM - k) ? ~0ull : 0ull;
-  const float slack = e_row * nmax * 0.5f;  // >= 2^-14 ||qbar|| max ||mu||
+  const float slack = e_row * nmax * 0.5f;  // >= (eps / 2) ||qbar|| max ||mu||
   float filt = L - slack;
   int nq = 0;
   auto rescore = [&](int c) -> float {

@@ -44,6 +44,25 @@ __global__ void probe_wait_kernel(uint64_t timeout_ns) {
   }
   __syncthreads();
 }
+// Issue-rate probe of the exponential the softmax uses (ex2.approx): every
+// thread runs 8 independent chains y <- 2^(-y), which stay in [0.5, 1], so
+// the special-function pipe is the only busy unit.  The sum is written only
+// when it is negative, which it never is, so nothing reaches memory but the
+// work cannot be dropped.
+__global__ void __launch_bounds__(256) ex2_rate_kernel(int32_t iters, float* sink) {
+  float y[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = 0.5f + 0.0625f * i + 1e-4f * (threadIdx.x & 15);
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = ex2_approx(-y[i]);
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s += y[i];
+  if (s < 0.f) *sink = s;
+}
+
 // Scratch of ssa_forward_static: summaries, routed lists and counts live
 // here instead of in a caller-provided workspace.  It is part of the loaded
 // module, so every device that loads this library holds these bytes until the
@@ -913,23 +932,63 @@ ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const 
   return ok();
 }
 
-// Device address of the static scratch on the current device, looked up
-// once per device (the first call on a device does the lookup).
+// Device address of the static scratch on the current device.  It is looked
+// up once per device and context: the first call on a device does the
+// lookup, and so does the first call after the device's context was made
+// anew (after cudaDeviceReset the module is loaded again and the array may
+// sit at another address).  Contexts are told apart by the driver's context
+// ID, which is unique for the life of the process.
 std::mutex g_static_mu;
 constexpr int kMaxDevices = 256;
 void* g_static_ptr[kMaxDevices] = {};
+unsigned long long g_static_ctx[kMaxDevices] = {};
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+// ID of the context current on this thread (0 if there is none yet)
+ssa_status current_context_id(unsigned long long* id) {
+  std::call_once(g_ctx_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+  });
+  if (g_ctx_current == nullptr || g_ctx_id == nullptr)
+    return fail(SSA_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId are unavailable (no CUDA driver?)");
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS) return fail(SSA_ERR_CUDA, "cuCtxGetCurrent failed");
+  *id = 0;
+  if (ctx != nullptr && g_ctx_id(ctx, id) != CUDA_SUCCESS)
+    return fail(SSA_ERR_CUDA, "cuCtxGetId failed");
+  return SSA_OK;
+}
 
 ssa_status static_scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(SSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  unsigned long long ctx = 0;
+  ssa_status s = current_context_id(&ctx);
+  if (s != SSA_OK) return s;
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_ptr[dev] == nullptr) {
+  if (g_static_ptr[dev] == nullptr || ctx == 0 || ctx != g_static_ctx[dev]) {
     void* ptr = nullptr;
+    // with this device current; makes its primary context current when no
+    // context is yet
     e = cudaGetSymbolAddress(&ptr, ssa::g_static_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    if ((s = current_context_id(&ctx)) != SSA_OK) return s;
     g_static_ptr[dev] = ptr;
+    g_static_ctx[dev] = ctx;
   }
   *out = g_static_ptr[dev];
   return SSA_OK;
@@ -1112,6 +1171,16 @@ ssa_status ssa_probe_wait_timeout(int32_t timeout_us, ssa_stream_t stream) {
       static_cast<uint64_t>(timeout_us) * 1000ull);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "probe_wait_kernel launch");
+  return ok();
+}
+
+ssa_status ssa_probe_ex2_rate(int32_t n_ctas, int32_t iters, float* sink,
+                              ssa_stream_t stream) {
+  if (n_ctas < 1 || n_ctas > (1 << 20) || iters < 1 || iters > (1 << 24) || sink == nullptr)
+    return fail(SSA_ERR_INVALID_ARG, "n_ctas in 1..2^20, iters in 1..2^24, sink non-NULL");
+  ssa::ex2_rate_kernel<<<n_ctas, 256, 0, static_cast<cudaStream_t>(stream)>>>(iters, sink);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "ex2_rate_kernel launch");
   return ok();
 }
 

@@ -18,7 +18,7 @@ __all__ = [
     "route", "route_consensus", "route_features", "route_cumulant", "tree_summary", "route_tree",
     "attend", "forward",
     "forward_host", "backward", "decode", "decode_workspace_size", "check_error",
-    "probe_wait_timeout",
+    "probe_wait_timeout", "probe_ex2_rate",
     "declared_functions", "LIB_PATH", "HEADER_PATH",
 ]
 
@@ -110,6 +110,7 @@ def lib() -> ctypes.CDLL:
         "ssa_decode": (i32, [P, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_check_error": (i32, [vp]),
         "ssa_probe_wait_timeout": (i32, [i32, vp]),
+        "ssa_probe_ex2_rate": (i32, [i32, i32, vp, vp]),
         "ssa_status_string": (ctypes.c_char_p, [i32]),
         "ssa_last_error_message": (ctypes.c_char_p, []),
         "ssa_version": (i32, []),
@@ -423,3 +424,10 @@ def check_error(stream=None):
 
 def probe_wait_timeout(timeout_us: int):
     _check(lib().ssa_probe_wait_timeout(int(timeout_us), _stream()))
+
+
+def probe_ex2_rate(n_ctas: int, iters: int, sink: torch.Tensor):
+    """Launch the exponential-rate probe (``ssa_probe_ex2_rate``) on the
+    current stream; the caller times it.  ``sink``: a device float32 tensor."""
+    _need(sink, torch.float32, (1,), "sink")
+    _check(lib().ssa_probe_ex2_rate(int(n_ctas), int(iters), _ptr(sink), _stream()))

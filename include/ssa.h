@@ -97,7 +97,14 @@ size_t ssa_workspace_size(const ssa_params* p);
  *        c*block .. c*block + block - 1, summed in fp32 then scaled by
  *        1/block (exact: block is a power of two).
  * H is the head count of x (Hq for queries, Hkv for keys); block is Bk or Bq.
- * B, N and D are taken from p.  One kernel launch. */
+ * B, N and D are taken from p.  One kernel launch.
+ * Non-finite inputs are outside the method's domain.  A summary with a NaN or
+ * infinite entry is still written and is reported through ssa_check_error
+ * (SSA_ERR_DEVICE_CHECK); ssa_forward reports it the same way.  Routing never
+ * selects a block whose score is NaN (so a count may fall below
+ * min(top_k, admissible blocks)), and the outputs of rows that read a
+ * non-finite key or value are unspecified; no kernel waits on data, so
+ * nothing hangs. */
 ssa_status ssa_block_summary(const ssa_params* p, const void* x, int32_t H,
                              int32_t block, float* out, ssa_stream_t stream);
 
@@ -250,7 +257,11 @@ ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const 
  * nothing is launched.  The call allocates nothing: no cudaMalloc, cudaFree or
  * allocating library routine.  The first call on each device looks up the
  * scratch's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture.  All calls share the one
+ * make that first call before any stream capture.  The address is kept per
+ * device and context: the first call after the device's context was made anew
+ * (cudaDeviceReset, or the primary context released and retaken) looks it up
+ * again, since the reloaded module may place the array elsewhere.  All calls
+ * share the one
  * scratch, which keeps the previous call's contents (every byte the path reads
  * is rewritten first, so nothing needs clearing); calls that can overlap on the
  * GPU -- on different streams, or from different host threads -- race on it
@@ -329,6 +340,15 @@ ssa_status ssa_check_error(ssa_stream_t stream);
  * timeout_us microseconds and records SSA_ERR_TIMEOUT in the error word.
  * Lets a caller check the timeout path without a hang. */
 ssa_status ssa_probe_wait_timeout(int32_t timeout_us, ssa_stream_t stream);
+
+/* Measurement: one launch of n_ctas blocks of 256 threads, each thread
+ * evaluating iters x 8 exponentials with the instruction the attend kernel's
+ * softmax uses (ex2.approx.ftz.f32, in 8 independent chains y <- 2^-y).
+ * Timing the launch gives the device's exponential rate, a ceiling of the
+ * softmax: n_ctas * 256 * iters * 8 / seconds.  sink is a device float that
+ * is never written in practice (the results only feed a branch that cannot
+ * be taken); it must still be valid device memory. */
+ssa_status ssa_probe_ex2_rate(int32_t n_ctas, int32_t iters, float* sink, ssa_stream_t stream);
 
 const char* ssa_status_string(ssa_status s);
 const char* ssa_last_error_message(void);

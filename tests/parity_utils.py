@@ -97,6 +97,49 @@ def check_route_rows(case: Case, idx_g: np.ndarray, cnt_g: np.ndarray, rows):
     return idx, cnt, alt
 
 
+def check_route_every_row(case: Case, idx_g: np.ndarray, cnt_g: np.ndarray):
+    """Compare the GPU's lists with the oracle's on every row (flat
+    mean-score route, ``O.route_flat_all``).  A row may differ only at a
+    counted near-tie, and there the GPU's selection must be one the oracle
+    enumerates (``O.acceptable_selections``).  Returns the oracle's idx/cnt
+    with the GPU's accepted alternatives in place, the number of such rows,
+    and the oracle's near-tie mask [B, Hq, NQB]."""
+    op = case.op
+    r = O.route_flat_all(case.qsum64, case.ksum64, op)
+    near = O.near_tie_rows(r)
+    assert (cnt_g == r.cnt).all(), "GPU counts differ from the oracle's"
+    diff = (idx_g != r.idx).any(axis=-1) if op.top_k else np.zeros_like(near)
+    idx = r.idx.copy()
+    alt = 0
+    for b, h, qb in zip(*np.nonzero(diff)):
+        n = int(cnt_g[b, h, qb])
+        g = idx_g[b, h, qb, :n]
+        assert near[b, h, qb], (f"row {(b, h, qb)}: GPU selection {g.tolist()} != "
+                                f"{r.idx[b, h, qb, :n].tolist()} outside a near-tie")
+        accepted = O.acceptable_selections(case.qsum64[b, h, qb], case.ksum64[b, h // op.group],
+                                           O.admissible_blocks(qb, op), op.top_k)
+        assert any(np.array_equal(a, g) for a in accepted), \
+            f"row {(b, h, qb)}: GPU selection {g.tolist()} is not an acceptable alternative"
+        idx[b, h, qb, :n] = g
+        alt += 1
+    return idx, r.cnt, alt, near
+
+
+def output_rows(case: Case, near: np.ndarray, seed: int = 0):
+    """Query blocks whose outputs are compared at full size: one random block
+    of every (b, head), the first and last blocks of every (b, head), and
+    every near-tie row."""
+    op = case.op
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for b in range(op.B):
+        for h in range(op.Hq):
+            rows.update({(b, h, 0), (b, h, op.n_qblocks - 1),
+                         (b, h, int(rng.integers(op.n_qblocks)))})
+    rows.update((int(b), int(h), int(q)) for b, h, q in zip(*np.nonzero(near)))
+    return sorted(rows)
+
+
 def oracle_attend_rows(case: Case, idx, cnt, rows):
     """fp64 oracle outputs for the query blocks ``rows`` -> ([n, Bq, D], [n, Bq])."""
     return O.attend_masked_dense(case.q64, case.k64, case.v64, idx, cnt, case.op, blocks=rows)

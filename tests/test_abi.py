@@ -249,3 +249,25 @@ def test_binding_checks_backward_and_tree_tensors_before_calling():
         ssa.tree_summary(ksum, t)
     with pytest.raises(ValueError):
         ssa.route_tree(torch.zeros(1, 2, 16, 64), ksum, torch.zeros(1, 1, 3, 64), t)
+
+
+def test_static_forward_rejects_oversized_shapes_before_any_cuda_call(L):
+    # the scratch size check comes first: no pointer is looked at and no CUDA
+    # call is made, so NULL pointers are never dereferenced or launched on
+    fn = L.ssa_forward_static
+    vp = ctypes.c_void_p
+    fn.restype = ctypes.c_int32
+    fn.argtypes = [ctypes.POINTER(ssa.Params), vp, vp, vp, vp, vp, vp, vp, vp]
+    p = _p(N=1 << 20, window=1024)
+    assert ssa.workspace_size(p) > (32 << 20)
+    assert fn(ctypes.byref(p), None, None, None, None, None, None, None, None) == 3
+    assert "scratch" in L.ssa_last_error_message().decode()
+    bad = _p(D=96)
+    assert fn(ctypes.byref(bad), None, None, None, None, None, None, None, None) == 2
+
+
+def test_ex2_probe_rejects_bad_arguments_before_launch(L):
+    good = ctypes.c_void_p(1 << 20)
+    assert L.ssa_probe_ex2_rate(0, 10, good, None) == 1
+    assert L.ssa_probe_ex2_rate(10, 0, good, None) == 1
+    assert L.ssa_probe_ex2_rate(10, 10, None, None) == 1

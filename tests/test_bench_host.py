@@ -41,6 +41,8 @@ def test_mode_flags_dispatch_to_their_arms(monkeypatch):
 
 def test_default_run_is_the_headline_workload():
     args = bench.parse_args([])
-    assert (args.gpus, args.config, args.steps >= 1, args.warmup >= 3) == (1, 2, True, True)
+    # the largest workload that fits one GPU: the million-token prefill
+    assert (args.gpus, args.config, args.steps >= 1, args.warmup >= 3) == (1, 5, True, True)
     w = bench.workload_of(args)
-    assert (w.name, w.tree_fanout, w.consensus, w.beta) == ("gqa-clustered-32k", 0, False, 0.0)
+    assert (w.name, w.tree_fanout, w.consensus, w.beta) == ("gqa-clustered-1m", 0, False, 0.0)
+    assert w.N == 1 << 20

@@ -5,7 +5,8 @@ selections against the oracle's top-k (bit-exact except at counted near-ties,
 where the GPU's choice must be one the oracle itself enumerates as
 acceptable), K3 fed the oracle's own selections against the oracle's attend.
 Then the whole forward on small shapes (every row) and on the five workloads
-at full size (sampled query blocks, plus properties that hold for every row).
+at full size: every row's list against the oracle's route, outputs on
+sampled query blocks and on every near-tie row.
 """
 import numpy as np
 import pytest
@@ -14,8 +15,8 @@ import torch
 import oracle as O
 from content_routed_block_b200 import build, ssa
 from content_routed_block_b200.workloads import CONFIGS, Workload, make_inputs
-from parity_utils import (Case, assert_close, check_forward, check_route_rows, gpu_rows,
-                          oracle_attend_rows, to_dev)
+from parity_utils import (Case, assert_close, check_forward, check_route_every_row,
+                          check_route_rows, gpu_rows, oracle_attend_rows, output_rows, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -163,19 +164,26 @@ def _route_properties_all_rows(case, idx, cnt):
     assert (np.where(vpair, d > 0, True)).all()
 
 
-@pytest.mark.parametrize("cfg,rows", [(2, 48), (3, 48), (4, 48)])
-def test_forward_full_size_sampled(cfg, rows):
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+def test_forward_full_size_every_row_routed_like_the_oracle(cfg):
+    # every row's list against the oracle's fp64 route (exact outside counted
+    # near-ties); outputs on one random, the first and the last query block of
+    # every (b, head) and on every near-tie row, through the oracle's
+    # block-gathered read
     case = Case(CONFIGS[cfg])
-    rep = check_forward(case, rows=case.sample_rows(rows, seed=cfg))
-    _route_properties_all_rows(case, rep["idx"], rep["cnt"])
-    assert torch.isfinite(rep["o"]).all()
-
-
-def test_forward_million_tokens_sampled():
-    case = Case(CONFIGS[5])
-    rep = check_forward(case, rows=case.sample_rows(16, seed=5))
-    _route_properties_all_rows(case, rep["idx"], rep["cnt"])
-    assert torch.isfinite(rep["o"]).all()
+    o, lse, idx, cnt = ssa.forward(case.qd, case.kd, case.vd, case.p)
+    ssa.check_error()
+    idx_g, cnt_g = idx.cpu().numpy(), cnt.cpu().numpy()
+    _route_properties_all_rows(case, idx_g, cnt_g)
+    r_idx, r_cnt, alt, near = check_route_every_row(case, idx_g, cnt_g)
+    rows = output_rows(case, near, seed=cfg)
+    print(f"{case.w.name}: {near.size} rows, {int(near.sum())} counted near-ties, "
+          f"{alt} GPU near-tie alternatives, outputs on {len(rows)} query blocks")
+    o_ref, l_ref = O.attend_gathered_blocks(case.q64, case.k64, case.v64, r_idx, r_cnt, case.op,
+                                            rows)
+    assert_close(gpu_rows(o, rows, case.op.block_q), o_ref, gpu_rows(lse, rows, case.op.block_q),
+                 l_ref, what=case.w.name)
+    assert torch.isfinite(o).all()
 
 
 def test_forward_is_deterministic():
@@ -275,3 +283,94 @@ def test_tensor_core_router_on_flat_and_tied_scores():
     i2, c2 = _route_with("tc", case)
     assert torch.equal(i1, i2) and torch.equal(c1, c2)
     check_route_rows(case, i2.cpu().numpy(), c2.cpu().numpy(), case.sample_rows(40, seed=1))
+
+
+def test_non_finite_key_block_is_reported_and_the_oracle_refuses_it():
+    # non-finite inputs are outside the method's domain: the oracle refuses
+    # to route them, and the GPU path reports them through the error word
+    # (pool kernel) without hanging; the context stays usable
+    case = Case(CONFIGS[1])
+    x = {n: case.u16[n].copy() for n in "qkv"}
+    x["k"][0, 1, 3 * 64 + 5, 7] = 0x7FC0            # a bf16 NaN in key block 3 of KV head 1
+    bad = Case(CONFIGS[1], x)
+    with pytest.raises(ValueError):
+        O.route(bad.qsum64, bad.ksum64, bad.op)
+    o, _, idx, cnt = ssa.forward(bad.qd, bad.kd, bad.vd, bad.p)
+    with pytest.raises(ssa.SsaError) as e:
+        ssa.check_error()
+    assert e.value.status == 6
+    # KV head 1's routing never picks the NaN block; head 0 is unaffected
+    idx = idx.cpu().numpy()
+    assert not (idx[0, 1] == 3).any()
+    rows = [(0, 0, qb) for qb in range(case.op.n_qblocks)]
+    r_idx, r_cnt, _ = check_route_rows(case, idx, cnt.cpu().numpy(), rows)
+    o_ref, l_ref = oracle_attend_rows(case, r_idx, r_cnt, rows)
+    assert_close(gpu_rows(o, rows, 64), o_ref, what="the finite head")
+    check_forward(Case(CONFIGS[1]))
+
+
+def _band_inputs(N, seed):
+    """Keys 10 + integer offsets whose sum over each 64-row block is a planted
+    j_c in [-6, 6]; every query row is 0 or 2 (heads 0) / 0 or 4 (head 1) with
+    a block mean of exactly 1 (2).  Block means are multiples of 1/64 that
+    bf16 does not hold (so both split parts are non-zero), and every score is
+    exactly (640 + j_c / 64) * {1, 2} in fp32 as in fp64: the order is known
+    exactly, every candidate lies within the tensor-core bound E_c of the
+    k-th score, and equal j_c are exact ties."""
+    from content_routed_block_b200.workloads import to_bf16_bits
+    rng = np.random.default_rng(seed)
+    D, nb = 64, N // 64
+    k = np.full((1, 1, N, D), 10.0, np.float32)
+    for c in range(nb):
+        j = int(rng.integers(-6, 7))
+        off = np.zeros(64 * D, np.float32)
+        pos = rng.choice(64 * D, size=80 + abs(j), replace=False)
+        off[pos[:40]] += 1.0
+        off[pos[40:80]] -= 1.0
+        off[pos[80:]] += np.sign(j)
+        k[0, 0, c * 64:(c + 1) * 64] += off.reshape(64, D)
+    q = np.zeros((1, 2, N, D), np.float32)
+    q[0, 0, 0::2] = 2.0
+    q[0, 1, 1::2] = 4.0
+    v = rng.standard_normal((1, 1, N, D)).astype(np.float32)
+    return {"q": to_bf16_bits(q), "k": to_bf16_bits(k), "v": to_bf16_bits(v)}
+
+
+def test_tensor_core_router_with_every_candidate_inside_its_bound():
+    # the filter / queue / rescoring path with whole rows inside the bound and
+    # many exact ties: both routers must give the exact lexicographic order
+    # (no near-tie allowance: the fp32 scores here are exact)
+    w = W("band-tc", N=16384, Hq=2, Hkv=1, top_k=16, window=64)
+    case = Case(w, _band_inputs(16384, seed=13))
+    i1, c1 = _route_with("fp32", case)
+    i2, c2 = _route_with("tc", case)
+    assert torch.equal(c1, c2) and torch.equal(i1, i2)
+    r = O.route_flat_all(case.qsum64, case.ksum64, case.op)
+    np.testing.assert_array_equal(c2.cpu().numpy(), r.cnt)
+    np.testing.assert_array_equal(i2.cpu().numpy(), r.idx)
+    # the planted scores are what the construction says
+    mu = case.ksum64[0, 0]
+    s = mu @ case.qsum64[0, 0, 5]
+    assert np.all(np.abs(s * 64 - np.round(s * 64)) == 0) and np.ptp(s) <= 12 / 64
+
+
+def test_tensor_core_router_on_near_duplicate_blocks():
+    # blocks that copy another block's keys with one bf16 step changed in one
+    # element: fp32 scores within the tensor-core bound of each other and not
+    # exact; the two routers must agree bit for bit, and with the oracle
+    # outside counted near-ties
+    w = W("dup-tc", N=16384, Hq=2, Hkv=1, top_k=16, window=64, kind="clustered", centres=8)
+    x = make_inputs(w)
+    kk = x["k"].reshape(1, 1, 256, 64, 64)
+    rng = np.random.default_rng(17)
+    for c in rng.choice(np.arange(1, 256), size=120, replace=False):
+        src = int(rng.integers(0, 256))
+        kk[0, 0, c] = kk[0, 0, src]
+        t, d = int(rng.integers(64)), int(rng.integers(64))
+        kk[0, 0, c, t, d] = kk[0, 0, c, t, d] + np.uint16(1)   # one bf16 step
+    case = Case(w, x)
+    i1, c1 = _route_with("fp32", case)
+    i2, c2 = _route_with("tc", case)
+    assert torch.equal(c1, c2) and torch.equal(i1, i2)
+    _, _, alt, near = check_route_every_row(case, i2.cpu().numpy(), c2.cpu().numpy())
+    print(f"near-duplicate blocks: {int(near.sum())} counted near-ties, {alt} alternatives")
