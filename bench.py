@@ -987,7 +987,16 @@ def run_backward(args):
     pairs = work["keys_per_query"] * w.B * w.Hq * w.N
     flops = 10.0 * w.D * pairs            # S, dP, dq, dk, dv: 2 D flops each per (query, key) pair
     achieved = flops / (ms * 1e-3) / 1e12
-    fma_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    simt = os.environ.get("SSA_BWD") == "simt"
+    peaks, peak_kind = load_peaks()
+    if simt:
+        roof = {"bound": "alu", "kernel": "bwd_kernel (CUDA-core fp32 FMA)",
+                "peak": 148 * 128 * 2 * 1.965e9 / 1e12,
+                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz"}
+    else:
+        roof = {"bound": "tensor", "kernel": "bwd_dq_kernel + bwd_dkdv_kernel (tcgen05)",
+                "peak": float(peaks["bf16_tflops"]),
+                "peak_source": f"{peak_kind} bf16_tflops (burst)"}
 
     e2e = None
     if not args.no_e2e:
@@ -1047,14 +1056,20 @@ def run_backward(args):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ssa", "config": cfg,
         "keys_per_query": work["keys_per_query"],
-        "roofline": {"bound": "alu", "kernel": "bwd_kernel (CUDA-core fp32 FMA)",
-                     "achieved": achieved, "peak": fma_peak, "unit": "TFLOP/s",
-                     "frac": achieved / fma_peak, "traffic": None,
-                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz",
+        "roofline": {"bound": roof["bound"], "kernel": roof["kernel"],
+                     "achieved": achieved, "peak": roof["peak"], "unit": "TFLOP/s",
+                     "frac": achieved / roof["peak"], "traffic": None,
+                     "peak_source": roof["peak_source"],
+                     "frac_basis": "algorithmic flops (10 D per (query, key) pair: S, dP, dq, dk, "
+                                   "dv) over the whole backward step",
                      "flops_per_launch": flops},
         "cpu_baseline": cpu, "e2e": e2e,
-        # per step: two memsets (dk, dv), the delta kernel and the gradient kernel
-        "gpu_launches": 2 * args.steps, "clocks": clocks,
+        # per step: CUDA-core form -- two memsets (dk, dv), the delta kernel
+        # and the gradient kernel; tensor-core form -- delta, the list
+        # transpose, dq, dk / dv and (GQA) the group sum kernels (the
+        # transpose's memset is not a kernel of ours)
+        "gpu_launches": (2 if simt else (4 if w.top_k else 3) + (1 if w.Hq > w.Hkv else 0))
+                        * args.steps, "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
 

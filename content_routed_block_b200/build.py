@@ -18,7 +18,7 @@ SRC = os.path.join(HERE, "csrc", "ssa.cu")
 OUT = os.path.join(HERE, "libssa.so")
 DEPS = [os.path.join(HERE, "csrc", f) for f in
         ("ssa.cu", "common.cuh", "pool.cuh", "route.cuh", "route_tc.cuh", "consensus.cuh",
-         "cumulant.cuh", "decode.cuh", "tree.cuh", "backward.cuh",
+         "cumulant.cuh", "decode.cuh", "tree.cuh", "backward.cuh", "backward_tc.cuh",
          "attend.cuh")] + \
        [os.path.join(ROOT, "include", "ssa.h")]
 

@@ -110,125 +110,23 @@ __device__ __forceinline__ uint64_t bit_range(int lo, int hi) {
   return m << lo;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kAtThreads, 2)
-    attend_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                  const __grid_constant__ CUtensorMap tv, const AttendArgs a) {
-  using L = AtLayout<D>;
-  constexpr int S = L::STAGES;
-  extern __shared__ uint8_t at_smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(at_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const uint32_t sbase = smem_u32(smem);
-  uint32_t* win = reinterpret_cast<uint32_t*>(smem + L::OFF_WIN);
-  int32_t* far = reinterpret_cast<int32_t*>(smem + L::OFF_FAR);
-  int32_t* faru = reinterpret_cast<int32_t*>(smem + L::OFF_FARU);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* bar_q = bars;
-  uint64_t* bar_kv_full = bars + 1;
-  uint64_t* bar_kv_empty = bars + 1 + S;
-  constexpr int NS = L::NS;
-  uint64_t* bar_s_full = bars + 1 + 2 * S;
-  uint64_t* bar_p_full = bar_s_full + NS;
-  uint64_t* bar_pv_done = bar_p_full + NS;
-  uint64_t* bar_drain = bar_pv_done + NS;
-  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
-  // misc[0] TMEM base, misc[1] raw far count, misc[2] unique far count,
-  // misc[3] abort flag
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[3]);
-
+// Union of a query tile's routed blocks and its window blocks, in shared
+// memory: every key block the tile's R query blocks read, once, each routed
+// entry carrying a bitmask of which query blocks routed it (bit r: query
+// block qb0 + r), ordered so that chunks needed by different softmax warps
+// alternate (see the comments inside).  On return (after a block-wide
+// barrier) misc[2] holds the number of routed entries outside the window
+// range, stored in faru[]; the window range's blocks wlo .. wlo + nwin - 1
+// carry their routed bits in win[].  Called by every thread of a 192-thread
+// CTA; used by the forward read and by the query-major kernel of its
+// backward, so both walk exactly the same key sets.
+__device__ __forceinline__ void at_build_union(const AttendArgs& a, int R, int RH, int q0, int qb0,
+                                               int64_t ibh, int wlo, int nwin, int pre_n,
+                                               int pre_c, uint32_t* win, int32_t* far,
+                                               int32_t* faru, uint32_t* misc) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // The tile is RH consecutive query positions of `pack` query heads: rows
-  // 0..RH-1 belong to head h0, rows RH..2RH-1 (pack == 2) to head h1 of the
-  // same KV group, which shares h0's routed lists.  With an odd group the
-  // last pair has no h1: its rows are loaded from h0 and never written.
-  const int RH = kAtQT / a.pack;
-  const int tile_bh = blockIdx.x / a.n_qtiles;
-  const int qt = blockIdx.x % a.n_qtiles;
-  const int grp = a.Hq / a.Hkv;
-  int b, h0, h1;
-  bool has_h1 = false;
-  if (a.pack == 1) {
-    b = tile_bh / a.Hq;
-    h0 = tile_bh % a.Hq;
-    h1 = h0;
-  } else {
-    const int npair = (grp + 1) / 2;
-    const int bk = tile_bh / npair, pr = tile_bh % npair;
-    b = bk / a.Hkv;
-    h0 = (bk % a.Hkv) * grp + 2 * pr;
-    has_h1 = 2 * pr + 1 < grp;
-    h1 = has_h1 ? h0 + 1 : h0;
-  }
-  const int bh = b * a.Hq + h0;
-  const int bkv = b * a.Hkv + h0 / grp;
-  const int ibh = (a.idx_heads == a.Hq) ? bh : bkv;  // row block of the routed lists
-  const int q0 = qt * RH;
-  const int qend = min(a.N, q0 + RH);
-  const int qb0 = q0 / a.Bq;
-  const int R = min(max(RH / a.Bq, 1), a.NQB - qb0);
-  int wlo = 0, nwin = 0;
-  if (a.causal) {
-    wlo = max(0, q0 - a.window + 1) / a.Bk;
-    nwin = (qend - 1) / a.Bk - wlo + 1;
-  }
-
-  // this thread's first routed entry, loaded before the set-up so that the
-  // load latency overlaps the barrier and TMEM set-up (reading the entry
-  // past the row's count stays inside the row: rows are top_k long)
   const int total = R * a.top_k;
-  int pre_n = 0, pre_c = -1;
-  if (tid < total) {
-    const int64_t row = static_cast<int64_t>(ibh) * a.NQB + qb0 + tid / a.top_k;
-    pre_n = a.cnt[row];
-    pre_c = a.idx[row * a.top_k + tid % a.top_k];
-  }
-
-  // ---------------------------------------------------------------- setup
-  if (tid == 0) {
-    mbar_init(bar_q, 1);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&bar_kv_full[s], 1);
-      mbar_init(&bar_kv_empty[s], 1);
-    }
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&bar_s_full[s], 1);
-      mbar_init(&bar_p_full[s], 4);  // one arrival per softmax warp
-      mbar_init(&bar_pv_done[s], 1);
-    }
-    mbar_init(bar_drain, 1);
-    misc[1] = 0;
-    misc[2] = 0;
-    misc[3] = 0;
-    fence_barrier_init();
-  }
-  if (warp == 5) {
-    tmem_alloc(&misc[0], kAtTmemCols);
-    tmem_relinquish();
-  }
-  for (int w = tid; w < nwin; w += kAtThreads) win[w] = 0u;
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = misc[0];
-
-  // Q does not depend on the routing: start its load now
-  if (warp == 4 && lane == 0) {
-    tma_prefetch_desc(&tq);
-    tma_prefetch_desc(&tk);
-    tma_prefetch_desc(&tv);
-    mbar_arrive_expect_tx(bar_q, L::Q_BYTES);
-#pragma unroll
-    for (int half = 0; half < D / 64; ++half) {
-      // the tensor map's box is RH rows: one box per head
-      tma_load_3d(smem + L::OFF_Q + half * L::HALF_Q, &tq, bar_q, half * 64, q0, bh);
-      if (a.pack == 2)
-        tma_load_3d(smem + L::OFF_Q + half * L::HALF_Q + 64 * 128, &tq, bar_q, half * 64, q0,
-                    b * a.Hq + h1);
-    }
-  }
-
-  // ------------------------------------------ union of routed and window blocks
+  const int G = (a.Bk < kAtKT) ? kAtKT / a.Bk : 1;           // blocks per chunk
   {
     for (int t = tid; t < total; t += kAtThreads) {
       const int r = t / a.top_k, e = t % a.top_k;
@@ -255,7 +153,6 @@ __global__ void __launch_bounds__(kAtThreads, 2)
     }
   }
   __syncthreads();
-  const int G = (a.Bk < kAtKT) ? kAtKT / a.Bk : 1;           // blocks per chunk
   if (warp == 0 && static_cast<int>(misc[1]) <= 32 && G == 1) {
     // Few routed entries outside the window (the common case, e.g. 2 query
     // blocks x 16): the whole union list is built in registers, one entry
@@ -428,9 +325,135 @@ __global__ void __launch_bounds__(kAtThreads, 2)
   }
   __syncthreads();
 
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAtThreads, 2)
+    attend_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                  const __grid_constant__ CUtensorMap tv, const AttendArgs a) {
+  using L = AtLayout<D>;
+  constexpr int S = L::STAGES;
+  extern __shared__ uint8_t at_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(at_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint32_t* win = reinterpret_cast<uint32_t*>(smem + L::OFF_WIN);
+  int32_t* far = reinterpret_cast<int32_t*>(smem + L::OFF_FAR);
+  int32_t* faru = reinterpret_cast<int32_t*>(smem + L::OFF_FARU);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_kv_full = bars + 1;
+  uint64_t* bar_kv_empty = bars + 1 + S;
+  constexpr int NS = L::NS;
+  uint64_t* bar_s_full = bars + 1 + 2 * S;
+  uint64_t* bar_p_full = bar_s_full + NS;
+  uint64_t* bar_pv_done = bar_p_full + NS;
+  uint64_t* bar_drain = bar_pv_done + NS;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  // misc[0] TMEM base, misc[1] raw far count, misc[2] unique far count,
+  // misc[3] abort flag
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[3]);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // The tile is RH consecutive query positions of `pack` query heads: rows
+  // 0..RH-1 belong to head h0, rows RH..2RH-1 (pack == 2) to head h1 of the
+  // same KV group, which shares h0's routed lists.  With an odd group the
+  // last pair has no h1: its rows are loaded from h0 and never written.
+  const int RH = kAtQT / a.pack;
+  const int tile_bh = blockIdx.x / a.n_qtiles;
+  const int qt = blockIdx.x % a.n_qtiles;
+  const int grp = a.Hq / a.Hkv;
+  int b, h0, h1;
+  bool has_h1 = false;
+  if (a.pack == 1) {
+    b = tile_bh / a.Hq;
+    h0 = tile_bh % a.Hq;
+    h1 = h0;
+  } else {
+    const int npair = (grp + 1) / 2;
+    const int bk = tile_bh / npair, pr = tile_bh % npair;
+    b = bk / a.Hkv;
+    h0 = (bk % a.Hkv) * grp + 2 * pr;
+    has_h1 = 2 * pr + 1 < grp;
+    h1 = has_h1 ? h0 + 1 : h0;
+  }
+  const int bh = b * a.Hq + h0;
+  const int bkv = b * a.Hkv + h0 / grp;
+  const int ibh = (a.idx_heads == a.Hq) ? bh : bkv;  // row block of the routed lists
+  const int q0 = qt * RH;
+  const int qend = min(a.N, q0 + RH);
+  const int qb0 = q0 / a.Bq;
+  const int R = min(max(RH / a.Bq, 1), a.NQB - qb0);
+  int wlo = 0, nwin = 0;
+  if (a.causal) {
+    wlo = max(0, q0 - a.window + 1) / a.Bk;
+    nwin = (qend - 1) / a.Bk - wlo + 1;
+  }
+
+  // this thread's first routed entry, loaded before the set-up so that the
+  // load latency overlaps the barrier and TMEM set-up (reading the entry
+  // past the row's count stays inside the row: rows are top_k long)
+  const int total = R * a.top_k;
+  int pre_n = 0, pre_c = -1;
+  if (tid < total) {
+    const int64_t row = static_cast<int64_t>(ibh) * a.NQB + qb0 + tid / a.top_k;
+    pre_n = a.cnt[row];
+    pre_c = a.idx[row * a.top_k + tid % a.top_k];
+  }
+
+  // ---------------------------------------------------------------- setup
+  if (tid == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&bar_kv_full[s], 1);
+      mbar_init(&bar_kv_empty[s], 1);
+    }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar_s_full[s], 1);
+      mbar_init(&bar_p_full[s], 4);  // one arrival per softmax warp
+      mbar_init(&bar_pv_done[s], 1);
+    }
+    mbar_init(bar_drain, 1);
+    misc[1] = 0;
+    misc[2] = 0;
+    misc[3] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&misc[0], kAtTmemCols);
+    tmem_relinquish();
+  }
+  for (int w = tid; w < nwin; w += kAtThreads) win[w] = 0u;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  // Q does not depend on the routing: start its load now
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+    mbar_arrive_expect_tx(bar_q, L::Q_BYTES);
+#pragma unroll
+    for (int half = 0; half < D / 64; ++half) {
+      // the tensor map's box is RH rows: one box per head
+      tma_load_3d(smem + L::OFF_Q + half * L::HALF_Q, &tq, bar_q, half * 64, q0, bh);
+      if (a.pack == 2)
+        tma_load_3d(smem + L::OFF_Q + half * L::HALF_Q + 64 * 128, &tq, bar_q, half * 64, q0,
+                    b * a.Hq + h1);
+    }
+  }
+
+  // ------------------------------------------ union of routed and window blocks
+  at_build_union(a, R, RH, q0, qb0, ibh, wlo, nwin, pre_n, pre_c, win, far, faru, misc);
+  const int G = (a.Bk < kAtKT) ? kAtKT / a.Bk : 1;           // blocks per chunk
   const int nf = static_cast<int>(misc[2]);
   const int n_entries = nf + nwin;
   const int SUBS = (a.Bk > kAtKT) ? a.Bk / kAtKT : 1;        // chunks per block
+  // a power of two: chunk t is sub-chunk t % SUBS of entry t / SUBS, by shifts
+  // (a runtime division would cost a long dependent sequence in every chunk)
+  const int subs_sh = __ffs(SUBS) - 1;
   const int T = (a.Bk >= kAtKT) ? n_entries * SUBS : (n_entries + G - 1) / G;
   int issued = 0;  // chunks the producer has put in flight
 
@@ -446,7 +469,7 @@ __global__ void __launch_bounds__(kAtThreads, 2)
         uint8_t* kdst = smem + L::OFF_K + st * L::KV_BYTES;
         uint8_t* vdst = smem + L::OFF_V + st * L::KV_BYTES;
         if (a.Bk >= kAtKT) {
-          const int e = t / SUBS, sub = t % SUBS;
+          const int e = t >> subs_sh, sub = t & (SUBS - 1);
           const int c = static_cast<int>(at_entry(faru, win, nf, wlo, e) >> 8);
           const int row0 = c * a.Bk + sub * kAtKT;
 #pragma unroll
@@ -564,7 +587,7 @@ __global__ void __launch_bounds__(kAtThreads, 2)
       if (row_ok) {
         uint64_t mask = 0ull;
         if (a.Bk >= kAtKT) {
-          const int e = t / SUBS, sub = t % SUBS;
+          const int e = t >> subs_sh, sub = t & (SUBS - 1);
           const uint32_t ent = at_entry(faru, win, nf, wlo, e);
           const int j0 = static_cast<int>(ent >> 8) * a.Bk + sub * kAtKT;
           const bool routed = (ent >> qbr) & 1u;

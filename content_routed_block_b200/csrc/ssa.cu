@@ -19,6 +19,7 @@
 #include "../../include/ssa.h"
 #include "attend.cuh"
 #include "backward.cuh"
+#include "backward_tc.cuh"
 #include "common.cuh"
 #include "consensus.cuh"
 #include "cumulant.cuh"
@@ -451,8 +452,39 @@ ssa_status launch_route_tree(const ssa_params* p, const float* qsum, const float
 }
 
 // ------------------------------------------------------------------ backward
-size_t bwd_ws_bytes(const ssa_params* p) {
-  return align256(static_cast<size_t>(p->B) * p->Hq * p->N * sizeof(float));
+// The CUDA-core form (SSA_BWD=simt, kept as a comparison) needs delta only;
+// the tensor-core form also keeps the list transpose (one bit per key tile of
+// 128 keys and query chunk of 64 queries, per list head).
+struct BwdWs {
+  size_t delta, map, map_bytes, part_dk, part_dv, total;
+  int32_t n_ktiles, map_words;
+};
+
+BwdWs bwd_ws_layout(const ssa_params* p) {
+  BwdWs w;
+  w.delta = 0;
+  w.map = align256(static_cast<size_t>(p->B) * p->Hq * p->N * sizeof(float));
+  w.n_ktiles = (p->N + ssa::kBkKT - 1) / ssa::kBkKT;
+  const int32_t nqc = (p->N + ssa::kBkQC - 1) / ssa::kBkQC;
+  w.map_words = (nqc + 31) / 32;
+  const int32_t lh = p->consensus ? p->Hkv : p->Hq;
+  w.map_bytes = static_cast<size_t>(p->B) * lh * w.n_ktiles * w.map_words * sizeof(uint32_t);
+  // per-query-head shares of dk and dv when a KV head serves several query
+  // heads (summed in head order afterwards)
+  const size_t part = p->Hq > p->Hkv
+                          ? align256(static_cast<size_t>(p->B) * p->Hq * p->N * p->D * sizeof(float))
+                          : 0;
+  w.part_dk = w.map + align256(w.map_bytes);
+  w.part_dv = w.part_dk + part;
+  w.total = w.part_dv + part;
+  return w;
+}
+
+size_t bwd_ws_bytes(const ssa_params* p) { return bwd_ws_layout(p).total; }
+
+bool use_simt_backward() {
+  const char* env = std::getenv("SSA_BWD");
+  return env != nullptr && std::string(env) == "simt";
 }
 
 template <int D>
@@ -466,6 +498,35 @@ cudaError_t launch_backward_d(const ssa::BwdArgs& a, int B, cudaStream_t stream)
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   ssa::bwd_kernel<D><<<dim3(a.N / a.RT, B * a.Hq), ssa::kBwdThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// the two tensor-core kernels of the backward: maps[0..3] = Q, G (128-row
+// boxes), K, V (the forward's key boxes) for the query-major dq kernel;
+// maps[4..7] = Q, G (64-row boxes), K, V (128-row boxes) for the key-major
+// dk / dv kernel
+template <int D>
+cudaError_t launch_backward_tc_d(const CUtensorMap* maps, const ssa::BwdTcArgs& a, int B,
+                                 int Hkv, int64_t n_qctas, cudaStream_t stream) {
+  const uint32_t smem_dq = ssa::DqLayout<D>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(
+      ssa::bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_dq));
+  if (e != cudaSuccess) return e;
+  ssa::bwd_dq_kernel<D><<<static_cast<unsigned>(n_qctas), ssa::kAtThreads, smem_dq, stream>>>(
+      maps[0], maps[1], maps[2], maps[3], a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const uint32_t smem_kv = ssa::DkvLayout<D>::SMEM_BYTES;
+  e = cudaFuncSetAttribute(ssa::bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem_kv));
+  if (e != cudaSuccess) return e;
+  const int64_t n_kctas = static_cast<int64_t>(B) * a.at.Hq * a.n_ktiles;
+  ssa::bwd_dkdv_kernel<D><<<static_cast<unsigned>(n_kctas), ssa::kAtThreads, smem_kv, stream>>>(
+      maps[4], maps[5], maps[6], maps[7], a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.at.Hq == Hkv) return e;
+  const int64_t n4 = static_cast<int64_t>(B) * Hkv * a.at.N * (D / 4);
+  ssa::bwd_group_sum_kernel<D><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(a, n4);
   return cudaGetLastError();
 }
 
@@ -1038,10 +1099,7 @@ ssa_status ssa_attend_backward(const ssa_params* p, const void* q, const void* k
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(SSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t kv_bytes = static_cast<size_t>(p->B) * p->Hkv * p->N * p->D * sizeof(float);
-  cudaError_t e = cudaMemsetAsync(dk, 0, kv_bytes, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, st);
-  if (e != cudaSuccess) return cuda_fail(e, "clear dk / dv");
+  cudaError_t e;
   ssa::BwdArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k = static_cast<const __nv_bfloat16*>(k);
@@ -1069,7 +1127,89 @@ ssa_status ssa_attend_backward(const ssa_params* p, const void* q, const void* k
   a.RT = std::min(p->block_q, p->D == 64 ? ssa::bwd_rows<64>() : ssa::bwd_rows<128>());
   a.CK = std::min(p->block_k, p->D == 64 ? ssa::bwd_keys<64>() : ssa::bwd_keys<128>());
   a.scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
-  e = p->D == 64 ? launch_backward_d<64>(a, p->B, st) : launch_backward_d<128>(a, p->B, st);
+  if (use_simt_backward()) {
+    // CUDA-core form: dk / dv are accumulated with atomics, so clear them
+    const size_t kv_bytes = static_cast<size_t>(p->B) * p->Hkv * p->N * p->D * sizeof(float);
+    e = cudaMemsetAsync(dk, 0, kv_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "clear dk / dv");
+    e = p->D == 64 ? launch_backward_d<64>(a, p->B, st) : launch_backward_d<128>(a, p->B, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return ok();
+  }
+
+  // tensor-core form: delta, the list transpose, the query-major dq kernel
+  // and the key-major dk / dv kernel
+  const BwdWs w = bwd_ws_layout(p);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* map = reinterpret_cast<uint32_t*>(ws + w.map);
+  e = cudaMemsetAsync(map, 0, w.map_bytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clear the list transpose");
+  const int64_t rows = static_cast<int64_t>(p->B) * p->Hq * p->N;
+  if (p->D == 64)
+    ssa::bwd_delta_kernel<64><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a, rows);
+  else
+    ssa::bwd_delta_kernel<128><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a, rows);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "bwd_delta_kernel launch");
+
+  if ((s = get_encoder()) != SSA_OK) return s;
+  const int64_t hq = static_cast<int64_t>(p->B) * p->Hq, hkv = static_cast<int64_t>(p->B) * p->Hkv;
+  const uint32_t kv_rows = static_cast<uint32_t>(p->block_k < 64 ? p->block_k : 64);
+  CUtensorMap maps[8];
+  if ((s = make_map(&maps[0], q, hq, p->N, p->D, ssa::kAtQT)) != SSA_OK ||
+      (s = make_map(&maps[1], d_o, hq, p->N, p->D, ssa::kAtQT)) != SSA_OK ||
+      (s = make_map(&maps[2], k, hkv, p->N, p->D, kv_rows)) != SSA_OK ||
+      (s = make_map(&maps[3], v, hkv, p->N, p->D, kv_rows)) != SSA_OK ||
+      (s = make_map(&maps[4], q, hq, p->N, p->D, ssa::kBkQC)) != SSA_OK ||
+      (s = make_map(&maps[5], d_o, hq, p->N, p->D, ssa::kBkQC)) != SSA_OK ||
+      (s = make_map(&maps[6], k, hkv, p->N, p->D, ssa::kBkKT)) != SSA_OK ||
+      (s = make_map(&maps[7], v, hkv, p->N, p->D, ssa::kBkKT)) != SSA_OK)
+    return s;
+  ssa::BwdTcArgs t;
+  t.at.idx = idx;
+  t.at.cnt = cnt;
+  t.at.o = nullptr;
+  t.at.lse = nullptr;
+  t.at.Hq = p->Hq;
+  t.at.Hkv = p->Hkv;
+  t.at.N = p->N;
+  t.at.NQB = p->N / p->block_q;
+  t.at.NB = p->N / p->block_k;
+  t.at.Bq = p->block_q;
+  t.at.Bk = p->block_k;
+  t.at.top_k = p->top_k;
+  t.at.window = p->window;
+  t.at.causal = p->causal;
+  t.at.idx_heads = p->consensus ? p->Hkv : p->Hq;
+  t.at.pack = 1;
+  t.at.n_qtiles = (p->N + ssa::kAtQT - 1) / ssa::kAtQT;
+  t.at.scale_log2 = a.scale * 1.4426950408889634f;
+  t.at.timeout_ns = timeout_ns(p);
+  t.lse = lse;
+  t.delta = a.delta;
+  t.dq = dq;
+  t.dk = dk;
+  t.dv = dv;
+  t.map = map;
+  t.map_w = map;
+  t.n_ktiles = w.n_ktiles;
+  t.map_words = w.map_words;
+  t.B = p->B;
+  t.part_dk = p->Hq > p->Hkv ? reinterpret_cast<float*>(ws + w.part_dk) : nullptr;
+  t.part_dv = p->Hq > p->Hkv ? reinterpret_cast<float*>(ws + w.part_dv) : nullptr;
+  t.scale = a.scale;
+  if (p->top_k > 0) {
+    const int64_t slots = static_cast<int64_t>(p->B) * t.at.idx_heads * t.at.NQB * p->top_k;
+    ssa::bwd_map_kernel<<<static_cast<unsigned>((slots + 255) / 256), 256, 0, st>>>(t, slots);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "bwd_map_kernel launch");
+  }
+  const int64_t n_qctas = hq * t.at.n_qtiles;
+  if (n_qctas > 0x7FFFFFFF || hq * w.n_ktiles > 0x7FFFFFFF)
+    return fail(SSA_ERR_UNSUPPORTED, "too many tiles");
+  e = p->D == 64 ? launch_backward_tc_d<64>(maps, t, p->B, p->Hkv, n_qctas, st)
+                 : launch_backward_tc_d<128>(maps, t, p->B, p->Hkv, n_qctas, st);
   if (e != cudaSuccess) return cuda_fail(e, "backward launch");
   return ok();
 }

@@ -272,7 +272,10 @@ ssa_status ssa_forward_static(const ssa_params* p, const void* q, const void* k,
                               ssa_stream_t stream);
 
 /* Bytes of device workspace ssa_attend_backward needs (0 if the parameters
- * are invalid): one fp32 per query row. */
+ * are invalid): one fp32 per query row, the lists' transpose (one bit per
+ * list head, 128-key tile and 64-query chunk: 235 MB for 14 heads at 1M
+ * tokens, 0.23 MB at 32K) and, when Hq > Hkv, each query head's fp32 share
+ * of dk and dv (2 * B * Hq * N * D * 4 bytes: 7.5 GB at 1M tokens). */
 size_t ssa_backward_workspace_size(const ssa_params* p);
 
 /* Backward of the read with the selection held fixed (jonsmirl/ssa README,
@@ -289,13 +292,24 @@ size_t ssa_backward_workspace_size(const ssa_params* p);
  *   idx/cnt     the lists the forward read (per head, or per KV group with
  *               p->consensus), as for ssa_attend
  *   dq          fp32 [B, Hq, N, D] (device, out)
- *   dk, dv      fp32 [B, Hkv, N, D] (device, out; cleared by the call, then
- *               accumulated with atomic adds, so their summation order -- and
- *               the last bits -- can vary from run to run)
- *   workspace   ssa_backward_workspace_size(p) bytes (device, 256-byte aligned)
+ *   dk, dv      fp32 [B, Hkv, N, D] (device, out; every entry is written)
+ *   workspace   ssa_backward_workspace_size(p) bytes (device, 256-byte aligned):
+ *               delta [B, Hq, N] fp32, the lists' transpose (one bit per list
+ *               head, 128-key tile and 64-query chunk) and, when Hq > Hkv,
+ *               every query head's share of dk and dv
+ * The products run on the tensor cores (tcgen05, bf16 operands, fp32
+ * accumulation in TMEM): a query-major kernel for dq over the forward's key
+ * sets and a key-major kernel for dk / dv over the transposed lists.  P and
+ * dS enter the MMAs as two bf16 parts each (hi + lo, about 16 significant
+ * bits).  Every gradient is summed in a fixed order, so results are
+ * reproducible bit for bit.  Launches: one memset (the transpose), delta,
+ * the transpose (when top_k > 0), dq, dk / dv per (key tile, query head),
+ * and (when Hq > Hkv) the sum of the heads' shares in head order.  The
+ * environment variable SSA_BWD=simt selects the earlier CUDA-core form
+ * instead (fp32 FMA, dk / dv cleared and accumulated with atomic adds, so
+ * their last bits can vary).
  * List entries that are out of range, not ascending or not admissible are
- * reported through ssa_check_error (SSA_ERR_DEVICE_CHECK) and skipped.  Two
- * memsets and two launches (delta, then the gradients). */
+ * reported through ssa_check_error (SSA_ERR_DEVICE_CHECK) and skipped. */
 ssa_status ssa_attend_backward(const ssa_params* p, const void* q, const void* k, const void* v,
                                const void* o, const float* lse, const void* d_o,
                                const int32_t* idx, const int32_t* cnt, float* dq, float* dk,

@@ -14,9 +14,14 @@ which moves dS_ij by at most P_ij E_i.  Hence
     |err dk_jd| <= scale sum_i P_ij E_i |q_id|   (the oracle's dv for upstream E_i |q_i|)
 and dv does not depend on delta.  Each bound gets a slack of 1e-4 of the
 largest reference entry for fp32 arithmetic (scores, exponentials and sums
-over up to a few thousand terms).  dk and dv are accumulated with atomic
-adds, so their last bits are not reproducible; nothing here compares two GPU
-runs bit for bit.
+over up to a few thousand terms).
+
+The default (tensor-core) form feeds P and dS to bf16 MMAs as two bf16 parts
+each, hi + lo, which leaves a relative rounding of at most 2^-16 per term --
+below the fp32 arithmetic the slack covers -- so the same bounds apply to it
+and to the CUDA-core form (SSA_BWD=simt).  The tensor-core form sums every
+gradient in a fixed order (no atomics), so two runs agree bit for bit; the
+CUDA-core form adds dk and dv atomically, so only its tolerance is checked.
 """
 import numpy as np
 import pytest
@@ -183,3 +188,54 @@ def test_backward_full_size_sampled():
                       "dk block 300", bound_dk[0, g, lo:hi + 1])
     assert_grad_close(dv[0, g, lo:hi + 1].cpu().numpy().astype(np.float64), wdv[0, g, lo:hi + 1],
                       "dv block 300")
+
+
+def _with_form(form, fn):
+    import os
+    old = os.environ.get("SSA_BWD")
+    if form is None:
+        os.environ.pop("SSA_BWD", None)
+    else:
+        os.environ["SSA_BWD"] = form
+    try:
+        return fn()
+    finally:
+        if old is None:
+            os.environ.pop("SSA_BWD", None)
+        else:
+            os.environ["SSA_BWD"] = old
+
+
+@pytest.mark.parametrize("w", [SHAPES[0], SHAPES[3], SHAPES[8]], ids=lambda w: w.name)
+def test_cuda_core_form_matches_oracle(w):
+    # the CUDA-core form, kept for comparison, under the same bounds
+    case = Case(w)
+    p = case.p
+    o, lse, idx, cnt = ssa.forward(case.qd, case.kd, case.vd, p)
+    _, g_d, g64 = upstream(w, 7)
+    dq, dk, dv = _with_form("simt", lambda: ssa.backward(case.qd, case.kd, case.vd, o, lse, g_d,
+                                                         idx, cnt, p))
+    ssa.check_error()
+    r_idx, r_cnt = oracle_lists(case, idx.cpu().numpy(), cnt.cpu().numpy())
+    want = O.attend_backward(case.q64, case.k64, case.v64, g64, r_idx, r_cnt, case.op)
+    bq, bk = delta_bounds(case, g64, r_idx, r_cnt)
+    for got, ref, bound, name in zip((dq, dk, dv), want, (bq, bk, None), ("dq", "dk", "dv")):
+        assert_grad_close(got.cpu().numpy().astype(np.float64), ref, f"simt {w.name} {name}", bound)
+
+
+@pytest.mark.parametrize("w", [SHAPES[0], SHAPES[2], SHAPES[8], SHAPES[9], CONFIGS[2]],
+                         ids=lambda w: w.name)
+def test_tensor_core_backward_is_bit_reproducible(w):
+    # every gradient is summed by one CTA in a fixed order: two runs (with a
+    # different call in between) agree bit for bit
+    case = Case(w)
+    p = case.p
+    o, lse, idx, cnt = ssa.forward(case.qd, case.kd, case.vd, p)
+    _, g_d, _ = upstream(w, 5)
+    first = ssa.backward(case.qd, case.kd, case.vd, o, lse, g_d, idx, cnt, p)
+    _, g2, _ = upstream(w, 6)
+    ssa.backward(case.qd, case.kd, case.vd, o, lse, g2, idx, cnt, p)
+    second = ssa.backward(case.qd, case.kd, case.vd, o, lse, g_d, idx, cnt, p)
+    ssa.check_error()
+    for name, a, b in zip(("dq", "dk", "dv"), first, second):
+        assert torch.equal(a, b), f"{w.name}: {name} differs between two runs"
