@@ -58,6 +58,10 @@ struct BwdTcArgs {
   AttendArgs at;          // lists, shapes and the forward's tiling (o / lse unused)
   const float* lse;       // [B*Hq, N] the forward's natural-log LSE
   const float* delta;     // [B*Hq, N] <g_i, o_i>
+  float* delta_w;         // the same, written by bwd_prep_kernel
+  float* lse2;            // [B*Hq, N] lse * log2(e), written by bwd_prep_kernel
+  const __nv_bfloat16* o;     // [B*Hq, N, D] the forward's output
+  const __nv_bfloat16* d_o;   // [B*Hq, N, D] upstream gradient
   float* dq;              // [B*Hq, N, D] (out)
   float* dk;              // [B*Hkv, N, D] (out)
   float* dv;              // [B*Hkv, N, D] (out)
@@ -546,26 +550,29 @@ __global__ void __launch_bounds__(256) bwd_map_kernel(const BwdTcArgs ba, int64_
 // ===========================================================================
 template <int D>
 struct DkvLayout {
-  static constexpr int STG = (D == 64) ? 3 : 2;       // visit stages
+  static constexpr int STG = 4;                       // visit stages
+  static constexpr int NSW = 8;                       // softmax warps (2 per TMEM lane quarter)
+  static constexpr int THREADS = (NSW + 2) * 32;      // + producer warp + MMA warp
   static constexpr uint32_t HALF_K = kBkKT * 128;     // one 64-column half of the K tile
   static constexpr uint32_t K_BYTES = kBkKT * D * 2;
   static constexpr uint32_t HALF_Q = kBkQC * 128;     // one 64-column half of a Q chunk
   static constexpr uint32_t Q_BYTES = kBkQC * D * 2;
-  // a stage: Q chunk | G chunk | lse (64 f32) | delta (64 f32) | descriptor
+  // a stage: Q chunk | G chunk | lse * log2(e) (64 f32) | delta (64 f32) | descriptor
   static constexpr uint32_t ST_Q = 0, ST_G = Q_BYTES, ST_LSE = 2 * Q_BYTES;
   static constexpr uint32_t ST_DEL = ST_LSE + kBkQC * 4, ST_DESC = ST_DEL + kBkQC * 4;
   static constexpr uint32_t STAGE_BYTES = (ST_DESC + 16 + 1023) / 1024 * 1024;
   static constexpr uint32_t OFF_K = 0, OFF_V = K_BYTES, OFF_ST = 2 * K_BYTES;
-  // kv | full[STG] | empty[STG] | sd_full | p_full | pd_done | drain
-  static constexpr int NBAR = 1 + 2 * STG + 4;
+  // kv | full[STG] | empty[STG] | sd_full[2] | p_full[2] | pd_done[2] | drain
+  static constexpr int NBAR = 1 + 2 * STG + 6 + 1;
   static constexpr uint32_t OFF_BAR = OFF_ST + STG * STAGE_BYTES;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t USED = OFF_MISC + 64;
-  static constexpr uint32_t MIN_REQ = 80 * 1024;
+  // one CTA per SM: it holds all 512 TMEM columns
+  static constexpr uint32_t MIN_REQ = 120 * 1024;
   static constexpr uint32_t SMEM_BYTES = (USED + 1024 > MIN_REQ) ? USED + 1024 : MIN_REQ;
-  // TMEM: S^T (P^T over it), dP^T (dS^T over it), dk, dv
-  static constexpr uint32_t TM_S = 0, TM_DP = 64, TM_DK = 128, TM_DV = 128 + D;
-  static constexpr uint32_t COLS = (D == 64) ? 256 : 512;
+  // TMEM: two S^T buffers (P^T over them), two dP^T buffers (dS^T over them), dk, dv
+  static constexpr uint32_t TM_S0 = 0, TM_DP0 = 128, TM_DK = 256, TM_DV = 256 + D;
+  static constexpr uint32_t COLS = 512;
   static_assert(TM_DV + D <= COLS, "TMEM budget");
 };
 
@@ -576,13 +583,22 @@ struct DkvDesc {
   int32_t end;      // 1: no more visits
 };
 
+// 4 consecutive floats of shared memory
+__device__ __forceinline__ float4 lds_f4(uint32_t saddr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(saddr));
+  return v;
+}
+
 template <int D>
-__global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
+__global__ void __launch_bounds__(DkvLayout<D>::THREADS, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tg,
                     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                     const BwdTcArgs ba) {
   using L = DkvLayout<D>;
-  constexpr int STG = L::STG;
+  constexpr int STG = L::STG, NSW = L::NSW;
   const AttendArgs& a = ba.at;
   extern __shared__ uint8_t kv_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -592,10 +608,10 @@ __global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
   uint64_t* bar_kv = bars;
   uint64_t* bar_full = bars + 1;
   uint64_t* bar_empty = bars + 1 + STG;
-  uint64_t* bar_sd_full = bars + 1 + 2 * STG;
-  uint64_t* bar_p_full = bar_sd_full + 1;
-  uint64_t* bar_pd_done = bar_p_full + 1;
-  uint64_t* bar_drain = bar_pd_done + 1;
+  uint64_t* bar_sd_full = bars + 1 + 2 * STG;   // [2]
+  uint64_t* bar_p_full = bar_sd_full + 2;        // [2]
+  uint64_t* bar_pd_done = bar_p_full + 2;        // [2]
+  uint64_t* bar_drain = bar_pd_done + 2;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[3]);
   auto stage = [&](int st) { return smem + L::OFF_ST + st * L::STAGE_BYTES; };
@@ -620,14 +636,16 @@ __global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
       mbar_init(&bar_full[s], 1);
       mbar_init(&bar_empty[s], 1);
     }
-    mbar_init(bar_sd_full, 1);
-    mbar_init(bar_p_full, 4);
-    mbar_init(bar_pd_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_sd_full[s], 1);
+      mbar_init(&bar_p_full[s], NSW);   // one arrival per softmax warp
+      mbar_init(&bar_pd_done[s], 1);
+    }
     mbar_init(bar_drain, 1);
     misc[3] = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == NSW + 1) {
     tmem_alloc(&misc[0], L::COLS);
     tmem_relinquish();
   }
@@ -637,7 +655,7 @@ __global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
   const uint32_t tmem = misc[0];
   int produced = 0;   // visits put in flight (producer lane 0)
 
-  if (warp == 4) {
+  if (warp == NSW) {
     // ------------------------------------------------------- visit producer
     if (lane == 0) {
       tma_prefetch_desc(&tq);
@@ -711,7 +729,7 @@ __global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
               tma_load_3d(sp + L::ST_Q + half * L::HALF_Q, &tq, &bar_full[st], half * 64, i0, bh);
               tma_load_3d(sp + L::ST_G + half * L::HALF_Q, &tg, &bar_full[st], half * 64, i0, bh);
             }
-            bulk_load(sp + L::ST_LSE, ba.lse + static_cast<int64_t>(bh) * a.N + i0, vb,
+            bulk_load(sp + L::ST_LSE, ba.lse2 + static_cast<int64_t>(bh) * a.N + i0, vb,
                       &bar_full[st]);
             bulk_load(sp + L::ST_DEL, ba.delta + static_cast<int64_t>(bh) * a.N + i0, vb,
                       &bar_full[st]);
@@ -758,66 +776,100 @@ __global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
         mbar_arrive(&bar_full[st]);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == NSW + 1) {
     // ------------------------------------------------------- MMA issuer
+    // Event-driven, two visits in flight: the products of visit v (S^T, dP^T
+    // into buffer v % 2) go out once its chunk has landed and visit v - 2's
+    // dv / dk products (which read that buffer) are done; visit u's dv / dk
+    // products go out once its P^T / dS^T are written.  The loop gives up
+    // after timeout_ns without progress.
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(kBkKT, kBkQC, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(kBkKT, D, false, true);
       bool ok = mbar_wait(bar_kv, 0, a.timeout_ns, abort_flag, kSiteQFull);
-      for (int v = 0; ok; ++v) {
-        const int st = v % STG;
-        if (!mbar_wait(&bar_full[st], (v / STG) & 1, a.timeout_ns, abort_flag, kSiteKvFull)) break;
-        if (reinterpret_cast<const DkvDesc*>(stage(st) + L::ST_DESC)->end) break;
-        // S^T / dP^T buffers are free once the previous visit's dv / dk
-        // MMAs (which read P^T / dS^T from them) are done
-        if (v > 0 && !mbar_wait(bar_pd_done, (v - 1) & 1, a.timeout_ns, abort_flag, kSiteMma))
-          break;
-        tc_fence_after();
-        const uint32_t qs = smem_u32(stage(st) + L::ST_Q), gs = smem_u32(stage(st) + L::ST_G);
+      int n1 = 0, n2 = 0;      // visits whose first / second products are issued
+      bool ended = false;
+      uint64_t t_last = globaltimer_ns();
+      while (ok && (!ended || n2 < n1)) {
+        bool progress = false;
+        if (!ended && n1 < n2 + 2) {
+          const int st = n1 % STG;
+          bool ready = mbar_test(&bar_full[st], (n1 / STG) & 1);
+          if (ready && reinterpret_cast<const DkvDesc*>(stage(st) + L::ST_DESC)->end) {
+            ended = true;
+            ready = false;
+            progress = true;
+          }
+          if (ready && n1 >= 2) ready = mbar_test(&bar_pd_done[n1 & 1], ((n1 - 2) >> 1) & 1);
+          if (ready) {
+            tc_fence_after();
+            const uint32_t qs = smem_u32(stage(st) + L::ST_Q), gs = smem_u32(stage(st) + L::ST_G);
+            const uint32_t buf = static_cast<uint32_t>(n1 & 1) * 64;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off_k = (kk / 4) * L::HALF_K + (kk % 4) * 32;
-          const uint32_t off_q = (kk / 4) * L::HALF_Q + (kk % 4) * 32;
-          mma_ss(tmem + L::TM_S, sdesc_sw128(sbase + L::OFF_K + off_k, 16, 1024),
-                 sdesc_sw128(qs + off_q, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
-        }
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off_k = (kk / 4) * L::HALF_K + (kk % 4) * 32;
+              const uint32_t off_q = (kk / 4) * L::HALF_Q + (kk % 4) * 32;
+              mma_ss(tmem + L::TM_S0 + buf, sdesc_sw128(sbase + L::OFF_K + off_k, 16, 1024),
+                     sdesc_sw128(qs + off_q, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+            }
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off_k = (kk / 4) * L::HALF_K + (kk % 4) * 32;
-          const uint32_t off_q = (kk / 4) * L::HALF_Q + (kk % 4) * 32;
-          mma_ss(tmem + L::TM_DP, sdesc_sw128(sbase + L::OFF_V + off_k, 16, 1024),
-                 sdesc_sw128(gs + off_q, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar_sd_full);
-        if (!mbar_wait(bar_p_full, v & 1, a.timeout_ns, abort_flag, kSitePFull)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-#pragma unroll
-          for (int kk = 0; kk < kBkQC / 16; ++kk) {
-            const uint32_t acc = (v > 0 || kk > 0 || part > 0) ? 1u : 0u;
-            mma_ts(tmem + L::TM_DV, tmem + L::TM_S + split_col(kk, part == 1),
-                   sdesc_sw128(gs + kk * 2048, L::HALF_Q, 1024), IDESC_O, acc);
-            mma_ts(tmem + L::TM_DK, tmem + L::TM_DP + split_col(kk, part == 1),
-                   sdesc_sw128(qs + kk * 2048, L::HALF_Q, 1024), IDESC_O, acc);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off_k = (kk / 4) * L::HALF_K + (kk % 4) * 32;
+              const uint32_t off_q = (kk / 4) * L::HALF_Q + (kk % 4) * 32;
+              mma_ss(tmem + L::TM_DP0 + buf, sdesc_sw128(sbase + L::OFF_V + off_k, 16, 1024),
+                     sdesc_sw128(gs + off_q, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&bar_sd_full[n1 & 1]);
+            ++n1;
+            progress = true;
           }
         }
-        mma_commit(bar_pd_done);
-        mma_commit(&bar_empty[st]);
+        if (n2 < n1 && mbar_test(&bar_p_full[n2 & 1], (n2 >> 1) & 1)) {
+          tc_fence_after();
+          const int st = n2 % STG;
+          const uint32_t qs = smem_u32(stage(st) + L::ST_Q), gs = smem_u32(stage(st) + L::ST_G);
+          const uint32_t buf = static_cast<uint32_t>(n2 & 1) * 64;
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+#pragma unroll
+            for (int kk = 0; kk < kBkQC / 16; ++kk) {
+              const uint32_t acc = (n2 > 0 || kk > 0 || part > 0) ? 1u : 0u;
+              mma_ts(tmem + L::TM_DV, tmem + L::TM_S0 + buf + split_col(kk, part == 1),
+                     sdesc_sw128(gs + kk * 2048, L::HALF_Q, 1024), IDESC_O, acc);
+              mma_ts(tmem + L::TM_DK, tmem + L::TM_DP0 + buf + split_col(kk, part == 1),
+                     sdesc_sw128(qs + kk * 2048, L::HALF_Q, 1024), IDESC_O, acc);
+            }
+          }
+          mma_commit(&bar_pd_done[n2 & 1]);
+          mma_commit(&bar_empty[st]);
+          ++n2;
+          progress = true;
+        }
+        if (progress) {
+          t_last = globaltimer_ns();
+        } else {
+          if (*abort_flag) break;
+          if (globaltimer_ns() - t_last > a.timeout_ns) {
+            *abort_flag = 1;
+            record_error(kErrTimeout, kSiteMma);
+            break;
+          }
+        }
       }
       mma_commit(bar_drain);
       mbar_wait(bar_drain, 0, a.timeout_ns, nullptr, kSiteDrain);
     }
   } else {
     // ------------------------------------------------------- softmax warps
-    const int r = tid;                   // key row in the tile == TMEM lane
+    // warp w: keys of TMEM lane quarter w % 4, query columns of half w / 4
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;   // key row in the tile == TMEM lane
     const int j = j0 + r;
     const bool row_ok = j < a.N;
     const int cl = (a.Bk < kBkKT) ? r / a.Bk : 0;           // key block within the tile
     const int bq_c = a.Bq < kBkQC ? a.Bq : kBkQC;           // columns of one query block
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float sl2 = a.scale_log2;
-    constexpr float kLog2e = 1.4426950408889634f;
     bool ok = true;
     int v = 0;
     for (;; ++v) {
@@ -831,81 +883,78 @@ __global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
       const uint8_t* sp = stage(st);
       const DkvDesc dsc = *reinterpret_cast<const DkvDesc*>(sp + L::ST_DESC);
       if (dsc.end) break;
-      const bool got2 = mbar_wait(bar_sd_full, v & 1, a.timeout_ns, abort_flag, kSiteSFull);
+      const bool got2 = mbar_wait(&bar_sd_full[v & 1], (v >> 1) & 1, a.timeout_ns, abort_flag,
+                                  kSiteSFull);
       if (!__all_sync(0xffffffffu, got2)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int i0 = dsc.qc * kBkQC;
-      // queries of the chunk that read this key
-      uint64_t m = 0ull;
+      // queries of this warp's half that read this key
+      uint32_t m = 0u;
       if (row_ok) {
+        uint64_t mm = 0ull;
         const int nq = min(kBkQC, a.N - i0);
 #pragma unroll 1
         for (int lq = 0; lq * bq_c < kBkQC; ++lq)
-          if ((dsc.routed >> (lq * 8 + cl)) & 1u) m |= bit_range(lq * bq_c, (lq + 1) * bq_c);
-        if (a.causal) m |= bit_range(max(0, j - i0), min(kBkQC, j + a.window - i0));
-        m &= bit_range(0, nq);
+          if ((dsc.routed >> (lq * 8 + cl)) & 1u) mm |= bit_range(lq * bq_c, (lq + 1) * bq_c);
+        if (a.causal) mm |= bit_range(max(0, j - i0), min(kBkQC, j + a.window - i0));
+        mm &= bit_range(0, nq);
+        m = static_cast<uint32_t>(mm >> (32 * half));
       }
-      const uint32_t mlo = static_cast<uint32_t>(m), mhi = static_cast<uint32_t>(m >> 32);
-      const float* lse_s = reinterpret_cast<const float*>(sp + L::ST_LSE);
-      const float* del_s = reinterpret_cast<const float*>(sp + L::ST_DEL);
-
-      if (__all_sync(0xffffffffu, m == 0ull)) {
-        uint32_t z[32];
+      const uint32_t scol = trow + L::TM_S0 + (v & 1) * 64 + half * 32;
+      const uint32_t dcol = trow + L::TM_DP0 + (v & 1) * 64 + half * 32;
+      if (__all_sync(0xffffffffu, m == 0u)) {
+        uint32_t z[16];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) z[c] = 0u;
-        tmem_st32(trow + L::TM_S, z);
-        tmem_st32(trow + L::TM_S + 32, z);
-        tmem_st32(trow + L::TM_DP, z);
-        tmem_st32(trow + L::TM_DP + 32, z);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_p_full);
-        continue;
-      }
-
-      // half by half (32 queries each): the half's S^T and dP^T come in one
-      // TMEM round trip; P^T and dS^T (split into bf16 hi / lo parts) go over
-      // the halves just read
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const uint32_t mm = half ? mhi : mlo;
+        for (int c = 0; c < 16; ++c) z[c] = 0u;
+        tmem_st16(scol, z);
+        tmem_st16(scol + 16, z);
+        tmem_st16(dcol, z);
+        tmem_st16(dcol + 16, z);
+      } else {
         uint32_t sv[32], dv32[32];
-        tmem_ld32(trow + L::TM_S + half * 32, sv);
-        tmem_ld32(trow + L::TM_DP + half * 32, dv32);
+        tmem_ld32(scol, sv);
+        tmem_ld32(dcol, dv32);
+        // the half's lse * log2(e) and delta, 4 at a time
+        const uint32_t lsa = smem_u32(sp + L::ST_LSE) + half * 128;
+        const uint32_t dla = smem_u32(sp + L::ST_DEL) + half * 128;
+        float ls[32], dl[32];
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 x = lds_f4(lsa + c4 * 16), y = lds_f4(dla + c4 * 16);
+          ls[4 * c4] = x.x; ls[4 * c4 + 1] = x.y; ls[4 * c4 + 2] = x.z; ls[4 * c4 + 3] = x.w;
+          dl[4 * c4] = y.x; dl[4 * c4 + 1] = y.y; dl[4 * c4 + 2] = y.z; dl[4 * c4 + 3] = y.w;
+        }
         tmem_ld_wait(sv);
         tmem_ld_wait(dv32);
-        // P^T and dS^T in place of S^T and dP^T (float bits), so that only
-        // the two loaded arrays are live
+        // P^T and dS^T in place of S^T and dP^T (float bits)
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const bool on = (mm >> c) & 1u;
-          const float pc = ex2_approx(
-              fmaf(__uint_as_float(sv[c]), sl2, -lse_s[half * 32 + c] * kLog2e));
-          dv32[c] = __float_as_uint(on ? pc * (__uint_as_float(dv32[c]) - del_s[half * 32 + c])
-                                       : 0.f);
+          const bool on = (m >> c) & 1u;
+          const float pc = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -ls[c]));
+          dv32[c] = __float_as_uint(on ? pc * (__uint_as_float(dv32[c]) - dl[c]) : 0.f);
           sv[c] = __float_as_uint(on ? pc : 0.f);
         }
         uint32_t hi[16], lo[16];
         split_pack32_bits(dv32, hi, lo);
-        tmem_st16(trow + L::TM_DP + half * 32, hi);
-        tmem_st16(trow + L::TM_DP + half * 32 + 16, lo);
+        tmem_st16(dcol, hi);
+        tmem_st16(dcol + 16, lo);
         split_pack32_bits(sv, hi, lo);
-        tmem_st16(trow + L::TM_S + half * 32, hi);
-        tmem_st16(trow + L::TM_S + half * 32 + 16, lo);
+        tmem_st16(scol, hi);
+        tmem_st16(scol + 16, lo);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p_full);
+      if (lane == 0) mbar_arrive(&bar_p_full[v & 1]);
     }
 
     // ------------------------------------------------------- epilogue
     if (ok && v > 0) {
-      const bool got = mbar_wait(bar_pd_done, (v - 1) & 1, a.timeout_ns, abort_flag, kSitePvDone);
+      const bool got = mbar_wait(&bar_pd_done[(v - 1) & 1], ((v - 1) >> 1) & 1, a.timeout_ns,
+                                 abort_flag, kSitePvDone);
       ok = __all_sync(0xffffffffu, got);
     }
     if (ok && !*abort_flag) {
@@ -919,9 +968,9 @@ __global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
         float* dst_row = (which == 0 ? (direct ? ba.dk : ba.part_dk)
                                      : (direct ? ba.dv : ba.part_dv)) + off;
         const float f = which == 0 ? ba.scale : 1.f;
-        const uint32_t col = which == 0 ? L::TM_DK : L::TM_DV;
+        const uint32_t col = (which == 0 ? L::TM_DK : L::TM_DV) + half * (D / 2);
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
+        for (int cc = 0; cc < D / 64; ++cc) {
           uint32_t x[32];
           if (v > 0) {
             tmem_ld32(trow + col + cc * 32, x);
@@ -931,7 +980,7 @@ __global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
             for (int c = 0; c < 32; ++c) x[c] = 0u;
           }
           if (row_ok) {
-            float4* dst = reinterpret_cast<float4*>(dst_row + cc * 32);
+            float4* dst = reinterpret_cast<float4*>(dst_row + half * (D / 2) + cc * 32);
 #pragma unroll
             for (int c = 0; c < 8; ++c)
               dst[c] = make_float4(__uint_as_float(x[4 * c]) * f, __uint_as_float(x[4 * c + 1]) * f,
@@ -946,7 +995,7 @@ __global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 4 && lane == 0) {
+  if (warp == NSW && lane == 0) {
     // after an abort, copies in flight must land before the CTA exits; on the
     // normal path every stage and the K/V tile were consumed
     if (*abort_flag) {
@@ -956,9 +1005,34 @@ __global__ void __launch_bounds__(kAtThreads, D == 64 ? 2 : 1)
     }
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == NSW + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, L::COLS);
+  }
+}
+
+// delta_i = <g_i, o_i> (fp32, from the bf16 output and gradient) and
+// lse_i * log2(e), the exponent offset the key-major kernel reads; one warp
+// per row
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdTcArgs ba, int64_t n_rows) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= n_rows) return;
+  const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(ba.o + row * D);
+  const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(ba.d_o + row * D);
+  float s = 0.f;
+#pragma unroll
+  for (int c = lane; c < D / 2; c += 32) {
+    const float2 x = __bfloat1622float2(o2[c]), y = __bfloat1622float2(g2[c]);
+    s = fmaf(x.x, y.x, s);
+    s = fmaf(x.y, y.y, s);
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+  if (lane == 0) {
+    ba.delta_w[row] = s;
+    ba.lse2[row] = ba.lse[row] * 1.4426950408889634f;
   }
 }
 

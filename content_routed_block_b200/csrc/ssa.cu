@@ -456,14 +456,16 @@ ssa_status launch_route_tree(const ssa_params* p, const float* qsum, const float
 // the tensor-core form also keeps the list transpose (one bit per key tile of
 // 128 keys and query chunk of 64 queries, per list head).
 struct BwdWs {
-  size_t delta, map, map_bytes, part_dk, part_dv, total;
+  size_t delta, lse2, map, map_bytes, part_dk, part_dv, total;
   int32_t n_ktiles, map_words;
 };
 
 BwdWs bwd_ws_layout(const ssa_params* p) {
   BwdWs w;
+  const size_t rows = align256(static_cast<size_t>(p->B) * p->Hq * p->N * sizeof(float));
   w.delta = 0;
-  w.map = align256(static_cast<size_t>(p->B) * p->Hq * p->N * sizeof(float));
+  w.lse2 = rows;
+  w.map = 2 * rows;
   w.n_ktiles = (p->N + ssa::kBkKT - 1) / ssa::kBkKT;
   const int32_t nqc = (p->N + ssa::kBkQC - 1) / ssa::kBkQC;
   w.map_words = (nqc + 31) / 32;
@@ -521,8 +523,9 @@ cudaError_t launch_backward_tc_d(const CUtensorMap* maps, const ssa::BwdTcArgs& 
                            static_cast<int>(smem_kv));
   if (e != cudaSuccess) return e;
   const int64_t n_kctas = static_cast<int64_t>(B) * a.at.Hq * a.n_ktiles;
-  ssa::bwd_dkdv_kernel<D><<<static_cast<unsigned>(n_kctas), ssa::kAtThreads, smem_kv, stream>>>(
-      maps[4], maps[5], maps[6], maps[7], a);
+  ssa::bwd_dkdv_kernel<D>
+      <<<static_cast<unsigned>(n_kctas), ssa::DkvLayout<D>::THREADS, smem_kv, stream>>>(
+          maps[4], maps[5], maps[6], maps[7], a);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.at.Hq == Hkv) return e;
   const int64_t n4 = static_cast<int64_t>(B) * Hkv * a.at.N * (D / 4);
@@ -1145,14 +1148,6 @@ ssa_status ssa_attend_backward(const ssa_params* p, const void* q, const void* k
   uint32_t* map = reinterpret_cast<uint32_t*>(ws + w.map);
   e = cudaMemsetAsync(map, 0, w.map_bytes, st);
   if (e != cudaSuccess) return cuda_fail(e, "clear the list transpose");
-  const int64_t rows = static_cast<int64_t>(p->B) * p->Hq * p->N;
-  if (p->D == 64)
-    ssa::bwd_delta_kernel<64><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a, rows);
-  else
-    ssa::bwd_delta_kernel<128><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a, rows);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "bwd_delta_kernel launch");
-
   if ((s = get_encoder()) != SSA_OK) return s;
   const int64_t hq = static_cast<int64_t>(p->B) * p->Hq, hkv = static_cast<int64_t>(p->B) * p->Hkv;
   const uint32_t kv_rows = static_cast<uint32_t>(p->block_k < 64 ? p->block_k : 64);
@@ -1188,6 +1183,10 @@ ssa_status ssa_attend_backward(const ssa_params* p, const void* q, const void* k
   t.at.timeout_ns = timeout_ns(p);
   t.lse = lse;
   t.delta = a.delta;
+  t.delta_w = a.delta;
+  t.lse2 = reinterpret_cast<float*>(ws + w.lse2);
+  t.o = static_cast<const __nv_bfloat16*>(o);
+  t.d_o = static_cast<const __nv_bfloat16*>(d_o);
   t.dq = dq;
   t.dk = dk;
   t.dv = dv;
@@ -1199,6 +1198,13 @@ ssa_status ssa_attend_backward(const ssa_params* p, const void* q, const void* k
   t.part_dk = p->Hq > p->Hkv ? reinterpret_cast<float*>(ws + w.part_dk) : nullptr;
   t.part_dv = p->Hq > p->Hkv ? reinterpret_cast<float*>(ws + w.part_dv) : nullptr;
   t.scale = a.scale;
+  const int64_t rows = static_cast<int64_t>(p->B) * p->Hq * p->N;
+  if (p->D == 64)
+    ssa::bwd_prep_kernel<64><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(t, rows);
+  else
+    ssa::bwd_prep_kernel<128><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(t, rows);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "bwd_prep_kernel launch");
   if (p->top_k > 0) {
     const int64_t slots = static_cast<int64_t>(p->B) * t.at.idx_heads * t.at.NQB * p->top_k;
     ssa::bwd_map_kernel<<<static_cast<unsigned>((slots + 255) / 256), 256, 0, st>>>(t, slots);

@@ -272,7 +272,7 @@ ssa_status ssa_forward_static(const ssa_params* p, const void* q, const void* k,
                               ssa_stream_t stream);
 
 /* Bytes of device workspace ssa_attend_backward needs (0 if the parameters
- * are invalid): one fp32 per query row, the lists' transpose (one bit per
+ * are invalid): two fp32 per query row, the lists' transpose (one bit per
  * list head, 128-key tile and 64-query chunk: 235 MB for 14 heads at 1M
  * tokens, 0.23 MB at 32K) and, when Hq > Hkv, each query head's fp32 share
  * of dk and dv (2 * B * Hq * N * D * 4 bytes: 7.5 GB at 1M tokens). */
@@ -294,9 +294,9 @@ size_t ssa_backward_workspace_size(const ssa_params* p);
  *   dq          fp32 [B, Hq, N, D] (device, out)
  *   dk, dv      fp32 [B, Hkv, N, D] (device, out; every entry is written)
  *   workspace   ssa_backward_workspace_size(p) bytes (device, 256-byte aligned):
- *               delta [B, Hq, N] fp32, the lists' transpose (one bit per list
- *               head, 128-key tile and 64-query chunk) and, when Hq > Hkv,
- *               every query head's share of dk and dv
+ *               delta and lse * log2(e) [B, Hq, N] fp32, the lists' transpose
+ *               (one bit per list head, 128-key tile and 64-query chunk) and,
+ *               when Hq > Hkv, every query head's share of dk and dv
  * The products run on the tensor cores (tcgen05, bf16 operands, fp32
  * accumulation in TMEM): a query-major kernel for dq over the forward's key
  * sets and a key-major kernel for dk / dv over the transposed lists.  P and

@@ -210,10 +210,10 @@ def test_backward_entry_point_rejects_bad_arguments_before_launch(L):
     odd = ctypes.c_void_p((1 << 20) + 4)
     p = _p()
     ws = L.ssa_backward_workspace_size(ctypes.byref(p))
-    # one fp32 per query row (delta), one bit per (head, 128-key tile,
+    # two fp32 per query row (delta, lse * log2 e), one bit per (head, 128-key tile,
     # 64-query chunk): 14 heads x 256 tiles x 16 words of 32 chunks, then
     # each query head's share of dk and dv (fp32 [14, 32768, 64] each)
-    assert ws == (1 * 14 * 32768 * 4 + 255) // 256 * 256 + 14 * 256 * 16 * 4 + \
+    assert ws == 2 * ((1 * 14 * 32768 * 4 + 255) // 256 * 256) + 14 * 256 * 16 * 4 + \
         2 * 14 * 32768 * 64 * 4
     f = L.ssa_attend_backward
 
