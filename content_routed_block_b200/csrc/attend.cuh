@@ -334,8 +334,10 @@ __global__ void __launch_bounds__(kAtThreads, 2)
   using L = AtLayout<D>;
   constexpr int S = L::STAGES;
   extern __shared__ uint8_t at_smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(at_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned start, as an offset into the shared array (not through an
+  // integer cast, which would drop the shared address space from every pointer
+  // derived from it and turn their loads into generic ones)
+  uint8_t* smem = at_smem_raw + ((1024u - (smem_u32(at_smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   uint32_t* win = reinterpret_cast<uint32_t*>(smem + L::OFF_WIN);
   int32_t* far = reinterpret_cast<int32_t*>(smem + L::OFF_FAR);
@@ -584,7 +586,7 @@ __global__ void __launch_bounds__(kAtThreads, 2)
 
       // allowed keys of this row within the chunk, as two 32-bit words
       uint32_t mlo = 0u, mhi = 0u;
-      if (row_ok) {
+      {
         uint64_t mask = 0ull;
         if (a.Bk >= kAtKT) {
           const int e = t >> subs_sh, sub = t & (SUBS - 1);
@@ -598,12 +600,13 @@ __global__ void __launch_bounds__(kAtThreads, 2)
           } else {
             hi = routed ? kAtKT : 0;
           }
-          mask = bit_range(lo, hi);
+          mask = row_ok ? bit_range(lo, hi) : 0ull;
         } else {
           for (int s = 0; s < G; ++s) {
             const int e = t * G + s;
             if (e >= n_entries) break;
             const uint32_t ent = at_entry(faru, win, nf, wlo, e);
+            if (!row_ok) continue;
             const int j0 = static_cast<int>(ent >> 8) * a.Bk;
             const bool routed = (ent >> qbr) & 1u;
             int lo = 0, hi = 0;

@@ -129,8 +129,10 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
   constexpr int NT = Lay::NT;
   constexpr uint32_t IDESC = idesc_bf16_f32(kRtcRows, NT, false, false);
   extern __shared__ uint8_t rtc_smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(rtc_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned start, as an offset into the shared array (not through an
+  // integer cast, which would drop the shared address space from every pointer
+  // derived from it and turn their loads into generic ones)
+  uint8_t* smem = rtc_smem_raw + ((1024u - (smem_u32(rtc_smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   float* qf = reinterpret_cast<float*>(smem + Lay::OFF_QF);     // [D][128]
   float* nrm = reinterpret_cast<float*>(smem + Lay::OFF_NRM);   // [NT]
