@@ -45,8 +45,8 @@
 //          the bounds sa_c - E_c themselves, at most an ulp of the score.)
 //
 // One CTA owns 128 query blocks of one (b, head): thread r = row r = TMEM
-// lane r runs the per-row tests straight out of TMEM; all 256 threads split
-// and stage each key-summary tile; one thread issues the MMAs.
+// lane r runs the per-row tests straight out of TMEM, while four other warps
+// stage the next key-summary tiles and issue their MMAs (see the kernel).
 #pragma once
 
 #include "common.cuh"
@@ -65,21 +65,23 @@ constexpr int kRtcCap = 32;               // queued candidates per row before a 
 template <int D>
 struct RtcLayout {
   static constexpr int NT = kRtcNT;
+  static constexpr int KSTAGES = 2;                   // key-summary tiles in flight
   static constexpr uint32_t HALF_Q = kRtcRows * 128;  // one 64-column bf16 half of a Q tile
   static constexpr uint32_t Q_BYTES = kRtcRows * D * 2;
   static constexpr uint32_t HALF_K = NT * 128;
   static constexpr uint32_t K_BYTES = NT * D * 2;
   static constexpr uint32_t OFF_QH = 0;
   static constexpr uint32_t OFF_QL = OFF_QH + Q_BYTES;
-  static constexpr uint32_t OFF_KH = OFF_QL + Q_BYTES;
-  static constexpr uint32_t OFF_KL = OFF_KH + K_BYTES;
-  static constexpr uint32_t OFF_QF = OFF_KL + K_BYTES;            // fp32 [D][128] query summaries
-  static constexpr uint32_t OFF_NRM = OFF_QF + D * kRtcRows * 4;  // fp32 [NT] key-summary norms
-  static constexpr uint32_t OFF_LIST = OFF_NRM + NT * 4;          // uint16 [kRtcCap][128]
+  static constexpr uint32_t OFF_K = OFF_QL + Q_BYTES;              // stage s: hi, then lo
+  static constexpr uint32_t OFF_NRM = OFF_K + KSTAGES * 2 * K_BYTES;  // fp32 [KSTAGES][NT]
+  static constexpr uint32_t OFF_LIST = OFF_NRM + KSTAGES * NT * 4;    // uint16 [kRtcCap][128]
   static constexpr uint32_t OFF_BAR = OFF_LIST + kRtcCap * kRtcRows * 2;
-  static constexpr uint32_t USED = OFF_BAR + 32;
+  // acc_full[2] | acc_empty[2] | TMEM base
+  static constexpr uint32_t USED = OFF_BAR + 48;
   static constexpr uint32_t SMEM_BYTES = USED + 1024;
-  static constexpr uint32_t TMEM_COLS = NT;
+  static constexpr uint32_t TMEM_COLS = KSTAGES * NT;             // two accumulators
+  static __device__ __forceinline__ uint32_t kh(int st) { return OFF_K + st * 2 * K_BYTES; }
+  static __device__ __forceinline__ uint32_t kl(int st) { return OFF_K + st * 2 * K_BYTES + K_BYTES; }
 };
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -122,6 +124,14 @@ __device__ __forceinline__ void sorted_insert(T (&arr)[KM], T v) {
   arr[0] = v > arr[0] ? v : arr[0];
 }
 
+// Warp roles: warps 0-3 are the rows (thread r = query block qb0 + r = TMEM
+// lane r) and scan every tile's scores; warps 4-7 stage the key-summary tiles
+// (one thread per key block: load, split into bf16 hi / lo, norm) into one of
+// two stages, and their first thread issues the tile's three MMAs into one of
+// two TMEM accumulators.  The tiles of both passes form one stream, so the
+// staging of the next tiles overlaps the scan of the current one.  Barriers:
+// acc_full[b] (MMAs of a tile into accumulator b done), acc_empty[b] (the rows
+// have read accumulator b and the norms of stage b).
 template <int D, int KM>
 __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     route_tc_kernel(const RouteArgs a) {
@@ -134,11 +144,11 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
   // derived from it and turn their loads into generic ones)
   uint8_t* smem = rtc_smem_raw + ((1024u - (smem_u32(rtc_smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
-  float* qf = reinterpret_cast<float*>(smem + Lay::OFF_QF);     // [D][128]
-  float* nrm = reinterpret_cast<float*>(smem + Lay::OFF_NRM);   // [NT]
+  float* nrm = reinterpret_cast<float*>(smem + Lay::OFF_NRM);   // [2][NT]
   uint16_t* qlist = reinterpret_cast<uint16_t*>(smem + Lay::OFF_LIST);
-  uint64_t* bar_mma = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_BAR + 8);
+  uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);       // [2]
+  uint64_t* bar_empty = bar_full + 2;                                          // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_BAR + 32);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int bh = blockIdx.y;
@@ -157,17 +167,20 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
   const float* ksrc = a.ksum + static_cast<int64_t>(bkv) * a.NB * D;
 
   if (tid == 0) {
-    mbar_init(bar_mma, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_empty[i], 4);   // one arrival per row warp
+    }
     fence_barrier_init();
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, Lay::TMEM_COLS);
     tmem_relinquish();
   }
-  // query summaries: bf16 hi / lo (MMA A operands) and fp32 transposed
+  // query summaries: bf16 hi / lo (MMA A operands), 2 threads per row
   {
-    constexpr int TPR = kRtcThreads / kRtcRows;   // 2 threads per row
-    constexpr int CPT = (D / 8) / TPR;            // 16-byte chunks per thread
+    constexpr int TPR = kRtcThreads / kRtcRows;
+    constexpr int CPT = (D / 8) / TPR;
     const int r = tid / TPR, part = tid % TPR;
     const bool ok = qb0 + r < a.NQB;
     const float* src = qsrc + static_cast<int64_t>(qb0 + r) * D;
@@ -184,9 +197,6 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
       split8_bf16(v0, v1, hi, lo, sq);
       *reinterpret_cast<uint4*>(smem + Lay::OFF_QH + sw128_offset(r, g, Lay::HALF_Q)) = hi;
       *reinterpret_cast<uint4*>(smem + Lay::OFF_QL + sw128_offset(r, g, Lay::HALF_Q)) = lo;
-      const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) qf[(g * 8 + e) * kRtcRows + r] = vv[e];
     }
   }
   fence_proxy_async_smem();
@@ -194,39 +204,20 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int total = 2 * n_tiles;     // pass 1 tiles, then pass 2 tiles
 
-  // per-row state (threads 0..127)
-  const int r = tid;
-  const bool is_row = tid < kRtcRows;
-  const int qb = qb0 + r;
-  int lim = 0;
-  float e_row = 0.f;
-  if (is_row && qb < a.NQB) {
-    lim = a.causal ? min(a.NB, static_cast<int>((static_cast<int64_t>(qb) * a.Bq) / a.Bk)) : a.NB;
-    float sq = 0.f;
-#pragma unroll 8
-    for (int d = 0; d < D; ++d) sq = fmaf(qf[d * kRtcRows + r], qf[d * kRtcRows + r], sq);
-    e_row = rtc_eps<D>() * sqrtf(sq) * 1.001f;  // slack for the fp32 norms themselves
-  }
-  const int k = a.top_k;
-  const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-  uint32_t phase = 0;
-
-  // one tile: split and stage key summaries, three MMAs, then for every
-  // 32-column group `group(cb, scores, nrm32, full)`: full means every column
-  // of the group is admissible for this row
-  auto run_tile = [&](int tile, auto&& group) {
-    const int c0 = tile * NT;
-    {
-      constexpr int TPR = kRtcThreads / NT;          // 2 threads per key row
-      constexpr int CPT = (D / 8) / TPR;
-      const int cr = tid / TPR, part = tid % TPR;
-      const bool ok = c0 + cr < a.NB;
-      const float* src = ksrc + static_cast<int64_t>(c0 + cr) * D;
+  if (warp >= 4) {
+    // ------------------------------------------------ key-summary stagers
+    const int sid = tid - kRtcRows;   // key row of the tile
+    for (int t = 0; t < total; ++t) {
+      const int st = t & 1;
+      if (t >= 2) mbar_wait(&bar_empty[st], ((t - 2) >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
+      const int c0 = (t % n_tiles) * NT;
+      const bool ok = c0 + sid < a.NB;
+      const float* src = ksrc + static_cast<int64_t>(c0 + sid) * D;
       float sq = 0.f;
 #pragma unroll
-      for (int c = 0; c < CPT; ++c) {
-        const int g = part * CPT + c;
+      for (int g = 0; g < D / 8; ++g) {
         float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
         if (ok) {
           v0 = *reinterpret_cast<const float4*>(src + g * 8);
@@ -234,175 +225,204 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
         }
         uint4 hi, lo;
         split8_bf16(v0, v1, hi, lo, sq);
-        *reinterpret_cast<uint4*>(smem + Lay::OFF_KH + sw128_offset(cr, g, Lay::HALF_K)) = hi;
-        *reinterpret_cast<uint4*>(smem + Lay::OFF_KL + sw128_offset(cr, g, Lay::HALF_K)) = lo;
+        *reinterpret_cast<uint4*>(smem + Lay::kh(st) + sw128_offset(sid, g, Lay::HALF_K)) = hi;
+        *reinterpret_cast<uint4*>(smem + Lay::kl(st) + sw128_offset(sid, g, Lay::HALF_K)) = lo;
       }
-      sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-      if (part == 0) nrm[cr] = sqrtf(sq) * 1.001f;
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == kRtcRows) {  // warp 4, lane 0
-      tc_fence_after();
-      const uint32_t oq[3] = {Lay::OFF_QH, Lay::OFF_QH, Lay::OFF_QL};
-      const uint32_t okk[3] = {Lay::OFF_KH, Lay::OFF_KL, Lay::OFF_KH};
+      nrm[st * NT + sid] = sqrtf(sq) * 1.001f;
+      fence_proxy_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");   // the stagers only
+      if (sid == 0) {
+        tc_fence_after();
+        const uint32_t oq[3] = {Lay::OFF_QH, Lay::OFF_QH, Lay::OFF_QL};
+        const uint32_t okk[3] = {Lay::kh(st), Lay::kl(st), Lay::kh(st)};
 #pragma unroll
-      for (int term = 0; term < 3; ++term) {
+        for (int term = 0; term < 3; ++term) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qa = sbase + oq[term] + (kk / 4) * Lay::HALF_Q + (kk % 4) * 32;
-          const uint32_t kb = sbase + okk[term] + (kk / 4) * Lay::HALF_K + (kk % 4) * 32;
-          mma_ss(tmem, sdesc_sw128(qa, 16, 1024), sdesc_sw128(kb, 16, 1024), IDESC,
-                 (term > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t qa = sbase + oq[term] + (kk / 4) * Lay::HALF_Q + (kk % 4) * 32;
+            const uint32_t kb = sbase + okk[term] + (kk / 4) * Lay::HALF_K + (kk % 4) * 32;
+            mma_ss(tmem + st * NT, sdesc_sw128(qa, 16, 1024), sdesc_sw128(kb, 16, 1024), IDESC,
+                   (term > 0 || kk > 0) ? 1u : 0u);
+          }
         }
+        mma_commit(&bar_full[st]);
       }
-      mma_commit(bar_mma);
     }
-    if (is_row) {
-      // the MMAs complete in bounded time; the wait is bounded anyway
-      mbar_wait(bar_mma, phase, a.timeout_ns, nullptr, kSiteMma);
+  } else {
+    // ------------------------------------------------------------ rows
+    const int r = tid;
+    const int qb = qb0 + r;
+    const bool row_valid = qb < a.NQB;
+    const float* qrow = qsrc + static_cast<int64_t>(row_valid ? qb : qb0) * D;
+    int lim = 0;
+    float e_row = 0.f;
+    if (row_valid) {
+      lim = a.causal ? min(a.NB, static_cast<int>((static_cast<int64_t>(qb) * a.Bq) / a.Bk)) : a.NB;
+      float sq = 0.f;
+#pragma unroll
+      for (int d4 = 0; d4 < D / 4; ++d4) {
+        const float4 v = reinterpret_cast<const float4*>(qrow)[d4];
+        sq = fmaf(v.x, v.x, sq);
+        sq = fmaf(v.y, v.y, sq);
+        sq = fmaf(v.z, v.z, sq);
+        sq = fmaf(v.w, v.w, sq);
+      }
+      e_row = rtc_eps<D>() * sqrtf(sq) * 1.001f;  // slack for the fp32 norms themselves
+    }
+    const int k = a.top_k;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+
+    // scan tile t of the stream: for every 32-column group `group(cb, scores,
+    // norms, full)` (full: every column of the group is admissible for this
+    // row), then hand the accumulator and the stage's norms back
+    auto scan_tile = [&](int t, auto&& group) {
+      const int st = t & 1;
+      mbar_wait(&bar_full[st], (t >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
       tc_fence_after();
+      const int c0 = (t % n_tiles) * NT;
 #pragma unroll 1
       for (int cc = 0; cc < NT / 32; ++cc) {
         uint32_t sv[32];
-        tmem_ld32(trow + cc * 32, sv);
+        tmem_ld32(trow + st * NT + cc * 32, sv);
         tmem_ld_wait(sv);
         const int cb = c0 + cc * 32;
-        group(cb, sv, nrm + cc * 32, cb + 32 <= lim);
+        group(cb, sv, nrm + st * NT + cc * 32, cb + 32 <= lim);
       }
-    }
-    phase ^= 1u;
-    tc_fence_before();
-    __syncthreads();
-  };
+      tc_fence_before();
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive(&bar_empty[st]);
+    };
 
-  // pass 1: L = k-th largest per-group maximum of the lower bounds (the
-  // first KM - k slots of lb are +inf sentinels, so slot KM-1 is the k-th)
-  float L = -INFINITY;
-  float nmax = 0.f;
-  {
-    float lb[KM];
+    // pass 1: L = k-th largest per-group maximum of the lower bounds (the
+    // first KM - k slots of lb are +inf sentinels, so slot KM-1 is the k-th)
+    float L = -INFINITY;
+    float nmax = 0.f;
+    {
+      float lb[KM];
 #pragma unroll
-    for (int j = 0; j < KM; ++j) lb[j] = (j < KM - k) ? INFINITY : -INFINITY;
-    for (int tile = 0; tile < n_tiles; ++tile) {
-      run_tile(tile, [&](int cb, const uint32_t (&sv)[32], const float* nc, bool full) {
-        if (cb >= lim) return;
-        float gmax = -INFINITY, gn = 0.f;
-        if (full) {
+      for (int j = 0; j < KM; ++j) lb[j] = (j < KM - k) ? INFINITY : -INFINITY;
+      for (int t = 0; t < n_tiles; ++t) {
+        scan_tile(t, [&](int cb, const uint32_t (&sv)[32], const float* nc, bool full) {
+          if (cb >= lim) return;
+          float gmax = -INFINITY, gn = 0.f;
+          if (full) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            gmax = fmaxf(gmax, fmaf(-e_row, nc[j], __uint_as_float(sv[j])));
-            gn = fmaxf(gn, nc[j]);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (cb + j < lim) {
+            for (int j = 0; j < 32; ++j) {
               gmax = fmaxf(gmax, fmaf(-e_row, nc[j], __uint_as_float(sv[j])));
               gn = fmaxf(gn, nc[j]);
             }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (cb + j < lim) {
+                gmax = fmaxf(gmax, fmaf(-e_row, nc[j], __uint_as_float(sv[j])));
+                gn = fmaxf(gn, nc[j]);
+              }
+            }
+          }
+          nmax = fmaxf(nmax, gn);
+          if (gmax > lb[KM - 1]) sorted_insert<KM>(lb, gmax);
+        });
+      }
+      L = lb[KM - 1];
+    }
+
+    // pass 2: queue every candidate whose upper bound reaches the filter and
+    // rescore the queues exactly in fp32, a warp's rows together
+    uint64_t keys[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) keys[j] = (j < KM - k) ? ~0ull : 0ull;
+    const float slack = e_row * nmax * 0.5f;  // >= (eps / 2) ||qbar|| max ||mu||
+    float filt = L - slack;
+    int nq = 0;
+    // the exact fp32 score: sequential fmaf over d, the FMA router's arithmetic
+    auto rescore = [&](int c) -> float {
+      const float4* mu = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(c) * D);
+      const float4* qv = reinterpret_cast<const float4*>(qrow);
+      float acc = 0.f;
+#pragma unroll 4
+      for (int d4 = 0; d4 < D / 4; ++d4) {
+        const float4 m = mu[d4], q = qv[d4];
+        acc = fmaf(q.x, m.x, acc);
+        acc = fmaf(q.y, m.y, acc);
+        acc = fmaf(q.z, m.z, acc);
+        acc = fmaf(q.w, m.w, acc);
+      }
+      return acc;
+    };
+    auto flush = [&]() {
+      int rounds = nq;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        rounds = max(rounds, __shfl_xor_sync(0xffffffffu, rounds, off));
+      for (int t = 0; t < rounds; t += 2) {
+        const bool h0 = t < nq, h1 = t + 1 < nq;
+        const int c0 = h0 ? qlist[t * kRtcRows + r] : 0;
+        const int c1 = h1 ? qlist[(t + 1) * kRtcRows + r] : c0;
+        float s0 = 0.f, s1 = 0.f;
+        if (h0) s0 = rescore(c0);
+        if (h1) s1 = rescore(c1);
+        if (h0) {
+          const uint64_t key = route_key(s0, c0);
+          if (key > keys[KM - 1]) sorted_insert<KM>(keys, key);
+        }
+        if (h1) {
+          const uint64_t key = route_key(s1, c1);
+          if (key > keys[KM - 1]) sorted_insert<KM>(keys, key);
+        }
+      }
+      nq = 0;
+      // once k exact candidates are known, the k-th exact score bounds the rest
+      if (keys[KM - 1] != 0ull && keys[KM - 1] != ~0ull)
+        filt = fmaxf(filt, key_score(keys[KM - 1]) - slack);
+    };
+    for (int t = n_tiles; t < total; ++t) {
+      scan_tile(t, [&](int cb, const uint32_t (&sv)[32], const float* nc, bool full) {
+        uint32_t m = 0u;
+        if (cb < lim) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const bool adm = full || (cb + j < lim);
+            if (adm && fmaf(e_row, nc[j], __uint_as_float(sv[j])) >= filt) m |= 1u << j;
           }
         }
-        nmax = fmaxf(nmax, gn);
-        if (gmax > lb[KM - 1]) sorted_insert<KM>(lb, gmax);
+        // flush (warp-uniform) only when a queue would overflow
+        if (__any_sync(0xffffffffu, nq + __popc(m) > kRtcCap)) flush();
+        while (m) {
+          const int j = __ffs(m) - 1;
+          m &= m - 1;
+          qlist[nq * kRtcRows + r] = static_cast<uint16_t>(cb + j);
+          ++nq;
+        }
       });
     }
-    L = lb[KM - 1];
-  }
+    flush();
 
-  // pass 2: queue every candidate whose upper bound reaches the filter and
-  // rescore the queues exactly in fp32, a warp's rows together
-  uint64_t keys[KM];
+    // output: the real entries, ascending by block index
+    if (row_valid) {
+      int sel[KM];
+      int n = 0;
 #pragma unroll
-  for (int j = 0; j < KM; ++j) keys[j] = (j < KM - k) ? ~0ull : 0ull;
-  const float slack = e_row * nmax * 0.5f;  // >= (eps / 2) ||qbar|| max ||mu||
-  float filt = L - slack;
-  int nq = 0;
-  auto rescore = [&](int c) -> float {
-    const float4* mu = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(c) * D);
-    float acc = 0.f;
-#pragma unroll 4
-    for (int d4 = 0; d4 < D / 4; ++d4) {
-      const float4 m = mu[d4];
-      acc = fmaf(qf[(d4 * 4 + 0) * kRtcRows + r], m.x, acc);
-      acc = fmaf(qf[(d4 * 4 + 1) * kRtcRows + r], m.y, acc);
-      acc = fmaf(qf[(d4 * 4 + 2) * kRtcRows + r], m.z, acc);
-      acc = fmaf(qf[(d4 * 4 + 3) * kRtcRows + r], m.w, acc);
-    }
-    return acc;
-  };
-  auto flush = [&]() {
-    int rounds = nq;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-      rounds = max(rounds, __shfl_xor_sync(0xffffffffu, rounds, off));
-    for (int t = 0; t < rounds; t += 2) {
-      const bool h0 = t < nq, h1 = t + 1 < nq;
-      const int c0 = h0 ? qlist[t * kRtcRows + r] : 0;
-      const int c1 = h1 ? qlist[(t + 1) * kRtcRows + r] : c0;
-      float s0 = 0.f, s1 = 0.f;
-      if (h0) s0 = rescore(c0);
-      if (h1) s1 = rescore(c1);
-      if (h0) {
-        const uint64_t key = route_key(s0, c0);
-        if (key > keys[KM - 1]) sorted_insert<KM>(keys, key);
+      for (int j = 0; j < KM; ++j) {
+        const bool real = (j >= KM - k) && keys[j] != 0ull;
+        sel[j] = real ? static_cast<int>(~static_cast<uint32_t>(keys[j] & 0xFFFFFFFFull)) : 0x7FFFFFFF;
+        n += real ? 1 : 0;
       }
-      if (h1) {
-        const uint64_t key = route_key(s1, c1);
-        if (key > keys[KM - 1]) sorted_insert<KM>(keys, key);
-      }
-    }
-    nq = 0;
-    // once k exact candidates are known, the k-th exact score bounds the rest
-    if (keys[KM - 1] != 0ull && keys[KM - 1] != ~0ull)
-      filt = fmaxf(filt, key_score(keys[KM - 1]) - slack);
-  };
-  for (int tile = 0; tile < n_tiles; ++tile) {
-    run_tile(tile, [&](int cb, const uint32_t (&sv)[32], const float* nc, bool full) {
-      uint32_t m = 0u;
-      if (cb < lim) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const bool adm = full || (cb + j < lim);
-          if (adm && fmaf(e_row, nc[j], __uint_as_float(sv[j])) >= filt) m |= 1u << j;
+      for (int x = 1; x < KM; ++x) {
+#pragma unroll
+        for (int y = x; y > 0; --y) {
+          const int lo = min(sel[y - 1], sel[y]), hi = max(sel[y - 1], sel[y]);
+          sel[y - 1] = lo;
+          sel[y] = hi;
         }
       }
-      // flush (warp-uniform) only when a queue would overflow
-      if (__any_sync(0xffffffffu, nq + __popc(m) > kRtcCap)) flush();
-      while (m) {
-        const int j = __ffs(m) - 1;
-        m &= m - 1;
-        qlist[nq * kRtcRows + r] = static_cast<uint16_t>(cb + j);
-        ++nq;
-      }
-    });
-  }
-  if (is_row) flush();
-
-  // output: the real entries, ascending by block index
-  if (is_row && qb < a.NQB) {
-    int sel[KM];
-    int n = 0;
+      int32_t* dst = a.idx + (static_cast<int64_t>(bh) * a.NQB + qb) * k;
 #pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      const bool real = (j >= KM - k) && keys[j] != 0ull;
-      sel[j] = real ? static_cast<int>(~static_cast<uint32_t>(keys[j] & 0xFFFFFFFFull)) : 0x7FFFFFFF;
-      n += real ? 1 : 0;
+      for (int j = 0; j < KM; ++j)
+        if (j < k) dst[j] = j < n ? sel[j] : -1;
+      a.cnt[static_cast<int64_t>(bh) * a.NQB + qb] = n;
     }
-#pragma unroll
-    for (int x = 1; x < KM; ++x) {
-#pragma unroll
-      for (int y = x; y > 0; --y) {
-        const int lo = min(sel[y - 1], sel[y]), hi = max(sel[y - 1], sel[y]);
-        sel[y - 1] = lo;
-        sel[y] = hi;
-      }
-    }
-    int32_t* dst = a.idx + (static_cast<int64_t>(bh) * a.NQB + qb) * k;
-#pragma unroll
-    for (int j = 0; j < KM; ++j)
-      if (j < k) dst[j] = j < n ? sel[j] : -1;
-    a.cnt[static_cast<int64_t>(bh) * a.NQB + qb] = n;
   }
 
   tc_fence_before();
