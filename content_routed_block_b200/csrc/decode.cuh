@@ -6,7 +6,7 @@
 // top_k (score desc, index asc), and reads exact softmax over the routed
 // blocks' keys united with the window i - W < j <= i, cut at i.
 //
-// B200 design (flash-decoding with routing in front; three launches):
+// B200 design (flash-decoding with routing in front; two launches):
 //  * decode_route_kernel: grid (candidate splits, b * KV head).  One warp per
 //    query head of the group (the group's block means are read once per CTA
 //    and hit L1 for the other heads); lanes take strided candidates and keep
@@ -19,9 +19,10 @@
 //    keys into the top_k, lays the key set out as the routed blocks' keys
 //    below the window followed by the window, and runs an online softmax in
 //    the exp2 domain over its share: 32 keys per warp step with lanes = keys
-//    for q.k, then lanes = dims for p.v.  Writes a partial (m, l, o).
-//  * decode_combine_kernel: merges the key splits' partials, writes O (bf16)
-//    and the natural-log LSE.
+//    for q.k, then lanes = dims for p.v.  Writes a partial (m, l, o); the
+//    last split of a head to finish (counted atomically; the route kernel
+//    zeroes the counts) merges the partials and writes O (bf16) and the
+//    natural-log LSE.
 // The work is memory-bound: the block means of the admissible blocks
 // (A * D * 4 bytes per KV head) and the gathered K/V rows (k*Bk + W rows per
 // head).
@@ -42,6 +43,7 @@ struct DecodeArgs {
   float* ksum;              // [B*Hkv, Ncap/Bk, D] (in / out)
   uint64_t* part_keys;      // [B*Hq, S, KM]
   float* part_attn;         // [B*Hq, KS, D + 2]: m, l, o
+  uint32_t* done;           // [B*Hq] key splits finished (zeroed by the route kernel)
   __nv_bfloat16* o;         // [B*Hq, D]
   float* lse;               // [B*Hq] or null
   int32_t* idx;             // [B*Hq, top_k] or null
@@ -74,6 +76,7 @@ __global__ void __launch_bounds__(kDecThreads, (KM <= 16) ? 2 : 1) decode_route_
   const int nc = max(0, c1 - c0);
   float* qs = dec_smem;                       // [g][D]
   float* sc = dec_smem + g * D;               // [g][cands_per_split]
+  if (s == 0 && tid < g) a.done[static_cast<int64_t>(b) * a.Hq + kv * g + tid] = 0u;
   float* ksum = a.ksum + static_cast<int64_t>(bkv) * (a.Ncap / a.Bk) * D;
   // the newest admissible block's mean (its last key is i - 1 or earlier):
   // thread t sums rows t / D, t / D + 256 / D, ... of column t % D (the loads
@@ -398,38 +401,43 @@ __global__ void __launch_bounds__(kDecThreads) decode_attend_kernel(const Decode
     }
 #pragma unroll
     for (int d = 0; d < DL; ++d) dst[2 + lane + 32 * d] = oo[d];
+    // 4. the last key split of this head to finish merges all splits'
+    // partials and writes O and the LSE: each split's partial is visible
+    // device-wide before its count, and the last one sees every count
+    __threadfence();
+    __syncwarp();
+    uint32_t prev = 0;
+    if (lane == 0) prev = atomicAdd(&a.done[bh], 1u);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev == static_cast<uint32_t>(a.KS - 1)) {
+      __threadfence();
+      const volatile float* src = a.part_attn + static_cast<int64_t>(bh) * a.KS * (D + 2);
+      float Mx = -INFINITY;
+      for (int y = 0; y < a.KS; ++y) Mx = fmaxf(Mx, src[y * (D + 2)]);
+      float L = 0.f;
+      float acc[DL];
+#pragma unroll
+      for (int d = 0; d < DL; ++d) acc[d] = 0.f;
+      for (int y = 0; y < a.KS; ++y) {
+        const float my = src[y * (D + 2)];
+        const float f = (my == -INFINITY) ? 0.f : exp2f(my - Mx);
+        L += src[y * (D + 2) + 1] * f;
+#pragma unroll
+        for (int d = 0; d < DL; ++d) acc[d] += src[y * (D + 2) + 2 + lane + 32 * d] * f;
+      }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+      for (int d = 0; d < DL; ++d)
+        a.o[static_cast<int64_t>(bh) * D + lane + 32 * d] = __float2bfloat16_rn(acc[d] * inv);
+      if (lane == 0 && a.lse != nullptr)
+        a.lse[bh] = L > 0.f ? (Mx + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
+    }
   }
 }
 
 template <int D>
 __host__ __device__ constexpr size_t decode_attend_smem() {
   return static_cast<size_t>(kDecThreads / 32) * 32 * D * 2;
-}
-
-template <int D>
-__global__ void __launch_bounds__(32) decode_combine_kernel(const DecodeArgs a) {
-  constexpr int DL = D / 32;
-  const int bh = blockIdx.x, lane = threadIdx.x;
-  const float* src = a.part_attn + static_cast<int64_t>(bh) * a.KS * (D + 2);
-  float M = -INFINITY;
-  for (int x = 0; x < a.KS; ++x) M = fmaxf(M, src[x * (D + 2)]);
-  float L = 0.f;
-  float o[DL];
-#pragma unroll
-  for (int d = 0; d < DL; ++d) o[d] = 0.f;
-  for (int x = 0; x < a.KS; ++x) {
-    const float mx = src[x * (D + 2)];
-    const float f = (mx == -INFINITY) ? 0.f : exp2f(mx - M);
-    L += src[x * (D + 2) + 1] * f;
-#pragma unroll
-    for (int d = 0; d < DL; ++d) o[d] += src[x * (D + 2) + 2 + lane + 32 * d] * f;
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-  for (int d = 0; d < DL; ++d)
-    a.o[static_cast<int64_t>(bh) * D + lane + 32 * d] = __float2bfloat16_rn(o[d] * inv);
-  if (lane == 0 && a.lse != nullptr)
-    a.lse[bh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
 }
 
 }  // namespace ssa

@@ -767,7 +767,8 @@ int decode_km(int32_t top_k) { return top_k <= 8 ? 8 : top_k <= 16 ? 16 : top_k 
 size_t decode_ws_bytes(const ssa_params* p) {
   const size_t heads = static_cast<size_t>(p->B) * p->Hq;
   return align256(heads * ssa::kDecMaxSplits * decode_km(p->top_k) * sizeof(uint64_t)) +
-         align256(heads * ssa::kDecMaxSplits * (p->D + 2) * sizeof(float));
+         align256(heads * ssa::kDecMaxSplits * (p->D + 2) * sizeof(float)) +
+         align256(heads * sizeof(uint32_t));
 }
 
 ssa_status validate_decode(const ssa_params* p) {
@@ -797,8 +798,6 @@ cudaError_t launch_decode_t(const ssa::DecodeArgs& a, int B, cudaStream_t stream
                            cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(as));
   if (e != cudaSuccess) return e;
   ssa::decode_attend_kernel<D, KM><<<dim3(a.KS, B * a.Hq), ssa::kDecThreads, as, stream>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  ssa::decode_combine_kernel<D><<<B * a.Hq, 32, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -1252,8 +1251,10 @@ ssa_status ssa_decode(const ssa_params* p, const void* q, const void* k_cache, c
   const size_t heads = static_cast<size_t>(p->B) * p->Hq;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.part_keys = reinterpret_cast<uint64_t*>(ws);
-  a.part_attn = reinterpret_cast<float*>(
-      ws + align256(heads * ssa::kDecMaxSplits * decode_km(p->top_k) * sizeof(uint64_t)));
+  const size_t keys_bytes = align256(heads * ssa::kDecMaxSplits * decode_km(p->top_k) * sizeof(uint64_t));
+  a.part_attn = reinterpret_cast<float*>(ws + keys_bytes);
+  a.done = reinterpret_cast<uint32_t*>(
+      ws + keys_bytes + align256(heads * ssa::kDecMaxSplits * (p->D + 2) * sizeof(float)));
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.idx = idx_out;

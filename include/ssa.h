@@ -338,8 +338,11 @@ size_t ssa_decode_workspace_size(const ssa_params* p);
  *   o          bf16 [B, Hq, D] (device, out); lse fp32 [B, Hq] (nullable)
  *   idx_out    int32 [B, Hq, top_k] (nullable): the selection, ascending,
  *              -1 padded; cnt_out int32 [B, Hq] (nullable)
- *   workspace  ssa_decode_workspace_size(p) bytes (device, 256-byte aligned)
- * Three launches (routing splits, attend splits, combine). */
+ *   workspace  ssa_decode_workspace_size(p) bytes (device, 256-byte aligned):
+ *              the splits' partial lists and reads and one counter per
+ *              (b, query head); nothing needs clearing between calls
+ * Two launches: the routing splits, then the attend splits, of which the
+ * last to finish for a head merges the splits' reads and writes o and lse. */
 ssa_status ssa_decode(const ssa_params* p, const void* q, const void* k_cache, const void* v_cache,
                       int32_t n_ctx, float* ksum_cache, void* o, float* lse, int32_t* idx_out,
                       int32_t* cnt_out, void* workspace, size_t workspace_bytes,
