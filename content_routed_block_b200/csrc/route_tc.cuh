@@ -126,9 +126,9 @@ __device__ __forceinline__ void sorted_insert(T (&arr)[KM], T v) {
 
 // Warp roles: warps 0-3 are the rows (thread r = query block qb0 + r = TMEM
 // lane r) and scan every tile's scores; warps 4-7 stage the key-summary tiles
-// (one thread per key block: load, split into bf16 hi / lo, norm) into one of
-// two stages, and their first thread issues the tile's three MMAs into one of
-// two TMEM accumulators.  The tiles of both passes form one stream, so the
+// (eight lanes per key block: load, split into bf16 hi / lo, norm) into one of
+// two stages, and thread 128 issues the tile's three MMAs into one of two
+// TMEM accumulators.  The tiles of both passes form one stream, so the
 // staging of the next tiles overlaps the scan of the current one.  Barriers:
 // acc_full[b] (MMAs of a tile into accumulator b done), acc_empty[b] (the rows
 // have read accumulator b and the norms of stage b).
@@ -208,30 +208,45 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
 
   if (warp >= 4) {
     // ------------------------------------------------ key-summary stagers
-    const int sid = tid - kRtcRows;   // key row of the tile
+    // warp w stages key rows 32(w-4) .. +31, four rows per step: lane = (row
+    // of the four, 16-byte bf16 chunk g), so one load instruction covers four
+    // consecutive rows (one contiguous span for D = 64) instead of 32 rows
+    const int lane = tid & 31;
+    const int g0 = lane & 7, rsub = lane >> 3;
+    const int rbase = (warp - 4) * 32 + rsub;
     for (int t = 0; t < total; ++t) {
       const int st = t & 1;
       if (t >= 2) mbar_wait(&bar_empty[st], ((t - 2) >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
       const int c0 = (t % n_tiles) * NT;
-      const bool ok = c0 + sid < a.NB;
-      const float* src = ksrc + static_cast<int64_t>(c0 + sid) * D;
-      float sq = 0.f;
+#pragma unroll 4
+      for (int i = 0; i < 8; ++i) {
+        const int row = rbase + i * 4;
+        const bool ok = c0 + row < a.NB;
+        const float* src = ksrc + static_cast<int64_t>(c0 + row) * D;
+        float sq = 0.f;
 #pragma unroll
-      for (int g = 0; g < D / 8; ++g) {
-        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-        if (ok) {
-          v0 = *reinterpret_cast<const float4*>(src + g * 8);
-          v1 = *reinterpret_cast<const float4*>(src + g * 8 + 4);
+        for (int hh = 0; hh < D / 64; ++hh) {
+          const int g = hh * 8 + g0;
+          float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+          if (ok) {
+            v0 = *reinterpret_cast<const float4*>(src + g * 8);
+            v1 = *reinterpret_cast<const float4*>(src + g * 8 + 4);
+          }
+          uint4 hi, lo;
+          split8_bf16(v0, v1, hi, lo, sq);
+          *reinterpret_cast<uint4*>(smem + Lay::kh(st) + sw128_offset(row, g, Lay::HALF_K)) = hi;
+          *reinterpret_cast<uint4*>(smem + Lay::kl(st) + sw128_offset(row, g, Lay::HALF_K)) = lo;
         }
-        uint4 hi, lo;
-        split8_bf16(v0, v1, hi, lo, sq);
-        *reinterpret_cast<uint4*>(smem + Lay::kh(st) + sw128_offset(sid, g, Lay::HALF_K)) = hi;
-        *reinterpret_cast<uint4*>(smem + Lay::kl(st) + sw128_offset(sid, g, Lay::HALF_K)) = lo;
+        // the row's sum of squares over its 8 (or 16) chunks: the summation
+        // order differs from a sequential one by far less than the 1.001 slack
+        sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+        if (g0 == 0) nrm[st * NT + row] = sqrtf(sq) * 1.001f;
       }
-      nrm[st * NT + sid] = sqrtf(sq) * 1.001f;
       fence_proxy_async_smem();
       asm volatile("bar.sync 1, 128;" ::: "memory");   // the stagers only
-      if (sid == 0) {
+      if (tid == kRtcRows) {
         tc_fence_after();
         const uint32_t oq[3] = {Lay::OFF_QH, Lay::OFF_QH, Lay::OFF_QL};
         const uint32_t okk[3] = {Lay::kh(st), Lay::kl(st), Lay::kh(st)};
@@ -306,11 +321,14 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
           if (cb >= lim) return;
           float gmax = -INFINITY, gn = 0.f;
           if (full) {
+            // four partial maxima keep the dependent chain short (max is exact)
+            float gm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              gmax = fmaxf(gmax, fmaf(-e_row, nc[j], __uint_as_float(sv[j])));
+              gm[j & 3] = fmaxf(gm[j & 3], fmaf(-e_row, nc[j], __uint_as_float(sv[j])));
               gn = fmaxf(gn, nc[j]);
             }
+            gmax = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -335,40 +353,53 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     const float slack = e_row * nmax * 0.5f;  // >= (eps / 2) ||qbar|| max ||mu||
     float filt = L - slack;
     int nq = 0;
-    // the exact fp32 score: sequential fmaf over d, the FMA router's arithmetic
-    auto rescore = [&](int c) -> float {
-      const float4* mu = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(c) * D);
+    // the exact fp32 scores of up to four candidates: per candidate a
+    // sequential fmaf over d (the FMA router's arithmetic); the four share
+    // each load of the row's query summary
+    auto rescore4 = [&](const int (&c)[4], const bool (&h)[4], float (&s)[4]) {
       const float4* qv = reinterpret_cast<const float4*>(qrow);
-      float acc = 0.f;
-#pragma unroll 4
-      for (int d4 = 0; d4 < D / 4; ++d4) {
-        const float4 m = mu[d4], q = qv[d4];
-        acc = fmaf(q.x, m.x, acc);
-        acc = fmaf(q.y, m.y, acc);
-        acc = fmaf(q.z, m.z, acc);
-        acc = fmaf(q.w, m.w, acc);
+      const float4* mu[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        mu[u] = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(c[u]) * D);
+        s[u] = 0.f;
       }
-      return acc;
+#pragma unroll 2
+      for (int d4 = 0; d4 < D / 4; ++d4) {
+        const float4 q = qv[d4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (h[u]) {
+            const float4 m = mu[u][d4];
+            s[u] = fmaf(q.x, m.x, s[u]);
+            s[u] = fmaf(q.y, m.y, s[u]);
+            s[u] = fmaf(q.z, m.z, s[u]);
+            s[u] = fmaf(q.w, m.w, s[u]);
+          }
+        }
+      }
     };
     auto flush = [&]() {
       int rounds = nq;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1)
         rounds = max(rounds, __shfl_xor_sync(0xffffffffu, rounds, off));
-      for (int t = 0; t < rounds; t += 2) {
-        const bool h0 = t < nq, h1 = t + 1 < nq;
-        const int c0 = h0 ? qlist[t * kRtcRows + r] : 0;
-        const int c1 = h1 ? qlist[(t + 1) * kRtcRows + r] : c0;
-        float s0 = 0.f, s1 = 0.f;
-        if (h0) s0 = rescore(c0);
-        if (h1) s1 = rescore(c1);
-        if (h0) {
-          const uint64_t key = route_key(s0, c0);
-          if (key > keys[KM - 1]) sorted_insert<KM>(keys, key);
+      for (int t = 0; t < rounds; t += 4) {
+        int c[4];
+        bool h[4];
+        float sc[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          h[u] = t + u < nq;
+          c[u] = h[u] ? qlist[(t + u) * kRtcRows + r] : 0;
         }
-        if (h1) {
-          const uint64_t key = route_key(s1, c1);
-          if (key > keys[KM - 1]) sorted_insert<KM>(keys, key);
+        rescore4(c, h, sc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (h[u]) {
+            const uint64_t key = route_key(sc[u], c[u]);
+            if (key > keys[KM - 1]) sorted_insert<KM>(keys, key);
+          }
         }
       }
       nq = 0;
