@@ -35,6 +35,27 @@ namespace ssa {
 
 constexpr int kDecThreads = 256;
 constexpr int kDecMaxSplits = 128;
+constexpr int kDecSurvivors = 64;   // keys a fast selection sorts (two per lane)
+
+// bitonic sort of 64 keys, element e = lane + 32 h (x0: h = 0, x1: h = 1),
+// descending over e: both halves sorted, the second reversed (the 64 form a
+// bitonic sequence), one exchange at distance 32, then each half merged
+__device__ __forceinline__ void warp_sort64_desc(uint64_t& x0, uint64_t& x1, int lane) {
+  x0 = warp_sort_desc(x0, lane);
+  x1 = warp_sort_desc(x1, lane);
+  const uint64_t r1 = __shfl_sync(0xffffffffu, x1, 31 - lane);
+  uint64_t a = umax64(x0, r1), b = umin64(x0, r1);
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const uint64_t ya = __shfl_xor_sync(0xffffffffu, a, j);
+    const uint64_t yb = __shfl_xor_sync(0xffffffffu, b, j);
+    const bool low = (lane & j) == 0;
+    a = low ? umax64(a, ya) : umin64(a, ya);
+    b = low ? umax64(b, yb) : umin64(b, yb);
+  }
+  x0 = a;
+  x1 = b;
+}
 
 struct DecodeArgs {
   const __nv_bfloat16* q;   // [B*Hq, D]
@@ -134,8 +155,11 @@ __global__ void __launch_bounds__(kDecThreads, (KM <= 16) ? 2 : 1) decode_route_
   __syncthreads();
 
   // 2. per head, the top KM of the split: a lower bound L from the lanes'
-  //    maxima (the KM-th largest of them is reached by >= KM candidates)
-  //    admits few candidates into the per-lane register lists
+  //    maxima (the KM-th largest of them is reached by >= KM candidates).
+  //    The candidates at or above L hold the top KM; when at most 64 do, the
+  //    warp compacts them and sorts them (the usual case), otherwise they go
+  //    through per-lane register lists and shuffle merges
+  __shared__ uint64_t surv[NW][kDecSurvivors];
   for (int j = warp; j < g; j += NW) {
     const int bh = b * a.Hq + kv * g + j;
     const float* sj = sc + j * a.cands_per_split;
@@ -157,6 +181,33 @@ __global__ void __launch_bounds__(kDecThreads, (KM <= 16) ? 2 : 1) decode_route_
       }
       L = __shfl_sync(0xffffffffu, x, KM - 1);
     }
+    uint64_t* dst = a.part_keys + (static_cast<int64_t>(bh) * a.S + s) * KM;
+    if (KM <= 32 && a.top_k > 0) {
+      int nsv = 0;
+      for (int r0 = 0; r0 < nc; r0 += 32) {
+        const int r = r0 + lane;
+        const float v = r < nc ? sj[r] : 0.f;
+        const bool take = r < nc && v >= L;
+        const uint32_t bal = __ballot_sync(0xffffffffu, take);
+        const int pos = nsv + __popc(bal & ((1u << lane) - 1u));
+        if (take && pos < kDecSurvivors) surv[warp][pos] = route_key(v, c0 + r);
+        nsv += __popc(bal);
+      }
+      __syncwarp();
+      if (nsv <= kDecSurvivors) {
+        uint64_t x0 = lane < nsv ? surv[warp][lane] : 0ull;
+        if (nsv <= 32) {
+          x0 = warp_sort_desc(x0, lane);
+        } else {
+          uint64_t x1 = lane + 32 < nsv ? surv[warp][lane + 32] : 0ull;
+          warp_sort64_desc(x0, x1, lane);
+        }
+        __syncwarp();
+        if (lane < KM) dst[lane] = x0;   // zeros past the split's candidates
+        continue;
+      }
+      __syncwarp();
+    }
     uint64_t keys[KM];
 #pragma unroll
     for (int e = 0; e < KM; ++e) keys[e] = 0ull;
@@ -172,7 +223,6 @@ __global__ void __launch_bounds__(kDecThreads, (KM <= 16) ? 2 : 1) decode_route_
 #pragma unroll
     for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);
     if (lane == 0) {
-      uint64_t* dst = a.part_keys + (static_cast<int64_t>(bh) * a.S + s) * KM;
 #pragma unroll
       for (int e = 0; e < KM; ++e) dst[e] = keys[e];
     }
@@ -198,35 +248,85 @@ __global__ void __launch_bounds__(kDecThreads) decode_attend_kernel(const Decode
   const int lo = max(0, i - a.window + 1);
 
   for (int d = tid; d < D; d += kDecThreads) qs[d] = __bfloat162float(a.q[static_cast<int64_t>(bh) * D + d]);
-  // 1. merge the splits' keys (warp 0) and list the selection ascending
+  // 1. the top_k of the splits' keys, listed ascending.  Each split's list is
+  //    sorted descending, so L = the largest of the splits' top_k-th keys is
+  //    reached by top_k keys of one split: the selection lies among the keys
+  //    >= L, and only in the first top_k entries of each list.  When at most
+  //    64 keys pass (the usual case) the whole CTA collects them and warp 0
+  //    sorts them; otherwise warp 0 merges the lists.
+  __shared__ uint64_t surv[kDecSurvivors];
+  __shared__ uint64_t wmax[NW];
+  __shared__ int n_surv;
+  bool fast = false;
+  if constexpr (KM <= 32) {
+    if (a.top_k > 0) {
+      const uint64_t* lists = a.part_keys + static_cast<int64_t>(bh) * a.S * KM;
+      uint64_t kth = 0ull;
+      for (int sp = tid; sp < a.S; sp += kDecThreads) kth = umax64(kth, lists[sp * KM + a.top_k - 1]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) kth = umax64(kth, __shfl_xor_sync(0xffffffffu, kth, off));
+      if (lane == 0) wmax[warp] = kth;
+      if (tid == 0) n_surv = 0;
+      __syncthreads();
+      uint64_t L = wmax[0];
+#pragma unroll
+      for (int w = 1; w < NW; ++w) L = umax64(L, wmax[w]);
+      const int total = a.S * a.top_k;
+      for (int e = tid; e < total; e += kDecThreads) {
+        const int sp = e / a.top_k, jj = e - sp * a.top_k;
+        const uint64_t key = lists[sp * KM + jj];
+        if (key != 0ull && key >= L) {
+          const int pos = atomicAdd(&n_surv, 1);
+          if (pos < kDecSurvivors) surv[pos] = key;
+        }
+      }
+      __syncthreads();
+      fast = n_surv <= kDecSurvivors;
+    } else {
+      fast = true;   // nothing is routed
+    }
+  }
   if (warp == 0) {
     uint64_t keys[KM];
 #pragma unroll
     for (int j = 0; j < KM; ++j) keys[j] = 0ull;
-    // lane l folds splits l, l + 32, ... (each sorted descending) into its
-    // list with in-register bitonic merges; the shuffle merges then keep the
-    // top KM of all of them
-    for (int sp = lane; sp < a.S; sp += 32) {
-      const uint64_t* src = a.part_keys + (static_cast<int64_t>(bh) * a.S + sp) * KM;
-      uint64_t other[KM];
+    uint64_t mine = 0ull;
+    int n = 0;
+    if (fast) {
+      const int ns = a.top_k > 0 ? n_surv : 0;
+      uint64_t x0 = lane < ns ? surv[lane] : 0ull;
+      if (ns <= 32) {
+        x0 = warp_sort_desc(x0, lane);
+      } else {
+        uint64_t x1 = lane + 32 < ns ? surv[lane + 32] : 0ull;
+        warp_sort64_desc(x0, x1, lane);
+      }
+      mine = (lane < a.top_k) ? x0 : 0ull;
+      n = __popc(__ballot_sync(0xffffffffu, mine != 0ull));
+    } else {
+      // lane l folds splits l, l + 32, ... (each sorted descending) into its
+      // list with in-register bitonic merges; the shuffle merges then keep
+      // the top KM of all of them
+      for (int sp = lane; sp < a.S; sp += 32) {
+        const uint64_t* src = a.part_keys + (static_cast<int64_t>(bh) * a.S + sp) * KM;
+        uint64_t other[KM];
 #pragma unroll
-      for (int j = 0; j < KM; ++j) other[j] = src[j];
-      route_merge_lists<KM>(keys, other);
-    }
+        for (int j = 0; j < KM; ++j) other[j] = src[j];
+        route_merge_lists<KM>(keys, other);
+      }
 #pragma unroll
-    for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);
-    if constexpr (KM <= 32) {
-      // every lane now holds the top KM; lane j takes entry j (j < top_k), the
-      // warp sorts the block indices ascending and scans the far-segment
-      // lengths (the part of each routed block below the window)
-      int n = 0;
-      uint64_t mine = 0ull;
+      for (int mask = 1; mask < 32; mask <<= 1) route_merge_partner<KM>(keys, mask);
+      // every lane now holds the top KM; lane j takes entry j (j < top_k)
 #pragma unroll
       for (int j = 0; j < KM; ++j) {
         const bool real = j < a.top_k && keys[j] != 0ull;
         n += real ? 1 : 0;
         if (j == lane) mine = real ? keys[j] : 0ull;
       }
+    }
+    if constexpr (KM <= 32) {
+      // the warp sorts the selected block indices ascending and scans the
+      // far-segment lengths (the part of each routed block below the window)
       int c = mine != 0ull ? static_cast<int>(~static_cast<uint32_t>(mine & 0xFFFFFFFFull)) : 0x7FFFFFFF;
 #pragma unroll
       for (int k = 2; k <= 32; k <<= 1) {

@@ -142,3 +142,39 @@ def test_decode_million_token_cache_sampled():
     c = Cache(w)
     for n_ctx in (w.N, w.N - 4097, 300_001):
         check_step(c, n_ctx, *c.step(n_ctx))
+
+
+def _tied_cache(w, period_blocks, seed):
+    """Keys whose block means repeat every ``period_blocks`` blocks (a
+    constant cache for period 1): small integer keys, so every block mean is
+    exact in fp32 whatever the summation order, and equal means give exactly
+    equal scores on both sides."""
+    from content_routed_block_b200.workloads import to_bf16_bits
+    rng = np.random.default_rng(seed)
+    span = period_blocks * w.block_k
+    base = rng.integers(-2, 3, size=(w.B, w.Hkv, span, w.D)).astype(np.float32)
+    k = np.tile(base, (1, 1, w.N // span + 1, 1))[:, :, :w.N]
+    x = make_inputs(w)
+    x["k"] = to_bf16_bits(k)
+    return x
+
+
+def test_decode_selection_when_ties_defeat_the_fast_paths():
+    # Each routing split normally passes at most 64 keys to a sort; these
+    # caches push both kernels onto their merge paths and the result must not
+    # change.  (a) A constant cache: every score of a split ties, so all of a
+    # split's candidates (111 of them here: 8 KV heads give 37 splits of
+    # 4096 blocks) reach the split's threshold.  (b) Block means that repeat
+    # with the split length (32 blocks): every split holds the same scores, so
+    # about 7 keys of each of 16 splits reach the merge threshold.  Exact ties
+    # go to the lower block index on both sides.
+    wa = W("tied-constant", B=1, Hq=8, Hkv=8, N=4096 * 16 + 16, block_k=16, block_q=16,
+           top_k=8, window=32)
+    ca = Cache(wa, _tied_cache(wa, 1, 5))
+    for n_ctx in (wa.N, wa.N - 700):
+        check_step(ca, n_ctx, *ca.step(n_ctx))
+    wb = W("tied-periodic", B=1, Hq=2, Hkv=1, N=512 * 16 + 16, block_k=16, block_q=16,
+           top_k=8, window=32)
+    cb = Cache(wb, _tied_cache(wb, 32, 6))
+    for n_ctx in (wb.N, wb.N - 16 * 32):
+        check_step(cb, n_ctx, *cb.step(n_ctx))
