@@ -214,49 +214,68 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     const int lane = tid & 31;
     const int g0 = lane & 7, rsub = lane >> 3;
     const int rbase = (warp - 4) * 32 + rsub;
+    constexpr int RB = D == 64 ? 8 : 4;      // rows of a batch, all loads in flight
+    constexpr int HH = D / 64;               // 64-column halves of a row
+    // the descriptors of the Q parts and of stage 0's key parts; the other
+    // operands are these plus a shared-memory offset (>> 4 in the low field)
+    const uint64_t dq_hi = sdesc_sw128(sbase + Lay::OFF_QH, 16, 1024);
+    const uint64_t dq_lo = sdesc_sw128(sbase + Lay::OFF_QL, 16, 1024);
+    const uint64_t dk0 = sdesc_sw128(sbase + Lay::kh(0), 16, 1024);
     for (int t = 0; t < total; ++t) {
       const int st = t & 1;
-      if (t >= 2) mbar_wait(&bar_empty[st], ((t - 2) >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
       const int c0 = (t % n_tiles) * NT;
-#pragma unroll 4
-      for (int i = 0; i < 8; ++i) {
-        const int row = rbase + i * 4;
-        const bool ok = c0 + row < a.NB;
-        const float* src = ksrc + static_cast<int64_t>(c0 + row) * D;
-        float sq = 0.f;
+#pragma unroll 1
+      for (int i0 = 0; i0 < 8; i0 += RB) {
+        float4 va[RB][HH], vb[RB][HH];
 #pragma unroll
-        for (int hh = 0; hh < D / 64; ++hh) {
-          const int g = hh * 8 + g0;
-          float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-          if (ok) {
-            v0 = *reinterpret_cast<const float4*>(src + g * 8);
-            v1 = *reinterpret_cast<const float4*>(src + g * 8 + 4);
+        for (int i = 0; i < RB; ++i) {
+          const int row = rbase + (i0 + i) * 4;
+          const bool ok = c0 + row < a.NB;
+          const float* src = ksrc + static_cast<int64_t>(c0 + row) * D;
+#pragma unroll
+          for (int hh = 0; hh < HH; ++hh) {
+            const int g = hh * 8 + g0;
+            va[i][hh] = ok ? *reinterpret_cast<const float4*>(src + g * 8) : make_float4(0.f, 0.f, 0.f, 0.f);
+            vb[i][hh] = ok ? *reinterpret_cast<const float4*>(src + g * 8 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
-          uint4 hi, lo;
-          split8_bf16(v0, v1, hi, lo, sq);
-          *reinterpret_cast<uint4*>(smem + Lay::kh(st) + sw128_offset(row, g, Lay::HALF_K)) = hi;
-          *reinterpret_cast<uint4*>(smem + Lay::kl(st) + sw128_offset(row, g, Lay::HALF_K)) = lo;
         }
-        // the row's sum of squares over its 8 (or 16) chunks: the summation
-        // order differs from a sequential one by far less than the 1.001 slack
-        sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-        sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-        sq += __shfl_xor_sync(0xffffffffu, sq, 4);
-        if (g0 == 0) nrm[st * NT + row] = sqrtf(sq) * 1.001f;
+        // the stage is rewritten only after the rows have read it (the
+        // loads above are already in flight)
+        if (i0 == 0 && t >= 2) mbar_wait(&bar_empty[st], ((t - 2) >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
+#pragma unroll
+        for (int i = 0; i < RB; ++i) {
+          const int row = rbase + (i0 + i) * 4;
+          float sq = 0.f;
+#pragma unroll
+          for (int hh = 0; hh < HH; ++hh) {
+            const int g = hh * 8 + g0;
+            uint4 hi, lo;
+            split8_bf16(va[i][hh], vb[i][hh], hi, lo, sq);
+            *reinterpret_cast<uint4*>(smem + Lay::kh(st) + sw128_offset(row, g, Lay::HALF_K)) = hi;
+            *reinterpret_cast<uint4*>(smem + Lay::kl(st) + sw128_offset(row, g, Lay::HALF_K)) = lo;
+          }
+          // the row's sum of squares over its 8 (or 16) chunks: the summation
+          // order differs from a sequential one by far less than the 1.001 slack
+          sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+          sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+          sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+          if (g0 == 0) nrm[st * NT + row] = sqrtf(sq) * 1.001f;
+        }
       }
       fence_proxy_async_smem();
       asm volatile("bar.sync 1, 128;" ::: "memory");   // the stagers only
       if (tid == kRtcRows) {
         tc_fence_after();
-        const uint32_t oq[3] = {Lay::OFF_QH, Lay::OFF_QH, Lay::OFF_QL};
-        const uint32_t okk[3] = {Lay::kh(st), Lay::kl(st), Lay::kh(st)};
+        const uint64_t dk_st = dk0 + ((st * 2 * Lay::K_BYTES) >> 4);
+        const uint64_t da[3] = {dq_hi, dq_hi, dq_lo};
+        const uint64_t db[3] = {dk_st, dk_st + (Lay::K_BYTES >> 4), dk_st};
 #pragma unroll
         for (int term = 0; term < 3; ++term) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t qa = sbase + oq[term] + (kk / 4) * Lay::HALF_Q + (kk % 4) * 32;
-            const uint32_t kb = sbase + okk[term] + (kk / 4) * Lay::HALF_K + (kk % 4) * 32;
-            mma_ss(tmem + st * NT, sdesc_sw128(qa, 16, 1024), sdesc_sw128(kb, 16, 1024), IDESC,
+            const uint64_t qoff = ((kk / 4) * Lay::HALF_Q + (kk % 4) * 32) >> 4;
+            const uint64_t koff = ((kk / 4) * Lay::HALF_K + (kk % 4) * 32) >> 4;
+            mma_ss(tmem + st * NT, da[term] + qoff, db[term] + koff, IDESC,
                    (term > 0 || kk > 0) ? 1u : 0u);
           }
         }
@@ -319,25 +338,26 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
       for (int t = 0; t < n_tiles; ++t) {
         scan_tile(t, [&](int cb, const uint32_t (&sv)[32], const float* nc, bool full) {
           if (cb >= lim) return;
-          float gmax = -INFINITY, gn = 0.f;
-          if (full) {
-            // four partial maxima keep the dependent chain short (max is exact)
-            float gm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          // branch-free: inadmissible columns count as -inf (and norm 0);
+          // four partial maxima keep the dependent chain short (max is exact)
+          const int nadm = full ? 32 : lim - cb;
+          const float4* nc4 = reinterpret_cast<const float4*>(nc);
+          float gm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          float gq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              gm[j & 3] = fmaxf(gm[j & 3], fmaf(-e_row, nc[j], __uint_as_float(sv[j])));
-              gn = fmaxf(gn, nc[j]);
-            }
-            gmax = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
-          } else {
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 n4 = nc4[j4];
+            const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (cb + j < lim) {
-                gmax = fmaxf(gmax, fmaf(-e_row, nc[j], __uint_as_float(sv[j])));
-                gn = fmaxf(gn, nc[j]);
-              }
+            for (int u = 0; u < 4; ++u) {
+              const bool adm = 4 * j4 + u < nadm;
+              const float lbv = fmaf(-e_row, nn[u], __uint_as_float(sv[4 * j4 + u]));
+              gm[u] = fmaxf(gm[u], adm ? lbv : -INFINITY);
+              gq[u] = fmaxf(gq[u], adm ? nn[u] : 0.f);
             }
           }
+          const float gmax = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
+          const float gn = fmaxf(fmaxf(gq[0], gq[1]), fmaxf(gq[2], gq[3]));
           nmax = fmaxf(nmax, gn);
           if (gmax > lb[KM - 1]) sorted_insert<KM>(lb, gmax);
         });
@@ -409,13 +429,22 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     };
     for (int t = n_tiles; t < total; ++t) {
       scan_tile(t, [&](int cb, const uint32_t (&sv)[32], const float* nc, bool full) {
+        // branch-free: a bit per column whose upper bound reaches the filter,
+        // then the inadmissible columns cut off
         uint32_t m = 0u;
         if (cb < lim) {
+          const float4* nc4 = reinterpret_cast<const float4*>(nc);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const bool adm = full || (cb + j < lim);
-            if (adm && fmaf(e_row, nc[j], __uint_as_float(sv[j])) >= filt) m |= 1u << j;
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 n4 = nc4[j4];
+            const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float ub = fmaf(e_row, nn[u], __uint_as_float(sv[4 * j4 + u]));
+              m |= static_cast<uint32_t>(ub >= filt) << (4 * j4 + u);
+            }
           }
+          if (!full) m &= (1u << (lim - cb)) - 1u;   // 0 < lim - cb < 32 here
         }
         // flush (warp-uniform) only when a queue would overflow
         if (__any_sync(0xffffffffu, nq + __popc(m) > kRtcCap)) flush();
