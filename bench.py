@@ -530,6 +530,8 @@ def run_ssa(args):
     st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     pp = ctypes.byref(p)
     P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    rws_n = int(L.ssa_route_workspace_size(pp))         # the router's pre-split key image
+    rws = torch.empty(max(rws_n, 256), dtype=torch.uint8, device=dev)
     for s in range(n_split):
         flush.zero_()
         e = ev[s]
@@ -554,7 +556,8 @@ def run_ssa(args):
             assert L.ssa_route_tree(pp, P(qs), P(ks), P(ks2), P(sup), P(supc),
                                     P(ri) if w.top_k else None, P(rc), st) == 0
         else:
-            assert L.ssa_route(pp, P(qs), P(ks), P(ri) if w.top_k else None, P(rc), st) == 0
+            assert L.ssa_route_with_workspace(pp, P(qs), P(ks), P(ri) if w.top_k else None, P(rc),
+                                              P(rws), rws_n, st) == 0
         e[4].record()
         if w.consensus:
             assert L.ssa_route_consensus(pp, P(idx_h) if w.top_k else None, P(cnt_h),
@@ -743,7 +746,8 @@ def run_ssa(args):
         # per forward: pool (K and Q in one launch) + route + attend; with
         # beta: two feature launches + scores + select + attend; two-level:
         # pool + super-block pool + upper route + select + attend; +1 consensus
-        "gpu_launches": ((5 if (w.beta or tree) else 3) + (1 if w.consensus else 0)) * args.steps,
+        "gpu_launches": ((5 if (w.beta or tree) else 3) + (1 if w.consensus else 0)
+                         + (1 if (rws_n and not tree and not w.beta) else 0)) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -45,6 +45,11 @@ struct RouteArgs {
   int32_t Hq, Hkv, NQB, NB, Bq, Bk, top_k, causal;
   int32_t n_row_tiles;
   uint64_t timeout_ns;
+  // tensor-core form only: the key summaries already split into their bf16
+  // MMA image (rtc_split_kernel), or null to split them in the kernel
+  const uint8_t* kimg = nullptr;   // [B*Hkv, k_tiles, 2 * 128 * D * 2]
+  const float* knrm = nullptr;     // [B*Hkv, k_tiles * 128]
+  int32_t k_tiles = 0;
 };
 
 // orderable 64-bit key: larger key <=> (higher score, then lower index)

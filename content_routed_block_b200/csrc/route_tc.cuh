@@ -76,8 +76,10 @@ struct RtcLayout {
   static constexpr uint32_t OFF_NRM = OFF_K + KSTAGES * 2 * K_BYTES;  // fp32 [KSTAGES][NT]
   static constexpr uint32_t OFF_LIST = OFF_NRM + KSTAGES * NT * 4;    // uint16 [kRtcCap][128]
   static constexpr uint32_t OFF_BAR = OFF_LIST + kRtcCap * kRtcRows * 2;
-  // acc_full[2] | acc_empty[2] | TMEM base
-  static constexpr uint32_t USED = OFF_BAR + 48;
+  // acc_full[2] | acc_empty[2] | TMEM base (+ pad) | stage_loaded[2]
+  static constexpr uint32_t USED = OFF_BAR + 56;
+  // one tile of the pre-split image: hi then lo, each laid out as a stage
+  static constexpr uint32_t IMG_TILE = 2 * K_BYTES;
   static constexpr uint32_t SMEM_BYTES = USED + 1024;
   static constexpr uint32_t TMEM_COLS = KSTAGES * NT;             // two accumulators
   static __device__ __forceinline__ uint32_t kh(int st) { return OFF_K + st * 2 * K_BYTES; }
@@ -124,6 +126,42 @@ __device__ __forceinline__ void sorted_insert(T (&arr)[KM], T v) {
   arr[0] = v > arr[0] ? v : arr[0];
 }
 
+// The key summaries' MMA image, once per launch instead of once per CTA and
+// tile: tile t of KV head bkv holds rows c = 128 t .. 128 t + 127 as the bf16
+// hi parts then the lo parts, each in the shared-memory layout of a stage
+// (128B-swizzled, K-major), and their norms sqrt(sum mu^2) * 1.001.  Rows past
+// NB are zero.  D/8 lanes per row, one 16-byte chunk each.
+template <int D>
+__global__ void __launch_bounds__(256) rtc_split_kernel(const float* ksum, uint8_t* img, float* nrm,
+                                                        int32_t NB, int32_t k_tiles,
+                                                        int64_t n_rows) {
+  using Lay = RtcLayout<D>;
+  constexpr int G = D / 8;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = t / G;        // (bkv, tile, r) flattened
+  const int g = static_cast<int>(t % G);
+  if (row >= n_rows) return;        // whole warps: n_rows * G is a multiple of 32
+  const int64_t per_head = static_cast<int64_t>(k_tiles) * kRtcNT;
+  const int64_t bkv = row / per_head;
+  const int c = static_cast<int>(row - bkv * per_head);
+  const int tile = c / kRtcNT, r = c % kRtcNT;
+  float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+  if (c < NB) {
+    const float* src = ksum + (bkv * NB + c) * D + g * 8;
+    v0 = *reinterpret_cast<const float4*>(src);
+    v1 = *reinterpret_cast<const float4*>(src + 4);
+  }
+  uint4 hi, lo;
+  float sq = 0.f;
+  split8_bf16(v0, v1, hi, lo, sq);
+  uint8_t* base = img + (bkv * k_tiles + tile) * static_cast<int64_t>(Lay::IMG_TILE);
+  *reinterpret_cast<uint4*>(base + sw128_offset(r, g, Lay::HALF_K)) = hi;
+  *reinterpret_cast<uint4*>(base + Lay::K_BYTES + sw128_offset(r, g, Lay::HALF_K)) = lo;
+#pragma unroll
+  for (int off = 1; off < G; off <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+  if (g == 0) nrm[(bkv * k_tiles + tile) * kRtcNT + r] = sqrtf(sq) * 1.001f;
+}
+
 // Warp roles: warps 0-3 are the rows (thread r = query block qb0 + r = TMEM
 // lane r) and scan every tile's scores; warps 4-7 stage the key-summary tiles
 // (eight lanes per key block: load, split into bf16 hi / lo, norm) into one of
@@ -149,6 +187,8 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
   uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);       // [2]
   uint64_t* bar_empty = bar_full + 2;                                          // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_BAR + 32);
+  uint64_t* bar_load = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR + 40);  // [2]
+  const bool presplit = a.kimg != nullptr;
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int bh = blockIdx.y;
@@ -170,6 +210,7 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_full[i], 1);
       mbar_init(&bar_empty[i], 4);   // one arrival per row warp
+      mbar_init(&bar_load[i], 1);
     }
     fence_barrier_init();
   }
@@ -207,79 +248,107 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
   const int total = 2 * n_tiles;     // pass 1 tiles, then pass 2 tiles
 
   if (warp >= 4) {
-    // ------------------------------------------------ key-summary stagers
-    // warp w stages key rows 32(w-4) .. +31, four rows per step: lane = (row
-    // of the four, 16-byte bf16 chunk g), so one load instruction covers four
-    // consecutive rows (one contiguous span for D = 64) instead of 32 rows
+    // ------------------------------------------------ key-summary producers
     const int lane = tid & 31;
-    const int g0 = lane & 7, rsub = lane >> 3;
-    const int rbase = (warp - 4) * 32 + rsub;
-    constexpr int RB = D == 64 ? 8 : 4;      // rows of a batch, all loads in flight
-    constexpr int HH = D / 64;               // 64-column halves of a row
     // the descriptors of the Q parts and of stage 0's key parts; the other
     // operands are these plus a shared-memory offset (>> 4 in the low field)
     const uint64_t dq_hi = sdesc_sw128(sbase + Lay::OFF_QH, 16, 1024);
     const uint64_t dq_lo = sdesc_sw128(sbase + Lay::OFF_QL, 16, 1024);
     const uint64_t dk0 = sdesc_sw128(sbase + Lay::kh(0), 16, 1024);
-    for (int t = 0; t < total; ++t) {
-      const int st = t & 1;
-      const int c0 = (t % n_tiles) * NT;
-#pragma unroll 1
-      for (int i0 = 0; i0 < 8; i0 += RB) {
-        float4 va[RB][HH], vb[RB][HH];
+    // the tile's three MMAs (q_hi k_hi, q_hi k_lo, q_lo k_hi) into accumulator st
+    auto issue_mmas = [&](int st) {
+      const uint64_t dk_st = dk0 + ((st * 2 * Lay::K_BYTES) >> 4);
+      const uint64_t da[3] = {dq_hi, dq_hi, dq_lo};
+      const uint64_t db[3] = {dk_st, dk_st + (Lay::K_BYTES >> 4), dk_st};
 #pragma unroll
-        for (int i = 0; i < RB; ++i) {
-          const int row = rbase + (i0 + i) * 4;
-          const bool ok = c0 + row < a.NB;
-          const float* src = ksrc + static_cast<int64_t>(c0 + row) * D;
+      for (int term = 0; term < 3; ++term) {
 #pragma unroll
-          for (int hh = 0; hh < HH; ++hh) {
-            const int g = hh * 8 + g0;
-            va[i][hh] = ok ? *reinterpret_cast<const float4*>(src + g * 8) : make_float4(0.f, 0.f, 0.f, 0.f);
-            vb[i][hh] = ok ? *reinterpret_cast<const float4*>(src + g * 8 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-        // the stage is rewritten only after the rows have read it (the
-        // loads above are already in flight)
-        if (i0 == 0 && t >= 2) mbar_wait(&bar_empty[st], ((t - 2) >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
-#pragma unroll
-        for (int i = 0; i < RB; ++i) {
-          const int row = rbase + (i0 + i) * 4;
-          float sq = 0.f;
-#pragma unroll
-          for (int hh = 0; hh < HH; ++hh) {
-            const int g = hh * 8 + g0;
-            uint4 hi, lo;
-            split8_bf16(va[i][hh], vb[i][hh], hi, lo, sq);
-            *reinterpret_cast<uint4*>(smem + Lay::kh(st) + sw128_offset(row, g, Lay::HALF_K)) = hi;
-            *reinterpret_cast<uint4*>(smem + Lay::kl(st) + sw128_offset(row, g, Lay::HALF_K)) = lo;
-          }
-          // the row's sum of squares over its 8 (or 16) chunks: the summation
-          // order differs from a sequential one by far less than the 1.001 slack
-          sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-          sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-          sq += __shfl_xor_sync(0xffffffffu, sq, 4);
-          if (g0 == 0) nrm[st * NT + row] = sqrtf(sq) * 1.001f;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t qoff = ((kk / 4) * Lay::HALF_Q + (kk % 4) * 32) >> 4;
+          const uint64_t koff = ((kk / 4) * Lay::HALF_K + (kk % 4) * 32) >> 4;
+          mma_ss(tmem + st * NT, da[term] + qoff, db[term] + koff, IDESC,
+                 (term > 0 || kk > 0) ? 1u : 0u);
         }
       }
-      fence_proxy_async_smem();
-      asm volatile("bar.sync 1, 128;" ::: "memory");   // the stagers only
+      mma_commit(&bar_full[st]);
+    };
+    if (presplit) {
+      // ------------------------------------- pre-split image: one producer
+      // thread copies a tile's image and norms into stage st (untiled bulk
+      // copies) and issues its MMAs; the other stager warps have no work
       if (tid == kRtcRows) {
-        tc_fence_after();
-        const uint64_t dk_st = dk0 + ((st * 2 * Lay::K_BYTES) >> 4);
-        const uint64_t da[3] = {dq_hi, dq_hi, dq_lo};
-        const uint64_t db[3] = {dk_st, dk_st + (Lay::K_BYTES >> 4), dk_st};
+        const uint8_t* img = a.kimg + static_cast<int64_t>(bkv) * a.k_tiles * Lay::IMG_TILE;
+        const float* kn = a.knrm + static_cast<int64_t>(bkv) * a.k_tiles * NT;
+        for (int t = 0; t < total; ++t) {
+          const int st = t & 1, tile = t % n_tiles;
+          if (t >= 2) mbar_wait(&bar_empty[st], ((t - 2) >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
+          mbar_arrive_expect_tx(&bar_load[st], Lay::IMG_TILE + NT * 4);
+          bulk_load(smem + Lay::kh(st), img + static_cast<int64_t>(tile) * Lay::IMG_TILE,
+                    Lay::IMG_TILE, &bar_load[st]);
+          bulk_load(nrm + st * NT, kn + static_cast<int64_t>(tile) * NT, NT * 4, &bar_load[st]);
+          mbar_wait(&bar_load[st], (t >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
+          tc_fence_after();
+          issue_mmas(st);
+        }
+      }
+      __syncwarp();   // warp 4 converges before the final barrier
+    } else {
+      // ------------------- otherwise the four stager warps split the tiles:
+      // warp w stages key rows 32(w-4) .. +31, four rows per step: lane =
+      // (row of the four, 16-byte bf16 chunk g), so one load instruction
+      // covers four consecutive rows (one contiguous span for D = 64)
+      const int g0 = lane & 7, rsub = lane >> 3;
+      const int rbase = (warp - 4) * 32 + rsub;
+      constexpr int RB = D == 64 ? 8 : 4;      // rows of a batch, all loads in flight
+      constexpr int HH = D / 64;               // 64-column halves of a row
+      for (int t = 0; t < total; ++t) {
+        const int st = t & 1;
+        const int c0 = (t % n_tiles) * NT;
+#pragma unroll 1
+        for (int i0 = 0; i0 < 8; i0 += RB) {
+          float4 va[RB][HH], vb[RB][HH];
 #pragma unroll
-        for (int term = 0; term < 3; ++term) {
+          for (int i = 0; i < RB; ++i) {
+            const int row = rbase + (i0 + i) * 4;
+            const bool ok = c0 + row < a.NB;
+            const float* src = ksrc + static_cast<int64_t>(c0 + row) * D;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t qoff = ((kk / 4) * Lay::HALF_Q + (kk % 4) * 32) >> 4;
-            const uint64_t koff = ((kk / 4) * Lay::HALF_K + (kk % 4) * 32) >> 4;
-            mma_ss(tmem + st * NT, da[term] + qoff, db[term] + koff, IDESC,
-                   (term > 0 || kk > 0) ? 1u : 0u);
+            for (int hh = 0; hh < HH; ++hh) {
+              const int g = hh * 8 + g0;
+              va[i][hh] = ok ? *reinterpret_cast<const float4*>(src + g * 8) : make_float4(0.f, 0.f, 0.f, 0.f);
+              vb[i][hh] = ok ? *reinterpret_cast<const float4*>(src + g * 8 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          }
+          // the stage is rewritten only after the rows have read it (the
+          // loads above are already in flight)
+          if (i0 == 0 && t >= 2) mbar_wait(&bar_empty[st], ((t - 2) >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
+#pragma unroll
+          for (int i = 0; i < RB; ++i) {
+            const int row = rbase + (i0 + i) * 4;
+            float sq = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < HH; ++hh) {
+              const int g = hh * 8 + g0;
+              uint4 hi, lo;
+              split8_bf16(va[i][hh], vb[i][hh], hi, lo, sq);
+              *reinterpret_cast<uint4*>(smem + Lay::kh(st) + sw128_offset(row, g, Lay::HALF_K)) = hi;
+              *reinterpret_cast<uint4*>(smem + Lay::kl(st) + sw128_offset(row, g, Lay::HALF_K)) = lo;
+            }
+            // the row's sum of squares over its 8 (or 16) chunks: the
+            // summation order differs from a sequential one by far less than
+            // the 1.001 slack
+            sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+            sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+            sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+            if (g0 == 0) nrm[st * NT + row] = sqrtf(sq) * 1.001f;
           }
         }
-        mma_commit(&bar_full[st]);
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");   // the stagers only
+        if (tid == kRtcRows) {
+          tc_fence_after();
+          issue_mmas(st);
+        }
       }
     }
   } else {
@@ -312,6 +381,8 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     auto scan_tile = [&](int t, auto&& group) {
       const int st = t & 1;
       mbar_wait(&bar_full[st], (t >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
+      // the pre-split norms come by bulk copy: observe its completion here too
+      if (presplit) mbar_wait(&bar_load[st], (t >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
       tc_fence_after();
       const int c0 = (t % n_tiles) * NT;
 #pragma unroll 1

@@ -346,8 +346,31 @@ bool use_tc_router(const ssa_params* p) {
   return static_cast<int64_t>(p->B) * p->Hq * pairs >= (static_cast<int64_t>(1) << 25);
 }
 
+// bytes of the tensor-core router's pre-split key image (tiles of 128 key
+// blocks, bf16 hi / lo in the MMA layout) and of its norms, or 0 when the
+// fp32 form routes this problem
+size_t route_img_bytes(const ssa_params* p, size_t* nrm_offset) {
+  if (!use_tc_router(p)) return 0;
+  const size_t tiles = static_cast<size_t>(p->N / p->block_k + ssa::kRtcNT - 1) / ssa::kRtcNT;
+  const size_t heads_tiles = static_cast<size_t>(p->B) * p->Hkv * tiles;
+  const size_t img = align256(heads_tiles * 2 * ssa::kRtcNT * p->D * 2);
+  if (nrm_offset) *nrm_offset = img;
+  return img + align256(heads_tiles * ssa::kRtcNT * sizeof(float));
+}
+
+template <int D>
+cudaError_t launch_rtc_split(const ssa::RouteArgs& a, int B, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(B) * a.Hkv * a.k_tiles * ssa::kRtcNT;
+  const int64_t threads = rows * (D / 8);
+  ssa::rtc_split_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+      a.ksum, const_cast<uint8_t*>(a.kimg), const_cast<float*>(a.knrm), a.NB, a.k_tiles, rows);
+  return cudaGetLastError();
+}
+
+// img (optional, route_img_bytes of scratch): with the tensor-core form the
+// key summaries are split once into it and every CTA copies its tiles
 ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksum, int32_t* idx,
-                        int32_t* cnt, cudaStream_t stream) {
+                        int32_t* cnt, cudaStream_t stream, uint8_t* img = nullptr) {
   ssa::RouteArgs a;
   a.qsum = qsum;
   a.ksum = ksum;
@@ -365,6 +388,14 @@ ssa_status launch_route(const ssa_params* p, const float* qsum, const float* ksu
   a.timeout_ns = timeout_ns(p);
   cudaError_t e;
   if (use_tc_router(p)) {
+    size_t nrm_off = 0;
+    if (img != nullptr && route_img_bytes(p, &nrm_off) > 0) {
+      a.kimg = img;
+      a.knrm = reinterpret_cast<const float*>(img + nrm_off);
+      a.k_tiles = (a.NB + ssa::kRtcNT - 1) / ssa::kRtcNT;
+      e = p->D == 64 ? launch_rtc_split<64>(a, p->B, stream) : launch_rtc_split<128>(a, p->B, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "rtc_split_kernel launch");
+    }
     e = p->D == 64 ? launch_route_tc<64>(a, p->B, stream) : launch_route_tc<128>(a, p->B, stream);
   } else {
     e = p->D == 64 ? launch_route_fp32<64>(a, p->B, stream) : launch_route_fp32<128>(a, p->B, stream);
@@ -726,7 +757,7 @@ ssa_status launch_consensus(const ssa_params* p, const int32_t* idx, const int32
 // Workspace of ssa_forward: K and Q summaries, the per-head routed lists and
 // counts, and (consensus routing only) the per-group lists and counts.
 struct WsLayout {
-  size_t ksum, qsum, idx, cnt, idx_kv, cnt_kv, qf, kf, sc, ksum2, sup_idx, sup_cnt, total;
+  size_t ksum, qsum, idx, cnt, idx_kv, cnt_kv, qf, kf, sc, ksum2, sup_idx, sup_cnt, kimg, total;
 };
 
 WsLayout ws_layout(const ssa_params* p) {
@@ -762,7 +793,10 @@ WsLayout ws_layout(const ssa_params* p) {
   w.ksum2 = w.sc + align256(scb);
   w.sup_idx = w.ksum2 + align256(k2b);
   w.sup_cnt = w.sup_idx + align256(s2b);
-  w.total = w.sup_cnt + align256(c2b);
+  // flat routing in the tensor-core form: the pre-split key image
+  const size_t imgb = (!cum && !tree) ? route_img_bytes(p, nullptr) : 0;
+  w.kimg = w.sup_cnt + align256(c2b);
+  w.total = w.kimg + imgb;
   return w;
 }
 
@@ -851,6 +885,33 @@ ssa_status ssa_route(const ssa_params* p, const float* qsum, const float* ksum, 
   if (!aligned16(qsum) || !aligned16(ksum) || !aligned16(cnt) || (idx && !aligned16(idx)))
     return fail(SSA_ERR_INVALID_ARG, "routing buffers must be 16-byte aligned");
   s = launch_route(p, qsum, ksum, idx, cnt, static_cast<cudaStream_t>(stream));
+  return s == SSA_OK ? ok() : s;
+}
+
+size_t ssa_route_workspace_size(const ssa_params* p) {
+  if (validate(p) != SSA_OK || p->beta != 0.0f) return 0;
+  return route_img_bytes(p, nullptr);
+}
+
+ssa_status ssa_route_with_workspace(const ssa_params* p, const float* qsum, const float* ksum,
+                                    int32_t* idx, int32_t* cnt, void* workspace,
+                                    size_t workspace_bytes, ssa_stream_t stream) {
+  ssa_status s = validate(p);
+  if (s != SSA_OK) return s;
+  if (p->beta != 0.0f)
+    return fail(SSA_ERR_INVALID_ARG,
+                "beta != 0: route with ssa_route_features and ssa_route_cumulant");
+  if (qsum == nullptr || ksum == nullptr || cnt == nullptr || (p->top_k > 0 && idx == nullptr))
+    return fail(SSA_ERR_INVALID_ARG, "qsum, ksum, cnt (and idx when top_k > 0) must be non-NULL");
+  if (!aligned16(qsum) || !aligned16(ksum) || !aligned16(cnt) || (idx && !aligned16(idx)))
+    return fail(SSA_ERR_INVALID_ARG, "routing buffers must be 16-byte aligned");
+  const size_t need = route_img_bytes(p, nullptr);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return fail(SSA_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  s = launch_route(p, qsum, ksum, idx, cnt, static_cast<cudaStream_t>(stream),
+                   need > 0 ? static_cast<uint8_t*>(workspace) : nullptr);
   return s == SSA_OK ? ok() : s;
 }
 
@@ -990,7 +1051,7 @@ ssa_status ssa_forward(const ssa_params* p, const void* q, const void* k, const 
       if ((s = launch_route_tree(p, qsum, ksum, ksum2, sup_idx, sup_cnt, idx_h, cnt_h, st)) !=
           SSA_OK)
         return s;
-    } else if ((s = launch_route(p, qsum, ksum, idx_h, cnt_h, st)) != SSA_OK) {
+    } else if ((s = launch_route(p, qsum, ksum, idx_h, cnt_h, st, ws + w.kimg)) != SSA_OK) {
       return s;
     }
   }

@@ -15,7 +15,8 @@ import torch
 
 __all__ = [
     "Params", "SsaError", "lib", "make_params", "params_of", "workspace_size", "block_summary",
-    "route", "route_consensus", "route_features", "route_cumulant", "tree_summary", "route_tree",
+    "route", "route_workspace_size", "route_consensus", "route_features", "route_cumulant",
+    "tree_summary", "route_tree",
     "attend", "forward",
     "forward_host", "backward", "decode", "decode_workspace_size", "check_error",
     "probe_wait_timeout", "probe_ex2_rate",
@@ -97,6 +98,8 @@ def lib() -> ctypes.CDLL:
         "ssa_workspace_size": (sz, [P]),
         "ssa_block_summary": (i32, [P, vp, i32, i32, vp, vp]),
         "ssa_route": (i32, [P, vp, vp, vp, vp, vp]),
+        "ssa_route_workspace_size": (sz, [P]),
+        "ssa_route_with_workspace": (i32, [P, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_route_consensus": (i32, [P, vp, vp, vp, vp, vp]),
         "ssa_tree_summary": (i32, [P, vp, vp, vp]),
         "ssa_route_tree": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
@@ -167,15 +170,30 @@ def block_summary(x: torch.Tensor, block: int, p: Params) -> torch.Tensor:
     return out
 
 
-def route(qsum: torch.Tensor, ksum: torch.Tensor, p: Params):
-    """(idx int32 [B, Hq, NQB, top_k], cnt int32 [B, Hq, NQB])."""
+def route_workspace_size(p: Params) -> int:
+    return int(lib().ssa_route_workspace_size(ctypes.byref(p)))
+
+
+def route(qsum: torch.Tensor, ksum: torch.Tensor, p: Params, workspace: torch.Tensor | None = None,
+          in_kernel_split: bool = False):
+    """(idx int32 [B, Hq, NQB, top_k], cnt int32 [B, Hq, NQB]).  Routes through
+    ssa_route_with_workspace (scratch from ``workspace`` or a fresh buffer);
+    ``in_kernel_split`` calls ssa_route, which needs no scratch."""
     _need(qsum, torch.float32, (p.B, p.Hq, p.n_qblocks, p.D), "qsum")
     _need(ksum, torch.float32, (p.B, p.Hkv, p.n_kblocks, p.D), "ksum")
     dev = qsum.device
     idx = torch.empty((p.B, p.Hq, p.n_qblocks, p.top_k), dtype=torch.int32, device=dev)
     cnt = torch.empty((p.B, p.Hq, p.n_qblocks), dtype=torch.int32, device=dev)
-    _check(lib().ssa_route(ctypes.byref(p), _ptr(qsum), _ptr(ksum),
-                           _ptr(idx) if p.top_k else None, _ptr(cnt), _stream()))
+    if in_kernel_split:
+        _check(lib().ssa_route(ctypes.byref(p), _ptr(qsum), _ptr(ksum),
+                               _ptr(idx) if p.top_k else None, _ptr(cnt), _stream()))
+        return idx, cnt
+    ws = route_workspace_size(p)
+    if ws and (workspace is None or workspace.numel() < ws):
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+    _check(lib().ssa_route_with_workspace(
+        ctypes.byref(p), _ptr(qsum), _ptr(ksum), _ptr(idx) if p.top_k else None, _ptr(cnt),
+        _ptr(workspace) if ws else None, ws, _stream()))
     return idx, cnt
 
 

@@ -123,6 +123,24 @@ ssa_status ssa_block_summary(const ssa_params* p, const void* x, int32_t H,
 ssa_status ssa_route(const ssa_params* p, const float* qsum, const float* ksum,
                      int32_t* idx, int32_t* cnt, ssa_stream_t stream);
 
+/* ssa_route with caller scratch, the same result bit for bit.  Problems the
+ * tensor-core form routes (at least 2^25 admissible (query block, key block)
+ * pairs over all heads, or SSA_ROUTER=tc) split the key summaries once into
+ * the scratch -- tiles of 128 blocks as bf16 hi / lo parts in the MMA layout,
+ * and their norms -- instead of once per CTA and tile, and the route then
+ * copies each tile in with one bulk copy (two launches).  Elsewhere the
+ * scratch is unused and may be NULL.
+ *   workspace  device, 256-byte aligned, >= ssa_route_workspace_size(p)
+ *              bytes (SSA_ERR_WORKSPACE otherwise); contents undefined
+ *              before and after.  ssa_forward keeps the same image in its
+ *              own workspace.
+ * ssa_route_workspace_size returns 0 for invalid params, beta != 0, or when
+ * the fp32 form routes the problem. */
+size_t ssa_route_workspace_size(const ssa_params* p);
+ssa_status ssa_route_with_workspace(const ssa_params* p, const float* qsum, const float* ksum,
+                                    int32_t* idx, int32_t* cnt, void* workspace,
+                                    size_t workspace_bytes, ssa_stream_t stream);
+
 /* Second-cumulant routing features (jonsmirl/ssa README, "Algorithm and
  * complexity": r_c(q) = <q, mu_c> + (beta/2) q^T Sigma_c q with Sigma_c block
  * c's second cumulant).  A query block scores by the mean of its queries'
@@ -234,7 +252,9 @@ ssa_status ssa_attend(const ssa_params* p, const void* q, const void* k, const v
  * -- or, with p->beta != 0, the second-cumulant features of K and Q and
  * ssa_route_cumulant --, or, with p->tree_fanout > 0, the super-block
  * summaries and ssa_route_tree --, (with p->consensus) the consensus route, attend.  workspace must hold
- * ssa_workspace_size(p) bytes (device, 256-byte aligned).  idx_out / cnt_out
+ * ssa_workspace_size(p) bytes (device, 256-byte aligned); when the flat route
+ * takes the tensor-core form its last ssa_route_workspace_size(p) bytes hold
+ * the router's pre-split key image (one more launch).  idx_out / cnt_out
  * (device, may be NULL) receive the lists attend used when given -- per head
  * [B, Hq, N/Bq, top_k], or per KV group [B, Hkv, N/Bq, top_k] with
  * p->consensus; otherwise they live in the workspace.  lse may be NULL. */

@@ -45,6 +45,45 @@ def test_workspace_layout(L):
     assert ssa.workspace_size(p) == a(ks) + a(qs) + a(ix) + a(cn)
 
 
+def test_workspace_layout_with_the_routers_key_image(L, monkeypatch):
+    # the tensor-core router's pre-split key summaries (tiles of 128 key
+    # blocks: bf16 hi and lo parts of 128 x D each, and 128 fp32 norms) sit at
+    # the end of the forward's workspace when that form routes the problem
+    # (>= 2^25 admissible pairs over all heads) and form ssa_route's scratch
+    monkeypatch.delenv("SSA_ROUTER", raising=False)
+    a = lambda x: (x + 255) // 256 * 256
+    p = _p(N=1 << 20, window=1024)                      # 16,384 blocks, 14 heads
+    nb = 16384
+    ks, qs = 2 * nb * 64 * 4, 14 * nb * 64 * 4
+    ix, cn = 14 * nb * 16 * 4, 14 * nb * 4
+    tiles = 2 * (nb // 128)
+    img = a(tiles * 2 * 128 * 64 * 2) + a(tiles * 128 * 4)
+    assert ssa.route_workspace_size(p) == img
+    assert ssa.workspace_size(p) == a(ks) + a(qs) + a(ix) + a(cn) + img
+    assert ssa.route_workspace_size(_p()) == 0          # 32K tokens: the fp32 form
+    monkeypatch.setenv("SSA_ROUTER", "fp32")
+    assert ssa.route_workspace_size(p) == 0
+    monkeypatch.setenv("SSA_ROUTER", "tc")
+    t = 2 * 4                                           # 512 blocks: four tiles per head
+    assert ssa.route_workspace_size(_p()) == a(t * 2 * 128 * 64 * 2) + a(t * 128 * 4)
+    # a ragged last tile: 200 blocks are two tiles
+    q = _p(N=200 * 64, Hq=2, Hkv=1)
+    assert ssa.route_workspace_size(q) == a(2 * 2 * 128 * 64 * 2) + a(2 * 128 * 4)
+
+
+def test_route_with_workspace_rejects_bad_arguments_before_launch(L, monkeypatch):
+    monkeypatch.setenv("SSA_ROUTER", "tc")
+    p = _p()
+    good = ctypes.c_void_p(1 << 20)
+    need = ssa.route_workspace_size(p)
+    f = L.ssa_route_with_workspace
+    assert f(ctypes.byref(p), good, good, good, good, None, 0, None) == 3        # no scratch
+    assert f(ctypes.byref(p), good, good, good, good, good, need - 1, None) == 3  # too small
+    odd = ctypes.c_void_p((1 << 20) + 16)
+    assert f(ctypes.byref(p), good, good, good, good, odd, need, None) == 1      # unaligned
+    assert f(ctypes.byref(p), None, good, good, good, good, need, None) == 1     # no qsum
+
+
 def test_workspace_layout_with_consensus(L):
     p = _p(consensus=True)
     ks = 1 * 2 * 512 * 64 * 4

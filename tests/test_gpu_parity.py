@@ -230,7 +230,7 @@ def test_forward_host_roundtrip():
 
 
 # ------------------------------------------------------------------ router forms
-def _route_with(form, case):
+def _route_with(form, case, in_kernel_split=False):
     import os
     old = os.environ.get("SSA_ROUTER")
     os.environ["SSA_ROUTER"] = form
@@ -238,7 +238,7 @@ def _route_with(form, case):
         p = case.p
         ks = ssa.block_summary(case.kd, case.w.block_k, p)
         qs = ssa.block_summary(case.qd, case.w.block_q, p)
-        idx, cnt = ssa.route(qs, ks, p)
+        idx, cnt = ssa.route(qs, ks, p, in_kernel_split=in_kernel_split)
         ssa.check_error()
         return idx, cnt
     finally:
@@ -253,11 +253,15 @@ def _route_with(form, case):
 def test_tensor_core_router_equals_fp32_router(w):
     # the tensor-core router ranks on the same fp32 scores as the FMA router
     # (bf16 prefilter with a proven bound + exact rescoring): bit-identical lists
+    # The tensor-core form runs twice: with the key image split once into
+    # scratch (ssa_route_with_workspace, as in the forward) and split by each
+    # CTA (ssa_route, no scratch).
     case = Case(w)
     i1, c1 = _route_with("fp32", case)
     i2, c2 = _route_with("tc", case)
-    assert torch.equal(c1, c2)
-    assert torch.equal(i1, i2)
+    i3, c3 = _route_with("tc", case, in_kernel_split=True)
+    assert torch.equal(c1, c2) and torch.equal(c1, c3)
+    assert torch.equal(i1, i2) and torch.equal(i1, i3)
 
 
 def test_tensor_core_router_on_flat_and_tied_scores():
@@ -269,7 +273,9 @@ def test_tensor_core_router_on_flat_and_tied_scores():
     case = Case(w, x)
     i1, c1 = _route_with("fp32", case)
     i2, c2 = _route_with("tc", case)
+    i3, c3 = _route_with("tc", case, in_kernel_split=True)
     assert torch.equal(i1, i2) and torch.equal(c1, c2)
+    assert torch.equal(i1, i3) and torch.equal(c1, c3)
     idx = i2.cpu().numpy()
     for qb in (5, 40, 127):
         n = min(16, qb)
