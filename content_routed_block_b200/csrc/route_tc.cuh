@@ -408,27 +408,55 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
       for (int j = 0; j < KM; ++j) lb[j] = (j < KM - k) ? INFINITY : -INFINITY;
       for (int t = 0; t < n_tiles; ++t) {
         scan_tile(t, [&](int cb, const uint32_t (&sv)[32], const float* nc, bool full) {
+          // (the vote comes before any lane leaves: full implies cb < lim)
+          const bool warp_full = __all_sync(0xffffffffu, full);
           if (cb >= lim) return;
           // branch-free: inadmissible columns count as -inf (and norm 0);
           // four partial maxima keep the dependent chain short (max is exact)
-          const int nadm = full ? 32 : lim - cb;
           const float4* nc4 = reinterpret_cast<const float4*>(nc);
-          float gm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          float gq[4] = {0.f, 0.f, 0.f, 0.f};
+          float gmax, gn;
+          if (warp_full) {
+            // the usual case: three-input maxima, no per-column test
+            float gm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            float gq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 n4 = nc4[j4];
-            const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+            for (int j4 = 0; j4 < 8; j4 += 2) {
+              const float4 na = nc4[j4], nb = nc4[j4 + 1];
+              const float nn[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
+              float lbv[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const bool adm = 4 * j4 + u < nadm;
-              const float lbv = fmaf(-e_row, nn[u], __uint_as_float(sv[4 * j4 + u]));
-              gm[u] = fmaxf(gm[u], adm ? lbv : -INFINITY);
-              gq[u] = fmaxf(gq[u], adm ? nn[u] : 0.f);
+              for (int u = 0; u < 8; ++u)
+                lbv[u] = fmaf(-e_row, nn[u], __uint_as_float(sv[4 * j4 + u]));
+              gm[0] = fmax3(gm[0], lbv[0], lbv[1]);
+              gm[1] = fmax3(gm[1], lbv[2], lbv[3]);
+              gm[2] = fmax3(gm[2], lbv[4], lbv[5]);
+              gm[3] = fmax3(gm[3], lbv[6], lbv[7]);
+              gq[0] = fmax3(gq[0], nn[0], nn[1]);
+              gq[1] = fmax3(gq[1], nn[2], nn[3]);
+              gq[2] = fmax3(gq[2], nn[4], nn[5]);
+              gq[3] = fmax3(gq[3], nn[6], nn[7]);
             }
+            gmax = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
+            gn = fmaxf(fmaxf(gq[0], gq[1]), fmaxf(gq[2], gq[3]));
+          } else {
+            const int nadm = full ? 32 : lim - cb;
+            float gm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            float gq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 n4 = nc4[j4];
+              const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const bool adm = 4 * j4 + u < nadm;
+                const float lbv = fmaf(-e_row, nn[u], __uint_as_float(sv[4 * j4 + u]));
+                gm[u] = fmaxf(gm[u], adm ? lbv : -INFINITY);
+                gq[u] = fmaxf(gq[u], adm ? nn[u] : 0.f);
+              }
+            }
+            gmax = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
+            gn = fmaxf(fmaxf(gq[0], gq[1]), fmaxf(gq[2], gq[3]));
           }
-          const float gmax = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
-          const float gn = fmaxf(fmaxf(gq[0], gq[1]), fmaxf(gq[2], gq[3]));
           nmax = fmaxf(nmax, gn);
           if (gmax > lb[KM - 1]) sorted_insert<KM>(lb, gmax);
         });
@@ -502,20 +530,33 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
       scan_tile(t, [&](int cb, const uint32_t (&sv)[32], const float* nc, bool full) {
         // branch-free: a bit per column whose upper bound reaches the filter,
         // then the inadmissible columns cut off
+        // (few groups hold a candidate: the maximum upper bound is taken
+        // first, with three-input maxima, and the bits only where it passes)
         uint32_t m = 0u;
         if (cb < lim) {
           const float4* nc4 = reinterpret_cast<const float4*>(nc);
+          float ub[32];
 #pragma unroll
           for (int j4 = 0; j4 < 8; ++j4) {
             const float4 n4 = nc4[j4];
-            const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float ub = fmaf(e_row, nn[u], __uint_as_float(sv[4 * j4 + u]));
-              m |= static_cast<uint32_t>(ub >= filt) << (4 * j4 + u);
-            }
+            ub[4 * j4 + 0] = fmaf(e_row, n4.x, __uint_as_float(sv[4 * j4 + 0]));
+            ub[4 * j4 + 1] = fmaf(e_row, n4.y, __uint_as_float(sv[4 * j4 + 1]));
+            ub[4 * j4 + 2] = fmaf(e_row, n4.z, __uint_as_float(sv[4 * j4 + 2]));
+            ub[4 * j4 + 3] = fmaf(e_row, n4.w, __uint_as_float(sv[4 * j4 + 3]));
           }
-          if (!full) m &= (1u << (lim - cb)) - 1u;   // 0 < lim - cb < 32 here
+          float um[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            um[0] = fmax3(um[0], ub[j], ub[j + 1]);
+            um[1] = fmax3(um[1], ub[j + 2], ub[j + 3]);
+            um[2] = fmax3(um[2], ub[j + 4], ub[j + 5]);
+            um[3] = fmax3(um[3], ub[j + 6], ub[j + 7]);
+          }
+          if (fmaxf(fmaxf(um[0], um[1]), fmaxf(um[2], um[3])) >= filt) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) m |= static_cast<uint32_t>(ub[j] >= filt) << j;
+            if (!full) m &= (1u << (lim - cb)) - 1u;   // 0 < lim - cb < 32 here
+          }
         }
         // flush (warp-uniform) only when a queue would overflow
         if (__any_sync(0xffffffffu, nq + __popc(m) > kRtcCap)) flush();
