@@ -55,7 +55,8 @@
 namespace ssa {
 
 constexpr int kRtcRows = 128;
-constexpr int kRtcThreads = 256;
+constexpr int kRtcThreads = 256;          // in-kernel split: 4 row warps + 4 stager warps
+constexpr int kRtcThreadsPre = 160;       // pre-split image: 4 row warps + 1 producer warp
 constexpr int kRtcNT = 128;               // key blocks per MMA (N)
 // error-bound factor of the split tensor-core scores (see above)
 template <int D>
@@ -76,8 +77,8 @@ struct RtcLayout {
   static constexpr uint32_t OFF_NRM = OFF_K + KSTAGES * 2 * K_BYTES;  // fp32 [KSTAGES][NT]
   static constexpr uint32_t OFF_LIST = OFF_NRM + KSTAGES * NT * 4;    // uint16 [kRtcCap][128]
   static constexpr uint32_t OFF_BAR = OFF_LIST + kRtcCap * kRtcRows * 2;
-  // acc_full[2] | acc_empty[2] | TMEM base (+ pad) | stage_loaded[2]
-  static constexpr uint32_t USED = OFF_BAR + 56;
+  // acc_full[2] | acc_empty[2] | TMEM base (+ pad) | kload[2] | nrm_full[2]
+  static constexpr uint32_t USED = OFF_BAR + 72;
   // one tile of the pre-split image: hi then lo, each laid out as a stage
   static constexpr uint32_t IMG_TILE = 2 * K_BYTES;
   static constexpr uint32_t SMEM_BYTES = USED + 1024;
@@ -170,9 +171,10 @@ __global__ void __launch_bounds__(256) rtc_split_kernel(const float* ksum, uint8
 // staging of the next tiles overlaps the scan of the current one.  Barriers:
 // acc_full[b] (MMAs of a tile into accumulator b done), acc_empty[b] (the rows
 // have read accumulator b and the norms of stage b).
-template <int D, int KM>
-__global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
+template <int D, int KM, bool PRE>
+__global__ void __launch_bounds__(PRE ? kRtcThreadsPre : kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     route_tc_kernel(const RouteArgs a) {
+  constexpr int THREADS = PRE ? kRtcThreadsPre : kRtcThreads;
   using Lay = RtcLayout<D>;
   constexpr int NT = Lay::NT;
   constexpr uint32_t IDESC = idesc_bf16_f32(kRtcRows, NT, false, false);
@@ -187,8 +189,9 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
   uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);       // [2]
   uint64_t* bar_empty = bar_full + 2;                                          // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_BAR + 32);
-  uint64_t* bar_load = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR + 40);  // [2]
-  const bool presplit = a.kimg != nullptr;
+  uint64_t* bar_kload = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR + 40);  // [2]
+  uint64_t* nrm_full = bar_kload + 2;                                           // [2]
+  constexpr bool presplit = PRE;   // a.kimg holds the key image
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int bh = blockIdx.y;
@@ -210,7 +213,8 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_full[i], 1);
       mbar_init(&bar_empty[i], 4);   // one arrival per row warp
-      mbar_init(&bar_load[i], 1);
+      mbar_init(&bar_kload[i], 1);
+      mbar_init(&nrm_full[i], 1);
     }
     fence_barrier_init();
   }
@@ -218,9 +222,9 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     tmem_alloc(tmem_slot, Lay::TMEM_COLS);
     tmem_relinquish();
   }
-  // query summaries: bf16 hi / lo (MMA A operands), 2 threads per row
-  {
-    constexpr int TPR = kRtcThreads / kRtcRows;
+  // query summaries: bf16 hi / lo (MMA A operands), TPR threads per row
+  if (tid < kRtcRows * (THREADS / kRtcRows)) {
+    constexpr int TPR = THREADS / kRtcRows;
     constexpr int CPT = (D / 8) / TPR;
     const int r = tid / TPR, part = tid % TPR;
     const bool ok = qb0 + r < a.NQB;
@@ -272,24 +276,27 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
       }
       mma_commit(&bar_full[st]);
     };
-    if (presplit) {
+    if constexpr (PRE) {
       // ------------------------------------- pre-split image: one producer
       // thread copies a tile's image and norms into stage st (untiled bulk
-      // copies) and issues its MMAs; the other stager warps have no work
+      // copies) once the rows have released it, and issues its MMAs.
       if (tid == kRtcRows) {
         const uint8_t* img = a.kimg + static_cast<int64_t>(bkv) * a.k_tiles * Lay::IMG_TILE;
         const float* kn = a.knrm + static_cast<int64_t>(bkv) * a.k_tiles * NT;
         for (int t = 0; t < total; ++t) {
           const int st = t & 1, tile = t % n_tiles;
           if (t >= 2) mbar_wait(&bar_empty[st], ((t - 2) >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
-          mbar_arrive_expect_tx(&bar_load[st], Lay::IMG_TILE + NT * 4);
+          mbar_arrive_expect_tx(&bar_kload[st], Lay::IMG_TILE);
           bulk_load(smem + Lay::kh(st), img + static_cast<int64_t>(tile) * Lay::IMG_TILE,
-                    Lay::IMG_TILE, &bar_load[st]);
-          bulk_load(nrm + st * NT, kn + static_cast<int64_t>(tile) * NT, NT * 4, &bar_load[st]);
-          mbar_wait(&bar_load[st], (t >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
+                    Lay::IMG_TILE, &bar_kload[st]);
+          mbar_arrive_expect_tx(&nrm_full[st], NT * 4);
+          bulk_load(nrm + st * NT, kn + static_cast<int64_t>(tile) * NT, NT * 4, &nrm_full[st]);
+          mbar_wait(&bar_kload[st], (t >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
           tc_fence_after();
           issue_mmas(st);
         }
+        // every copy is waited for before the final barrier: the images
+        // here, the norms by the rows
       }
       __syncwarp();   // warp 4 converges before the final barrier
     } else {
@@ -382,16 +389,33 @@ __global__ void __launch_bounds__(kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
       const int st = t & 1;
       mbar_wait(&bar_full[st], (t >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
       // the pre-split norms come by bulk copy: observe its completion here too
-      if (presplit) mbar_wait(&bar_load[st], (t >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
+      const int ns = st;
+      if (presplit) mbar_wait(&nrm_full[st], (t >> 1) & 1, a.timeout_ns, nullptr, kSiteMma);
       tc_fence_after();
       const int c0 = (t % n_tiles) * NT;
+      if constexpr (PRE) {
+        // the next group's TMEM load is in flight while this group is tested
+        uint32_t sv0[32], sv1[32];
+        tmem_ld32(trow + st * NT, sv0);
+        tmem_ld_wait(sv0);
+#pragma unroll
+        for (int cc = 0; cc < NT / 32; ++cc) {
+          uint32_t(&cur)[32] = (cc & 1) ? sv1 : sv0;
+          uint32_t(&nxt)[32] = (cc & 1) ? sv0 : sv1;
+          if (cc + 1 < NT / 32) tmem_ld32(trow + st * NT + (cc + 1) * 32, nxt);
+          const int cb = c0 + cc * 32;
+          group(cb, cur, nrm + ns * NT + cc * 32, cb + 32 <= lim);
+          if (cc + 1 < NT / 32) tmem_ld_wait(nxt);
+        }
+      } else {
 #pragma unroll 1
-      for (int cc = 0; cc < NT / 32; ++cc) {
-        uint32_t sv[32];
-        tmem_ld32(trow + st * NT + cc * 32, sv);
-        tmem_ld_wait(sv);
-        const int cb = c0 + cc * 32;
-        group(cb, sv, nrm + st * NT + cc * 32, cb + 32 <= lim);
+        for (int cc = 0; cc < NT / 32; ++cc) {
+          uint32_t sv[32];
+          tmem_ld32(trow + st * NT + cc * 32, sv);
+          tmem_ld_wait(sv);
+          const int cb = c0 + cc * 32;
+          group(cb, sv, nrm + ns * NT + cc * 32, cb + 32 <= lim);
+        }
       }
       tc_fence_before();
       __syncwarp();

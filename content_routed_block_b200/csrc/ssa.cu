@@ -243,12 +243,21 @@ template <int D, int KM>
 cudaError_t launch_route_tc_t(ssa::RouteArgs a, int B, cudaStream_t stream) {
   a.n_row_tiles = (a.NQB + ssa::kRtcRows - 1) / ssa::kRtcRows;
   const uint32_t smem = ssa::RtcLayout<D>::SMEM_BYTES;
-  cudaError_t e = cudaFuncSetAttribute(ssa::route_tc_kernel<D, KM>,
+  dim3 grid(a.n_row_tiles, B * a.Hq);
+  // with the pre-split key image one producer thread replaces the stager warps
+  if (a.kimg != nullptr) {
+    cudaError_t e = cudaFuncSetAttribute(ssa::route_tc_kernel<D, KM, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    ssa::route_tc_kernel<D, KM, true><<<grid, ssa::kRtcThreadsPre, smem, stream>>>(a);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaFuncSetAttribute(ssa::route_tc_kernel<D, KM, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(a.n_row_tiles, B * a.Hq);
-  ssa::route_tc_kernel<D, KM><<<grid, ssa::kRtcThreads, smem, stream>>>(a);
+  ssa::route_tc_kernel<D, KM, false><<<grid, ssa::kRtcThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
