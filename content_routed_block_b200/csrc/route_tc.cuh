@@ -45,8 +45,10 @@
 //          the bounds sa_c - E_c themselves, at most an ulp of the score.)
 //
 // One CTA owns 128 query blocks of one (b, head): thread r = row r = TMEM
-// lane r runs the per-row tests straight out of TMEM, while four other warps
-// stage the next key-summary tiles and issue their MMAs (see the kernel).
+// lane r runs the per-row tests straight out of TMEM, while the next
+// key-summary tiles are staged and their MMAs issued: from the key image that
+// rtc_split_kernel writes once per launch (one producer thread, bulk copies),
+// or, without scratch, split by four stager warps in the kernel.
 #pragma once
 
 #include "common.cuh"
@@ -164,13 +166,16 @@ __global__ void __launch_bounds__(256) rtc_split_kernel(const float* ksum, uint8
 }
 
 // Warp roles: warps 0-3 are the rows (thread r = query block qb0 + r = TMEM
-// lane r) and scan every tile's scores; warps 4-7 stage the key-summary tiles
-// (eight lanes per key block: load, split into bf16 hi / lo, norm) into one of
-// two stages, and thread 128 issues the tile's three MMAs into one of two
-// TMEM accumulators.  The tiles of both passes form one stream, so the
-// staging of the next tiles overlaps the scan of the current one.  Barriers:
-// acc_full[b] (MMAs of a tile into accumulator b done), acc_empty[b] (the rows
-// have read accumulator b and the norms of stage b).
+// lane r) and scan every tile's scores.  PRE (160 threads): thread 128 copies
+// each tile's pre-split image and norms into one of two stages and issues its
+// three MMAs into one of two TMEM accumulators.  Otherwise (256 threads)
+// warps 4-7 stage the tiles themselves (eight lanes per key block: load,
+// split into bf16 hi / lo, norm) and thread 128 issues the MMAs.  The tiles of
+// both passes form one stream, so the staging of the next tile overlaps the
+// scan of the current one.  Barriers: acc_full[b] (MMAs of a tile into
+// accumulator b done), acc_empty[b] (the rows have read accumulator b and the
+// norms of stage b), and with PRE kload[b] / nrm_full[b] (the stage's image
+// and norms have landed).
 template <int D, int KM, bool PRE>
 __global__ void __launch_bounds__(PRE ? kRtcThreadsPre : kRtcThreads, (D == 64 && KM <= 16) ? 2 : 1)
     route_tc_kernel(const RouteArgs a) {
