@@ -1343,7 +1343,9 @@ ssa_status ssa_decode(const ssa_params* p, const void* q, const void* k_cache, c
   a.i = n_ctx - 1;
   a.nb = a.i / p->block_k;
   // about two CTAs per SM in each phase; a route split scans >= 32 blocks
-  // and a key split >= 256 keys (32 per warp)
+  // and a key split >= 128 keys (the attend kernel's warps take 32 keys a
+  // step; measured: 256-key minimum 42.4 us, 128-key 39.2 us per step on the
+  // 8K-token, 64-head needle cache; unchanged at 1M and 32K tokens)
   const int64_t want_s = (2 * 148 + static_cast<int64_t>(p->B) * p->Hkv - 1) /
                          (static_cast<int64_t>(p->B) * p->Hkv);
   int64_t S = std::min<int64_t>(std::min<int64_t>(ssa::kDecMaxSplits, want_s), (a.nb + 31) / 32);
@@ -1356,7 +1358,7 @@ ssa_status ssa_decode(const ssa_params* p, const void* q, const void* k_cache, c
   a.S = static_cast<int32_t>(S);
   const int64_t lmax = static_cast<int64_t>(p->top_k) * p->block_k + p->window;
   const int64_t want_ks = (2 * 148 + static_cast<int64_t>(heads) - 1) / static_cast<int64_t>(heads);
-  int64_t KS = std::min<int64_t>(std::min<int64_t>(ssa::kDecMaxSplits, want_ks), (lmax + 255) / 256);
+  int64_t KS = std::min<int64_t>(std::min<int64_t>(ssa::kDecMaxSplits, want_ks), (lmax + 127) / 128);
   a.KS = static_cast<int32_t>(std::max<int64_t>(KS, 1));
   const float scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
   a.scale_log2 = scale * 1.4426950408889634f;
